@@ -1,0 +1,214 @@
+/*
+ * fp8train.h — C ABI of the B200 (sm_100a) FP8 delayed-scaling Linear step and fused AdamW.
+ *
+ * One Linear layer's training step, HYBRID recipe, per-tensor delayed scaling:
+ *
+ *   cast X, W (E4M3) and dY (E5M2)      fp8_cast_transpose_amax   (x3)
+ *   Y  = X  . W        (fprop)          fp8_gemm
+ *   dX = dY . W^T      (dgrad)          fp8_gemm
+ *   dW = X^T . dY      (wgrad)          fp8_gemm
+ *   amax history roll + next scales     fp8_scale_update
+ *   unscale, clip, AdamW, BF16 weight   fused_adamw_multi_tensor
+ *
+ * Sources, cited by page title and section:
+ *   [P1] "算子与编译器：FP8 训练与优化器 Kernel" (charles2530.github.io)
+ *   [P2] "FP8 混合精度训练工程实践：从 H100 到大模型训练的范式跃迁" (ybb.press)
+ *   [P3] "LLM FP8 微调上线生产实战：用 Amax Scaling、层级白名单与 BF16 回退守住收敛" (oh-bug.com)
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer argument whose name starts with d_, and every tensor argument, is DEVICE
+ *     memory on the current CUDA device, owned by the caller. The library allocates no device
+ *     memory and keeps no pointer after a call returns.
+ *   - All matrices are row-major and contiguous. BF16 is stored as uint16 bit patterns, FP8 as
+ *     one byte per element (E4M3: 1-4-3 bits, bias 7, max 448; E5M2: 1-5-2 bits, bias 15,
+ *     max 57344 [P2 §一]).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*; NULL is the
+ *     legacy default stream). Scalars that the GPU produces (scales, amax, norms) travel by
+ *     device pointer, so a step never synchronises with the host.
+ *   - Arguments are validated on the host before anything is launched. An invalid argument
+ *     returns an error status and launches nothing. A launch failure returns FP8T_ERR_CUDA;
+ *     fp8t_last_error_message() describes the last failure on the calling thread.
+ *   - Waits inside kernels are bounded in time. When one expires the kernel records it in a
+ *     device error word and returns early; fp8t_check_device_error() reports it.
+ */
+#ifndef FP8TRAIN_H
+#define FP8TRAIN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum fp8t_status {
+    FP8T_OK = 0,
+    FP8T_ERR_INVALID_ARG = 1,       /* NULL pointer, non-positive size, unknown enum value     */
+    FP8T_ERR_UNSUPPORTED_SHAPE = 2, /* a dimension is not a multiple of 16, or is too large    */
+    FP8T_ERR_MISALIGNED = 3,        /* a pointer is not 16-byte aligned                          */
+    FP8T_ERR_UNSUPPORTED_DEVICE = 4,/* the current device is not sm_100                         */
+    FP8T_ERR_CUDA = 5,              /* a CUDA runtime or driver call failed                      */
+    FP8T_ERR_TIMEOUT = 6            /* a bounded wait inside a kernel expired                    */
+} fp8t_status;
+
+typedef enum fp8t_format {
+    FP8T_E4M3 = 0, /* forward tensors X and W under HYBRID [P3 核心原理, E4M3 与 E5M2 承担不同职责] */
+    FP8T_E5M2 = 1  /* the output gradient dY under HYBRID                                        */
+} fp8t_format;
+
+typedef enum fp8t_amax_algo {
+    FP8T_AMAX_MAX = 0,         /* representative amax = largest entry of the history window  */
+    FP8T_AMAX_MOST_RECENT = 1  /* representative amax = the newest entry                       */
+} fp8t_amax_algo;             /* [P3 核心原理, Delayed Scaling 用历史换取稳定性, strategy table] */
+
+/*
+ * fp8_cast_transpose_amax — quantise one BF16 matrix to FP8 with a given per-tensor scale,
+ * emit it row-major and transposed, and measure its amax.
+ *
+ * Defines: the saturating quantise q = sat(x * scale) of the FP8Tensor quantize step
+ * [P2 §四, Delayed Scaling 核心逻辑], the amax = max|x| statistic it records [same], and the
+ * zero-fraction / saturation / non-finite counts of [P3 工程落地, 第四步 metrics table].
+ *
+ *   x_bf16          rows x cols BF16, row-major (input).
+ *   rows, cols      > 0, multiples of 16, rows*cols < 2^40.
+ *   fmt             FP8T_E4M3 or FP8T_E5M2.
+ *   d_scale         1 float: the scale to apply (delayed scaling: produced by the previous
+ *                   fp8_scale_update). Read only.
+ *   q_rowmajor      rows x cols FP8 bytes, row-major, or NULL to skip.
+ *   q_transposed    cols x rows FP8 bytes (q^T, row-major), or NULL to skip.
+ *   d_amax_out      1 float, overwritten with max|x| over the BF16 input (NaN if any input is NaN).
+ *   d_scale_inv_out 1 float, overwritten with 1/scale (IEEE division), or NULL to skip.
+ *   d_counters      3 x uint64, or NULL: ADDED to [0] #saturated (|f32(x*scale)| > FP8 max),
+ *                   [1] #zero codes (q is +0 or -0), [2] #non-finite inputs.
+ *   Element rule:   q = encode_fmt(f32(x) * scale), one IEEE f32 multiply rounded to nearest,
+ *                   then round-to-nearest-even to the format with saturation to +-max (an
+ *                   infinite product saturates too); a NaN input gives the byte 0x7F.
+ *   Pointers must be 16-byte aligned (except d_* scalars, 4- or 8-byte aligned).
+ */
+fp8t_status fp8_cast_transpose_amax(const void* x_bf16, int64_t rows, int64_t cols, fp8t_format fmt,
+                                    const float* d_scale, void* q_rowmajor, void* q_transposed,
+                                    float* d_amax_out, float* d_scale_inv_out,
+                                    unsigned long long* d_counters, void* stream);
+
+/*
+ * fp8_gemm — per-tensor scaled FP8 GEMM, FP32 accumulation, BF16 output, "TN" layout:
+ *
+ *   D[i][j] = bf16_rn( (sum_k A[i][k] * B[j][k]) * (a_scale_inv * b_scale_inv) )
+ *
+ * Defines: the FP8 GEMM of the recipe table with an FP32 accumulator and a 16-bit output
+ * [P2 §三, 标准 FP8 Training Recipe], dequantised by the per-tensor scales [P2 §四, dequantize;
+ * P2 §五, per-tensor mode of the FP8 GEMM table: FP8 x FP8, FP32 accumulate, BF16 out].
+ * The three GEMMs of the step are all of this form (W stored in x out):
+ *   fprop  Y  = X.W     : A = Xq   (T x in),   B = Wq^T  (out x in), M=T,  N=out, K=in
+ *   dgrad  dX = dY.W^T  : A = dYq  (T x out),  B = Wq    (in x out), M=T,  N=in,  K=out
+ *   wgrad  dW = X^T.dY  : A = Xq^T (in x T),   B = dYq^T (out x T),  M=in, N=out, K=T
+ *
+ *   A               M x K FP8 bytes, row-major (K contiguous), format a_fmt.
+ *   B               N x K FP8 bytes, row-major (K contiguous), format b_fmt.
+ *   M, N, K         > 0, multiples of 16, each < 2^31.
+ *   d_a_scale_inv, d_b_scale_inv   1 float each (device); their f32 product scales the sum.
+ *   D_bf16          M x N BF16, row-major (output, overwritten).
+ *   A, B, D must be 16-byte aligned. The accumulation order over k is unspecified; the result is
+ *   within 2 BF16 ulp + 1e-5 * sum_k |A[i][k] B[j][k]| * scale of the exact value.
+ */
+fp8t_status fp8_gemm(const void* A, fp8t_format a_fmt, const void* B, fp8t_format b_fmt,
+                     int64_t M, int64_t N, int64_t K,
+                     const float* d_a_scale_inv, const float* d_b_scale_inv,
+                     void* D_bf16, void* stream);
+
+/*
+ * fp8_scale_update — roll each tensor's amax history and compute the next scale
+ * [P3 核心原理, Scale 决定数值是否进入可表示区间 (scale = (FP8_MAX / amax) / 2^margin) and
+ *  Delayed Scaling 用历史换取稳定性 (history window; max / most_recent; used next iteration)].
+ *
+ * For each tensor t in [0, n_tensors):
+ *   history row t is shifted by one (entry H-1 is dropped) and entry 0 becomes d_amax[t];
+ *   rep   = max over the row of |h| (NaN if any entry is NaN)   for FP8T_AMAX_MAX,
+ *           |h[0]|                                              for FP8T_AMAX_MOST_RECENT;
+ *   scale = (d_fp8_max[t] / rep) * 2^-margin   (IEEE f32 division, then an exact power-of-two
+ *           multiply; +inf becomes FLT_MAX)     if rep is finite and > 0,
+ *           1.0                                 if rep == 0,
+ *           unchanged                           if rep is NaN or inf;
+ *   scale_inv = 1 / scale (IEEE f32 division).
+ *
+ *   n_tensors       1 .. 65535.
+ *   d_amax          n floats (input).
+ *   d_amax_history  n x history_len floats, row-major, index 0 = newest (in/out).
+ *   history_len     1 .. 65536.
+ *   d_fp8_max       n floats: 448 for E4M3 tensors, 57344 for E5M2 tensors (input).
+ *   margin          0 .. 126.
+ *   d_scale, d_scale_inv   n floats each (in/out, out).
+ */
+fp8t_status fp8_scale_update(int32_t n_tensors, const float* d_amax, float* d_amax_history,
+                             int32_t history_len, const float* d_fp8_max, fp8t_amax_algo algo,
+                             int32_t margin, float* d_scale, float* d_scale_inv, void* stream);
+
+/* One parameter tensor of the multi-tensor AdamW: device pointers, 16-byte aligned. */
+typedef struct fp8t_adamw_tensor {
+    float* master;          /* FP32 master weight, numel (in/out)                 */
+    float* m;               /* FP32 first moment, numel (in/out)                  */
+    float* v;               /* FP32 second moment, numel (in/out)                 */
+    const void* grad_bf16;  /* BF16 gradient of the loss-scaled loss, numel (in)  */
+    void* weight_bf16;      /* BF16 copy of the updated master, numel (out)       */
+    int64_t numel;          /* > 0                                                */
+} fp8t_adamw_tensor;
+
+/*
+ * fused_adamw_multi_tensor — one fused AdamW step over many tensors [P1 Fused Optimizer 的意义
+ * (read grad, update first/second moments, bias correction, weight decay, parameter update in
+ * one kernel); P1 FP8 训练主路径图 (unscale / clip before the optimizer); P2 §四, precision flow
+ * (gradient un-scaling by the loss scale, FP32 AdamW)].
+ *
+ *   norm  = sqrt(sum over all tensors of f32(g)^2, accumulated in FP64) / loss_scale
+ *   If norm is not finite nothing is updated and *d_skipped_out = 1; otherwise *d_skipped_out = 0,
+ *   coef  = (max_grad_norm > 0 && norm > max_grad_norm) ? max_grad_norm / norm : 1
+ *   and each element, in f32 with every operation rounded separately (no fused multiply-add):
+ *     g = f32(grad) * (coef * (1/loss_scale))
+ *     m = beta1*m + (1-beta1)*g ;  v = beta2*v + (1-beta2)*g*g
+ *     p = p * (1 - lr*wd)                                           (decoupled weight decay)
+ *     p = p - (lr / (1-beta1^step)) * (m / (sqrt(v) / sqrt(1-beta2^step) + eps))
+ *     weight_bf16 = bf16_rne(p)
+ *   where 1-beta1, 1-beta2, 1-lr*wd, lr/(1-beta1^step) and sqrt(1-beta2^step) are computed
+ *   in double on the host and rounded once to f32.
+ *
+ *   tensors         HOST array of n_tensors descriptors (read during the call only).
+ *   n_tensors       1 .. 1<<20.
+ *   step            >= 1 (bias-correction step count).
+ *   loss_scale      > 0 and finite.  max_grad_norm <= 0 disables clipping.
+ *   d_grad_norm_out 1 float (device) or NULL: the unscaled global norm.
+ *   d_skipped_out   1 int32 (device) or NULL.
+ *   d_workspace     device scratch of at least fused_adamw_workspace_bytes() bytes, 16-byte
+ *                   aligned; its contents on entry are ignored.
+ */
+fp8t_status fused_adamw_multi_tensor(const fp8t_adamw_tensor* tensors, int32_t n_tensors,
+                                     float lr, float beta1, float beta2, float eps,
+                                     float weight_decay, int64_t step, float loss_scale,
+                                     float max_grad_norm, float* d_grad_norm_out,
+                                     int32_t* d_skipped_out, void* d_workspace,
+                                     size_t workspace_bytes, void* stream);
+
+/* Scratch bytes fused_adamw_multi_tensor needs for these tensors (0 on invalid input). */
+size_t fused_adamw_workspace_bytes(const fp8t_adamw_tensor* tensors, int32_t n_tensors);
+
+/* Synchronise `stream`, then read and clear the device error word: FP8T_ERR_TIMEOUT if a bounded
+ * wait in any kernel expired since the last check, FP8T_ERR_CUDA if the stream reports an error. */
+fp8t_status fp8t_check_device_error(void* stream);
+
+/* Override the time limit of the bounded waits in the GEMM (nanoseconds; 0 restores the default
+ * of 2 s). Meant for tests of the timeout path; takes effect for launches after the call. */
+fp8t_status fp8t_set_wait_timeout_ns(uint64_t ns);
+
+/* Human-readable name of a status code; never NULL. */
+const char* fp8t_status_string(fp8t_status status);
+
+/* Message describing the last failure on the calling thread ("" if none). */
+const char* fp8t_last_error_message(void);
+
+/* ABI version of this header: 1. */
+int32_t fp8t_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8TRAIN_H */

@@ -1,0 +1,27 @@
+"""Compile the CPU oracle (fp8_oracle.c) into liboracle.so with gcc.
+
+Test infrastructure: the oracle is the checker, never part of the product path.
+Plain IEEE arithmetic: -O2 -ffp-contract=off, no -ffast-math, no -march (no FMA contraction).
+"""
+import os
+import subprocess
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "fp8_oracle.c")
+LIB = os.path.join(HERE, "liboracle.so")
+
+
+def build_oracle(force: bool = False) -> str:
+    """Build liboracle.so if it is missing or older than its source; return its path."""
+    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
+        return LIB
+    tmp = LIB + ".tmp.%d" % os.getpid()
+    cmd = ["gcc", "-std=c11", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
+           "-Wall", "-Wextra", "-o", tmp, SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build_oracle(force=True))
