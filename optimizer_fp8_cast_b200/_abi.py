@@ -1,0 +1,42 @@
+"""ctypes declarations of the C ABI in include/fp8train.h (argument and return types only)."""
+import ctypes as C
+
+STATUS = {0: "FP8T_OK", 1: "FP8T_ERR_INVALID_ARG", 2: "FP8T_ERR_UNSUPPORTED_SHAPE",
+          3: "FP8T_ERR_MISALIGNED", 4: "FP8T_ERR_UNSUPPORTED_DEVICE", 5: "FP8T_ERR_CUDA",
+          6: "FP8T_ERR_TIMEOUT"}
+
+
+def status_name(s):
+    return STATUS.get(int(s), f"status {int(s)}")
+
+
+class AdamWTensor(C.Structure):
+    """fp8t_adamw_tensor."""
+    _fields_ = [("master", C.c_void_p), ("m", C.c_void_p), ("v", C.c_void_p),
+                ("grad_bf16", C.c_void_p), ("weight_bf16", C.c_void_p), ("numel", C.c_int64)]
+
+
+def declare(L):
+    vp, i32, i64, f32 = C.c_void_p, C.c_int32, C.c_int64, C.c_float
+    L.fp8_cast_transpose_amax.restype = C.c_int
+    L.fp8_cast_transpose_amax.argtypes = [vp, i64, i64, C.c_int, vp, vp, vp, vp, vp, vp, vp]
+    L.fp8_gemm.restype = C.c_int
+    L.fp8_gemm.argtypes = [vp, C.c_int, vp, C.c_int, i64, i64, i64, vp, vp, vp, vp]
+    L.fp8_scale_update.restype = C.c_int
+    L.fp8_scale_update.argtypes = [i32, vp, vp, i32, vp, C.c_int, i32, vp, vp, vp]
+    L.fused_adamw_multi_tensor.restype = C.c_int
+    L.fused_adamw_multi_tensor.argtypes = [C.POINTER(AdamWTensor), i32, f32, f32, f32, f32, f32,
+                                           i64, f32, f32, vp, vp, vp, C.c_size_t, vp]
+    L.fused_adamw_workspace_bytes.restype = C.c_size_t
+    L.fused_adamw_workspace_bytes.argtypes = [C.POINTER(AdamWTensor), i32]
+    L.fp8t_check_device_error.restype = C.c_int
+    L.fp8t_check_device_error.argtypes = [vp]
+    L.fp8t_set_wait_timeout_ns.restype = C.c_int
+    L.fp8t_set_wait_timeout_ns.argtypes = [C.c_uint64]
+    L.fp8t_status_string.restype = C.c_char_p
+    L.fp8t_status_string.argtypes = [C.c_int]
+    L.fp8t_last_error_message.restype = C.c_char_p
+    L.fp8t_last_error_message.argtypes = []
+    L.fp8t_abi_version.restype = i32
+    L.fp8t_abi_version.argtypes = []
+    return L

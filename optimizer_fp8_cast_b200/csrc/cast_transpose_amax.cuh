@@ -1,0 +1,166 @@
+// cast_transpose_amax.cuh — BF16 -> FP8 quantise with a per-tensor scale, row-major and
+// transposed outputs, amax and quality counters, in one pass over HBM.
+//
+// Method: the FP8Tensor quantize step of "FP8 混合精度训练工程实践" §四 (amax = max|x|;
+// q = clamp(x * scale) stored as FP8) with the HYBRID format choice of "LLM FP8 微调上线生产实战"
+// (核心原理: E4M3 forward, E5M2 gradients) and its saturation / zero-fraction metrics (第四步).
+//
+// Layout: one CTA per 128 x 128 tile. Each of 256 threads reads four 16-element row segments
+// with 16-byte loads (a warp covers four full 256-byte row segments), converts them, writes 16
+// FP8 bytes row-major and stages them in shared memory. The staged tile is 16-byte-chunk XOR
+// swizzled by (row / 16) so that the transposing read, in which thread (row group ig, word
+// column jg) gathers a 16 x 4 byte block, is free of bank conflicts. Blocks of 4 x 4 bytes are
+// transposed with byte permutes, and each thread writes four 16-byte pieces of q^T rows; the 8
+// threads of a row group write 128 contiguous bytes. Algorithmic traffic: 2 B read + 2 B
+// written per element.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace fp8t {
+namespace cast {
+
+constexpr int kTile = 128;
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) { return __reduce_max_sync(0xffffffffu, v); }
+__device__ __forceinline__ uint32_t warp_add_u32(uint32_t v) { return __reduce_add_sync(0xffffffffu, v); }
+
+template <int FMT, bool COUNT>
+__global__ void __launch_bounds__(kThreads)
+    k_cast_transpose_amax(const uint16_t* __restrict__ x, int64_t rows, int64_t cols,
+                          int64_t tiles_c, const float* __restrict__ d_scale,
+                          uint8_t* __restrict__ q, uint8_t* __restrict__ qT,
+                          unsigned int* __restrict__ amax_bits,
+                          unsigned long long* __restrict__ counters,
+                          float* __restrict__ scale_inv_out) {
+  __shared__ __align__(16) uint32_t tile[kTile * kTile / 4];  // 128 rows x 128 bytes
+  __shared__ uint32_t red[4][kThreads / 32];
+
+  constexpr float kMax = FMT == 0 ? 448.0f : 57344.0f;
+  const float s = __ldg(d_scale);
+  const int tid = threadIdx.x;
+  const int64_t r0 = (static_cast<int64_t>(blockIdx.x) / tiles_c) * kTile;
+  const int64_t c0 = (static_cast<int64_t>(blockIdx.x) % tiles_c) * kTile;
+
+  uint32_t vmax = 0, nsat = 0, nzero = 0, nnonfinite = 0;
+
+  // ---- phase 1: load 4 segments of 16 BF16 per thread, quantise, store row-major + stage
+  uint4 in[4][2];
+  bool ok[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int seg = tid + kThreads * k;
+    const int64_t gr = r0 + (seg >> 3), gc = c0 + 16 * (seg & 7);
+    ok[k] = gr < rows && gc < cols;
+    if (ok[k]) {
+      const uint16_t* p = x + gr * cols + gc;
+      in[k][0] = ld_stream_u4(p);
+      in[k][1] = ld_stream_u4(p + 8);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int seg = tid + kThreads * k;
+    const int row = seg >> 3, c16 = seg & 7;
+    uint32_t packed[4] = {0u, 0u, 0u, 0u};
+    if (ok[k]) {
+      const uint32_t* w = reinterpret_cast<const uint32_t*>(&in[k][0]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t h0 = w[j] & 0xFFFFu, h1 = w[j] >> 16;
+        const uint32_t m0 = h0 & 0x7FFFu, m1 = h1 & 0x7FFFu;
+        vmax = max(vmax, max(m0, m1));
+        const float p0 = __fmul_rn(__uint_as_float(h0 << 16), s);
+        const float p1 = __fmul_rn(__uint_as_float(w[j] & 0xFFFF0000u), s);
+        uint32_t pair = cvt_fp8x2<FMT>(p0, p1);
+        // a NaN input (or NaN product) is stored as 0x7F whatever its sign
+        if (p0 != p0) pair = (pair & 0xFF00u) | 0x7Fu;
+        if (p1 != p1) pair = (pair & 0x00FFu) | 0x7F00u;
+        packed[j >> 1] |= pair << (16 * (j & 1));
+        if (COUNT) {
+          nsat += (fabsf(p0) > kMax) + (fabsf(p1) > kMax);
+          nzero += ((pair & 0x7Fu) == 0) + ((pair & 0x7F00u) == 0);
+          nnonfinite += (m0 >= 0x7F80u) + (m1 >= 0x7F80u);
+        }
+      }
+      if (q) {
+        const int64_t gr = r0 + row, gc = c0 + 16 * c16;
+        *reinterpret_cast<uint4*>(q + gr * cols + gc) =
+            make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      }
+    }
+    const int pchunk = c16 ^ ((row >> 4) & 7);
+    *reinterpret_cast<uint4*>(&tile[row * 32 + pchunk * 4]) =
+        make_uint4(packed[0], packed[1], packed[2], packed[3]);
+  }
+
+  // ---- block reductions (partials to shared memory before the barrier)
+  const int lane = tid & 31, warp = tid >> 5;
+  vmax = warp_max_u32(vmax);
+  if (COUNT) {
+    nsat = warp_add_u32(nsat);
+    nzero = warp_add_u32(nzero);
+    nnonfinite = warp_add_u32(nnonfinite);
+  }
+  if (lane == 0) {
+    red[0][warp] = vmax;
+    red[1][warp] = nsat;
+    red[2][warp] = nzero;
+    red[3][warp] = nnonfinite;
+  }
+  __syncthreads();
+
+  if (tid == 0) {
+    uint32_t m = 0, a = 0, b = 0, c = 0;
+#pragma unroll
+    for (int i = 0; i < kThreads / 32; ++i) {
+      m = max(m, red[0][i]);
+      a += red[1][i];
+      b += red[2][i];
+      c += red[3][i];
+    }
+    if (m > 0x7F80u) m = 0x7FC0u;  // canonical NaN
+    atomicMax(amax_bits, m << 16);
+    if (COUNT) {
+      if (a) atomicAdd(counters + 0, static_cast<unsigned long long>(a));
+      if (b) atomicAdd(counters + 1, static_cast<unsigned long long>(b));
+      if (c) atomicAdd(counters + 2, static_cast<unsigned long long>(c));
+    }
+    if (scale_inv_out && blockIdx.x == 0) *scale_inv_out = __fdiv_rn(1.0f, s);
+  }
+
+  // ---- phase 2: transposed output, 16 q-rows x 4 q-columns per thread
+  if (qT) {
+    const int ig = lane & 7;                  // row group: q rows 16*ig .. 16*ig+15
+    const int jg = 4 * warp + (lane >> 3);    // word column: q columns 4*jg .. 4*jg+3
+    const int64_t grow = r0 + 16 * ig, gcol = c0 + 4 * jg;
+    if (grow < rows && gcol < cols) {
+      uint32_t v[16];
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        const int row = 16 * ig + r;
+        const int chunk = (jg >> 2) ^ ig;     // (row >> 4) & 7 == ig
+        v[r] = tile[row * 32 + chunk * 4 + (jg & 3)];
+      }
+      uint32_t o[4][4];
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint32_t a = v[4 * kk], b = v[4 * kk + 1], c = v[4 * kk + 2], d = v[4 * kk + 3];
+        const uint32_t t0 = __byte_perm(a, b, 0x5140), t1 = __byte_perm(a, b, 0x7362);
+        const uint32_t u0 = __byte_perm(c, d, 0x5140), u1 = __byte_perm(c, d, 0x7362);
+        o[0][kk] = __byte_perm(t0, u0, 0x5410);
+        o[1][kk] = __byte_perm(t0, u0, 0x7632);
+        o[2][kk] = __byte_perm(t1, u1, 0x5410);
+        o[3][kk] = __byte_perm(t1, u1, 0x7632);
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        *reinterpret_cast<uint4*>(qT + (gcol + c) * rows + grow) =
+            make_uint4(o[c][0], o[c][1], o[c][2], o[c][3]);
+    }
+  }
+}
+
+}  // namespace cast
+}  // namespace fp8t

@@ -1,0 +1,394 @@
+// fp8train.cu — the C ABI declared in include/fp8train.h: host-side validation, launch
+// configuration and tensor-map encoding for the four kernels of the FP8 delayed-scaling Linear
+// step. Every argument is checked before the first CUDA call, so invalid input returns an error
+// status and launches nothing; there is no fallback path.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "fp8train.h"
+#include "cast_transpose_amax.cuh"
+#include "fused_adamw.cuh"
+#include "gemm_tcgen05.cuh"
+#include "scale_update.cuh"
+
+namespace {
+
+thread_local std::string t_last_error;
+
+fp8t_status fail(fp8t_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return s;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  int state = 0;               // 0 unknown, 1 sm_100, 2 other
+  int sms = 0;
+  int adamw_blocks_per_sm = 0;
+  bool gemm_smem_set = false;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mutex;
+
+// Current device must be compute capability 10.0 (sm_100a code runs there only).
+fp8t_status current_device(DeviceInfo** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(FP8T_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(FP8T_ERR_UNSUPPORTED_DEVICE, "device index %d", dev);
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  DeviceInfo& d = g_dev[dev];
+  if (d.state == 0) {
+    int major = 0, minor = 0, sms = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return fail(FP8T_ERR_CUDA, "cudaDeviceGetAttribute: %s", cudaGetErrorString(e));
+    d.sms = sms;
+    d.state = (major == 10 && minor == 0) ? 1 : 2;
+    if (d.state == 1) {
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.adamw_blocks_per_sm,
+                                                        fp8t::adamw::k_adamw_update,
+                                                        fp8t::adamw::kThreads, 0);
+      if (e != cudaSuccess || d.adamw_blocks_per_sm < 1) d.adamw_blocks_per_sm = 1;
+      e = cudaFuncSetAttribute(fp8t::gemm::k_fp8_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fp8t::gemm::kSmemBytes);
+      if (e != cudaSuccess) {
+        d.state = 0;
+        return fail(FP8T_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+      }
+      d.gemm_smem_set = true;
+    }
+  }
+  if (d.state != 1) return fail(FP8T_ERR_UNSUPPORTED_DEVICE, "device %d is not sm_100", dev);
+  *out = &d;
+  return FP8T_OK;
+}
+
+fp8t_status after_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(FP8T_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return FP8T_OK;
+}
+
+// ------------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// rows x K bytes, row-major: boxes of box_rows rows x 128 bytes, 128-byte swizzle, zero fill.
+fp8t_status encode_kmajor(CUtensorMap* map, const void* ptr, int64_t rows, int64_t K,
+                          uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(FP8T_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(fp8t::gemm::kBK), box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box,
+                  es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FP8T_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return FP8T_OK;
+}
+
+// ------------------------------------------------------------------ AdamW helpers
+struct AdamWPlan {
+  int nbatches = 0;
+  int64_t nparts = 0;
+};
+
+int64_t chunks_of(int64_t numel) { return (numel + fp8t::adamw::kChunk - 1) / fp8t::adamw::kChunk; }
+
+AdamWPlan plan_adamw(const fp8t_adamw_tensor* t, int32_t n) {
+  AdamWPlan p;
+  for (int32_t b0 = 0; b0 < n; b0 += fp8t::adamw::kMaxTensors) {
+    int64_t chunks = 0;
+    const int32_t b1 = std::min<int32_t>(n, b0 + fp8t::adamw::kMaxTensors);
+    for (int32_t i = b0; i < b1; ++i) chunks += chunks_of(t[i].numel);
+    p.nparts += std::min<int64_t>(chunks, fp8t::adamw::kSumsqBlocks);
+    ++p.nbatches;
+  }
+  return p;
+}
+
+size_t workspace_for(const AdamWPlan& p) {
+  return static_cast<size_t>((p.nparts * 8 + 255) / 256 * 256);
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t fp8t_abi_version(void) { return 1; }
+
+const char* fp8t_last_error_message(void) { return t_last_error.c_str(); }
+
+const char* fp8t_status_string(fp8t_status s) {
+  switch (s) {
+    case FP8T_OK: return "FP8T_OK";
+    case FP8T_ERR_INVALID_ARG: return "FP8T_ERR_INVALID_ARG";
+    case FP8T_ERR_UNSUPPORTED_SHAPE: return "FP8T_ERR_UNSUPPORTED_SHAPE";
+    case FP8T_ERR_MISALIGNED: return "FP8T_ERR_MISALIGNED";
+    case FP8T_ERR_UNSUPPORTED_DEVICE: return "FP8T_ERR_UNSUPPORTED_DEVICE";
+    case FP8T_ERR_CUDA: return "FP8T_ERR_CUDA";
+    case FP8T_ERR_TIMEOUT: return "FP8T_ERR_TIMEOUT";
+  }
+  return "FP8T_UNKNOWN_STATUS";
+}
+
+// ------------------------------------------------------------------ cast / transpose / amax
+fp8t_status fp8_cast_transpose_amax(const void* x_bf16, int64_t rows, int64_t cols, fp8t_format fmt,
+                                    const float* d_scale, void* q_rowmajor, void* q_transposed,
+                                    float* d_amax_out, float* d_scale_inv_out,
+                                    unsigned long long* d_counters, void* stream) {
+  t_last_error.clear();
+  if (!x_bf16 || !d_scale || !d_amax_out)
+    return fail(FP8T_ERR_INVALID_ARG, "fp8_cast_transpose_amax: NULL input, scale or amax pointer");
+  if (fmt != FP8T_E4M3 && fmt != FP8T_E5M2)
+    return fail(FP8T_ERR_INVALID_ARG, "fp8_cast_transpose_amax: unknown format %d", (int)fmt);
+  if (rows <= 0 || cols <= 0)
+    return fail(FP8T_ERR_INVALID_ARG, "fp8_cast_transpose_amax: rows and cols must be > 0");
+  if (rows % 16 || cols % 16 || rows > (int64_t(1) << 31) || cols > (int64_t(1) << 31) ||
+      rows * cols >= (int64_t(1) << 40))
+    return fail(FP8T_ERR_UNSUPPORTED_SHAPE,
+                "fp8_cast_transpose_amax: rows and cols must be multiples of 16, rows*cols < 2^40");
+  if (!aligned(x_bf16, 16) || !aligned(q_rowmajor, 16) || !aligned(q_transposed, 16) ||
+      !aligned(d_scale, 4) || !aligned(d_amax_out, 4) || !aligned(d_scale_inv_out, 4) ||
+      !aligned(d_counters, 8))
+    return fail(FP8T_ERR_MISALIGNED, "fp8_cast_transpose_amax: misaligned pointer");
+  DeviceInfo* dev = nullptr;
+  fp8t_status st = current_device(&dev);
+  if (st != FP8T_OK) return st;
+
+  cudaStream_t s = as_stream(stream);
+  cudaError_t e = cudaMemsetAsync(d_amax_out, 0, sizeof(float), s);
+  if (e != cudaSuccess) return fail(FP8T_ERR_CUDA, "cudaMemsetAsync(amax): %s", cudaGetErrorString(e));
+  using namespace fp8t::cast;
+  const int64_t tiles_c = (cols + kTile - 1) / kTile;
+  const int64_t tiles = ((rows + kTile - 1) / kTile) * tiles_c;
+  auto* xq = static_cast<const uint16_t*>(x_bf16);
+  auto* q = static_cast<uint8_t*>(q_rowmajor);
+  auto* qT = static_cast<uint8_t*>(q_transposed);
+  auto* amax = reinterpret_cast<unsigned int*>(d_amax_out);
+  const dim3 grid(static_cast<unsigned>(tiles));
+  if (fmt == FP8T_E4M3) {
+    if (d_counters)
+      k_cast_transpose_amax<0, true><<<grid, kThreads, 0, s>>>(xq, rows, cols, tiles_c, d_scale, q, qT, amax, d_counters, d_scale_inv_out);
+    else
+      k_cast_transpose_amax<0, false><<<grid, kThreads, 0, s>>>(xq, rows, cols, tiles_c, d_scale, q, qT, amax, nullptr, d_scale_inv_out);
+  } else {
+    if (d_counters)
+      k_cast_transpose_amax<1, true><<<grid, kThreads, 0, s>>>(xq, rows, cols, tiles_c, d_scale, q, qT, amax, d_counters, d_scale_inv_out);
+    else
+      k_cast_transpose_amax<1, false><<<grid, kThreads, 0, s>>>(xq, rows, cols, tiles_c, d_scale, q, qT, amax, nullptr, d_scale_inv_out);
+  }
+  return after_launch("fp8_cast_transpose_amax launch");
+}
+
+// ------------------------------------------------------------------ GEMM
+fp8t_status fp8_gemm(const void* A, fp8t_format a_fmt, const void* B, fp8t_format b_fmt, int64_t M,
+                     int64_t N, int64_t K, const float* d_a_scale_inv, const float* d_b_scale_inv,
+                     void* D_bf16, void* stream) {
+  t_last_error.clear();
+  if (!A || !B || !D_bf16 || !d_a_scale_inv || !d_b_scale_inv)
+    return fail(FP8T_ERR_INVALID_ARG, "fp8_gemm: NULL pointer");
+  if ((a_fmt != FP8T_E4M3 && a_fmt != FP8T_E5M2) || (b_fmt != FP8T_E4M3 && b_fmt != FP8T_E5M2))
+    return fail(FP8T_ERR_INVALID_ARG, "fp8_gemm: unknown format");
+  if (M <= 0 || N <= 0 || K <= 0) return fail(FP8T_ERR_INVALID_ARG, "fp8_gemm: M, N, K must be > 0");
+  const int64_t lim = int64_t(1) << 31;
+  if (M % 16 || N % 16 || K % 16 || M >= lim || N >= lim || K >= lim)
+    return fail(FP8T_ERR_UNSUPPORTED_SHAPE, "fp8_gemm: M, N, K must be multiples of 16 below 2^31");
+  if (!aligned(A, 16) || !aligned(B, 16) || !aligned(D_bf16, 16) || !aligned(d_a_scale_inv, 4) ||
+      !aligned(d_b_scale_inv, 4))
+    return fail(FP8T_ERR_MISALIGNED, "fp8_gemm: misaligned pointer");
+  DeviceInfo* dev = nullptr;
+  fp8t_status st = current_device(&dev);
+  if (st != FP8T_OK) return st;
+
+  using namespace fp8t::gemm;
+  CUtensorMap ta, tb;
+  if ((st = encode_kmajor(&ta, A, M, K, kBM)) != FP8T_OK) return st;
+  if ((st = encode_kmajor(&tb, B, N, K, kBN)) != FP8T_OK) return st;
+  const int64_t tiles_n = (N + kBN - 1) / kBN;
+  const int64_t tiles = ((M + kBM - 1) / kBM) * tiles_n;
+  k_fp8_gemm<<<static_cast<unsigned>(tiles), kThreads, kSmemBytes, as_stream(stream)>>>(
+      ta, tb, static_cast<uint16_t*>(D_bf16), static_cast<int>(M), static_cast<int>(N),
+      static_cast<int>(K), d_a_scale_inv, d_b_scale_inv, make_idesc(a_fmt, b_fmt),
+      static_cast<int>(tiles_n));
+  return after_launch("fp8_gemm launch");
+}
+
+// ------------------------------------------------------------------ scale update
+fp8t_status fp8_scale_update(int32_t n_tensors, const float* d_amax, float* d_amax_history,
+                             int32_t history_len, const float* d_fp8_max, fp8t_amax_algo algo,
+                             int32_t margin, float* d_scale, float* d_scale_inv, void* stream) {
+  t_last_error.clear();
+  if (!d_amax || !d_amax_history || !d_fp8_max || !d_scale || !d_scale_inv)
+    return fail(FP8T_ERR_INVALID_ARG, "fp8_scale_update: NULL pointer");
+  if (n_tensors < 1 || n_tensors > 65535 || history_len < 1 || history_len > 65536)
+    return fail(FP8T_ERR_INVALID_ARG, "fp8_scale_update: n_tensors in 1..65535, history_len in 1..65536");
+  if (algo != FP8T_AMAX_MAX && algo != FP8T_AMAX_MOST_RECENT)
+    return fail(FP8T_ERR_INVALID_ARG, "fp8_scale_update: unknown amax algorithm %d", (int)algo);
+  if (margin < 0 || margin > 126) return fail(FP8T_ERR_INVALID_ARG, "fp8_scale_update: margin in 0..126");
+  if (!aligned(d_amax, 4) || !aligned(d_amax_history, 4) || !aligned(d_fp8_max, 4) ||
+      !aligned(d_scale, 4) || !aligned(d_scale_inv, 4))
+    return fail(FP8T_ERR_MISALIGNED, "fp8_scale_update: misaligned pointer");
+  DeviceInfo* dev = nullptr;
+  fp8t_status st = current_device(&dev);
+  if (st != FP8T_OK) return st;
+  fp8t::scale::k_scale_update<<<n_tensors, fp8t::scale::kThreads, 0, as_stream(stream)>>>(
+      d_amax, d_amax_history, history_len, d_fp8_max, algo == FP8T_AMAX_MAX ? 1 : 0, margin,
+      d_scale, d_scale_inv);
+  return after_launch("fp8_scale_update launch");
+}
+
+// ------------------------------------------------------------------ fused AdamW
+size_t fused_adamw_workspace_bytes(const fp8t_adamw_tensor* tensors, int32_t n_tensors) {
+  if (!tensors || n_tensors < 1 || n_tensors > (1 << 20)) return 0;
+  for (int32_t i = 0; i < n_tensors; ++i)
+    if (tensors[i].numel <= 0) return 0;
+  return workspace_for(plan_adamw(tensors, n_tensors));
+}
+
+fp8t_status fused_adamw_multi_tensor(const fp8t_adamw_tensor* tensors, int32_t n_tensors, float lr,
+                                     float beta1, float beta2, float eps, float weight_decay,
+                                     int64_t step, float loss_scale, float max_grad_norm,
+                                     float* d_grad_norm_out, int32_t* d_skipped_out,
+                                     void* d_workspace, size_t workspace_bytes, void* stream) {
+  t_last_error.clear();
+  if (!tensors || n_tensors < 1 || n_tensors > (1 << 20))
+    return fail(FP8T_ERR_INVALID_ARG, "fused_adamw_multi_tensor: tensors NULL or n_tensors out of range");
+  for (int32_t i = 0; i < n_tensors; ++i) {
+    const fp8t_adamw_tensor& t = tensors[i];
+    if (!t.master || !t.m || !t.v || !t.grad_bf16 || !t.weight_bf16 || t.numel <= 0)
+      return fail(FP8T_ERR_INVALID_ARG, "fused_adamw_multi_tensor: tensor %d has a NULL pointer or numel <= 0", i);
+    if (!aligned(t.master, 16) || !aligned(t.m, 16) || !aligned(t.v, 16) ||
+        !aligned(t.grad_bf16, 16) || !aligned(t.weight_bf16, 16))
+      return fail(FP8T_ERR_MISALIGNED, "fused_adamw_multi_tensor: tensor %d is not 16-byte aligned", i);
+  }
+  if (step < 1) return fail(FP8T_ERR_INVALID_ARG, "fused_adamw_multi_tensor: step must be >= 1");
+  if (!(loss_scale > 0.0f) || !std::isfinite(loss_scale) || !std::isfinite(lr) ||
+      !std::isfinite(beta1) || !std::isfinite(beta2) || !std::isfinite(eps) ||
+      !std::isfinite(weight_decay) || !std::isfinite(max_grad_norm))
+    return fail(FP8T_ERR_INVALID_ARG, "fused_adamw_multi_tensor: non-finite hyperparameter or loss_scale <= 0");
+  if (!aligned(d_grad_norm_out, 4) || !aligned(d_skipped_out, 4) || !aligned(d_workspace, 16))
+    return fail(FP8T_ERR_MISALIGNED, "fused_adamw_multi_tensor: misaligned output or workspace");
+  const AdamWPlan plan = plan_adamw(tensors, n_tensors);
+  const size_t need = workspace_for(plan);
+  if (!d_workspace || workspace_bytes < need)
+    return fail(FP8T_ERR_INVALID_ARG, "fused_adamw_multi_tensor: workspace of %zu bytes needed", need);
+  DeviceInfo* dev = nullptr;
+  fp8t_status st = current_device(&dev);
+  if (st != FP8T_OK) return st;
+
+  using namespace fp8t::adamw;
+  Scalars k;
+  k.beta1 = beta1;
+  k.beta2 = beta2;
+  k.omb1 = static_cast<float>(1.0 - static_cast<double>(beta1));
+  k.omb2 = static_cast<float>(1.0 - static_cast<double>(beta2));
+  k.decay = static_cast<float>(1.0 - static_cast<double>(lr) * static_cast<double>(weight_decay));
+  k.step_size = static_cast<float>(static_cast<double>(lr) /
+                                   (1.0 - std::pow(static_cast<double>(beta1), static_cast<double>(step))));
+  k.bc2_sqrt = static_cast<float>(std::sqrt(1.0 - std::pow(static_cast<double>(beta2), static_cast<double>(step))));
+  k.eps = eps;
+  k.inv_s_d = 1.0 / static_cast<double>(loss_scale);
+  k.inv_s = static_cast<float>(k.inv_s_d);
+  k.max_norm = max_grad_norm;
+
+  cudaStream_t s = as_stream(stream);
+  double* partials = static_cast<double*>(d_workspace);
+  static thread_local Batch batch;   // ~14 KB: kept off the stack
+  int64_t off = 0;
+  for (int pass = 0; pass < 2; ++pass) {
+    off = 0;
+    for (int32_t b0 = 0, bi = 0; b0 < n_tensors; b0 += kMaxTensors, ++bi) {
+      const int32_t b1 = std::min<int32_t>(n_tensors, b0 + kMaxTensors);
+      batch.n = b1 - b0;
+      batch.first = bi == 0 ? 1 : 0;
+      int64_t acc = 0;
+      for (int32_t i = b0; i < b1; ++i) {
+        const int j = i - b0;
+        batch.chunk_start[j] = acc;
+        acc += chunks_of(tensors[i].numel);
+        batch.numel[j] = tensors[i].numel;
+        batch.master[j] = tensors[i].master;
+        batch.m[j] = tensors[i].m;
+        batch.v[j] = tensors[i].v;
+        batch.g[j] = static_cast<const uint16_t*>(tensors[i].grad_bf16);
+        batch.w[j] = static_cast<uint16_t*>(tensors[i].weight_bf16);
+      }
+      batch.chunk_start[batch.n] = acc;
+      if (pass == 0) {
+        const int64_t grid = std::min<int64_t>(acc, kSumsqBlocks);
+        k_adamw_sumsq<<<static_cast<unsigned>(grid), kThreads, 0, s>>>(batch, partials + off);
+        off += grid;
+        if ((st = after_launch("adamw norm pass launch")) != FP8T_OK) return st;
+      } else {
+        const int64_t grid = std::min<int64_t>(acc, static_cast<int64_t>(dev->sms) * dev->adamw_blocks_per_sm);
+        k_adamw_update<<<static_cast<unsigned>(grid), kThreads, 0, s>>>(
+            batch, k, partials, static_cast<int>(plan.nparts), d_grad_norm_out, d_skipped_out);
+        if ((st = after_launch("adamw update launch")) != FP8T_OK) return st;
+      }
+    }
+  }
+  return FP8T_OK;
+}
+
+// ------------------------------------------------------------------ device error word
+fp8t_status fp8t_check_device_error(void* stream) {
+  t_last_error.clear();
+  cudaError_t e = cudaStreamSynchronize(as_stream(stream));
+  if (e != cudaSuccess) return fail(FP8T_ERR_CUDA, "stream: %s", cudaGetErrorString(e));
+  unsigned int word = 0;
+  e = cudaMemcpyFromSymbol(&word, fp8t::g_error_word, sizeof(word));
+  if (e != cudaSuccess) return fail(FP8T_ERR_CUDA, "reading the error word: %s", cudaGetErrorString(e));
+  if (word) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(fp8t::g_error_word, &zero, sizeof(zero));
+    if (e != cudaSuccess) return fail(FP8T_ERR_CUDA, "clearing the error word: %s", cudaGetErrorString(e));
+    if (word & fp8t::kErrTimeout) return fail(FP8T_ERR_TIMEOUT, "a bounded wait in a kernel expired");
+  }
+  return FP8T_OK;
+}
+
+fp8t_status fp8t_set_wait_timeout_ns(uint64_t ns) {
+  t_last_error.clear();
+  const unsigned long long v = ns;
+  cudaError_t e = cudaMemcpyToSymbol(fp8t::g_wait_timeout_ns, &v, sizeof(v));
+  if (e != cudaSuccess) return fail(FP8T_ERR_CUDA, "setting the wait limit: %s", cudaGetErrorString(e));
+  return FP8T_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,113 @@
+"""Device state and call sequence of one FP8 delayed-scaling training step of Linear layers.
+
+One step for each layer (W stored in x out, Y = X.W), following the precision flow of
+"FP8 混合精度训练工程实践" §四 and the HYBRID recipe of "LLM FP8 微调上线生产实战":
+
+  cast X, W -> E4M3 and dY -> E5M2 with the scales of the previous step (delayed scaling)
+  Y  = Xq . Wq      (fprop,  A = Xq,   B = Wq^T)
+  dX = dYq . Wq^T   (dgrad,  A = dYq,  B = Wq)
+  dW = Xq^T . dYq   (wgrad,  A = Xq^T, B = dYq^T)
+then, for all layers at once, the amax-history roll and next scales, and one fused AdamW over
+every dW (loss-scale unscale, global-norm clip, FP32 master/m/v, BF16 weight for the next step).
+All scalars stay on the device; nothing in a step synchronises with the host.
+"""
+import torch
+
+from . import (AMAX_MAX, AMAX_MOST_RECENT, E4M3, E5M2, FP8_MAX, fp8_cast_transpose_amax,
+               fp8_gemm, fp8_scale_update, fused_adamw_multi_tensor, fused_adamw_workspace_bytes)
+
+ROLE_X, ROLE_W, ROLE_DY = 0, 1, 2
+ROLE_FMT = (E4M3, E4M3, E5M2)
+
+
+class LinearLayerBuffers:
+    def __init__(self, fin, fout, tokens, w_init, device):
+        u8 = dict(dtype=torch.uint8, device=device)
+        bf = dict(dtype=torch.bfloat16, device=device)
+        self.fin, self.fout, self.tokens = fin, fout, tokens
+        self.W = w_init.to(device=device, dtype=torch.bfloat16).contiguous().clone()
+        self.master = self.W.float()
+        self.m = torch.zeros_like(self.master)
+        self.v = torch.zeros_like(self.master)
+        self.Xq = torch.empty(tokens, fin, **u8)
+        self.XqT = torch.empty(fin, tokens, **u8)
+        self.Wq = torch.empty(fin, fout, **u8)
+        self.WqT = torch.empty(fout, fin, **u8)
+        self.dYq = torch.empty(tokens, fout, **u8)
+        self.dYqT = torch.empty(fout, tokens, **u8)
+        self.Y = torch.empty(tokens, fout, **bf)
+        self.dX = torch.empty(tokens, fin, **bf)
+        self.dW = torch.empty(fin, fout, **bf)
+
+
+class Fp8LinearStep:
+    """A group of Linear layers sharing one scale update and one fused AdamW per step.
+
+    Scale state is indexed 3*layer + role (role 0 = X, 1 = W, 2 = dY)."""
+
+    def __init__(self, layer_shapes, tokens, history_len, algo="max", margin=0, adamw=None,
+                 w_init=None, device="cuda", counters=False):
+        self.device = torch.device(device)
+        self.tokens = tokens
+        self.algo = AMAX_MAX if algo == "max" else AMAX_MOST_RECENT
+        self.margin = int(margin)
+        self.hp = dict(adamw)
+        n = 3 * len(layer_shapes)
+        f32 = dict(dtype=torch.float32, device=self.device)
+        self.amax = torch.zeros(n, **f32)
+        self.history = torch.zeros(n, history_len, **f32)
+        self.scale = torch.ones(n, **f32)
+        self.scale_inv = torch.ones(n, **f32)
+        self.fp8_max = torch.tensor([FP8_MAX[ROLE_FMT[i % 3]] for i in range(n)], **f32)
+        self.counters = torch.zeros(n, 3, dtype=torch.int64, device=self.device) if counters else None
+        self.layers = [LinearLayerBuffers(fi, fo, tokens, w_init[k], self.device)
+                       for k, (fi, fo) in enumerate(layer_shapes)]
+        self.grad_norm = torch.zeros(1, **f32)
+        self.skipped = torch.zeros(1, dtype=torch.int32, device=self.device)
+        ws = fused_adamw_workspace_bytes([l.master.numel() for l in self.layers])
+        self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=self.device)
+        self.t = 0
+
+    def _slot(self, t, i):
+        return t[i:i + 1]
+
+    def cast(self, k, role, src, q, qT, stream=None):
+        i = 3 * k + role
+        fp8_cast_transpose_amax(src, ROLE_FMT[role], self._slot(self.scale, i), q, qT,
+                                self._slot(self.amax, i), self._slot(self.scale_inv, i),
+                                self.counters[i] if self.counters is not None else None,
+                                stream=stream)
+
+    def layer_forward_backward(self, k, X, dY, stream=None):
+        L = self.layers[k]
+        sx, sw, sdy = (self._slot(self.scale_inv, 3 * k + r) for r in (ROLE_X, ROLE_W, ROLE_DY))
+        self.cast(k, ROLE_X, X, L.Xq, L.XqT, stream)
+        self.cast(k, ROLE_W, L.W, L.Wq, L.WqT, stream)
+        self.cast(k, ROLE_DY, dY, L.dYq, L.dYqT, stream)
+        fp8_gemm(L.Xq, E4M3, L.WqT, E4M3, sx, sw, L.Y, stream=stream)       # fprop
+        fp8_gemm(L.dYq, E5M2, L.Wq, E4M3, sdy, sw, L.dX, stream=stream)     # dgrad
+        fp8_gemm(L.XqT, E4M3, L.dYqT, E5M2, sx, sdy, L.dW, stream=stream)   # wgrad
+
+    def update(self, stream=None):
+        fp8_scale_update(self.amax, self.history, self.fp8_max, self.algo, self.margin,
+                         self.scale, self.scale_inv, stream=stream)
+        hp = self.hp
+        fused_adamw_multi_tensor([l.master for l in self.layers], [l.m for l in self.layers],
+                                 [l.v for l in self.layers], [l.dW for l in self.layers],
+                                 [l.W for l in self.layers], lr=hp["lr"], beta1=hp["beta1"],
+                                 beta2=hp["beta2"], eps=hp["eps"], weight_decay=hp["weight_decay"],
+                                 step=self.t, loss_scale=hp["loss_scale"],
+                                 max_grad_norm=hp["max_grad_norm"], grad_norm=self.grad_norm,
+                                 skipped=self.skipped, workspace=self.workspace, stream=stream)
+
+    def step(self, xs, dys, stream=None):
+        """One training step; xs[k] = X [tokens, in_k], dys[k] = dY [tokens, out_k] (BF16, device)."""
+        self.t += 1
+        for k in range(len(self.layers)):
+            self.layer_forward_backward(k, xs[k], dys[k], stream)
+        self.update(stream)
+
+    # launches of the library's kernels per step (for the benchmark's launch count)
+    def kernels_per_step(self):
+        n_adamw_batches = (len(self.layers) + 255) // 256
+        return 6 * len(self.layers) + 1 + 2 * n_adamw_batches

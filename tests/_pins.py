@@ -71,11 +71,24 @@ def bf16_to_f32(bits):
 
 
 def bf16_ulp(v):
-    """Spacing of BF16 values at |v| (float64 array): 2^(e-7) for normals, 2^-133 below."""
+    """Spacing of BF16 values at |v| (float64 array): 2^(e-7) for normals, 2^-133 at and below
+    the smallest normal (zero included)."""
     v = np.abs(np.asarray(v, np.float64))
-    e = np.floor(np.log2(np.where(v > 0, v, 1.0)))
+    e = np.floor(np.log2(np.where(v > 0, v, 2.0 ** -126)))
     e = np.maximum(e, -126)
     return np.where(np.isfinite(v), np.exp2(e - 7), np.inf)
+
+
+def gemm_within_tolerance(d_gpu_bits, d_ref_bits, abs_sum):
+    """|D_gpu - D_ref| <= 2 BF16 ulp of D_ref + 1e-5 * sum_k |a_k b_k| * scale, per element;
+    NaN where and only where the reference is NaN. Returns the boolean mask of passing elements."""
+    g = bf16_to_f32(d_gpu_bits).astype(np.float64)
+    r = bf16_to_f32(d_ref_bits).astype(np.float64)
+    tol = 2 * bf16_ulp(r) + 1e-5 * np.asarray(abs_sum, np.float64)
+    with np.errstate(invalid="ignore"):
+        ok = (np.abs(g - r) <= tol) | (g == r)
+    both_nan = np.isnan(g) & np.isnan(r)
+    return (ok & ~np.isnan(g) & ~np.isnan(r)) | both_nan
 
 
 def nearest_f32(fr: Fraction) -> float:

@@ -1,0 +1,115 @@
+"""Parity of fp8_cast_transpose_amax (C ABI, sm_100a) with the oracle: bit-exact codes,
+transpose, amax, scale_inv and counters.
+
+[P2] "FP8 混合精度训练工程实践" §四 quantize; [P3] "LLM FP8 微调上线生产实战" 核心原理 (HYBRID) and
+工程落地 第四步 (saturation / zero metrics)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from optimizer_fp8_cast_b200 import synth
+from tests._gpu import bf16_bits, bf16_from_bits, dev_scalar, u8
+
+pytestmark = pytest.mark.gpu
+
+SCALES = [1.0, 2.0 ** -3, 3.7, 1.0 / 3.0, 16384.0, 2.0 ** 100, 2.0 ** -100]
+
+
+def run_gpu(fp8, x, fmt, scale, want_q=True, want_qT=True, counters=True):
+    rows, cols = x.shape
+    q = torch.empty(rows, cols, dtype=torch.uint8, device="cuda") if want_q else None
+    qT = torch.empty(cols, rows, dtype=torch.uint8, device="cuda") if want_qT else None
+    amax = torch.full((1,), 12345.0, device="cuda")                 # must be overwritten
+    sinv = torch.zeros(1, device="cuda")
+    cnt = torch.zeros(3, dtype=torch.int64, device="cuda") if counters else None
+    fp8.fp8_cast_transpose_amax(x, fmt, dev_scalar(scale), q, qT, amax, sinv, cnt)
+    fp8.fp8t_check_device_error()
+    return (u8(q) if want_q else None, u8(qT) if want_qT else None,
+            np.float32(amax.item()), np.float32(sinv.item()),
+            cnt.cpu().numpy().astype(np.uint64) if counters else None)
+
+
+def check(fp8, x_bits, fmt, scale):
+    x = bf16_from_bits(x_bits)
+    q, qT, amax, sinv, cnt = run_gpu(fp8, x, fmt, scale)
+    rq, rqT, ramax, rsinv, rcnt = oracle.cast_transpose_amax(x_bits, fmt, scale)
+    assert np.array_equal(q, rq), "row-major codes differ"
+    assert np.array_equal(qT, rqT), "transposed codes differ"
+    assert amax.view(np.uint32) == np.float32(ramax).view(np.uint32), (amax, ramax)
+    assert sinv.view(np.uint32) == np.float32(rsinv).view(np.uint32)
+    assert np.array_equal(cnt, rcnt), (cnt, rcnt)
+
+
+@pytest.mark.parametrize("fmt", [oracle.E4M3, oracle.E5M2])
+@pytest.mark.parametrize("scale", SCALES)
+def test_every_bf16_pattern(cuda_lib, fmt, scale):
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16).reshape(256, 256)
+    check(cuda_lib, bits, fmt, scale)
+    # the same values in a different arrangement (rows and columns swapped, tail tiles)
+    check(cuda_lib, np.ascontiguousarray(bits.reshape(128, 512)), fmt, scale)
+
+
+@pytest.mark.parametrize("shape", [(16, 16), (48, 80), (144, 272), (128, 128), (256, 384),
+                                   (1040, 2064), (16, 4096), (4096, 16)])
+@pytest.mark.parametrize("fmt", [oracle.E4M3, oracle.E5M2])
+def test_ragged_shapes(cuda_lib, shape, fmt):
+    g = torch.Generator().manual_seed(hash(shape) & 0xFFFF)
+    x = torch.randn(shape, generator=g) * 3
+    x[torch.rand(shape, generator=g) < 0.01] *= 1000
+    bits = bf16_bits(x.to(torch.bfloat16))
+    for scale in (1.0, 0.37, 200.0):
+        check(cuda_lib, bits, fmt, scale)
+
+
+def test_optional_outputs(cuda_lib):
+    x = torch.randn(272, 144).to(torch.bfloat16)
+    bits = bf16_bits(x)
+    xd = bf16_from_bits(bits)
+    rq, rqT, ramax, _, _ = oracle.cast_transpose_amax(bits, oracle.E4M3, 2.0)
+    q, qT, amax, _, _ = run_gpu(cuda_lib, xd, oracle.E4M3, 2.0, want_qT=False, counters=False)
+    assert qT is None and np.array_equal(q, rq) and amax == ramax
+    q, qT, amax, _, _ = run_gpu(cuda_lib, xd, oracle.E4M3, 2.0, want_q=False)
+    assert q is None and np.array_equal(qT, rqT)
+    q, qT, amax, _, _ = run_gpu(cuda_lib, xd, oracle.E4M3, 2.0, want_q=False, want_qT=False)
+    assert amax == ramax
+
+
+def test_counters_accumulate(cuda_lib):
+    x = torch.randn(512, 256) * 100
+    xd = x.to(torch.bfloat16).cuda()
+    cnt = torch.zeros(3, dtype=torch.int64, device="cuda")
+    amax = torch.zeros(1, device="cuda")
+    for _ in range(3):
+        cuda_lib.fp8_cast_transpose_amax(xd, oracle.E4M3, dev_scalar(4.0), None, None, amax, None, cnt)
+    _, _, _, _, rc = oracle.cast_transpose_amax(bf16_bits(xd), oracle.E4M3, 4.0)
+    assert np.array_equal(cnt.cpu().numpy(), 3 * rc.astype(np.int64))
+
+
+def test_special_values_and_nan_amax(cuda_lib):
+    bits = np.zeros((32, 32), np.uint16)
+    bits[0, :8] = [0x0000, 0x8000, 0x7F80, 0xFF80, 0x7FC0, 0xFFC1, 0x0001, 0x8001]
+    for fmt in (oracle.E4M3, oracle.E5M2):
+        check(cuda_lib, bits, fmt, 1.0)
+    bits2 = np.full((32, 32), 0x8000, np.uint16)      # all -0: amax +0
+    check(cuda_lib, bits2, oracle.E4M3, 1.0)
+
+
+@pytest.mark.parametrize("name,rows,cols,fmt", [
+    ("X linear4096", 8192, 4096, oracle.E4M3),
+    ("W linear4096", 4096, 4096, oracle.E4M3),
+    ("dY linear4096", 8192, 4096, oracle.E5M2),
+    ("X of down, block7b", 16384, 11008, oracle.E4M3),
+    ("dY of gate, block7b", 16384, 11008, oracle.E5M2),
+])
+def test_full_size_workload_shapes(cuda_lib, name, rows, cols, fmt):
+    """Full-size tensors of the 4096 x 4096 / 8192-token Linear and the 7B-block projections,
+    compared element by element."""
+    std = 1e-3 if fmt == oracle.E5M2 else (0.02 if name.startswith("W") else 1.0)
+    x = synth.normal_f32((rows, cols), std, synth.tensor_seed(0, name, 0), "cuda")
+    if fmt == oracle.E5M2:
+        x[torch.rand(rows, cols, device="cuda") < 1e-3] *= 1000
+    xb = x.to(torch.bfloat16)
+    del x
+    scale = 448.0 / 4.5 if fmt == oracle.E4M3 else 57344.0 / 1.1
+    check(cuda_lib, bf16_bits(xb), fmt, scale)

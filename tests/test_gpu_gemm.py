@@ -1,0 +1,105 @@
+"""Parity of fp8_gemm (C ABI, tcgen05 on sm_100a) with the oracle's exact GEMM:
+|D - D_ref| <= 2 BF16 ulp + 1e-5 * sum_k |a_k b_k| * scale for every compared element.
+
+[P2] "FP8 混合精度训练工程实践" §三 (FP8 GEMM, FP32 accumulation, 16-bit output), §五 (per-tensor
+mode)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from optimizer_fp8_cast_b200 import synth
+from tests._gpu import bf16_bits, dev_scalar, sample_positions, u8
+from tests._pins import gemm_within_tolerance
+
+pytestmark = pytest.mark.gpu
+PAIRS = [(oracle.E4M3, oracle.E4M3), (oracle.E5M2, oracle.E4M3), (oracle.E4M3, oracle.E5M2),
+         (oracle.E5M2, oracle.E5M2)]
+
+
+def codes_from_normal(fp8, rows, cols, fmt, std, seed):
+    """FP8 operand made by the library's own cast of seeded normal data (realistic codes)."""
+    x = synth.normal_f32((rows, cols), std, seed, "cuda").to(torch.bfloat16)
+    q = torch.empty(rows, cols, dtype=torch.uint8, device="cuda")
+    amax = torch.zeros(1, device="cuda")
+    scale = (448.0 if fmt == oracle.E4M3 else 57344.0) / (5.0 * std)
+    fp8.fp8_cast_transpose_amax(x, fmt, dev_scalar(scale), q, None, amax)
+    return q
+
+
+def random_codes(rows, cols, fmt, seed):
+    rng = np.random.default_rng(seed)
+    t = oracle.decode_table(fmt)
+    ok = np.flatnonzero(np.isfinite(t) & (np.abs(t) <= (64 if fmt == oracle.E5M2 else 448)))
+    return torch.from_numpy(rng.choice(ok, size=(rows, cols)).astype(np.uint8)).cuda()
+
+
+def run(fp8, A, af, B, bf, sa, sb):
+    M, N = A.shape[0], B.shape[0]
+    D = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    fp8.fp8_gemm(A, af, B, bf, dev_scalar(sa), dev_scalar(sb), D)
+    fp8.fp8t_check_device_error()
+    return bf16_bits(D)
+
+
+@pytest.mark.parametrize("af,bf", PAIRS)
+@pytest.mark.parametrize("M,N,K", [(128, 256, 128), (512, 256, 256), (256, 256, 512),
+                                   (16, 16, 16), (144, 272, 48), (400, 528, 1040),
+                                   (128, 256, 4096)])
+def test_full_compare_small(cuda_lib, af, bf, M, N, K):
+    A = random_codes(M, K, af, M * 7 + K)
+    B = random_codes(N, K, bf, N * 13 + K)
+    sa, sb = 0.013, 0.7
+    D = run(cuda_lib, A, af, B, bf, sa, sb)
+    R, ab = oracle.gemm(u8(A), af, u8(B), bf, sa, sb, want_abs=True)
+    ok = gemm_within_tolerance(D, R, ab)
+    assert ok.all(), f"{(~ok).sum()} of {ok.size} outside tolerance, first at {np.argwhere(~ok)[:3]}"
+
+
+def test_realistic_codes_and_step_shapes(cuda_lib):
+    """The three GEMMs of the 256 x 256 / 512-token Linear with codes from the library cast."""
+    T, fin, fout = 512, 256, 256
+    Xq = codes_from_normal(cuda_lib, T, fin, oracle.E4M3, 1.0, 1)
+    WqT = codes_from_normal(cuda_lib, fout, fin, oracle.E4M3, 0.02, 2)
+    dYq = codes_from_normal(cuda_lib, T, fout, oracle.E5M2, 1e-3, 3)
+    for A, af, B, bf in ((Xq, 0, WqT, 0), (dYq, 1, WqT.t().contiguous(), 0),
+                         (Xq.t().contiguous(), 0, dYq.t().contiguous(), 1)):
+        D = run(cuda_lib, A, af, B, bf, 0.01, 0.002)
+        R, ab = oracle.gemm(u8(A), af, u8(B), bf, 0.01, 0.002, want_abs=True)
+        assert gemm_within_tolerance(D, R, ab).all()
+
+
+def test_output_overwritten_and_nan_propagates(cuda_lib):
+    A = random_codes(128, 128, 0, 5)
+    B = random_codes(256, 128, 0, 6)
+    A[3, 7] = 0x7F                       # NaN code
+    D = run(cuda_lib, A, 0, B, 0, 1.0, 1.0)
+    R = oracle.gemm(u8(A), 0, u8(B), 0, 1.0, 1.0)
+    Df = (D.astype(np.uint32) << 16).view(np.float32)
+    assert np.all(np.isnan(Df[3])) and not np.isnan(np.delete(Df, 3, 0)).any()
+    assert gemm_within_tolerance(D, R, np.zeros(R.shape)).sum() > 0
+
+
+@pytest.mark.parametrize("M,N,K,af,bf,label", [
+    (8192, 4096, 4096, 0, 0, "fprop linear4096"),
+    (8192, 4096, 4096, 1, 0, "dgrad linear4096"),
+    (4096, 4096, 8192, 0, 1, "wgrad linear4096"),
+    (16384, 11008, 4096, 0, 0, "fprop gate/up block7b"),
+    (16384, 4096, 11008, 0, 0, "fprop down block7b"),
+    (4096, 11008, 16384, 0, 1, "wgrad gate/up block7b"),
+    (11008, 4096, 16384, 0, 1, "wgrad down block7b"),
+])
+def test_full_size_sampled(cuda_lib, M, N, K, af, bf, label):
+    """Full-size GEMMs of the benchmark workloads in the launch configuration the benchmark uses,
+    checked on ~6,000 seeded output positions including tile edges."""
+    A = codes_from_normal(cuda_lib, M, K, af, 1.0 if af == 0 else 1e-3, M + K)
+    B = codes_from_normal(cuda_lib, N, K, bf, 0.02 if bf == 0 else 1e-3, N + 3 * K)
+    sa, sb = 1.0 / 89.6, 1.0 / 4480.0
+    D = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    cuda_lib.fp8_gemm(A, af, B, bf, dev_scalar(sa), dev_scalar(sb), D)
+    cuda_lib.fp8t_check_device_error()
+    ii, jj = sample_positions(M, N, 4096, seed=M ^ N ^ K)
+    Dh = bf16_bits(D)[ii, jj]
+    R, ab = oracle.gemm_at(u8(A), af, u8(B), bf, sa, sb, ii, jj)
+    ok = gemm_within_tolerance(Dh, R, ab)
+    assert ok.all(), f"{label}: {(~ok).sum()} of {ok.size} samples outside tolerance"
