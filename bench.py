@@ -1,0 +1,448 @@
+#!/usr/bin/env python
+"""Benchmark of the FP8 delayed-scaling Linear training step and fused AdamW on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch of the 4096 x 4096 Linear with 8192
+tokens (batch 4 x sequence 2048): three casts (X, W to E4M3, dY to E5M2, each with its
+transposed copy and amax), fprop / dgrad / wgrad FP8 GEMMs, the amax-history roll and scale
+update (history 1024, algo max, margin 0), and one fused AdamW over dW. Inputs are synthetic
+(seeded normals of the stated shapes), resident in HBM when timing starts; L2 is flushed (a
+256 MiB write) before every timed step.
+
+Prints one JSON line (rank 0). `value` is the GEMM work of all ranks (3 x 2 x 8192 x 4096 x 4096
+FLOP per step per rank) divided by the max over ranks of the summed device time of the K steps.
+With N > 1 every rank runs an independent replica (the path has no data-path collective);
+the barrier and the max-over-ranks reduction use NCCL.
+
+--impl reference times the CPU oracle (single thread, as it stands) on a bounded sample of the
+same workload: each step runs every stage on 1/4096 of its rows and the sample's share of the
+GEMM work is scaled to the same TFLOP/s unit. Only rank 0 runs it.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "FP8 Linear fwd+bwd TFLOP/s; cast+amax & fused AdamW GB/s vs HBM peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP8_OVER_BF16 = 2.0        # nominal dense FP8 / BF16 tensor-core ratio (4.5 / 2.25 PFLOP/s)
+L2_FLUSH_BYTES = 256 << 20
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+REASON_NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+
+# ----------------------------------------------------------------------------- host helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=float(p["hbm_gbs"]), bf16_tflops=float(p["bf16_tflops"]),
+                    bf16_tflops_sustained=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                    source="measured")
+    return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def workload_numbers(wl):
+    """Algorithmic work per step of a one-layer workload."""
+    _, fin, fout = wl.layers[0]
+    T = wl.tokens
+    return dict(
+        gemm_flop=2 * T * fin * fout,                       # each of fprop, dgrad, wgrad
+        cast_bytes=[4 * T * fin, 4 * fin * fout, 4 * T * fout],   # X, W, dY: 2 B in + 1 + 1 out
+        adamw_bytes=30 * fin * fout,                        # 2 B norm pass + 28 B update
+        params=fin * fout,
+        h2d=2 * T * fin + 2 * T * fout,                     # X and dY, BF16
+        d2h=2 * T * fout + 2 * T * fin,                     # Y and dX, BF16
+    )
+
+
+def reduce_max(value, world_size, device=None):
+    """Max of a float over all ranks (identity when not distributed)."""
+    if world_size <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def throughput(flop_per_step_per_rank, steps, world_size, total_ms_max):
+    """Whole-job TFLOP/s: work of all ranks over the slowest rank's device time."""
+    return flop_per_step_per_rank * steps * world_size / (total_ms_max * 1e-3) / 1e12
+
+
+class ClockSampler:
+    """nvidia-smi sampling of one GPU's clocks and throttle reasons every 200 ms."""
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_id), f"--query-gpu={CLOCK_FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append(dict(sm=float(parts[1]), max=float(parts[2]),
+                                     power=float(parts[3]) if parts[3] not in ("[N/A]", "") else 0.0,
+                                     reasons={n: parts[5 + i] == "Active" for i, n in enumerate(REASON_NAMES)}))
+                except ValueError:
+                    continue
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        load = [r for r in rows if r["power"] > 250.0] or rows
+        reasons = sorted({n for r in load for n, a in r["reasons"].items() if a})
+        return {"sm_mhz": statistics.median(r["sm"] for r in load),
+                "sm_max_mhz": max(r["max"] for r in rows), "reasons": reasons,
+                "samples": len(rows), "samples_under_load": len(load)}
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import optimizer_fp8_cast_b200 as fp8
+    from optimizer_fp8_cast_b200 import synth
+    from optimizer_fp8_cast_b200.step import ROLE_DY, ROLE_W, ROLE_X, Fp8LinearStep
+
+    fp8.load()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = synth.WORKLOADS[args.workload]
+    nums = workload_numbers(wl)
+    peaks = load_peaks()
+
+    st = Fp8LinearStep([(i, o) for _, i, o in wl.layers], wl.tokens, wl.history_len, wl.algo,
+                       wl.margin, wl.adamw, [synth.linear_weight(wl, 0, dev)], dev)
+    batches = [synth.linear_inputs(wl, 0, t, dev) for t in range(2)]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    L = st.layers[0]
+    NEV = 9
+    stage_names = ["cast X", "cast W", "cast dY", "fprop", "dgrad", "wgrad", "scale update", "adamw"]
+
+    def one_step(X, dY, ev=None):
+        st.t += 1
+        rec = (lambda i: ev[i].record()) if ev is not None else (lambda i: None)
+        rec(0)
+        st.cast(0, ROLE_X, X, L.Xq, L.XqT); rec(1)
+        st.cast(0, ROLE_W, L.W, L.Wq, L.WqT); rec(2)
+        st.cast(0, ROLE_DY, dY, L.dYq, L.dYqT); rec(3)
+        st.gemm(0, 0); rec(4)
+        st.gemm(0, 1); rec(5)
+        st.gemm(0, 2); rec(6)
+        st.scale_update(); rec(7)
+        st.adamw(); rec(8)
+
+    for w in range(args.warmup):
+        flush.zero_()
+        one_step(*batches[w % 2])
+    torch.cuda.synchronize()
+    fp8.fp8t_check_device_error()
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(NEV)] for _ in range(args.steps)]
+    gpu_id = gpu_uuid(dev, local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    with ClockSampler(gpu_id) as clocks:
+        for t in range(args.steps):
+            flush.zero_()
+            one_step(*batches[t % 2], ev=events[t])
+        torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    if world > 1:
+        dist.barrier()
+    fp8.fp8t_check_device_error()
+
+    stage_ms = [[events[t][i].elapsed_time(events[t][i + 1]) for i in range(NEV - 1)]
+                for t in range(args.steps)]
+    step_ms = [events[t][0].elapsed_time(events[t][NEV - 1]) for t in range(args.steps)]
+    total_ms = reduce_max(sum(step_ms), world, dev)
+    flop_step = 3 * nums["gemm_flop"]
+    value = throughput(flop_step, args.steps, world, total_ms)
+
+    # per-kernel figures (this rank), averaged over the timed steps
+    avg = [statistics.mean(s[i] for s in stage_ms) for i in range(NEV - 1)]
+    gemm_ms = avg[3:6]
+    gemm_tflops = [nums["gemm_flop"] / (ms * 1e-3) / 1e12 for ms in gemm_ms]
+    cast_gbs = [b / (ms * 1e-3) / 1e9 for b, ms in zip(nums["cast_bytes"], avg[0:3])]
+    cast_all_gbs = sum(nums["cast_bytes"]) / (sum(avg[0:3]) * 1e-3) / 1e9
+    adamw_gbs = nums["adamw_bytes"] / (avg[7] * 1e-3) / 1e9
+    fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+    hbm = peaks["hbm_gbs"]
+    gemm_avg_ms = statistics.mean(gemm_ms)
+    gemm_achieved = nums["gemm_flop"] / (gemm_avg_ms * 1e-3) / 1e12
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "gemm_traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            tj = json.load(f)
+        if tj.get("workload") == wl.name and tj.get("kernel_source_sha") == kernel_source_sha():
+            traffic = tj.get("bytes_per_launch")
+
+    # end to end: host (pinned) inputs copied in and results copied out inside the timed region
+    hX = [b[0].cpu().pin_memory() for b in batches]
+    hdY = [b[1].cpu().pin_memory() for b in batches]
+    hY = torch.empty(L.Y.shape, dtype=torch.bfloat16).pin_memory()
+    hdX = torch.empty(L.dX.shape, dtype=torch.bfloat16).pin_memory()
+    X_dev = torch.empty_like(batches[0][0])
+    dY_dev = torch.empty_like(batches[0][1])
+    e2e_ms = []
+    for t in range(args.steps + 1):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        X_dev.copy_(hX[t % 2], non_blocking=True)
+        dY_dev.copy_(hdY[t % 2], non_blocking=True)
+        st.step([X_dev], [dY_dev])
+        hY.copy_(L.Y, non_blocking=True)
+        hdX.copy_(L.dX, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        if t > 0:                       # the first one warms the pinned paths
+            e2e_ms.append(e0.elapsed_time(e1))
+    fp8.fp8t_check_device_error()
+    e2e_total = reduce_max(sum(e2e_ms), world, dev)
+    e2e_value = throughput(flop_step, len(e2e_ms), world, e2e_total)
+
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp8 (e4m3/e5m2 operands, f32 accumulate)",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "tokens": wl.tokens, "in_features": wl.layers[0][1],
+                   "out_features": wl.layers[0][2], "recipe": "HYBRID, delayed per-tensor scaling",
+                   "history_len": wl.history_len, "amax_algo": wl.algo, "margin": wl.margin,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "flushed before every timed step (256 MiB write)"},
+        "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": nums["h2d"],
+                "d2h_bytes_per_step": nums["d2h"], "ms_per_step": round(e2e_total / len(e2e_ms), 4)},
+        "gpu_launches": args.steps * st.kernels_per_step(),
+        "roofline": {"kernel": "k_fp8_gemm (fprop, dgrad, wgrad)", "bound": "tensor",
+                     "achieved": round(gemm_achieved, 1), "peak": round(fp8_peak, 1),
+                     "unit": "TFLOP/s", "frac": round(gemm_achieved / fp8_peak, 4),
+                     "traffic": traffic,
+                     "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {FP8_OVER_BF16} (nominal FP8/BF16 ratio)"},
+        "kernels": {
+            "stage_ms": {n: round(a, 4) for n, a in zip(stage_names, avg)},
+            "gemm_tflops": {"fprop": round(gemm_tflops[0], 1), "dgrad": round(gemm_tflops[1], 1),
+                            "wgrad": round(gemm_tflops[2], 1)},
+            "cast_gbs": {"X": round(cast_gbs[0], 1), "W": round(cast_gbs[1], 1),
+                         "dY": round(cast_gbs[2], 1), "all": round(cast_all_gbs, 1),
+                         "frac_of_hbm": round(cast_all_gbs / hbm, 4)},
+            "adamw_gbs": round(adamw_gbs, 1), "adamw_frac_of_hbm": round(adamw_gbs / hbm, 4),
+            "hbm_peak_gbs": hbm, "peak_source": peaks["source"],
+        },
+        "clocks": clocks.summary(),
+        "wall_s_timed_region": round(wall, 3),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(st, wl, nums, batches[0], frac_rows=1024)
+    return result
+
+
+def gpu_uuid(dev, fallback):
+    """nvidia-smi identifier of a torch device (its UUID), independent of device renumbering."""
+    import torch
+    props = torch.cuda.get_device_properties(dev)
+    u = getattr(props, "uuid", None)
+    if u is None:
+        return fallback
+    s = str(u)
+    return s if s.startswith("GPU-") else "GPU-" + s
+
+
+def kernel_source_sha():
+    import hashlib
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "optimizer_fp8_cast_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_sample_step(oracle, host, wl, rows_div):
+    """Every stage of one step on a 1/rows_div row sample of the workload (CPU oracle).
+    Returns (seconds, GEMM FLOP of the sample)."""
+    import numpy as np
+    _, fin, fout = wl.layers[0]
+    T = wl.tokens
+    rt, rw = max(1, T // rows_div), max(1, fin // rows_div)
+    t0 = time.perf_counter()
+    # casts of the sampled rows (q, q^T of the sample, amax, counters)
+    oracle.cast_transpose_amax(host["X"][:rt], oracle.E4M3, 1.0)
+    oracle.cast_transpose_amax(host["W"][:rw], oracle.E4M3, 1.0)
+    oracle.cast_transpose_amax(host["dY"][:rt], oracle.E5M2, 1.0)
+    # GEMMs: rt (resp. rw) full output rows each
+    oracle.gemm(host["Xq"][:rt], 0, host["WqT"], 0, 1.0, 1.0)
+    oracle.gemm(host["dYq"][:rt], 1, host["Wq"], 0, 1.0, 1.0)
+    oracle.gemm(host["XqT"][:rw], 0, host["dYqT"], 1, 1.0, 1.0)
+    # scale update (whole: it is tiny) and AdamW on the sample's share of the parameters
+    hist = np.zeros((3, wl.history_len), np.float32)
+    sc = np.ones(3, np.float32)
+    si = np.ones(3, np.float32)
+    oracle.scale_update(np.ones(3, np.float32), hist, [448.0, 448.0, 57344.0], 0, 0, sc, si)
+    n = max(1, fin * fout // rows_div)
+    p = [host["master"][:n].copy()]
+    m = [np.zeros(n, np.float32)]
+    v = [np.zeros(n, np.float32)]
+    w = [np.zeros(n, np.uint16)]
+    oracle.fused_adamw(p, m, v, [host["dW"][:n]], w, dict(wl.adamw, step=1))
+    dt = time.perf_counter() - t0
+    flop = 2 * (rt * fout * fin + rt * fin * fout + rw * fout * T)
+    return dt, flop
+
+
+def host_copies(st, batch):
+    from optimizer_fp8_cast_b200.synth import bf16_bits, u8
+    L = st.layers[0]
+    return dict(X=bf16_bits(batch[0]), dY=bf16_bits(batch[1]), W=bf16_bits(L.W), Xq=u8(L.Xq),
+                XqT=u8(L.XqT), Wq=u8(L.Wq), WqT=u8(L.WqT), dYq=u8(L.dYq), dYqT=u8(L.dYqT),
+                master=L.master.detach().cpu().numpy().reshape(-1),
+                dW=bf16_bits(L.dW).reshape(-1))
+
+
+def cpu_baseline(st, wl, nums, batch, frac_rows):
+    import oracle
+    host = host_copies(st, batch)
+    dt, flop = oracle_sample_step(oracle, host, wl, frac_rows)
+    return {"value": round(flop / dt / 1e12, 9), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"every stage on 1/{frac_rows} of its rows ({flop / 1e9:.3f} GFLOP of GEMM "
+                      f"work, {dt:.1f} s), single-threaded C oracle on the host"}
+
+
+def run_reference(args):
+    """The CPU oracle as the reference arm: bounded samples, same metric and unit."""
+    import torch
+
+    import oracle
+    from optimizer_fp8_cast_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    _, fin, fout = wl.layers[0]
+    rows_div = 4096
+    # inputs: seeded CPU draws of the workload's shapes, quantised by the oracle itself
+    X, dY = synth.linear_inputs(wl, 0, 0, "cpu")
+    W = synth.linear_weight(wl, 0, "cpu")
+    host = dict(X=synth.bf16_bits(X), dY=synth.bf16_bits(dY), W=synth.bf16_bits(W))
+    q, qT, _, _, _ = oracle.cast_transpose_amax(host["X"], oracle.E4M3, 1.0)
+    host["Xq"], host["XqT"] = q, qT
+    q, qT, _, _, _ = oracle.cast_transpose_amax(host["W"], oracle.E4M3, 1.0)
+    host["Wq"], host["WqT"] = q, qT
+    q, qT, _, _, _ = oracle.cast_transpose_amax(host["dY"], oracle.E5M2, 1.0)
+    host["dYq"], host["dYqT"] = q, qT
+    host["master"] = W.float().numpy().reshape(-1)
+    host["dW"] = synth.bf16_bits(torch.randn(fin * fout, generator=torch.Generator().manual_seed(1)).to(torch.bfloat16))
+    for _ in range(args.warmup):
+        oracle_sample_step(oracle, host, wl, rows_div)
+    times, flops = [], []
+    for _ in range(args.steps):
+        dt, fl = oracle_sample_step(oracle, host, wl, rows_div)
+        times.append(dt)
+        flops.append(fl)
+    total = sum(times)
+    value = sum(flops) / total / 1e12
+    sample = (f"every stage on 1/{rows_div} of its rows per step ({flops[0] / 1e9:.3f} GFLOP of "
+              f"GEMM work), single-threaded C oracle")
+    return {
+        "metric": METRIC, "value": round(value, 9), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8 codes, exact integer accumulation (CPU oracle)", "data": "synthetic",
+        "config": {"workload": wl.name, "tokens": wl.tokens, "in_features": fin,
+                   "out_features": fout, "history_len": wl.history_len},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 9), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 9), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="linear4096_t8192")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        print("note: fewer than 3 warm-up steps", file=sys.stderr)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        result = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(result), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

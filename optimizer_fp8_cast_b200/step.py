@@ -78,19 +78,34 @@ class Fp8LinearStep:
                                 self.counters[i] if self.counters is not None else None,
                                 stream=stream)
 
-    def layer_forward_backward(self, k, X, dY, stream=None):
+    def gemm(self, k, which, stream=None):
+        """which: 0 = fprop Y = X.W, 1 = dgrad dX = dY.W^T, 2 = wgrad dW = X^T.dY."""
         L = self.layers[k]
         sx, sw, sdy = (self._slot(self.scale_inv, 3 * k + r) for r in (ROLE_X, ROLE_W, ROLE_DY))
+        if which == 0:
+            fp8_gemm(L.Xq, E4M3, L.WqT, E4M3, sx, sw, L.Y, stream=stream)
+        elif which == 1:
+            fp8_gemm(L.dYq, E5M2, L.Wq, E4M3, sdy, sw, L.dX, stream=stream)
+        else:
+            fp8_gemm(L.XqT, E4M3, L.dYqT, E5M2, sx, sdy, L.dW, stream=stream)
+
+    def layer_forward_backward(self, k, X, dY, stream=None):
+        L = self.layers[k]
         self.cast(k, ROLE_X, X, L.Xq, L.XqT, stream)
         self.cast(k, ROLE_W, L.W, L.Wq, L.WqT, stream)
         self.cast(k, ROLE_DY, dY, L.dYq, L.dYqT, stream)
-        fp8_gemm(L.Xq, E4M3, L.WqT, E4M3, sx, sw, L.Y, stream=stream)       # fprop
-        fp8_gemm(L.dYq, E5M2, L.Wq, E4M3, sdy, sw, L.dX, stream=stream)     # dgrad
-        fp8_gemm(L.XqT, E4M3, L.dYqT, E5M2, sx, sdy, L.dW, stream=stream)   # wgrad
+        for which in (0, 1, 2):
+            self.gemm(k, which, stream)
 
-    def update(self, stream=None):
+    def scale_update(self, stream=None):
         fp8_scale_update(self.amax, self.history, self.fp8_max, self.algo, self.margin,
                          self.scale, self.scale_inv, stream=stream)
+
+    def update(self, stream=None):
+        self.scale_update(stream)
+        self.adamw(stream)
+
+    def adamw(self, stream=None):
         hp = self.hp
         fused_adamw_multi_tensor([l.master for l in self.layers], [l.m for l in self.layers],
                                  [l.v for l in self.layers], [l.dW for l in self.layers],
