@@ -86,7 +86,8 @@ def throughput(flop_per_step_per_rank, steps, world_size, total_ms_max):
 
 
 class ClockSampler:
-    """nvidia-smi sampling of one GPU's clocks and throttle reasons every 200 ms."""
+    """nvidia-smi sampling of one GPU's clocks and throttle reasons every 20 ms; entering waits
+    (up to 15 s) until the first sample has been written, so the timed region is covered."""
 
     def __init__(self, gpu_id):
         self.gpu_id = gpu_id
@@ -99,10 +100,15 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu_id), f"--query-gpu={CLOCK_FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+            return self
+        t0 = time.time()
+        while time.time() - t0 < 15 and os.path.getsize(self.path) == 0 and self.proc.poll() is None:
+            time.sleep(0.02)
+        self.skip_lines = sum(1 for _ in open(self.path))     # samples taken before timing
         return self
 
     def __exit__(self, *exc):
@@ -116,7 +122,8 @@ class ClockSampler:
     def summary(self):
         rows = []
         if self.path and os.path.exists(self.path):
-            for line in open(self.path):
+            lines = open(self.path).readlines()[getattr(self, "skip_lines", 0):]
+            for line in lines:
                 parts = [p.strip() for p in line.split(",")]
                 if len(parts) < 9:
                     continue
@@ -229,7 +236,7 @@ def run_ours(args, rank, world, local_rank):
     X_dev = torch.empty_like(batches[0][0])
     dY_dev = torch.empty_like(batches[0][1])
     e2e_ms = []
-    for t in range(args.steps + 1):
+    for t in range(min(args.steps, 50) + 1):
         flush.zero_()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
@@ -407,7 +414,7 @@ def run_reference(args):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="linear4096_t8192")

@@ -76,7 +76,10 @@ typedef enum fp8t_amax_algo {
  *                   fp8_scale_update). Read only.
  *   q_rowmajor      rows x cols FP8 bytes, row-major, or NULL to skip.
  *   q_transposed    cols x rows FP8 bytes (q^T, row-major), or NULL to skip.
- *   d_amax_out      1 float, overwritten with max|x| over the BF16 input (NaN if any input is NaN).
+ *   d_amax_inout    1 float, MAX-ACCUMULATED like the counters: it becomes the larger of its
+ *                   previous content and max|x| over the BF16 input (NaN if any input is NaN),
+ *                   compared as non-negative f32 bit patterns. Start it at 0; fp8_scale_update
+ *                   resets each amax it consumes to 0, so a training step needs no memset.
  *   d_scale_inv_out 1 float, overwritten with 1/scale (IEEE division), or NULL to skip.
  *   d_counters      3 x uint64, or NULL: ADDED to [0] #saturated (|f32(x*scale)| > FP8 max),
  *                   [1] #zero codes (q is +0 or -0), [2] #non-finite inputs.
@@ -87,7 +90,7 @@ typedef enum fp8t_amax_algo {
  */
 fp8t_status fp8_cast_transpose_amax(const void* x_bf16, int64_t rows, int64_t cols, fp8t_format fmt,
                                     const float* d_scale, void* q_rowmajor, void* q_transposed,
-                                    float* d_amax_out, float* d_scale_inv_out,
+                                    float* d_amax_inout, float* d_scale_inv_out,
                                     unsigned long long* d_counters, void* stream);
 
 /*
@@ -122,7 +125,8 @@ fp8t_status fp8_gemm(const void* A, fp8t_format a_fmt, const void* B, fp8t_forma
  *  Delayed Scaling 用历史换取稳定性 (history window; max / most_recent; used next iteration)].
  *
  * For each tensor t in [0, n_tensors):
- *   history row t is shifted by one (entry H-1 is dropped) and entry 0 becomes d_amax[t];
+ *   history row t is shifted by one (entry H-1 is dropped) and entry 0 becomes d_amax[t],
+ *   after which d_amax[t] is reset to 0 (ready for the next step's max-accumulating casts);
  *   rep   = max over the row of |h| (NaN if any entry is NaN)   for FP8T_AMAX_MAX,
  *           |h[0]|                                              for FP8T_AMAX_MOST_RECENT;
  *   scale = (d_fp8_max[t] / rep) * 2^-margin   (IEEE f32 division, then an exact power-of-two
@@ -132,14 +136,14 @@ fp8t_status fp8_gemm(const void* A, fp8t_format a_fmt, const void* B, fp8t_forma
  *   scale_inv = 1 / scale (IEEE f32 division).
  *
  *   n_tensors       1 .. 65535.
- *   d_amax          n floats (input).
+ *   d_amax          n floats (input; reset to 0 on return).
  *   d_amax_history  n x history_len floats, row-major, index 0 = newest (in/out).
  *   history_len     1 .. 65536.
  *   d_fp8_max       n floats: 448 for E4M3 tensors, 57344 for E5M2 tensors (input).
  *   margin          0 .. 126.
  *   d_scale, d_scale_inv   n floats each (in/out, out).
  */
-fp8t_status fp8_scale_update(int32_t n_tensors, const float* d_amax, float* d_amax_history,
+fp8t_status fp8_scale_update(int32_t n_tensors, float* d_amax, float* d_amax_history,
                              int32_t history_len, const float* d_fp8_max, fp8t_amax_algo algo,
                              int32_t margin, float* d_scale, float* d_scale_inv, void* stream);
 

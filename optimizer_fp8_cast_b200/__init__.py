@@ -68,9 +68,10 @@ def fp8_cast_transpose_amax(x, fmt, scale, q=None, qT=None, amax=None, scale_inv
                             counters=None, stream=None):
     """Quantise BF16 ``x`` [rows, cols] with the device scalar ``scale`` (float32 [1]).
 
-    Writes ``q`` [rows, cols] and ``qT`` [cols, rows] (uint8, optional), ``amax`` (float32 [1],
-    overwritten), ``scale_inv`` (float32 [1], optional) and adds to ``counters`` (int64 [3],
-    optional: saturated, zero, non-finite)."""
+    Writes ``q`` [rows, cols] and ``qT`` [cols, rows] (uint8, optional) and ``scale_inv``
+    (float32 [1], optional); max-accumulates max|x| into ``amax`` (float32 [1]: start it at 0,
+    ``fp8_scale_update`` resets it after use) and adds to ``counters`` (int64 [3], optional:
+    saturated, zero, non-finite)."""
     assert x.dtype == torch.bfloat16 and x.dim() == 2
     rows, cols = x.shape
     _check(load().fp8_cast_transpose_amax(_ptr(x), rows, cols, int(fmt), _ptr(scale), _ptr(q),
@@ -88,7 +89,8 @@ def fp8_gemm(A, a_fmt, B, b_fmt, a_scale_inv, b_scale_inv, D, stream=None):
 
 
 def fp8_scale_update(amax, history, fp8_max, algo, margin, scale, scale_inv, stream=None):
-    """Roll ``history`` [n, H] (entry 0 newest) with ``amax`` [n] and write the next scales."""
+    """Roll ``history`` [n, H] (entry 0 newest) with ``amax`` [n] (reset to 0 afterwards) and
+    write the next scales."""
     n, H = history.shape
     _check(load().fp8_scale_update(n, _ptr(amax), _ptr(history), H, _ptr(fp8_max), int(algo),
                                    int(margin), _ptr(scale), _ptr(scale_inv), _stream(stream)),

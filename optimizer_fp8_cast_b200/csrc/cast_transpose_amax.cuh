@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(kThreads)
       c += red[3][i];
     }
     if (m > 0x7F80u) m = 0x7FC0u;  // canonical NaN
-    atomicMax(amax_bits, m << 16);
+    atomicMax(amax_bits, m << 16);  // max-accumulated into the caller's slot
     if (COUNT) {
       if (a) atomicAdd(counters + 0, static_cast<unsigned long long>(a));
       if (b) atomicAdd(counters + 1, static_cast<unsigned long long>(b));

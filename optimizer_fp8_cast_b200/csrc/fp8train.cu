@@ -41,7 +41,7 @@ struct DeviceInfo {
   int state = 0;               // 0 unknown, 1 sm_100, 2 other
   int sms = 0;
   int adamw_blocks_per_sm = 0;
-  bool gemm_smem_set = false;
+  int gemm_clusters = 0;       // co-resident 2-CTA clusters of the GEMM kernel
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
@@ -73,7 +73,17 @@ fp8t_status current_device(DeviceInfo** out) {
         d.state = 0;
         return fail(FP8T_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
       }
-      d.gemm_smem_set = true;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+      cfg.blockDim = dim3(fp8t::gemm::kThreads, 1, 1);
+      cfg.dynamicSmemBytes = fp8t::gemm::kSmemBytes;
+      int clusters = 0;
+      e = cudaOccupancyMaxActiveClusters(&clusters, fp8t::gemm::k_fp8_gemm, &cfg);
+      if (e != cudaSuccess || clusters < 1) {
+        (void)cudaGetLastError();
+        clusters = sms / 2;
+      }
+      d.gemm_clusters = clusters;
     }
   }
   if (d.state != 1) return fail(FP8T_ERR_UNSUPPORTED_DEVICE, "device %d is not sm_100", dev);
@@ -170,10 +180,10 @@ const char* fp8t_status_string(fp8t_status s) {
 // ------------------------------------------------------------------ cast / transpose / amax
 fp8t_status fp8_cast_transpose_amax(const void* x_bf16, int64_t rows, int64_t cols, fp8t_format fmt,
                                     const float* d_scale, void* q_rowmajor, void* q_transposed,
-                                    float* d_amax_out, float* d_scale_inv_out,
+                                    float* d_amax_inout, float* d_scale_inv_out,
                                     unsigned long long* d_counters, void* stream) {
   t_last_error.clear();
-  if (!x_bf16 || !d_scale || !d_amax_out)
+  if (!x_bf16 || !d_scale || !d_amax_inout)
     return fail(FP8T_ERR_INVALID_ARG, "fp8_cast_transpose_amax: NULL input, scale or amax pointer");
   if (fmt != FP8T_E4M3 && fmt != FP8T_E5M2)
     return fail(FP8T_ERR_INVALID_ARG, "fp8_cast_transpose_amax: unknown format %d", (int)fmt);
@@ -184,7 +194,7 @@ fp8t_status fp8_cast_transpose_amax(const void* x_bf16, int64_t rows, int64_t co
     return fail(FP8T_ERR_UNSUPPORTED_SHAPE,
                 "fp8_cast_transpose_amax: rows and cols must be multiples of 16, rows*cols < 2^40");
   if (!aligned(x_bf16, 16) || !aligned(q_rowmajor, 16) || !aligned(q_transposed, 16) ||
-      !aligned(d_scale, 4) || !aligned(d_amax_out, 4) || !aligned(d_scale_inv_out, 4) ||
+      !aligned(d_scale, 4) || !aligned(d_amax_inout, 4) || !aligned(d_scale_inv_out, 4) ||
       !aligned(d_counters, 8))
     return fail(FP8T_ERR_MISALIGNED, "fp8_cast_transpose_amax: misaligned pointer");
   DeviceInfo* dev = nullptr;
@@ -192,15 +202,13 @@ fp8t_status fp8_cast_transpose_amax(const void* x_bf16, int64_t rows, int64_t co
   if (st != FP8T_OK) return st;
 
   cudaStream_t s = as_stream(stream);
-  cudaError_t e = cudaMemsetAsync(d_amax_out, 0, sizeof(float), s);
-  if (e != cudaSuccess) return fail(FP8T_ERR_CUDA, "cudaMemsetAsync(amax): %s", cudaGetErrorString(e));
   using namespace fp8t::cast;
   const int64_t tiles_c = (cols + kTile - 1) / kTile;
   const int64_t tiles = ((rows + kTile - 1) / kTile) * tiles_c;
   auto* xq = static_cast<const uint16_t*>(x_bf16);
   auto* q = static_cast<uint8_t*>(q_rowmajor);
   auto* qT = static_cast<uint8_t*>(q_transposed);
-  auto* amax = reinterpret_cast<unsigned int*>(d_amax_out);
+  auto* amax = reinterpret_cast<unsigned int*>(d_amax_inout);
   const dim3 grid(static_cast<unsigned>(tiles));
   if (fmt == FP8T_E4M3) {
     if (d_counters)
@@ -238,19 +246,21 @@ fp8t_status fp8_gemm(const void* A, fp8t_format a_fmt, const void* B, fp8t_forma
 
   using namespace fp8t::gemm;
   CUtensorMap ta, tb;
-  if ((st = encode_kmajor(&ta, A, M, K, kBM)) != FP8T_OK) return st;
-  if ((st = encode_kmajor(&tb, B, N, K, kBN)) != FP8T_OK) return st;
+  if ((st = encode_kmajor(&ta, A, M, K, kHalf)) != FP8T_OK) return st;
+  if ((st = encode_kmajor(&tb, B, N, K, kHalf)) != FP8T_OK) return st;
   const int64_t tiles_n = (N + kBN - 1) / kBN;
-  const int64_t tiles = ((M + kBM - 1) / kBM) * tiles_n;
-  k_fp8_gemm<<<static_cast<unsigned>(tiles), kThreads, kSmemBytes, as_stream(stream)>>>(
+  const int64_t tiles = ((M + kBM - 1) / kBM) * tiles_n;        // 256 x 256 tiles, one per pair
+  if (tiles >= (int64_t(1) << 30)) return fail(FP8T_ERR_UNSUPPORTED_SHAPE, "fp8_gemm: too many tiles");
+  const int64_t grid = 2 * std::min<int64_t>(tiles, dev->gemm_clusters);   // persistent pairs
+  k_fp8_gemm<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, as_stream(stream)>>>(
       ta, tb, static_cast<uint16_t*>(D_bf16), static_cast<int>(M), static_cast<int>(N),
       static_cast<int>(K), d_a_scale_inv, d_b_scale_inv, make_idesc(a_fmt, b_fmt),
-      static_cast<int>(tiles_n));
+      static_cast<int>(tiles_n), static_cast<int>(tiles));
   return after_launch("fp8_gemm launch");
 }
 
 // ------------------------------------------------------------------ scale update
-fp8t_status fp8_scale_update(int32_t n_tensors, const float* d_amax, float* d_amax_history,
+fp8t_status fp8_scale_update(int32_t n_tensors, float* d_amax, float* d_amax_history,
                              int32_t history_len, const float* d_fp8_max, fp8t_amax_algo algo,
                              int32_t margin, float* d_scale, float* d_scale_inv, void* stream) {
   t_last_error.clear();

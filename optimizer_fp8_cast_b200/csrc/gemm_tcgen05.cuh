@@ -3,21 +3,29 @@
 // Method: the FP8 GEMM of "FP8 混合精度训练工程实践" §三 (FP8 inputs, FP32 accumulation,
 // 16-bit output) with per-tensor dequantisation (§四 dequantize; §五 per-tensor mode:
 // FP8 x FP8, FP32 accumulate, BF16 out). The pages' kernel design is Hopper WGMMA (m64nNk32
-// warpgroup MMA reading shared memory); on sm_100a the same contraction runs as
-// tcgen05.mma.kind::f8f6f4 issued by one thread, with the accumulator in tensor memory.
+// warpgroup MMA reading shared memory, one SM per tile); on sm_100a the same contraction runs
+// as tcgen05.mma.kind::f8f6f4 issued by one thread for a PAIR of SMs, with the accumulator in
+// tensor memory.
 //
 // D[M x N] = bf16((A[M x K] . B[N x K]^T) * sa * sb), A and B K-major ("TN").
-// One CTA of 128 threads computes a 128 x 256 tile:
-//   warp 0, lane 0  TMA producer: 128-byte-swizzled 128 x 128 (A) and 256 x 128 (B) byte tiles
-//                   into a 4-stage ring (48 KB per stage), one mbarrier per stage;
-//   warp 1, lane 0  MMA issuer: 4 x tcgen05.mma (M=128, N=256, K=32) per stage into a
-//                   128 x 256 f32 accumulator in TMEM (256 columns), tcgen05.commit frees the
-//                   stage; a final commit signals the epilogue;
-//   warps 0-3       epilogue: tcgen05.ld 32 lanes x 32 columns per warp-chunk, scale by sa*sb,
-//                   round to BF16, 16-byte stores (rows >= M and columns >= N masked).
-// Every mbarrier wait is bounded (globaltimer). On expiry the CTA records kErrTimeout, stops
-// issuing, waits (with a separate fixed bound) for the TMA loads and MMAs it already issued,
-// frees its TMEM and returns without writing D.
+// A cluster of two CTAs (one per SM) computes a 256 x 256 tile: CTA r loads A rows
+// [128r, 128r+128) and B rows (N columns) [128r, 128r+128) of the tile, 128-byte swizzled
+// 128 x 128-byte boxes, into its own 6-stage ring (32 KB per stage). Both CTAs' loads count on
+// the even CTA's "full" barrier; the even CTA's MMA thread issues tcgen05.mma.cta_group::2
+// (M=256, N=256, K=32), which reads A and B halves from both CTAs' shared memory, and releases
+// each stage in both CTAs with one multicast tcgen05.commit. Per SM that is 32 KB of operands per
+// 512 tensor-core cycles, two thirds of what a single-SM 128 x 256 tile needs.
+// Persistent: cluster c walks the tiles c, c + clusters, ...; two TMEM accumulators (2 x 256
+// columns) let the epilogue of one tile overlap the main loop of the next.
+// Warp roles (192 threads per CTA):
+//   warp 0, lane 0  TMA producer (both CTAs)
+//   warp 1, lane 0  MMA issuer (even CTA only); warp 1 also owns the TMEM allocation
+//   warps 2-5       epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 of its own CTA (rows of
+//                   its half), scales by sa*sb, rounds to BF16, stores, and tells the even CTA
+//                   that the accumulator is free again (4 warps x 2 CTAs = 8 arrivals).
+// Every mbarrier wait is bounded (globaltimer). On expiry a CTA records kErrTimeout and stops
+// issuing; issued MMAs are awaited with a fixed bound, loads in flight are given time to land,
+// and both CTAs meet at a cluster barrier before TMEM is freed; D is then incomplete.
 #pragma once
 
 #include "ptx.cuh"
@@ -25,11 +33,14 @@
 namespace fp8t {
 namespace gemm {
 
-constexpr int kBM = 128, kBN = 256, kBK = 128, kStages = 4, kUmmaK = 32;
-constexpr int kThreads = 128;
-constexpr int kABytes = kBM * kBK, kBBytes = kBN * kBK, kStageBytes = kABytes + kBBytes;
-constexpr int kTmemCols = 256;
+constexpr int kBM = 256, kBN = 256, kBK = 128, kStages = 6, kUmmaK = 32;
+constexpr int kHalf = 128;                               // rows of A and of B per CTA
+constexpr int kThreads = 192;
+constexpr int kABytes = kHalf * kBK, kBBytes = kHalf * kBK, kStageBytes = kABytes + kBBytes;
+constexpr uint32_t kPairTxBytes = 2 * kStageBytes;       // both CTAs' boxes of one stage
+constexpr int kAccCols = 256, kTmemCols = 2 * kAccCols;
 constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*alignment slack*/ + 256 /*barriers*/;
+constexpr uint64_t kSettleNs = 200000;                   // let loads in flight land on abort
 
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, 8-row groups 1024 B apart.
 __device__ __forceinline__ uint64_t make_sw128_desc(uint32_t saddr) {
@@ -42,7 +53,8 @@ __device__ __forceinline__ uint64_t make_sw128_desc(uint32_t saddr) {
   return d;
 }
 
-// Instruction descriptor: FP32 accumulator, FP8 A/B formats (0 = E4M3, 1 = E5M2), both K-major.
+// Instruction descriptor: FP32 accumulator, FP8 A/B formats (0 = E4M3, 1 = E5M2), both K-major,
+// M = 256 (pair), N = 256.
 __host__ __device__ constexpr uint32_t make_idesc(int a_fmt, int b_fmt) {
   return (1u << 4) | (static_cast<uint32_t>(a_fmt) << 7) | (static_cast<uint32_t>(b_fmt) << 10) |
          (static_cast<uint32_t>(kBN >> 3) << 17) | (static_cast<uint32_t>(kBM >> 4) << 24);
@@ -55,127 +67,177 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+struct Smem {
+  uint64_t full[kStages];     // even CTA: both CTAs' loads of a stage have landed
+  uint64_t empty[kStages];    // both CTAs: the pair MMA has consumed a stage
+  uint64_t acc_full[2];       // both CTAs: an accumulator holds a finished tile
+  uint64_t acc_empty[2];      // even CTA: both epilogues have drained an accumulator
+  uint64_t mma_done;          // even CTA: every issued MMA has completed
+  uint32_t tmem_base;
+  int abort;
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     k_fp8_gemm(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                uint16_t* __restrict__ D, int M, int N, int K, const float* __restrict__ d_sa,
-               const float* __restrict__ d_sb, uint32_t idesc, int n_tiles_n) {
+               const float* __restrict__ d_sb, uint32_t idesc, int n_tiles_n, int n_tiles) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   uint8_t* sA = smem;
   uint8_t* sB = smem + kStages * kABytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
-  uint64_t* empty = full + kStages;
-  uint64_t* accum = empty + kStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  Smem* S = reinterpret_cast<Smem*>(smem + kStages * kStageBytes);
+  volatile int* abort_flag = &S->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int mt = blockIdx.x / n_tiles_n, nt = blockIdx.x % n_tiles_n;
-  const int m0 = mt * kBM, n0 = nt * kBN;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
   const int num_kb = (K + kBK - 1) / kBK;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_u32(&full[s]), 1);
-      mbar_init(smem_u32(&empty[s]), 1);
+      mbar_init(smem_u32(&S->full[s]), 1);
+      mbar_init(smem_u32(&S->empty[s]), 1);
     }
-    mbar_init(smem_u32(accum), 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&S->acc_full[a]), 1);
+      mbar_init(smem_u32(&S->acc_empty[a]), 8);      // 4 epilogue warps x 2 CTAs
+    }
+    mbar_init(smem_u32(&S->mma_done), 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tma_a);
     tma_prefetch_desc(&tma_b);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(smem_u32(&S->tmem_base), kTmemCols);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();                 // barriers initialised and TMEM allocated in both CTAs
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem = S->tmem_base;
   const uint64_t limit = wait_limit_ns();
 
-  if (warp == 0 && lane == 0) {
-    // ---------------- TMA producer
-    int issued = 0;
-    for (int kb = 0; kb < num_kb; ++kb) {
-      const int s = kb % kStages;
-      const uint32_t ph = (kb / kStages) & 1;
-      if (*abort_flag) break;
-      if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1, limit)) {
-        *abort_flag = 1;
-        record_error(kErrTimeout);
-        break;
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer (both CTAs)
+      uint32_t it = 0, issued = 0;
+      for (int tile = cluster; tile < n_tiles && !*abort_flag; tile += n_clusters) {
+        const int m0 = (tile / n_tiles_n) * kBM + static_cast<int>(rank) * kHalf;
+        const int n0 = (tile % n_tiles_n) * kBN + static_cast<int>(rank) * kHalf;
+        for (int kb = 0; kb < num_kb; ++kb, ++it) {
+          const uint32_t s = it % kStages, ph = (it / kStages) & 1;
+          if (*abort_flag) break;
+          if (!mbar_wait(smem_u32(&S->empty[s]), ph ^ 1, limit)) {
+            *abort_flag = 1;
+            record_error(kErrTimeout);
+            break;
+          }
+          const uint32_t full_leader = mapa_shared(smem_u32(&S->full[s]), 0);
+          if (leader) mbar_arrive_expect_tx(smem_u32(&S->full[s]), kPairTxBytes);
+          tma_load_2d_pair(smem_u32(sA + s * kABytes), &tma_a, kb * kBK, m0, full_leader);
+          tma_load_2d_pair(smem_u32(sB + s * kBBytes), &tma_b, kb * kBK, n0, full_leader);
+          ++issued;
+        }
       }
-      mbar_arrive_expect_tx(smem_u32(&full[s]), kStageBytes);
-      tma_load_2d(smem_u32(sA + s * kABytes), &tma_a, kb * kBK, m0, smem_u32(&full[s]));
-      tma_load_2d(smem_u32(sB + s * kBBytes), &tma_b, kb * kBK, n0, smem_u32(&full[s]));
-      ++issued;
+      // the even CTA can see its own stages land: wait for the last ones it armed
+      if (leader)
+        for (uint32_t i = issued > kStages ? issued - kStages : 0; i < issued; ++i)
+          mbar_wait(smem_u32(&S->full[i % kStages]), (i / kStages) & 1, kDrainLimitNs);
     }
-    // every issued load must land before the CTA may exit (only the last kStages can be open)
-    for (int kb = issued > kStages ? issued - kStages : 0; kb < issued; ++kb)
-      mbar_wait(smem_u32(&full[kb % kStages]), (kb / kStages) & 1, kDrainLimitNs);
-  } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer
-    for (int kb = 0; kb < num_kb; ++kb) {
-      const int s = kb % kStages;
-      const uint32_t ph = (kb / kStages) & 1;
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ---------------- MMA issuer (even CTA)
+      uint32_t it = 0, local = 0;
+      for (int tile = cluster; tile < n_tiles && !*abort_flag; tile += n_clusters, ++local) {
+        const uint32_t acc = local & 1, aph = (local >> 1) & 1;
+        if (!mbar_wait(smem_u32(&S->acc_empty[acc]), aph ^ 1, limit)) {
+          *abort_flag = 1;
+          record_error(kErrTimeout);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + acc * kAccCols;
+        bool ok = true;
+        for (int kb = 0; kb < num_kb; ++kb, ++it) {
+          const uint32_t s = it % kStages, ph = (it / kStages) & 1;
+          if (*abort_flag || !mbar_wait(smem_u32(&S->full[s]), ph, limit)) {
+            if (!*abort_flag) record_error(kErrTimeout);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sA + s * kABytes);
+          const uint32_t b_base = smem_u32(sB + s * kBBytes);
+#pragma unroll
+          for (int k = 0; k < kBK / kUmmaK; ++k)
+            tc_mma_f8_pair(d_tmem, make_sw128_desc(a_base + k * kUmmaK),
+                           make_sw128_desc(b_base + k * kUmmaK), idesc, (kb | k) != 0 ? 1u : 0u);
+          tc_commit_pair_mc(smem_u32(&S->empty[s]), 0x3);
+        }
+        if (!ok) break;
+        tc_commit_pair_mc(smem_u32(&S->acc_full[acc]), 0x3);
+      }
+      // every MMA issued here must complete before either CTA frees TMEM or shared memory
+      tc_commit_pair(smem_u32(&S->mma_done));
+      mbar_wait(smem_u32(&S->mma_done), 0, kDrainLimitNs);
+    }
+  } else {
+    // ---------------- epilogue warps 2..5 (both CTAs)
+    const int quad = warp & 3;                       // TMEM lanes 32*quad .. 32*quad+31
+    const float alpha = __fmul_rn(__ldg(d_sa), __ldg(d_sb));
+    uint32_t local = 0;
+    for (int tile = cluster; tile < n_tiles; tile += n_clusters, ++local) {
+      const uint32_t acc = local & 1, aph = (local >> 1) & 1;
       if (*abort_flag) break;
-      if (!mbar_wait(smem_u32(&full[s]), ph, limit)) {
+      if (!mbar_wait(smem_u32(&S->acc_full[acc]), aph, limit)) {
         *abort_flag = 1;
         record_error(kErrTimeout);
         break;
       }
       tc_fence_after();
-      const uint32_t a_base = smem_u32(sA + s * kABytes);
-      const uint32_t b_base = smem_u32(sB + s * kBBytes);
+      const int row = (tile / n_tiles_n) * kBM + static_cast<int>(rank) * kHalf + quad * 32 + lane;
+      const int n0 = (tile % n_tiles_n) * kBN;
+      const uint32_t t_base = tmem + (static_cast<uint32_t>(quad * 32) << 16) + acc * kAccCols;
+#pragma unroll 1
+      for (int c = 0; c < kBN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(t_base + c * 32, r);
+        tmem_ld_wait();
+        const int col = n0 + c * 32;
+        if (row < M && col < N) {
+          uint32_t packed[16];
 #pragma unroll
-      for (int k = 0; k < kBK / kUmmaK; ++k)
-        tc_mma_f8(tmem, make_sw128_desc(a_base + k * kUmmaK), make_sw128_desc(b_base + k * kUmmaK),
-                  idesc, (kb | k) != 0 ? 1u : 0u);
-      tc_commit(smem_u32(&empty[s]));
+          for (int j = 0; j < 16; ++j)
+            packed[j] = pack_bf16x2(__fmul_rn(__uint_as_float(r[2 * j]), alpha),
+                                    __fmul_rn(__uint_as_float(r[2 * j + 1]), alpha));
+          uint16_t* dst = D + static_cast<int64_t>(row) * N + col;
+#pragma unroll
+          for (int qd = 0; qd < 4; ++qd)
+            if (col + 8 * qd < N)
+              *reinterpret_cast<uint4*>(dst + 8 * qd) = make_uint4(
+                  packed[4 * qd], packed[4 * qd + 1], packed[4 * qd + 2], packed[4 * qd + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&S->acc_empty[acc]), 0));
     }
-    tc_commit(smem_u32(accum));  // arrives when every MMA issued above has completed
   }
   __syncwarp();
-
-  // ---------------- epilogue (all four warps)
-  if (!mbar_wait(smem_u32(accum), 0, limit)) {
-    record_error(kErrTimeout);
-    *abort_flag = 1;
-    mbar_wait(smem_u32(accum), 0, kDrainLimitNs);  // MMAs must finish before TMEM is freed
-  }
-  tc_fence_after();
   __syncthreads();
-  const bool aborted = *abort_flag != 0;
-
-  const float alpha = __fmul_rn(__ldg(d_sa), __ldg(d_sb));
-  const int row = m0 + warp * 32 + lane;
-#pragma unroll 1
-  for (int c = 0; c < kBN / 32; ++c) {
-    uint32_t r[32];
-    tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c * 32, r);
-    tmem_ld_wait();
-    const int col = n0 + c * 32;
-    if (!aborted && row < M && col < N) {
-      uint32_t packed[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j)
-        packed[j] = pack_bf16x2(__fmul_rn(__uint_as_float(r[2 * j]), alpha),
-                                __fmul_rn(__uint_as_float(r[2 * j + 1]), alpha));
-      uint16_t* dst = D + static_cast<int64_t>(row) * N + col;
-#pragma unroll
-      for (int qd = 0; qd < 4; ++qd)
-        if (col + 8 * qd < N)
-          *reinterpret_cast<uint4*>(dst + 8 * qd) =
-              make_uint4(packed[4 * qd], packed[4 * qd + 1], packed[4 * qd + 2], packed[4 * qd + 3]);
+  if (*abort_flag && threadIdx.x == 0) {           // loads of either CTA may still be in flight
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < kSettleNs) {
     }
   }
-
   tc_fence_before();
-  __syncthreads();
-  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+  cluster_sync();                 // neither CTA leaves while the pair MMA may still read it
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem, kTmemCols);
 }
 
 }  // namespace gemm

@@ -5,7 +5,8 @@
 // scale used by the next iteration. History row t is [H] floats, entry 0 newest; the roll moves
 // entries i-1 -> i from the top down in chunks of the block size (read, barrier, write,
 // barrier), so no entry is overwritten before it is read. The window max is a u32 max of the
-// magnitude bits, which orders non-negative floats and puts NaN above infinity.
+// magnitude bits, which orders non-negative floats and puts NaN above infinity. Each consumed
+// amax slot is reset to 0 so that the next step's casts can max-accumulate into it.
 // Latency-bound: n * (8H + 16) bytes.
 #pragma once
 
@@ -17,7 +18,7 @@ namespace scale {
 constexpr int kThreads = 256;
 
 __global__ void __launch_bounds__(kThreads)
-    k_scale_update(const float* __restrict__ amax, float* __restrict__ hist, int H,
+    k_scale_update(float* __restrict__ amax, float* __restrict__ hist, int H,
                    const float* __restrict__ fp8_max, int algo_max, int margin,
                    float* __restrict__ scale, float* __restrict__ scale_inv) {
   __shared__ uint32_t red[kThreads / 32];
@@ -59,6 +60,7 @@ __global__ void __launch_bounds__(kThreads)
     }
     scale[t] = s;
     scale_inv[t] = __fdiv_rn(1.0f, s);
+    amax[t] = 0.0f;                                           // consumed: ready to accumulate
   }
 }
 

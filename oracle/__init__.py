@@ -112,15 +112,16 @@ def encode_array(x_f32: np.ndarray, fmt: int) -> np.ndarray:
 
 
 # ----------------------------------------------------------------------------- cast
-def cast_transpose_amax(x_bf16: np.ndarray, fmt: int, scale: float, want_q=True, want_qT=True):
+def cast_transpose_amax(x_bf16: np.ndarray, fmt: int, scale: float, want_q=True, want_qT=True,
+                        amax_in=0.0):
     """Oracle of fp8_cast_transpose_amax on a 2-D uint16 (BF16 bits) array.
 
-    Returns (q, qT, amax, scale_inv, counters[3])."""
+    Returns (q, qT, amax, scale_inv, counters[3]); amax is max-accumulated onto amax_in."""
     x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
     rows, cols = x.shape
     q = np.empty((rows, cols), np.uint8) if want_q else None
     qT = np.empty((cols, rows), np.uint8) if want_qT else None
-    amax = np.zeros(1, np.float32)
+    amax = np.array([amax_in], np.float32)
     sinv = np.zeros(1, np.float32)
     cnt = np.zeros(3, np.uint64)
     lib().orc_cast_transpose_amax(_ptr(x, C.c_uint16), rows, cols, int(fmt),
@@ -132,8 +133,10 @@ def cast_transpose_amax(x_bf16: np.ndarray, fmt: int, scale: float, want_q=True,
 
 # ----------------------------------------------------------------------------- scale update
 def scale_update(amax, hist, fp8_max, algo, margin, scale, scale_inv):
-    """Oracle of fp8_scale_update. hist [n, H], scale and scale_inv [n] are updated in place."""
-    amax = np.ascontiguousarray(amax, np.float32)
+    """Oracle of fp8_scale_update. hist [n, H], scale and scale_inv [n] are updated in place;
+    amax is reset to 0 in place when it is a float32 array (a copy is consumed otherwise)."""
+    if not (isinstance(amax, np.ndarray) and amax.dtype == np.float32 and amax.flags["C_CONTIGUOUS"]):
+        amax = np.ascontiguousarray(amax, np.float32)
     fp8_max = np.ascontiguousarray(fp8_max, np.float32)
     assert hist.dtype == np.float32 and hist.flags["C_CONTIGUOUS"] and hist.ndim == 2
     assert scale.dtype == np.float32 and scale_inv.dtype == np.float32

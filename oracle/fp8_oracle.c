@@ -155,6 +155,8 @@ void orc_fp8_encode_array(const float* x, int64_t n, int fmt, uint8_t* out)
  * amax = max |x| over the BF16 input [P2 §四, quantize records max(abs(x))] — taken on the
  * unscaled input. Computed as the largest magnitude bit pattern (bits & 0x7FFF), which orders
  * non-negative BF16 values exactly and puts NaN above infinity; a NaN result is 0x7FC0.
+ * The amax slot is max-accumulated: it becomes the larger of its previous content and max|x|,
+ * both non-negative f32 values or NaN, compared as bit patterns (so NaN dominates).
  * Counters [P3 工程落地, 第四步 量化质量: fraction near the FP8 maximum, fraction of zeros
  * after quantisation; 梯度健康: NaN/Inf counts]:
  *   c[0] += #{ |f32(x*scale)| > FP8 max }   (infinite products included, NaN not)
@@ -184,7 +186,10 @@ void orc_cast_transpose_amax(const uint16_t* x, int64_t rows, int64_t cols, int 
         }
     }
     if (amax_bits > 0x7F80u) amax_bits = 0x7FC0u;
-    if (amax_out) *amax_out = bits_f32(amax_bits << 16);
+    if (amax_out) {
+        const uint32_t prev = f32_bits(*amax_out), cur = amax_bits << 16;
+        *amax_out = bits_f32(prev > cur ? prev : cur);
+    }
     if (scale_inv_out) *scale_inv_out = 1.0f / scale;
     if (counters) {
         counters[0] += nsat;
@@ -201,7 +206,8 @@ void orc_cast_transpose_amax(const uint16_t* x, int64_t rows, int64_t cols, int 
  * includes the amax just recorded; rep = 0 gives scale 1.0 (the fallback the ScalingFactor
  * sketch of [P2 §四] uses for an empty history); a NaN or infinite rep keeps the previous
  * scale; a scale that overflows f32 becomes FLT_MAX. History entries are magnitudes, and rep
- * is taken over |h| with NaN propagating.
+ * is taken over |h| with NaN propagating. Each consumed amax entry is reset to 0 afterwards
+ * (the state a step starts from: casts max-accumulate into zeroed slots).
  * ------------------------------------------------------------------------------------- */
 static float mag_max(float a, float b)  /* NaN-propagating max of |a|, |b| */
 {
@@ -210,7 +216,7 @@ static float mag_max(float a, float b)  /* NaN-propagating max of |a|, |b| */
     return a > b ? a : b;
 }
 
-void orc_scale_update(int32_t n, const float* amax, float* hist, int32_t H, const float* fp8_max,
+void orc_scale_update(int32_t n, float* amax, float* hist, int32_t H, const float* fp8_max,
                       int algo, int32_t margin, float* scale, float* scale_inv)
 {
     const float pow2_neg_margin = (float)ldexp(1.0, -margin); /* exact for 0 <= margin <= 126 */
@@ -233,6 +239,7 @@ void orc_scale_update(int32_t n, const float* amax, float* hist, int32_t H, cons
         }
         scale[t] = s;
         scale_inv[t] = 1.0f / s;
+        amax[t] = 0.0f;
     }
 }
 

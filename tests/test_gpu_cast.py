@@ -20,7 +20,7 @@ def run_gpu(fp8, x, fmt, scale, want_q=True, want_qT=True, counters=True):
     rows, cols = x.shape
     q = torch.empty(rows, cols, dtype=torch.uint8, device="cuda") if want_q else None
     qT = torch.empty(cols, rows, dtype=torch.uint8, device="cuda") if want_qT else None
-    amax = torch.full((1,), 12345.0, device="cuda")                 # must be overwritten
+    amax = torch.zeros(1, device="cuda")                            # max-accumulated from 0
     sinv = torch.zeros(1, device="cuda")
     cnt = torch.zeros(3, dtype=torch.int64, device="cuda") if counters else None
     fp8.fp8_cast_transpose_amax(x, fmt, dev_scalar(scale), q, qT, amax, sinv, cnt)
@@ -84,6 +84,19 @@ def test_counters_accumulate(cuda_lib):
         cuda_lib.fp8_cast_transpose_amax(xd, oracle.E4M3, dev_scalar(4.0), None, None, amax, None, cnt)
     _, _, _, _, rc = oracle.cast_transpose_amax(bf16_bits(xd), oracle.E4M3, 4.0)
     assert np.array_equal(cnt.cpu().numpy(), 3 * rc.astype(np.int64))
+
+
+def test_amax_is_max_accumulated(cuda_lib):
+    """The amax slot keeps the larger of its content and max|x|; NaN dominates."""
+    x = (torch.randn(64, 64) * 3).to(torch.bfloat16)
+    bits = bf16_bits(x)
+    xd = bf16_from_bits(bits)
+    for start in (0.0, 1e-3, 1e6, float("inf"), float("nan")):
+        amax = torch.tensor([start], device="cuda")
+        cuda_lib.fp8_cast_transpose_amax(xd, oracle.E4M3, dev_scalar(1.0), None, None, amax)
+        _, _, ref, _, _ = oracle.cast_transpose_amax(bits, oracle.E4M3, 1.0, False, False, amax_in=start)
+        got = np.float32(amax.item())
+        assert got.view(np.uint32) == np.float32(ref).view(np.uint32), (start, got, ref)
 
 
 def test_special_values_and_nan_amax(cuda_lib):

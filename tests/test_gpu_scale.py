@@ -25,9 +25,11 @@ def test_random_histories(cuda_lib, H, algo, margin):
         amax = rng.lognormal(0, 3, n).astype(np.float32)
         amax[:3] = [0.0, np.nan, np.inf] if step == 1 else amax[:3]
         amax[3] = 1e-40
-        cuda_lib.fp8_scale_update(torch.from_numpy(amax).cuda(), dh, dm, algo, margin, ds, dsi)
+        damax = torch.from_numpy(amax.copy()).cuda()
+        cuda_lib.fp8_scale_update(damax, dh, dm, algo, margin, ds, dsi)
         oracle.scale_update(amax, hist, fp8_max, algo, margin, scale, sinv)
         cuda_lib.fp8t_check_device_error()
+        assert not damax.any().item() and not amax.any()         # consumed slots reset to 0
         assert np.array_equal(dh.cpu().numpy().view(np.uint32), hist.view(np.uint32))
         assert np.array_equal(ds.cpu().numpy().view(np.uint32), scale.view(np.uint32))
         assert np.array_equal(dsi.cpu().numpy().view(np.uint32), sinv.view(np.uint32))

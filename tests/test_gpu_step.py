@@ -70,8 +70,9 @@ def check_step(st, pre, xs, dys, gemm_full=True, gemm_samples=2048, cast_check=T
                 ii, jj = sample_positions(Dh.shape[0], Dh.shape[1], gemm_samples, seed=k)
                 R, ab = oracle.gemm_at(Ah, af, Bh, bf, sa, sb, ii, jj)
                 assert gemm_within_tolerance(Dh[ii, jj], R, ab).all()
-    # amax and the scale update
-    assert np.array_equal(f32(st.amax).view(np.uint32), amax_ref.view(np.uint32))
+    # amax (entry 0 of each history row) and the scale update; consumed amax slots are reset
+    assert np.array_equal(f32(st.history)[:, 0].view(np.uint32), amax_ref.view(np.uint32))
+    assert not st.amax.any().item()
     hist, scale = pre["hist"].copy(), pre["scale"].copy()
     sinv = np.zeros_like(scale)
     oracle.scale_update(amax_ref, hist, f32(st.fp8_max), st.algo, st.margin, scale, sinv)

@@ -68,6 +68,16 @@ def test_amax_special_cases():
     assert oracle.cast_transpose_amax(x, E, 1.0)[2] == bf16_to_f32(np.uint16(0x0003))
 
 
+def test_amax_slot_is_max_accumulated():
+    x = np.full((16, 16), 0x4000, np.uint16)                      # all 2.0
+    E = oracle.E4M3
+    assert oracle.cast_transpose_amax(x, E, 1.0, amax_in=0.0)[2] == 2.0
+    assert oracle.cast_transpose_amax(x, E, 1.0, amax_in=5.0)[2] == 5.0
+    assert oracle.cast_transpose_amax(x, E, 1.0, amax_in=1.5)[2] == 2.0
+    assert np.isnan(oracle.cast_transpose_amax(x, E, 1.0, amax_in=float("nan"))[2])
+    assert oracle.cast_transpose_amax(x, E, 1.0, amax_in=float("inf"))[2] == np.inf
+
+
 def test_counters_accumulate_and_hand_case():
     """Counters add to what the caller passes in; a hand-made 16x16 case."""
     x = np.zeros((16, 16), np.uint16)

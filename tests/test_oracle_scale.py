@@ -58,6 +58,14 @@ def test_history_sequence_h4():
             assert scale[0] == np.float32(nearest_f32(Fraction(448) / Fraction(g[key][t])))
 
 
+def test_consumed_amax_is_reset():
+    amax = np.array([3.0, np.nan, 0.5], np.float32)
+    hist = np.zeros((3, 4), np.float32)
+    s = np.ones(3, np.float32); si = np.ones(3, np.float32)
+    oracle.scale_update(amax, hist, [448.0] * 3, oracle.AMAX_MAX, 0, s, si)
+    assert np.all(amax == 0) and hist[0, 0] == 3.0 and np.isnan(hist[1, 0])
+
+
 def test_h1_max_equals_most_recent():
     rng = np.random.default_rng(5)
     seq = rng.uniform(0, 10, 20).astype(np.float32)
