@@ -194,6 +194,37 @@ fp8t_status fused_adamw_multi_tensor(const fp8t_adamw_tensor* tensors, int32_t n
 /* Scratch bytes fused_adamw_multi_tensor needs for these tensors (0 on invalid input). */
 size_t fused_adamw_workspace_bytes(const fp8t_adamw_tensor* tensors, int32_t n_tensors);
 
+/* Size of the scratch array built into the library for fused_adamw_multi_tensor_noalloc. */
+#define FP8T_NOALLOC_SCRATCH_BYTES 65536
+
+/*
+ * fused_adamw_multi_tensor_noalloc — the same AdamW step as fused_adamw_multi_tensor (same
+ * arguments, same results), for callers that have no way to give the library scratch memory.
+ * The pages have no counterpart to this entry point; it only changes where the scratch lives.
+ *
+ * Who needs it: a plugin or extension that receives the parameter, moment and gradient buffers
+ * from a host framework but has no handle on that framework's device allocator, and code that
+ * must not allocate once it is running because all device memory was reserved up front by a
+ * pool. Neither can call cudaMalloc for the few kilobytes of per-block norm partials.
+ *
+ * Scratch: a file-scope device array of FP8T_NOALLOC_SCRATCH_BYTES (64 KiB) inside the library;
+ * every GPU that loads the library keeps it until the process exits. It holds at most 8192 norm
+ * partials: any call with up to 3328 tensors fits, and larger calls fit when their tensors are
+ * small. A call that needs more (fused_adamw_workspace_bytes() > FP8T_NOALLOC_SCRATCH_BYTES)
+ * returns FP8T_ERR_UNSUPPORTED_SHAPE with a message and launches nothing.
+ * Set-up: the first call on each device looks up the array's device address (with that device
+ * current); make that first call before any stream capture on the device.
+ * Sharing: every call uses the same array, which keeps the last call's contents. Each call
+ * writes every slot it reads before reading it, so nothing has to be cleared, but two calls
+ * whose kernels overlap on the GPU (different streams with no ordering between them) race on it.
+ * It allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ */
+fp8t_status fused_adamw_multi_tensor_noalloc(const fp8t_adamw_tensor* tensors, int32_t n_tensors,
+                                             float lr, float beta1, float beta2, float eps,
+                                             float weight_decay, int64_t step, float loss_scale,
+                                             float max_grad_norm, float* d_grad_norm_out,
+                                             int32_t* d_skipped_out, void* stream);
+
 /* Synchronise `stream`, then read and clear the device error word: FP8T_ERR_TIMEOUT if a bounded
  * wait in any kernel expired since the last check, FP8T_ERR_CUDA if the stream reports an error. */
 fp8t_status fp8t_check_device_error(void* stream);

@@ -14,7 +14,8 @@ import torch
 from . import _abi
 
 __all__ = ["fp8_cast_transpose_amax", "fp8_gemm", "fp8_scale_update", "fused_adamw_multi_tensor",
-           "fused_adamw_workspace_bytes", "fp8t_check_device_error", "fp8t_set_wait_timeout_ns",
+           "fused_adamw_workspace_bytes", "fused_adamw_multi_tensor_noalloc",
+           "fp8t_check_device_error", "fp8t_set_wait_timeout_ns",
            "Fp8TrainError", "E4M3", "E5M2", "AMAX_MAX", "AMAX_MOST_RECENT", "FP8_MAX", "load",
            "LIB_PATH"]
 
@@ -134,6 +135,21 @@ def fused_adamw_multi_tensor(master, m, v, grads, weights, *, lr, beta1, beta2, 
                                            _ptr(grad_norm), _ptr(skipped), _ptr(workspace),
                                            workspace.numel(), _stream(stream)),
            "fused_adamw_multi_tensor")
+
+
+def fused_adamw_multi_tensor_noalloc(master, m, v, grads, weights, *, lr, beta1, beta2, eps,
+                                     weight_decay, step, loss_scale, max_grad_norm,
+                                     grad_norm=None, skipped=None, stream=None):
+    """The same AdamW step, with no scratch buffer from the caller: for code that cannot
+    allocate device memory (for instance a plugin that is handed the parameter buffers but not
+    the framework's allocator). The library uses a 64 KiB array of its own instead; calls share
+    it, so calls that overlap on the GPU race. Allocates nothing."""
+    arr, n = _tensor_table(master, m, v, grads, weights)
+    _check(load().fused_adamw_multi_tensor_noalloc(arr, n, float(lr), float(beta1), float(beta2),
+                                                   float(eps), float(weight_decay), int(step),
+                                                   float(loss_scale), float(max_grad_norm),
+                                                   _ptr(grad_norm), _ptr(skipped), _stream(stream)),
+           "fused_adamw_multi_tensor_noalloc")
 
 
 def fp8t_check_device_error(stream=None):

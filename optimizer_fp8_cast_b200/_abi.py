@@ -27,6 +27,9 @@ def declare(L):
     L.fused_adamw_multi_tensor.restype = C.c_int
     L.fused_adamw_multi_tensor.argtypes = [C.POINTER(AdamWTensor), i32, f32, f32, f32, f32, f32,
                                            i64, f32, f32, vp, vp, vp, C.c_size_t, vp]
+    L.fused_adamw_multi_tensor_noalloc.restype = C.c_int
+    L.fused_adamw_multi_tensor_noalloc.argtypes = [C.POINTER(AdamWTensor), i32, f32, f32, f32, f32,
+                                                   f32, i64, f32, f32, vp, vp, vp]
     L.fused_adamw_workspace_bytes.restype = C.c_size_t
     L.fused_adamw_workspace_bytes.argtypes = [C.POINTER(AdamWTensor), i32]
     L.fp8t_check_device_error.restype = C.c_int

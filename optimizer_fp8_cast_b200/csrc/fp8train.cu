@@ -42,6 +42,7 @@ struct DeviceInfo {
   int sms = 0;
   int adamw_blocks_per_sm = 0;
   int gemm_clusters = 0;       // co-resident 2-CTA clusters of the GEMM kernel
+  void* noalloc_scratch = nullptr;   // device address of g_adamw_noalloc_scratch
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
@@ -157,6 +158,11 @@ size_t workspace_for(const AdamWPlan& p) {
 }
 
 }  // namespace
+
+// Scratch of fused_adamw_multi_tensor_noalloc, for callers that cannot allocate: a file-scope
+// device array, present on every GPU that loads the library until the process exits. In host
+// code this name is only a stand-in; its device address comes from cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_adamw_noalloc_scratch[FP8T_NOALLOC_SCRATCH_BYTES];
 
 extern "C" {
 
@@ -374,6 +380,43 @@ fp8t_status fused_adamw_multi_tensor(const fp8t_adamw_tensor* tensors, int32_t n
     }
   }
   return FP8T_OK;
+}
+
+// Same step as fused_adamw_multi_tensor, with the built-in scratch array as its workspace.
+fp8t_status fused_adamw_multi_tensor_noalloc(const fp8t_adamw_tensor* tensors, int32_t n_tensors,
+                                             float lr, float beta1, float beta2, float eps,
+                                             float weight_decay, int64_t step, float loss_scale,
+                                             float max_grad_norm, float* d_grad_norm_out,
+                                             int32_t* d_skipped_out, void* stream) {
+  t_last_error.clear();
+  const size_t need = fused_adamw_workspace_bytes(tensors, n_tensors);
+  if (need == 0)   // invalid tensor table: the regular entry point reports it, launching nothing
+    return fused_adamw_multi_tensor(tensors, n_tensors, lr, beta1, beta2, eps, weight_decay, step,
+                                    loss_scale, max_grad_norm, d_grad_norm_out, d_skipped_out,
+                                    nullptr, 0, stream);
+  if (need > FP8T_NOALLOC_SCRATCH_BYTES)
+    return fail(FP8T_ERR_UNSUPPORTED_SHAPE,
+                "fused_adamw_multi_tensor_noalloc: needs %zu bytes of scratch, the built-in array "
+                "holds %d; split the tensors over several calls or use fused_adamw_multi_tensor",
+                need, FP8T_NOALLOC_SCRATCH_BYTES);
+  DeviceInfo* dev = nullptr;
+  fp8t_status st = current_device(&dev);
+  if (st != FP8T_OK) return st;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (!dev->noalloc_scratch) {       // once per device, with that device current
+      void* p = nullptr;
+      cudaError_t e = cudaGetSymbolAddress(&p, g_adamw_noalloc_scratch);
+      if (e != cudaSuccess || !p)
+        return fail(FP8T_ERR_CUDA, "cudaGetSymbolAddress(noalloc scratch): %s", cudaGetErrorString(e));
+      dev->noalloc_scratch = p;
+    }
+    scratch = dev->noalloc_scratch;
+  }
+  return fused_adamw_multi_tensor(tensors, n_tensors, lr, beta1, beta2, eps, weight_decay, step,
+                                  loss_scale, max_grad_norm, d_grad_norm_out, d_skipped_out,
+                                  scratch, FP8T_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 // ------------------------------------------------------------------ device error word
