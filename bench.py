@@ -220,13 +220,7 @@ def run_ours(args, rank, world, local_rank):
     hbm = peaks["hbm_gbs"]
     gemm_avg_ms = statistics.mean(gemm_ms)
     gemm_achieved = nums["gemm_flop"] / (gemm_avg_ms * 1e-3) / 1e12
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", "gemm_traffic.json")
-    if os.path.exists(tpath):
-        with open(tpath) as f:
-            tj = json.load(f)
-        if tj.get("workload") == wl.name and tj.get("kernel_source_sha") == kernel_source_sha():
-            traffic = tj.get("bytes_per_launch")
+    traffic = gemm_traffic_from_profile(wl.name)
 
     # end to end: host (pinned) inputs copied in and results copied out inside the timed region
     hX = [b[0].cpu().pin_memory() for b in batches]
@@ -302,11 +296,27 @@ def gpu_uuid(dev, fallback):
     return s if s.startswith("GPU-") else "GPU-" + s
 
 
-def kernel_source_sha():
+def gemm_traffic_from_profile(workload):
+    """DRAM bytes (read + write) per GEMM launch from the committed ncu summary, or None when the
+    summary is missing or was taken on different kernel sources."""
+    import re
+    path = os.path.join(ROOT, "profiles", f"k_fp8_gemm_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    t = re.search(r"traffic_bytes_per_launch[^:]*:\s*(\d+)", text)
+    sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text)
+    if not t or not sha or sha.group(1) != kernel_source_sha():
+        return None
+    return int(t.group(1))
+
+
+def kernel_source_sha(files=("gemm_tcgen05.cuh", "ptx.cuh")):
+    """Hash of the GEMM kernel's source files (what the committed counters were taken on)."""
     import hashlib
     h = hashlib.sha256()
     d = os.path.join(ROOT, "optimizer_fp8_cast_b200", "csrc")
-    for f in sorted(os.listdir(d)):
+    for f in files:
         with open(os.path.join(d, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
