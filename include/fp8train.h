@@ -93,6 +93,29 @@ fp8t_status fp8_cast_transpose_amax(const void* x_bf16, int64_t rows, int64_t co
                                     float* d_amax_inout, float* d_scale_inv_out,
                                     unsigned long long* d_counters, void* stream);
 
+/* One tensor of fp8_cast_transpose_amax_multi: the arguments of fp8_cast_transpose_amax. */
+typedef struct fp8t_cast_tensor {
+    const void* x_bf16;
+    int64_t rows, cols;
+    fp8t_format fmt;
+    const float* d_scale;
+    void* q_rowmajor;                  /* may be NULL */
+    void* q_transposed;                /* may be NULL */
+    float* d_amax_inout;
+    float* d_scale_inv_out;            /* may be NULL */
+    unsigned long long* d_counters;    /* may be NULL */
+} fp8t_cast_tensor;
+
+/*
+ * fp8_cast_transpose_amax_multi — fp8_cast_transpose_amax for several tensors in one launch
+ * (the X, W and dY casts of a step, for instance), with the same per-tensor semantics and
+ * validation. Up to 8 tensors share a launch; longer lists are split into several launches.
+ *   tensors     HOST array of n_tensors descriptors (read during the call only).
+ *   n_tensors   1 .. 4096.
+ */
+fp8t_status fp8_cast_transpose_amax_multi(const fp8t_cast_tensor* tensors, int32_t n_tensors,
+                                          void* stream);
+
 /*
  * fp8_gemm — per-tensor scaled FP8 GEMM, FP32 accumulation, BF16 output, "TN" layout:
  *
@@ -177,7 +200,13 @@ typedef struct fp8t_adamw_tensor {
  *
  *   tensors         HOST array of n_tensors descriptors (read during the call only).
  *   n_tensors       1 .. 1<<20.
- *   step            >= 1 (bias-correction step count).
+ *   step            >= 1 (bias-correction step count); used when d_step_inout is NULL.
+ *   d_step_inout    1 int64 in device memory holding the number of completed steps, or NULL.
+ *                   When given, `step` is ignored: the call performs step counter+1 and stores
+ *                   that back into the counter unless the update is skipped, so a CUDA graph that
+ *                   captured the call advances the optimizer on every replay. lr/(1-beta1^t) and
+ *                   sqrt(1-beta2^t) are then formed on the device, in double with the same
+ *                   formulas (a one-ulp difference from host-formed ones is possible).
  *   loss_scale      > 0 and finite.  max_grad_norm <= 0 disables clipping.
  *   d_grad_norm_out 1 float (device) or NULL: the unscaled global norm.
  *   d_skipped_out   1 int32 (device) or NULL.
@@ -186,10 +215,10 @@ typedef struct fp8t_adamw_tensor {
  */
 fp8t_status fused_adamw_multi_tensor(const fp8t_adamw_tensor* tensors, int32_t n_tensors,
                                      float lr, float beta1, float beta2, float eps,
-                                     float weight_decay, int64_t step, float loss_scale,
-                                     float max_grad_norm, float* d_grad_norm_out,
-                                     int32_t* d_skipped_out, void* d_workspace,
-                                     size_t workspace_bytes, void* stream);
+                                     float weight_decay, int64_t step, int64_t* d_step_inout,
+                                     float loss_scale, float max_grad_norm,
+                                     float* d_grad_norm_out, int32_t* d_skipped_out,
+                                     void* d_workspace, size_t workspace_bytes, void* stream);
 
 /* Scratch bytes fused_adamw_multi_tensor needs for these tensors (0 on invalid input). */
 size_t fused_adamw_workspace_bytes(const fp8t_adamw_tensor* tensors, int32_t n_tensors);
@@ -208,9 +237,9 @@ size_t fused_adamw_workspace_bytes(const fp8t_adamw_tensor* tensors, int32_t n_t
  * pool. Neither can call cudaMalloc for the few kilobytes of per-block norm partials.
  *
  * Scratch: a file-scope device array of FP8T_NOALLOC_SCRATCH_BYTES (64 KiB) inside the library;
- * every GPU that loads the library keeps it until the process exits. It holds at most 8192 norm
- * partials: any call with up to 3328 tensors fits, and larger calls fit when their tensors are
- * small. A call that needs more (fused_adamw_workspace_bytes() > FP8T_NOALLOC_SCRATCH_BYTES)
+ * every GPU that loads the library keeps it until the process exits. It holds 8191 norm
+ * partials and one step slot: any call with up to 3328 tensors fits, and larger calls fit when
+ * their tensors are small. A call that needs more (fused_adamw_workspace_bytes() > FP8T_NOALLOC_SCRATCH_BYTES)
  * returns FP8T_ERR_UNSUPPORTED_SHAPE with a message and launches nothing.
  * Set-up: the first call on each device looks up the array's device address (with that device
  * current); make that first call before any stream capture on the device.
@@ -221,7 +250,8 @@ size_t fused_adamw_workspace_bytes(const fp8t_adamw_tensor* tensors, int32_t n_t
  */
 fp8t_status fused_adamw_multi_tensor_noalloc(const fp8t_adamw_tensor* tensors, int32_t n_tensors,
                                              float lr, float beta1, float beta2, float eps,
-                                             float weight_decay, int64_t step, float loss_scale,
+                                             float weight_decay, int64_t step,
+                                             int64_t* d_step_inout, float loss_scale,
                                              float max_grad_norm, float* d_grad_norm_out,
                                              int32_t* d_skipped_out, void* stream);
 

@@ -13,7 +13,7 @@ import torch
 
 from . import _abi
 
-__all__ = ["fp8_cast_transpose_amax", "fp8_gemm", "fp8_scale_update", "fused_adamw_multi_tensor",
+__all__ = ["fp8_cast_transpose_amax", "fp8_cast_transpose_amax_multi", "fp8_gemm", "fp8_scale_update", "fused_adamw_multi_tensor",
            "fused_adamw_workspace_bytes", "fused_adamw_multi_tensor_noalloc",
            "fp8t_check_device_error", "fp8t_set_wait_timeout_ns",
            "Fp8TrainError", "E4M3", "E5M2", "AMAX_MAX", "AMAX_MOST_RECENT", "FP8_MAX", "load",
@@ -80,6 +80,20 @@ def fp8_cast_transpose_amax(x, fmt, scale, q=None, qT=None, amax=None, scale_inv
                                           _stream(stream)), "fp8_cast_transpose_amax")
 
 
+def fp8_cast_transpose_amax_multi(casts, stream=None):
+    """Several casts in one launch. ``casts`` is a list of dicts with the keyword arguments of
+    fp8_cast_transpose_amax (x, fmt, scale and optionally q, qT, amax, scale_inv, counters)."""
+    arr = (_abi.CastTensor * len(casts))()
+    for i, c in enumerate(casts):
+        x = c["x"]
+        assert x.dtype == torch.bfloat16 and x.dim() == 2
+        arr[i] = _abi.CastTensor(_ptr(x), x.shape[0], x.shape[1], int(c["fmt"]), _ptr(c["scale"]),
+                                 _ptr(c.get("q")), _ptr(c.get("qT")), _ptr(c.get("amax")),
+                                 _ptr(c.get("scale_inv")), _ptr(c.get("counters")))
+    _check(load().fp8_cast_transpose_amax_multi(arr, len(casts), _stream(stream)),
+           "fp8_cast_transpose_amax_multi")
+
+
 def fp8_gemm(A, a_fmt, B, b_fmt, a_scale_inv, b_scale_inv, D, stream=None):
     """D [M, N] bf16 = (A [M, K] . B [N, K]^T) * a_scale_inv * b_scale_inv; A, B uint8 FP8 codes."""
     M, K = A.shape
@@ -121,17 +135,21 @@ def fused_adamw_workspace_bytes(numels):
 
 def fused_adamw_multi_tensor(master, m, v, grads, weights, *, lr, beta1, beta2, eps,
                              weight_decay, step, loss_scale, max_grad_norm, grad_norm=None,
-                             skipped=None, workspace=None, stream=None):
+                             skipped=None, workspace=None, step_counter=None, stream=None):
     """One fused AdamW step over lists of tensors (see include/fp8train.h for the arithmetic).
 
-    ``workspace`` is a uint8 CUDA tensor of at least ``fused_adamw_workspace_bytes`` bytes."""
+    ``workspace`` is a uint8 CUDA tensor of at least ``fused_adamw_workspace_bytes`` bytes.
+    ``step_counter`` (int64 [1] on the device, completed steps) replaces ``step``: the call
+    performs step counter+1 and stores it back unless the update is skipped, which lets a
+    captured CUDA graph replay successive steps."""
     arr, n = _tensor_table(master, m, v, grads, weights)
     need = int(load().fused_adamw_workspace_bytes(arr, n))
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=master[0].device)
     _check(load().fused_adamw_multi_tensor(arr, n, float(lr), float(beta1), float(beta2),
                                            float(eps), float(weight_decay), int(step),
-                                           float(loss_scale), float(max_grad_norm),
+                                           _ptr(step_counter), float(loss_scale),
+                                           float(max_grad_norm),
                                            _ptr(grad_norm), _ptr(skipped), _ptr(workspace),
                                            workspace.numel(), _stream(stream)),
            "fused_adamw_multi_tensor")
@@ -139,7 +157,7 @@ def fused_adamw_multi_tensor(master, m, v, grads, weights, *, lr, beta1, beta2, 
 
 def fused_adamw_multi_tensor_noalloc(master, m, v, grads, weights, *, lr, beta1, beta2, eps,
                                      weight_decay, step, loss_scale, max_grad_norm,
-                                     grad_norm=None, skipped=None, stream=None):
+                                     grad_norm=None, skipped=None, step_counter=None, stream=None):
     """The same AdamW step, with no scratch buffer from the caller: for code that cannot
     allocate device memory (for instance a plugin that is handed the parameter buffers but not
     the framework's allocator). The library uses a 64 KiB array of its own instead; calls share
@@ -147,7 +165,8 @@ def fused_adamw_multi_tensor_noalloc(master, m, v, grads, weights, *, lr, beta1,
     arr, n = _tensor_table(master, m, v, grads, weights)
     _check(load().fused_adamw_multi_tensor_noalloc(arr, n, float(lr), float(beta1), float(beta2),
                                                    float(eps), float(weight_decay), int(step),
-                                                   float(loss_scale), float(max_grad_norm),
+                                                   _ptr(step_counter), float(loss_scale),
+                                                   float(max_grad_norm),
                                                    _ptr(grad_norm), _ptr(skipped), _stream(stream)),
            "fused_adamw_multi_tensor_noalloc")
 

@@ -16,20 +16,30 @@ class AdamWTensor(C.Structure):
                 ("grad_bf16", C.c_void_p), ("weight_bf16", C.c_void_p), ("numel", C.c_int64)]
 
 
+class CastTensor(C.Structure):
+    """fp8t_cast_tensor."""
+    _fields_ = [("x_bf16", C.c_void_p), ("rows", C.c_int64), ("cols", C.c_int64),
+                ("fmt", C.c_int), ("d_scale", C.c_void_p), ("q_rowmajor", C.c_void_p),
+                ("q_transposed", C.c_void_p), ("d_amax_inout", C.c_void_p),
+                ("d_scale_inv_out", C.c_void_p), ("d_counters", C.c_void_p)]
+
+
 def declare(L):
     vp, i32, i64, f32 = C.c_void_p, C.c_int32, C.c_int64, C.c_float
     L.fp8_cast_transpose_amax.restype = C.c_int
     L.fp8_cast_transpose_amax.argtypes = [vp, i64, i64, C.c_int, vp, vp, vp, vp, vp, vp, vp]
+    L.fp8_cast_transpose_amax_multi.restype = C.c_int
+    L.fp8_cast_transpose_amax_multi.argtypes = [C.POINTER(CastTensor), i32, vp]
     L.fp8_gemm.restype = C.c_int
     L.fp8_gemm.argtypes = [vp, C.c_int, vp, C.c_int, i64, i64, i64, vp, vp, vp, vp]
     L.fp8_scale_update.restype = C.c_int
     L.fp8_scale_update.argtypes = [i32, vp, vp, i32, vp, C.c_int, i32, vp, vp, vp]
     L.fused_adamw_multi_tensor.restype = C.c_int
     L.fused_adamw_multi_tensor.argtypes = [C.POINTER(AdamWTensor), i32, f32, f32, f32, f32, f32,
-                                           i64, f32, f32, vp, vp, vp, C.c_size_t, vp]
+                                           i64, vp, f32, f32, vp, vp, vp, C.c_size_t, vp]
     L.fused_adamw_multi_tensor_noalloc.restype = C.c_int
     L.fused_adamw_multi_tensor_noalloc.argtypes = [C.POINTER(AdamWTensor), i32, f32, f32, f32, f32,
-                                                   f32, i64, f32, f32, vp, vp, vp]
+                                                   f32, i64, vp, f32, f32, vp, vp, vp]
     L.fused_adamw_workspace_bytes.restype = C.c_size_t
     L.fused_adamw_workspace_bytes.argtypes = [C.POINTER(AdamWTensor), i32]
     L.fp8t_check_device_error.restype = C.c_int

@@ -42,6 +42,7 @@ struct DeviceInfo {
   int sms = 0;
   int adamw_blocks_per_sm = 0;
   int gemm_clusters = 0;       // co-resident 2-CTA clusters of the GEMM kernel
+  int cast_blocks_per_sm = 0;
   void* noalloc_scratch = nullptr;   // device address of g_adamw_noalloc_scratch
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -85,6 +86,22 @@ fp8t_status current_device(DeviceInfo** out) {
         clusters = sms / 2;
       }
       d.gemm_clusters = clusters;
+      e = cudaFuncSetAttribute(fp8t::cast::k_cast_transpose_amax<false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, fp8t::cast::kSmemBytes);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(fp8t::cast::k_cast_transpose_amax<true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, fp8t::cast::kSmemBytes);
+      if (e != cudaSuccess) {
+        d.state = 0;
+        return fail(FP8T_ERR_CUDA, "cudaFuncSetAttribute(cast): %s", cudaGetErrorString(e));
+      }
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.cast_blocks_per_sm,
+                                                        fp8t::cast::k_cast_transpose_amax<true>,
+                                                        fp8t::cast::kThreads, fp8t::cast::kSmemBytes);
+      if (e != cudaSuccess || d.cast_blocks_per_sm < 1) {
+        (void)cudaGetLastError();
+        d.cast_blocks_per_sm = 1;
+      }
     }
   }
   if (d.state != 1) return fail(FP8T_ERR_UNSUPPORTED_DEVICE, "device %d is not sm_100", dev);
@@ -153,8 +170,9 @@ AdamWPlan plan_adamw(const fp8t_adamw_tensor* t, int32_t n) {
   return p;
 }
 
+// One double per norm partial, then one int64 slot for the step a device-counted call performs.
 size_t workspace_for(const AdamWPlan& p) {
-  return static_cast<size_t>((p.nparts * 8 + 255) / 256 * 256);
+  return static_cast<size_t>(((p.nparts + 1) * 8 + 255) / 256 * 256);
 }
 
 }  // namespace
@@ -184,50 +202,98 @@ const char* fp8t_status_string(fp8t_status s) {
 }
 
 // ------------------------------------------------------------------ cast / transpose / amax
+fp8t_status fp8_cast_transpose_amax_multi(const fp8t_cast_tensor* tensors, int32_t n_tensors,
+                                          void* stream) {
+  t_last_error.clear();
+  if (!tensors || n_tensors < 1 || n_tensors > 4096)
+    return fail(FP8T_ERR_INVALID_ARG, "fp8_cast_transpose_amax: tensors NULL or n_tensors out of range");
+  for (int32_t i = 0; i < n_tensors; ++i) {
+    const fp8t_cast_tensor& t = tensors[i];
+    if (!t.x_bf16 || !t.d_scale || !t.d_amax_inout)
+      return fail(FP8T_ERR_INVALID_ARG, "fp8_cast_transpose_amax: tensor %d: NULL input, scale or amax pointer", i);
+    if (t.fmt != FP8T_E4M3 && t.fmt != FP8T_E5M2)
+      return fail(FP8T_ERR_INVALID_ARG, "fp8_cast_transpose_amax: tensor %d: unknown format %d", i, (int)t.fmt);
+    if (t.rows <= 0 || t.cols <= 0)
+      return fail(FP8T_ERR_INVALID_ARG, "fp8_cast_transpose_amax: tensor %d: rows and cols must be > 0", i);
+    if (t.rows % 16 || t.cols % 16 || t.rows > (int64_t(1) << 31) || t.cols > (int64_t(1) << 31) ||
+        t.rows * t.cols >= (int64_t(1) << 40))
+      return fail(FP8T_ERR_UNSUPPORTED_SHAPE,
+                  "fp8_cast_transpose_amax: tensor %d: rows and cols must be multiples of 16, rows*cols < 2^40", i);
+    if (!aligned(t.x_bf16, 16) || !aligned(t.q_rowmajor, 16) || !aligned(t.q_transposed, 16) ||
+        !aligned(t.d_scale, 4) || !aligned(t.d_amax_inout, 4) || !aligned(t.d_scale_inv_out, 4) ||
+        !aligned(t.d_counters, 8))
+      return fail(FP8T_ERR_MISALIGNED, "fp8_cast_transpose_amax: tensor %d: misaligned pointer", i);
+  }
+  DeviceInfo* dev = nullptr;
+  fp8t_status st = current_device(&dev);
+  if (st != FP8T_OK) return st;
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(FP8T_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+
+  using namespace fp8t::cast;
+  static thread_local Group group;
+  for (int32_t b0 = 0; b0 < n_tensors; b0 += kMaxTensors) {
+    const int32_t b1 = std::min<int32_t>(n_tensors, b0 + kMaxTensors);
+    std::memset(&group, 0, sizeof(group));
+    group.n = b1 - b0;
+    int64_t tiles = 0;
+    for (int32_t i = b0; i < b1; ++i) {
+      const fp8t_cast_tensor& t = tensors[i];
+      Tensor& T = group.t[i - b0];
+      {
+        cuuint64_t dims[2] = {static_cast<cuuint64_t>(t.cols), static_cast<cuuint64_t>(t.rows)};
+        cuuint64_t strides[1] = {static_cast<cuuint64_t>(t.cols) * 2};
+        cuuint32_t box[2] = {kTile, kTile};
+        cuuint32_t es[2] = {1, 1};
+        CUresult r = fn(&T.x_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(t.x_bf16),
+                        dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return fail(FP8T_ERR_CUDA, "cuTensorMapEncodeTiled (cast input) failed (%d)", (int)r);
+      }
+      if (t.q_transposed) {
+        cuuint64_t dims[2] = {static_cast<cuuint64_t>(t.rows), static_cast<cuuint64_t>(t.cols)};
+        cuuint64_t strides[1] = {static_cast<cuuint64_t>(t.rows)};
+        cuuint32_t box[2] = {kTile, kTile};
+        cuuint32_t es[2] = {1, 1};
+        CUresult r = fn(&T.qt_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, t.q_transposed, dims, strides,
+                        box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return fail(FP8T_ERR_CUDA, "cuTensorMapEncodeTiled (q^T store) failed (%d)", (int)r);
+      }
+      T.scale = t.d_scale;
+      T.amax_bits = reinterpret_cast<unsigned int*>(t.d_amax_inout);
+      T.scale_inv = t.d_scale_inv_out;
+      T.counters = t.d_counters;
+      T.q = static_cast<uint8_t*>(t.q_rowmajor);
+      T.rows = t.rows;
+      T.cols = t.cols;
+      T.tiles_c = (t.cols + kTile - 1) / kTile;
+      T.tile_start = tiles;
+      T.fmt = t.fmt;
+      T.has_qt = t.q_transposed ? 1 : 0;
+      tiles += ((t.rows + kTile - 1) / kTile) * T.tiles_c;
+    }
+    group.total_tiles = tiles;
+    bool count = false;
+    for (int32_t i = b0; i < b1; ++i) count |= tensors[i].d_counters != nullptr;
+    const int64_t grid = std::min<int64_t>(tiles, static_cast<int64_t>(dev->sms) * dev->cast_blocks_per_sm);
+    if (count)
+      k_cast_transpose_amax<true><<<static_cast<unsigned>(grid), kThreads, kSmemBytes, as_stream(stream)>>>(group);
+    else
+      k_cast_transpose_amax<false><<<static_cast<unsigned>(grid), kThreads, kSmemBytes, as_stream(stream)>>>(group);
+    if ((st = after_launch("fp8_cast_transpose_amax launch")) != FP8T_OK) return st;
+  }
+  return FP8T_OK;
+}
+
 fp8t_status fp8_cast_transpose_amax(const void* x_bf16, int64_t rows, int64_t cols, fp8t_format fmt,
                                     const float* d_scale, void* q_rowmajor, void* q_transposed,
                                     float* d_amax_inout, float* d_scale_inv_out,
                                     unsigned long long* d_counters, void* stream) {
-  t_last_error.clear();
-  if (!x_bf16 || !d_scale || !d_amax_inout)
-    return fail(FP8T_ERR_INVALID_ARG, "fp8_cast_transpose_amax: NULL input, scale or amax pointer");
-  if (fmt != FP8T_E4M3 && fmt != FP8T_E5M2)
-    return fail(FP8T_ERR_INVALID_ARG, "fp8_cast_transpose_amax: unknown format %d", (int)fmt);
-  if (rows <= 0 || cols <= 0)
-    return fail(FP8T_ERR_INVALID_ARG, "fp8_cast_transpose_amax: rows and cols must be > 0");
-  if (rows % 16 || cols % 16 || rows > (int64_t(1) << 31) || cols > (int64_t(1) << 31) ||
-      rows * cols >= (int64_t(1) << 40))
-    return fail(FP8T_ERR_UNSUPPORTED_SHAPE,
-                "fp8_cast_transpose_amax: rows and cols must be multiples of 16, rows*cols < 2^40");
-  if (!aligned(x_bf16, 16) || !aligned(q_rowmajor, 16) || !aligned(q_transposed, 16) ||
-      !aligned(d_scale, 4) || !aligned(d_amax_inout, 4) || !aligned(d_scale_inv_out, 4) ||
-      !aligned(d_counters, 8))
-    return fail(FP8T_ERR_MISALIGNED, "fp8_cast_transpose_amax: misaligned pointer");
-  DeviceInfo* dev = nullptr;
-  fp8t_status st = current_device(&dev);
-  if (st != FP8T_OK) return st;
-
-  cudaStream_t s = as_stream(stream);
-  using namespace fp8t::cast;
-  const int64_t tiles_c = (cols + kTile - 1) / kTile;
-  const int64_t tiles = ((rows + kTile - 1) / kTile) * tiles_c;
-  auto* xq = static_cast<const uint16_t*>(x_bf16);
-  auto* q = static_cast<uint8_t*>(q_rowmajor);
-  auto* qT = static_cast<uint8_t*>(q_transposed);
-  auto* amax = reinterpret_cast<unsigned int*>(d_amax_inout);
-  const dim3 grid(static_cast<unsigned>(tiles));
-  if (fmt == FP8T_E4M3) {
-    if (d_counters)
-      k_cast_transpose_amax<0, true><<<grid, kThreads, 0, s>>>(xq, rows, cols, tiles_c, d_scale, q, qT, amax, d_counters, d_scale_inv_out);
-    else
-      k_cast_transpose_amax<0, false><<<grid, kThreads, 0, s>>>(xq, rows, cols, tiles_c, d_scale, q, qT, amax, nullptr, d_scale_inv_out);
-  } else {
-    if (d_counters)
-      k_cast_transpose_amax<1, true><<<grid, kThreads, 0, s>>>(xq, rows, cols, tiles_c, d_scale, q, qT, amax, d_counters, d_scale_inv_out);
-    else
-      k_cast_transpose_amax<1, false><<<grid, kThreads, 0, s>>>(xq, rows, cols, tiles_c, d_scale, q, qT, amax, nullptr, d_scale_inv_out);
-  }
-  return after_launch("fp8_cast_transpose_amax launch");
+  const fp8t_cast_tensor t = {x_bf16, rows, cols, fmt, d_scale, q_rowmajor, q_transposed,
+                              d_amax_inout, d_scale_inv_out, d_counters};
+  return fp8_cast_transpose_amax_multi(&t, 1, stream);
 }
 
 // ------------------------------------------------------------------ GEMM
@@ -299,9 +365,10 @@ size_t fused_adamw_workspace_bytes(const fp8t_adamw_tensor* tensors, int32_t n_t
 
 fp8t_status fused_adamw_multi_tensor(const fp8t_adamw_tensor* tensors, int32_t n_tensors, float lr,
                                      float beta1, float beta2, float eps, float weight_decay,
-                                     int64_t step, float loss_scale, float max_grad_norm,
-                                     float* d_grad_norm_out, int32_t* d_skipped_out,
-                                     void* d_workspace, size_t workspace_bytes, void* stream) {
+                                     int64_t step, int64_t* d_step_inout, float loss_scale,
+                                     float max_grad_norm, float* d_grad_norm_out,
+                                     int32_t* d_skipped_out, void* d_workspace,
+                                     size_t workspace_bytes, void* stream) {
   t_last_error.clear();
   if (!tensors || n_tensors < 1 || n_tensors > (1 << 20))
     return fail(FP8T_ERR_INVALID_ARG, "fused_adamw_multi_tensor: tensors NULL or n_tensors out of range");
@@ -313,12 +380,14 @@ fp8t_status fused_adamw_multi_tensor(const fp8t_adamw_tensor* tensors, int32_t n
         !aligned(t.grad_bf16, 16) || !aligned(t.weight_bf16, 16))
       return fail(FP8T_ERR_MISALIGNED, "fused_adamw_multi_tensor: tensor %d is not 16-byte aligned", i);
   }
-  if (step < 1) return fail(FP8T_ERR_INVALID_ARG, "fused_adamw_multi_tensor: step must be >= 1");
+  if (!d_step_inout && step < 1)
+    return fail(FP8T_ERR_INVALID_ARG, "fused_adamw_multi_tensor: step must be >= 1");
   if (!(loss_scale > 0.0f) || !std::isfinite(loss_scale) || !std::isfinite(lr) ||
       !std::isfinite(beta1) || !std::isfinite(beta2) || !std::isfinite(eps) ||
       !std::isfinite(weight_decay) || !std::isfinite(max_grad_norm))
     return fail(FP8T_ERR_INVALID_ARG, "fused_adamw_multi_tensor: non-finite hyperparameter or loss_scale <= 0");
-  if (!aligned(d_grad_norm_out, 4) || !aligned(d_skipped_out, 4) || !aligned(d_workspace, 16))
+  if (!aligned(d_grad_norm_out, 4) || !aligned(d_skipped_out, 4) || !aligned(d_workspace, 16) ||
+      !aligned(d_step_inout, 8))
     return fail(FP8T_ERR_MISALIGNED, "fused_adamw_multi_tensor: misaligned output or workspace");
   const AdamWPlan plan = plan_adamw(tensors, n_tensors);
   const size_t need = workspace_for(plan);
@@ -335,9 +404,19 @@ fp8t_status fused_adamw_multi_tensor(const fp8t_adamw_tensor* tensors, int32_t n
   k.omb1 = static_cast<float>(1.0 - static_cast<double>(beta1));
   k.omb2 = static_cast<float>(1.0 - static_cast<double>(beta2));
   k.decay = static_cast<float>(1.0 - static_cast<double>(lr) * static_cast<double>(weight_decay));
-  k.step_size = static_cast<float>(static_cast<double>(lr) /
-                                   (1.0 - std::pow(static_cast<double>(beta1), static_cast<double>(step))));
-  k.bc2_sqrt = static_cast<float>(std::sqrt(1.0 - std::pow(static_cast<double>(beta2), static_cast<double>(step))));
+  k.d_step = d_step_inout;
+  k.step_slot = reinterpret_cast<const int64_t*>(static_cast<double*>(d_workspace) + plan.nparts);
+  k.lr_d = lr;
+  k.beta1_d = beta1;
+  k.beta2_d = beta2;
+  if (!d_step_inout) {
+    k.step_size = static_cast<float>(static_cast<double>(lr) /
+                                     (1.0 - std::pow(static_cast<double>(beta1), static_cast<double>(step))));
+    k.bc2_sqrt = static_cast<float>(std::sqrt(1.0 - std::pow(static_cast<double>(beta2), static_cast<double>(step))));
+  } else {
+    k.step_size = 0.0f;      // formed on the device from the counter
+    k.bc2_sqrt = 0.0f;
+  }
   k.eps = eps;
   k.inv_s_d = 1.0 / static_cast<double>(loss_scale);
   k.inv_s = static_cast<float>(k.inv_s_d);
@@ -368,7 +447,9 @@ fp8t_status fused_adamw_multi_tensor(const fp8t_adamw_tensor* tensors, int32_t n
       batch.chunk_start[batch.n] = acc;
       if (pass == 0) {
         const int64_t grid = std::min<int64_t>(acc, kSumsqBlocks);
-        k_adamw_sumsq<<<static_cast<unsigned>(grid), kThreads, 0, s>>>(batch, partials + off);
+        k_adamw_sumsq<<<static_cast<unsigned>(grid), kThreads, 0, s>>>(
+            batch, partials + off, bi == 0 ? d_step_inout : nullptr,
+            reinterpret_cast<int64_t*>(partials + plan.nparts));
         off += grid;
         if ((st = after_launch("adamw norm pass launch")) != FP8T_OK) return st;
       } else {
@@ -385,15 +466,16 @@ fp8t_status fused_adamw_multi_tensor(const fp8t_adamw_tensor* tensors, int32_t n
 // Same step as fused_adamw_multi_tensor, with the built-in scratch array as its workspace.
 fp8t_status fused_adamw_multi_tensor_noalloc(const fp8t_adamw_tensor* tensors, int32_t n_tensors,
                                              float lr, float beta1, float beta2, float eps,
-                                             float weight_decay, int64_t step, float loss_scale,
+                                             float weight_decay, int64_t step,
+                                             int64_t* d_step_inout, float loss_scale,
                                              float max_grad_norm, float* d_grad_norm_out,
                                              int32_t* d_skipped_out, void* stream) {
   t_last_error.clear();
   const size_t need = fused_adamw_workspace_bytes(tensors, n_tensors);
   if (need == 0)   // invalid tensor table: the regular entry point reports it, launching nothing
     return fused_adamw_multi_tensor(tensors, n_tensors, lr, beta1, beta2, eps, weight_decay, step,
-                                    loss_scale, max_grad_norm, d_grad_norm_out, d_skipped_out,
-                                    nullptr, 0, stream);
+                                    d_step_inout, loss_scale, max_grad_norm, d_grad_norm_out,
+                                    d_skipped_out, nullptr, 0, stream);
   if (need > FP8T_NOALLOC_SCRATCH_BYTES)
     return fail(FP8T_ERR_UNSUPPORTED_SHAPE,
                 "fused_adamw_multi_tensor_noalloc: needs %zu bytes of scratch, the built-in array "
@@ -415,8 +497,8 @@ fp8t_status fused_adamw_multi_tensor_noalloc(const fp8t_adamw_tensor* tensors, i
     scratch = dev->noalloc_scratch;
   }
   return fused_adamw_multi_tensor(tensors, n_tensors, lr, beta1, beta2, eps, weight_decay, step,
-                                  loss_scale, max_grad_norm, d_grad_norm_out, d_skipped_out,
-                                  scratch, FP8T_NOALLOC_SCRATCH_BYTES, stream);
+                                  d_step_inout, loss_scale, max_grad_norm, d_grad_norm_out,
+                                  d_skipped_out, scratch, FP8T_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 // ------------------------------------------------------------------ device error word

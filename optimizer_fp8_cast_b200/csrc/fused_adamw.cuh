@@ -43,6 +43,12 @@ struct Batch {
 struct Scalars {            // host-computed, rounded once to f32 (double where noted)
   float beta1, beta2, omb1, omb2, decay, step_size, bc2_sqrt, eps, inv_s, max_norm;
   double inv_s_d;
+  // device step counter (may be null): the step is read from step_slot (counter + 1, written by
+  // the norm pass), step_size and bc2_sqrt are formed on the device, and the counter is advanced
+  // by the first CTA of the first update launch unless the step is skipped
+  int64_t* d_step;
+  const int64_t* step_slot;
+  double lr_d, beta1_d, beta2_d;
 };
 
 __device__ __forceinline__ int find_tensor(const Batch& b, int64_t chunk) {
@@ -77,8 +83,11 @@ __device__ __forceinline__ T block_sum_fixed(T v, T* sh) {  // deterministic tre
 }
 
 __global__ void __launch_bounds__(kThreads)
-    k_adamw_sumsq(const __grid_constant__ Batch b, double* __restrict__ partials) {
+    k_adamw_sumsq(const __grid_constant__ Batch b, double* __restrict__ partials,
+                  const int64_t* __restrict__ step_counter, int64_t* __restrict__ step_slot) {
   __shared__ double sh[kThreads];
+  // the step this call performs, for the update kernels that run after this one
+  if (step_counter && blockIdx.x == 0 && threadIdx.x == 0) *step_slot = *step_counter + 1;
   double acc = 0.0;
   const int64_t nchunks = b.chunk_start[b.n];
   for (int64_t c = blockIdx.x; c < nchunks; c += gridDim.x) {
@@ -133,7 +142,7 @@ __global__ void __launch_bounds__(kThreads)
                    const double* __restrict__ partials, int nparts, float* __restrict__ norm_out,
                    int32_t* __restrict__ skipped_out) {
   __shared__ double sh[kThreads];
-  __shared__ float s_f;
+  __shared__ float s_f, s_step_size, s_bc2_sqrt;
   __shared__ int s_skip;
   {
     double acc = 0.0;
@@ -146,6 +155,16 @@ __global__ void __launch_bounds__(kThreads)
           (k.max_norm > 0.0f && norm > k.max_norm) ? __fdiv_rn(k.max_norm, norm) : 1.0f;
       s_f = __fmul_rn(coef, k.inv_s);
       s_skip = skip;
+      if (k.d_step) {
+        const int64_t step = *k.step_slot;
+        const double t = static_cast<double>(step);
+        s_step_size = static_cast<float>(__ddiv_rn(k.lr_d, 1.0 - pow(k.beta1_d, t)));
+        s_bc2_sqrt = static_cast<float>(__dsqrt_rn(1.0 - pow(k.beta2_d, t)));
+        if (b.first && blockIdx.x == 0 && !skip) *k.d_step = step;   // no CTA reads the counter
+      } else {
+        s_step_size = k.step_size;
+        s_bc2_sqrt = k.bc2_sqrt;
+      }
       if (b.first && blockIdx.x == 0) {
         if (norm_out) *norm_out = norm;
         if (skipped_out) *skipped_out = skip;
@@ -155,6 +174,9 @@ __global__ void __launch_bounds__(kThreads)
   }
   if (s_skip) return;
   const float f = s_f;
+  Scalars kk = k;
+  kk.step_size = s_step_size;
+  kk.bc2_sqrt = s_bc2_sqrt;
   const int64_t nchunks = b.chunk_start[b.n];
   for (int64_t c = blockIdx.x; c < nchunks; c += gridDim.x) {
     const int t = find_tensor(b, c);
@@ -195,8 +217,8 @@ __global__ void __launch_bounds__(kThreads)
           uint32_t wout[4];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            adam_one(pp[2 * j], mm[2 * j], vq[2 * j], bf16_to_f32(gw[j] & 0xFFFFu), k, f);
-            adam_one(pp[2 * j + 1], mm[2 * j + 1], vq[2 * j + 1], bf16_to_f32(gw[j] >> 16), k, f);
+            adam_one(pp[2 * j], mm[2 * j], vq[2 * j], bf16_to_f32(gw[j] & 0xFFFFu), kk, f);
+            adam_one(pp[2 * j + 1], mm[2 * j + 1], vq[2 * j + 1], bf16_to_f32(gw[j] >> 16), kk, f);
             wout[j] = f32_to_bf16_rne(pp[2 * j]) | (f32_to_bf16_rne(pp[2 * j + 1]) << 16);
           }
           __stcs(reinterpret_cast<float4*>(M + e), mv[u][0]);
@@ -209,7 +231,7 @@ __global__ void __launch_bounds__(kThreads)
         } else {
           for (int64_t i = e; i < n && i < e + kVec; ++i) {
             float p = P[i], mq = M[i], vq1 = V[i];
-            adam_one(p, mq, vq1, bf16_to_f32(G[i]), k, f);
+            adam_one(p, mq, vq1, bf16_to_f32(G[i]), kk, f);
             P[i] = p;
             M[i] = mq;
             V[i] = vq1;

@@ -10,7 +10,7 @@
 // D[M x N] = bf16((A[M x K] . B[N x K]^T) * sa * sb), A and B K-major ("TN").
 // A cluster of two CTAs (one per SM) computes a 256 x 256 tile: CTA r loads A rows
 // [128r, 128r+128) and B rows (N columns) [128r, 128r+128) of the tile, 128-byte swizzled
-// 128 x 128-byte boxes, into its own 6-stage ring (32 KB per stage). Both CTAs' loads count on
+// 128 x 128-byte boxes, into its own 7-stage ring (32 KB per stage, 224 KB). Both CTAs' loads count on
 // the even CTA's "full" barrier; the even CTA's MMA thread issues tcgen05.mma.cta_group::2
 // (M=256, N=256, K=32), which reads A and B halves from both CTAs' shared memory, and releases
 // each stage in both CTAs with one multicast tcgen05.commit. Per SM that is 32 KB of operands per
@@ -33,7 +33,7 @@
 namespace fp8t {
 namespace gemm {
 
-constexpr int kBM = 256, kBN = 256, kBK = 128, kStages = 6, kUmmaK = 32;
+constexpr int kBM = 256, kBN = 256, kBK = 128, kStages = 7, kUmmaK = 32;
 constexpr int kHalf = 128;                               // rows of A and of B per CTA
 constexpr int kThreads = 192;
 constexpr int kABytes = kHalf * kBK, kBBytes = kHalf * kBK, kStageBytes = kABytes + kBBytes;

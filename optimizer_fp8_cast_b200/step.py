@@ -14,7 +14,8 @@ All scalars stay on the device; nothing in a step synchronises with the host.
 import torch
 
 from . import (AMAX_MAX, AMAX_MOST_RECENT, E4M3, E5M2, FP8_MAX, fp8_cast_transpose_amax,
-               fp8_gemm, fp8_scale_update, fused_adamw_multi_tensor, fused_adamw_workspace_bytes)
+               fp8_cast_transpose_amax_multi, fp8_gemm, fp8_scale_update,
+               fused_adamw_multi_tensor, fused_adamw_workspace_bytes)
 
 ROLE_X, ROLE_W, ROLE_DY = 0, 1, 2
 ROLE_FMT = (E4M3, E4M3, E5M2)
@@ -46,7 +47,7 @@ class Fp8LinearStep:
     Scale state is indexed 3*layer + role (role 0 = X, 1 = W, 2 = dY)."""
 
     def __init__(self, layer_shapes, tokens, history_len, algo="max", margin=0, adamw=None,
-                 w_init=None, device="cuda", counters=False):
+                 w_init=None, device="cuda", counters=False, device_step=False):
         self.device = torch.device(device)
         self.tokens = tokens
         self.algo = AMAX_MAX if algo == "max" else AMAX_MOST_RECENT
@@ -67,6 +68,9 @@ class Fp8LinearStep:
         ws = fused_adamw_workspace_bytes([l.master.numel() for l in self.layers])
         self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=self.device)
         self.t = 0
+        # device_step: AdamW counts steps in device memory, so a captured graph can be replayed
+        self.step_counter = (torch.zeros(1, dtype=torch.int64, device=self.device)
+                             if device_step else None)
 
     def _slot(self, t, i):
         return t[i:i + 1]
@@ -77,6 +81,21 @@ class Fp8LinearStep:
                                 self._slot(self.amax, i), self._slot(self.scale_inv, i),
                                 self.counters[i] if self.counters is not None else None,
                                 stream=stream)
+
+    def cast_desc(self, k, role, src, q, qT):
+        i = 3 * k + role
+        return dict(x=src, fmt=ROLE_FMT[role], scale=self._slot(self.scale, i), q=q, qT=qT,
+                    amax=self._slot(self.amax, i), scale_inv=self._slot(self.scale_inv, i),
+                    counters=self.counters[i] if self.counters is not None else None)
+
+    def cast_all(self, xs, dys, stream=None):
+        """Every layer's X, W and dY casts, grouped into launches of up to 8 tensors."""
+        descs = []
+        for k, L in enumerate(self.layers):
+            descs += [self.cast_desc(k, ROLE_X, xs[k], L.Xq, L.XqT),
+                      self.cast_desc(k, ROLE_W, L.W, L.Wq, L.WqT),
+                      self.cast_desc(k, ROLE_DY, dys[k], L.dYq, L.dYqT)]
+        fp8_cast_transpose_amax_multi(descs, stream=stream)
 
     def gemm(self, k, which, stream=None):
         """which: 0 = fprop Y = X.W, 1 = dgrad dX = dY.W^T, 2 = wgrad dW = X^T.dY."""
@@ -113,16 +132,20 @@ class Fp8LinearStep:
                                  beta2=hp["beta2"], eps=hp["eps"], weight_decay=hp["weight_decay"],
                                  step=self.t, loss_scale=hp["loss_scale"],
                                  max_grad_norm=hp["max_grad_norm"], grad_norm=self.grad_norm,
-                                 skipped=self.skipped, workspace=self.workspace, stream=stream)
+                                 skipped=self.skipped, workspace=self.workspace,
+                                 step_counter=self.step_counter, stream=stream)
 
     def step(self, xs, dys, stream=None):
         """One training step; xs[k] = X [tokens, in_k], dys[k] = dY [tokens, out_k] (BF16, device)."""
         self.t += 1
+        self.cast_all(xs, dys, stream)
         for k in range(len(self.layers)):
-            self.layer_forward_backward(k, xs[k], dys[k], stream)
+            for which in (0, 1, 2):
+                self.gemm(k, which, stream)
         self.update(stream)
 
     # launches of the library's kernels per step (for the benchmark's launch count)
     def kernels_per_step(self):
         n_adamw_batches = (len(self.layers) + 255) // 256
-        return 6 * len(self.layers) + 1 + 2 * n_adamw_batches
+        n_cast_launches = (3 * len(self.layers) + 7) // 8
+        return n_cast_launches + 3 * len(self.layers) + 1 + 2 * n_adamw_batches

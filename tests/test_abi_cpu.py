@@ -53,6 +53,15 @@ def test_invalid_arguments_rejected_on_host(lib):
     assert lib.fp8_cast_transpose_amax(P, 24, 16, 0, P, P, P, P, P, P, z) == 2
     assert lib.fp8_cast_transpose_amax(U, 16, 16, 0, P, P, P, P, P, P, z) == 3
     assert b"misaligned" in lib.fp8t_last_error_message()
+    # grouped cast: validated per tensor before anything runs
+    arr = (_abi.CastTensor * 2)()
+    arr[0] = _abi.CastTensor(P, 16, 16, 0, P, P, P, P, P, None)
+    arr[1] = _abi.CastTensor(P, 16, 24, 1, P, P, P, P, P, None)
+    assert lib.fp8_cast_transpose_amax_multi(arr, 2, z) == 2
+    assert b"tensor 1" in lib.fp8t_last_error_message()
+    assert lib.fp8_cast_transpose_amax_multi(arr, 0, z) == 1
+    arr[1] = _abi.CastTensor(P, 16, 16, 1, P, U, P, P, P, None)
+    assert lib.fp8_cast_transpose_amax_multi(arr, 2, z) == 3
     # gemm
     assert lib.fp8_gemm(z, 0, P, 0, 16, 16, 16, P, P, P, z) == 1
     assert lib.fp8_gemm(P, 0, P, 9, 16, 16, 16, P, P, P, z) == 1
@@ -70,9 +79,10 @@ def test_invalid_arguments_rejected_on_host(lib):
     arr[0] = _abi.AdamWTensor(P, P, P, P, P, 1000)
     need = lib.fused_adamw_workspace_bytes(arr, 1)
     assert need >= 8 and need % 256 == 0
-    call = lambda a, n=1, step=1, S=1.0, ws=P, wsb=need: lib.fused_adamw_multi_tensor(
-        a, n, 1e-3, 0.9, 0.999, 1e-8, 0.0, step, S, 1.0, z, z, ws, wsb, z)
+    call = lambda a, n=1, step=1, S=1.0, ws=P, wsb=need, dstep=z: lib.fused_adamw_multi_tensor(
+        a, n, 1e-3, 0.9, 0.999, 1e-8, 0.0, step, dstep, S, 1.0, z, z, ws, wsb, z)
     assert call(arr, step=0) == 1
+    assert call(arr, step=0, dstep=C.c_void_p(16 * 1024 + 4)) == 3   # misaligned step counter
     assert call(arr, S=0.0) == 1
     assert call(arr, S=float("inf")) == 1
     assert call(arr, ws=None) == 1

@@ -91,6 +91,31 @@ def test_nonfinite_gradient_skips_update(cuda_lib, bad):
     assert all(int(w.abs().sum().item()) == 0 for w in W)
 
 
+def test_device_step_counter(cuda_lib):
+    """With a device step counter the call performs counter+1, stores it back, and leaves it
+    unchanged on a skipped step; results match the oracle at that step within 4 ulp."""
+    P, M, V, G, W = make([5000, 70000], seed=6)
+    counter = torch.tensor([41], dtype=torch.int64, device="cuda")
+    host = [[f32(t) for t in P], [f32(t) for t in M], [f32(t) for t in V]]
+    for k in range(3):
+        norm = torch.zeros(1, device="cuda")
+        cuda_lib.fused_adamw_multi_tensor(P, M, V, G, W, grad_norm=norm, step_counter=counter,
+                                          step=0, **HP)
+        cuda_lib.fp8t_check_device_error()
+        assert counter.item() == 42 + k
+        gbits = [bf16_bits(g) for g in G]
+        oracle.fused_adamw(host[0], host[1], host[2], gbits, [np.zeros(g.size, np.uint16) for g in gbits],
+                           dict(HP, step=42 + k))
+        for i in range(2):
+            for got, ref in ((P[i], host[0][i]), (M[i], host[1][i]), (V[i], host[2][i])):
+                assert ulp_distance_f32(f32(got), ref).max() <= 4
+    G[0][3] = float("nan")
+    skipped = torch.zeros(1, dtype=torch.int32, device="cuda")
+    cuda_lib.fused_adamw_multi_tensor(P, M, V, G, W, skipped=skipped, step_counter=counter, step=0, **HP)
+    cuda_lib.fp8t_check_device_error()
+    assert skipped.item() == 1 and counter.item() == 44
+
+
 def test_adamw4e9_full_size_sampled(cuda_lib):
     """The 4.0e9-parameter, 512-tensor workload at full size in the benchmark's launch
     configuration. The oracle computes the global norm over every gradient (host copies) and

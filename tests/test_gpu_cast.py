@@ -126,3 +126,34 @@ def test_full_size_workload_shapes(cuda_lib, name, rows, cols, fmt):
     del x
     scale = 448.0 / 4.5 if fmt == oracle.E4M3 else 57344.0 / 1.1
     check(cuda_lib, bf16_bits(xb), fmt, scale)
+
+
+def test_multi_tensor_launch(cuda_lib):
+    """Several casts in one launch (mixed shapes, formats and optional outputs) equal the
+    per-tensor oracle, including more tensors than one launch table holds."""
+    rng = np.random.default_rng(21)
+    specs = [((272, 144), oracle.E4M3, 3.0, True, True), ((16, 4096), oracle.E5M2, 1000.0, True, True),
+             ((1040, 48), oracle.E4M3, 0.5, False, True), ((128, 128), oracle.E5M2, 7.0, True, False)]
+    specs = specs * 3                                   # 12 tensors: two launch tables
+    casts, refs = [], []
+    for (shape, fmt, scale, want_q, want_qT) in specs:
+        x = torch.from_numpy((rng.standard_normal(shape) * 3).astype(np.float32)).to(torch.bfloat16)
+        bits = bf16_bits(x)
+        rows, cols = shape
+        c = dict(x=bf16_from_bits(bits), fmt=fmt, scale=dev_scalar(scale),
+                 q=torch.empty(rows, cols, dtype=torch.uint8, device="cuda") if want_q else None,
+                 qT=torch.empty(cols, rows, dtype=torch.uint8, device="cuda") if want_qT else None,
+                 amax=torch.zeros(1, device="cuda"), scale_inv=torch.zeros(1, device="cuda"),
+                 counters=torch.zeros(3, dtype=torch.int64, device="cuda"))
+        casts.append(c)
+        refs.append(oracle.cast_transpose_amax(bits, fmt, scale))
+    cuda_lib.fp8_cast_transpose_amax_multi(casts)
+    cuda_lib.fp8t_check_device_error()
+    for c, (rq, rqT, ramax, rsinv, rcnt) in zip(casts, refs):
+        if c["q"] is not None:
+            assert np.array_equal(u8(c["q"]), rq)
+        if c["qT"] is not None:
+            assert np.array_equal(u8(c["qT"]), rqT)
+        assert np.float32(c["amax"].item()).view(np.uint32) == np.float32(ramax).view(np.uint32)
+        assert np.float32(c["scale_inv"].item()) == rsinv
+        assert np.array_equal(c["counters"].cpu().numpy().astype(np.uint64), rcnt)

@@ -69,6 +69,6 @@ def test_noalloc_rejects_calls_beyond_its_array(cuda_lib):
     for i in range(n):
         arr[i] = _abi.AdamWTensor(P, P, P, P, P, 592 * 8192)
     assert lib.fused_adamw_workspace_bytes(arr, n) > 65536
-    st = lib.fused_adamw_multi_tensor_noalloc(arr, n, 1e-3, 0.9, 0.999, 1e-8, 0.0, 1, 1.0, 1.0,
-                                              None, None, None)
+    st = lib.fused_adamw_multi_tensor_noalloc(arr, n, 1e-3, 0.9, 0.999, 1e-8, 0.0, 1, None, 1.0,
+                                              1.0, None, None, None)
     assert st == 2 and b"built-in array" in lib.fp8t_last_error_message()
