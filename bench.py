@@ -249,31 +249,30 @@ def run_ours(args, rank, world, local_rank):
     for g, _ in graphs:
         del g
     graphs.clear()
-    # end to end: host (pinned) inputs copied in and results copied out inside the timed region
+    # End to end: X and dY start in pinned host memory and Y, dX end there; every step's copies
+    # are inside the timed region. The host-streamed runner overlaps step t's kernels with the
+    # copy-in of step t+1 and the copy-out of step t-1 (separate streams and copy engines).
+    from optimizer_fp8_cast_b200.host_stream import HostStreamedStep
+    runner = HostStreamedStep(st)
     hX = [b[0].cpu().pin_memory() for b in batches]
     hdY = [b[1].cpu().pin_memory() for b in batches]
-    hY = torch.empty(L.Y.shape, dtype=torch.bfloat16).pin_memory()
-    hdX = torch.empty(L.dX.shape, dtype=torch.bfloat16).pin_memory()
-    X_dev = torch.empty_like(batches[0][0])
-    dY_dev = torch.empty_like(batches[0][1])
-    e2e_ms = []
-    for t in range(min(args.steps, 50) + 1):
-        flush.zero_()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record()
-        X_dev.copy_(hX[t % 2], non_blocking=True)
-        dY_dev.copy_(hdY[t % 2], non_blocking=True)
-        st.step([X_dev], [dY_dev])
-        hY.copy_(L.Y, non_blocking=True)
-        hdX.copy_(L.dX, non_blocking=True)
-        e1.record()
-        torch.cuda.synchronize()
-        if t > 0:                       # the first one warms the pinned paths
-            e2e_ms.append(e0.elapsed_time(e1))
+    hY = [torch.empty(L.Y.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    hdX = [torch.empty(L.dX.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    for t in range(2):                                   # warm the pinned paths
+        runner.step([hX[t]], [hdY[t]], [hY[t]], [hdX[t]])
+    runner.finish()
+    n_e2e = min(args.steps, 50)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(runner.s_in)
+    for t in range(n_e2e):
+        runner.step([hX[t % 2]], [hdY[t % 2]], [hY[t % 2]], [hdX[t % 2]])
+    e1.record(runner.s_out)
+    runner.finish()
     fp8.fp8t_check_device_error()
-    e2e_total = reduce_max(sum(e2e_ms), world, dev)
-    e2e_value = throughput(flop_step, len(e2e_ms), world, e2e_total)
+    e2e_total = reduce_max(e0.elapsed_time(e1), world, dev)
+    e2e_value = throughput(flop_step, n_e2e, world, e2e_total)
+    e2e_ms = [e2e_total / n_e2e] * n_e2e
 
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
@@ -288,7 +287,9 @@ def run_ours(args, rank, world, local_rank):
                    "launch": "eager" if args.eager else "CUDA graph per step (AdamW step counter on the device)",
                    "l2": "flushed before every timed step (256 MiB write)"},
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": nums["h2d"],
-                "d2h_bytes_per_step": nums["d2h"], "ms_per_step": round(e2e_total / len(e2e_ms), 4)},
+                "d2h_bytes_per_step": nums["d2h"], "ms_per_step": round(e2e_total / len(e2e_ms), 4),
+                "how": "pinned host X, dY in and Y, dX out every step; copies overlapped with "
+                       "the previous/next step's kernels on separate streams"},
         "gpu_launches": args.steps * st.kernels_per_step(),
         "roofline": {"kernel": "k_fp8_gemm (fprop, dgrad, wgrad)", "bound": "tensor",
                      "achieved": round(gemm_achieved, 1), "peak": round(fp8_peak, 1),

@@ -263,6 +263,13 @@ fp8t_status fp8t_check_device_error(void* stream);
  * of 2 s). Meant for tests of the timeout path; takes effect for launches after the call. */
 fp8t_status fp8t_set_wait_timeout_ns(uint64_t ns);
 
+/* Test hook for failure detection: mode 1 makes every bounded wait inside the cast and GEMM
+ * kernels behave as if its barrier were never signalled, so each runs out its time limit and
+ * the kernel takes its abort path (FP8T_ERR_TIMEOUT); mode 2 does this for the GEMM epilogue's
+ * waits only, so loads and MMAs are in flight when the kernel drains them; 0 turns it off.
+ * The drains of work already issued are never affected. Takes effect for later launches. */
+fp8t_status fp8t_debug_expire_waits(int32_t mode);
+
 /* Human-readable name of a status code; never NULL. */
 const char* fp8t_status_string(fp8t_status status);
 

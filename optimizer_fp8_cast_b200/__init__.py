@@ -15,7 +15,7 @@ from . import _abi
 
 __all__ = ["fp8_cast_transpose_amax", "fp8_cast_transpose_amax_multi", "fp8_gemm", "fp8_scale_update", "fused_adamw_multi_tensor",
            "fused_adamw_workspace_bytes", "fused_adamw_multi_tensor_noalloc",
-           "fp8t_check_device_error", "fp8t_set_wait_timeout_ns",
+           "fp8t_check_device_error", "fp8t_debug_expire_waits", "fp8t_set_wait_timeout_ns",
            "Fp8TrainError", "E4M3", "E5M2", "AMAX_MAX", "AMAX_MOST_RECENT", "FP8_MAX", "load",
            "LIB_PATH"]
 
@@ -174,6 +174,11 @@ def fused_adamw_multi_tensor_noalloc(master, m, v, grads, weights, *, lr, beta1,
 def fp8t_check_device_error(stream=None):
     """Synchronise the stream and raise if a bounded wait in a kernel expired."""
     _check(load().fp8t_check_device_error(_stream(stream)), "fp8t_check_device_error")
+
+
+def fp8t_debug_expire_waits(mode):
+    """Test hook: 1 = every bounded kernel wait expires, 2 = only the GEMM epilogue's, 0 = off."""
+    _check(load().fp8t_debug_expire_waits(int(mode)), "fp8t_debug_expire_waits")
 
 
 def fp8t_set_wait_timeout_ns(ns):

@@ -44,6 +44,8 @@ def declare(L):
     L.fused_adamw_workspace_bytes.argtypes = [C.POINTER(AdamWTensor), i32]
     L.fp8t_check_device_error.restype = C.c_int
     L.fp8t_check_device_error.argtypes = [vp]
+    L.fp8t_debug_expire_waits.restype = C.c_int
+    L.fp8t_debug_expire_waits.argtypes = [i32]
     L.fp8t_set_wait_timeout_ns.restype = C.c_int
     L.fp8t_set_wait_timeout_ns.argtypes = [C.c_uint64]
     L.fp8t_status_string.restype = C.c_char_p

@@ -152,13 +152,14 @@ __global__ void __launch_bounds__(kThreads, 2) k_cast_transpose_amax(const __gri
   }
   __syncthreads();
   const uint64_t limit = wait_limit_ns();
+  const bool expire = expire_mode() != kExpireNone;
 
   for (int64_t i = 0;; ++i) {
     const int64_t tile = blockIdx.x + i * stride;
     if (tile >= g.total_tiles) break;
     const int buf = static_cast<int>(i & 1);
     if (tid == 0) {
-      if (!mbar_wait(smem_u32(&full[buf]), static_cast<uint32_t>((i >> 1) & 1), limit)) {
+      if (!mbar_wait(smem_u32(&full[buf]), static_cast<uint32_t>((i >> 1) & 1), limit, expire)) {
         record_error(kErrTimeout);
         s_abort = 1;
       } else {

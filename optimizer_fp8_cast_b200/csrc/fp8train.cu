@@ -518,6 +518,14 @@ fp8t_status fp8t_check_device_error(void* stream) {
   return FP8T_OK;
 }
 
+fp8t_status fp8t_debug_expire_waits(int32_t mode) {
+  t_last_error.clear();
+  if (mode < 0 || mode > 2) return fail(FP8T_ERR_INVALID_ARG, "fp8t_debug_expire_waits: mode in 0..2");
+  cudaError_t e = cudaMemcpyToSymbol(fp8t::g_expire_waits, &mode, sizeof(mode));
+  if (e != cudaSuccess) return fail(FP8T_ERR_CUDA, "setting the test hook: %s", cudaGetErrorString(e));
+  return FP8T_OK;
+}
+
 fp8t_status fp8t_set_wait_timeout_ns(uint64_t ns) {
   t_last_error.clear();
   const unsigned long long v = ns;

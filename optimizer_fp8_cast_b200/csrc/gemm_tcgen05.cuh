@@ -41,6 +41,7 @@ constexpr uint32_t kPairTxBytes = 2 * kStageBytes;       // both CTAs' boxes of 
 constexpr int kAccCols = 256, kTmemCols = 2 * kAccCols;
 constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*alignment slack*/ + 256 /*barriers*/;
 constexpr uint64_t kSettleNs = 200000;                   // let loads in flight land on abort
+constexpr uint64_t kPairDrainNs = 1000000;               // producer drain budget (1 ms)
 
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, 8-row groups 1024 B apart.
 __device__ __forceinline__ uint64_t make_sw128_desc(uint32_t saddr) {
@@ -119,6 +120,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = S->tmem_base;
   const uint64_t limit = wait_limit_ns();
+  const int expire = expire_mode();
+  const bool expire_main = expire == kExpireAll;
+  const bool expire_epi = expire == kExpireAll || expire == kExpireGemmEpilogue;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -130,7 +134,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < num_kb; ++kb, ++it) {
           const uint32_t s = it % kStages, ph = (it / kStages) & 1;
           if (*abort_flag) break;
-          if (!mbar_wait(smem_u32(&S->empty[s]), ph ^ 1, limit)) {
+          if (!mbar_wait(smem_u32(&S->empty[s]), ph ^ 1, limit, expire_main)) {
             *abort_flag = 1;
             record_error(kErrTimeout);
             break;
@@ -142,10 +146,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           ++issued;
         }
       }
-      // the even CTA can see its own stages land: wait for the last ones it armed
-      if (leader)
-        for (uint32_t i = issued > kStages ? issued - kStages : 0; i < issued; ++i)
-          mbar_wait(smem_u32(&S->full[i % kStages]), (i / kStages) & 1, kDrainLimitNs);
+      // the even CTA can see its own stages land: wait for the last ones it armed (one shared
+      // budget; after an abort a stage may miss the peer's bytes, and the settle delay below
+      // covers loads still in flight)
+      if (leader) {
+        const uint64_t t0 = globaltimer_ns();
+        for (uint32_t i = issued > kStages ? issued - kStages : 0; i < issued; ++i) {
+          const uint64_t spent = globaltimer_ns() - t0;
+          if (spent >= kPairDrainNs) break;
+          mbar_wait(smem_u32(&S->full[i % kStages]), (i / kStages) & 1, kPairDrainNs - spent);
+        }
+      }
     }
   } else if (warp == 1) {
     if (lane == 0 && leader) {
@@ -153,7 +164,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       uint32_t it = 0, local = 0;
       for (int tile = cluster; tile < n_tiles && !*abort_flag; tile += n_clusters, ++local) {
         const uint32_t acc = local & 1, aph = (local >> 1) & 1;
-        if (!mbar_wait(smem_u32(&S->acc_empty[acc]), aph ^ 1, limit)) {
+        if (!mbar_wait(smem_u32(&S->acc_empty[acc]), aph ^ 1, limit, expire_main)) {
           *abort_flag = 1;
           record_error(kErrTimeout);
           break;
@@ -163,7 +174,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int kb = 0; kb < num_kb; ++kb, ++it) {
           const uint32_t s = it % kStages, ph = (it / kStages) & 1;
-          if (*abort_flag || !mbar_wait(smem_u32(&S->full[s]), ph, limit)) {
+          if (*abort_flag || !mbar_wait(smem_u32(&S->full[s]), ph, limit, expire_main)) {
             if (!*abort_flag) record_error(kErrTimeout);
             *abort_flag = 1;
             ok = false;
@@ -193,7 +204,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int tile = cluster; tile < n_tiles; tile += n_clusters, ++local) {
       const uint32_t acc = local & 1, aph = (local >> 1) & 1;
       if (*abort_flag) break;
-      if (!mbar_wait(smem_u32(&S->acc_full[acc]), aph, limit)) {
+      if (!mbar_wait(smem_u32(&S->acc_full[acc]), aph, limit, expire_epi)) {
         *abort_flag = 1;
         record_error(kErrTimeout);
         break;

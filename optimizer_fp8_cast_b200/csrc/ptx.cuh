@@ -15,6 +15,9 @@ enum : unsigned { kErrTimeout = 1u };
 __device__ unsigned int g_error_word = 0;
 // Time limit of a bounded wait in nanoseconds (0 = default of 2 s). Set by the host.
 __device__ unsigned long long g_wait_timeout_ns = 0;
+// Test hook (fp8t_debug_expire_waits): bounded waits behave as if never signalled.
+enum : int { kExpireNone = 0, kExpireAll = 1, kExpireGemmEpilogue = 2 };
+__device__ int g_expire_waits = 0;
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
@@ -27,6 +30,10 @@ __device__ __forceinline__ uint64_t wait_limit_ns() {
 }
 // Limit for draining work already in flight after an abort: never shortened by the host.
 constexpr uint64_t kDrainLimitNs = 4000000000ull;
+
+__device__ __forceinline__ int expire_mode() {
+  return *reinterpret_cast<volatile int*>(&g_expire_waits);
+}
 
 __device__ __forceinline__ void record_error(unsigned e) { atomicOr(&g_error_word, e); }
 
@@ -41,6 +48,8 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
 __device__ __forceinline__ void fence_mbar_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
+// One probe: the thread may be suspended for a hardware-defined time waiting for the phase
+// (an explicit suspend-time hint slowed the GEMM's producer/MMA wake-ups measurably).
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -53,13 +62,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 // Wait until the phase with the given parity has completed; false if limit_ns elapsed first.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+// `expired` (the test hook) makes the wait behave as if the phase never completed.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns,
+                                          bool expired = false) {
+  if (!expired && mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
+    if (!expired) {
 #pragma unroll 1
-    for (int i = 0; i < 16; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+      for (int i = 0; i < 16; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    }
     if (globaltimer_ns() - t0 > limit_ns) return false;
   }
 }

@@ -94,3 +94,4 @@ def test_invalid_arguments_rejected_on_host(lib):
     assert call(bad) == 1
     assert lib.fused_adamw_workspace_bytes(bad, 1) == 0
     assert b"numel" in lib.fp8t_last_error_message()
+    assert lib.fp8t_debug_expire_waits(3) == 1 and lib.fp8t_debug_expire_waits(-1) == 1

@@ -173,3 +173,31 @@ def test_block7b_one_step(cuda_lib):
     st.step(xs, dys)
     cuda_lib.fp8t_check_device_error()
     check_step(st, pre, xs, dys, gemm_full=False, gemm_samples=1024)
+
+
+def test_host_streamed_steps_match_eager(cuda_lib):
+    """Three steps fed from pinned host memory through the overlapped runner give bit for bit
+    the Y, dX and weights of three eager steps on device-resident copies of the same inputs."""
+    from optimizer_fp8_cast_b200.host_stream import HostStreamedStep
+    wl = synth.LINEAR256
+    inputs = [synth.linear_inputs(wl, 0, t, "cpu") for t in range(3)]
+    eager = make_step(wl, counters=False)
+    ref = []
+    for X, dY in inputs:
+        eager.step([X.cuda()], [dY.cuda()])
+        ref.append((eager.layers[0].Y.cpu(), eager.layers[0].dX.cpu()))
+    streamed = make_step(wl, counters=False)
+    runner = HostStreamedStep(streamed)
+    outs = []
+    for X, dY in inputs:
+        hy = torch.empty(wl.tokens, 256, dtype=torch.bfloat16).pin_memory()
+        hdx = torch.empty(wl.tokens, 256, dtype=torch.bfloat16).pin_memory()
+        runner.step([X.pin_memory()], [dY.pin_memory()], [hy], [hdx])
+        outs.append((hy, hdx))
+    runner.finish()
+    cuda_lib.fp8t_check_device_error()
+    for (ry, rdx), (gy, gdx) in zip(ref, outs):
+        assert torch.equal(ry.view(torch.int16), gy.view(torch.int16))
+        assert torch.equal(rdx.view(torch.int16), gdx.view(torch.int16))
+    assert torch.equal(eager.layers[0].W.view(torch.int16), streamed.layers[0].W.view(torch.int16))
+    assert torch.equal(eager.history, streamed.history)
