@@ -56,16 +56,15 @@ def load_peaks():
 
 
 def workload_numbers(wl):
-    """Algorithmic work per step of a one-layer workload."""
-    _, fin, fout = wl.layers[0]
+    """Algorithmic work per step of a (multi-layer) Linear workload."""
     T = wl.tokens
     return dict(
-        gemm_flop=2 * T * fin * fout,                       # each of fprop, dgrad, wgrad
-        cast_bytes=[4 * T * fin, 4 * fin * fout, 4 * T * fout],   # X, W, dY: 2 B in + 1 + 1 out
-        adamw_bytes=30 * fin * fout,                        # 2 B norm pass + 28 B update
-        params=fin * fout,
-        h2d=2 * T * fin + 2 * T * fout,                     # X and dY, BF16
-        d2h=2 * T * fout + 2 * T * fin,                     # Y and dX, BF16
+        gemm_flop=[2 * T * fin * fout for _, fin, fout in wl.layers],   # each of fprop/dgrad/wgrad
+        cast_bytes=sum(4 * (T * fin + fin * fout + T * fout) for _, fin, fout in wl.layers),
+        adamw_bytes=30 * sum(fin * fout for _, fin, fout in wl.layers),   # 2 B norm + 28 B update
+        params=sum(fin * fout for _, fin, fout in wl.layers),
+        h2d=sum(2 * T * fin + 2 * T * fout for _, fin, fout in wl.layers),   # X and dY, BF16
+        d2h=sum(2 * T * fout + 2 * T * fin for _, fin, fout in wl.layers),   # Y and dX, BF16
     )
 
 
@@ -158,26 +157,34 @@ def run_ours(args, rank, world, local_rank):
     wl = synth.WORKLOADS[args.workload]
     nums = workload_numbers(wl)
     peaks = load_peaks()
+    nl = len(wl.layers)
 
     st = Fp8LinearStep([(i, o) for _, i, o in wl.layers], wl.tokens, wl.history_len, wl.algo,
-                       wl.margin, wl.adamw, [synth.linear_weight(wl, 0, dev)], dev,
-                       device_step=True)
-    batches = [synth.linear_inputs(wl, 0, t, dev) for t in range(2)]
+                       wl.margin, wl.adamw, [synth.linear_weight(wl, k, dev) for k in range(nl)],
+                       dev, device_step=True)
+    batches = [list(zip(*[synth.linear_inputs(wl, k, t, dev) for k in range(nl)])) for t in range(2)]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    L = st.layers[0]
-    NEV = 7
-    stage_names = ["cast X, W, dY", "fprop", "dgrad", "wgrad", "scale update", "adamw"]
+    # one timing window per kernel launch of the step
+    stages = [("cast", None)]
+    for k, (lname, _, _) in enumerate(wl.layers):
+        stages += [(f"fprop/{lname}", (k, 0)), (f"dgrad/{lname}", (k, 1)), (f"wgrad/{lname}", (k, 2))]
+    stages += [("scale update", None), ("adamw", None)]
+    NEV = len(stages) + 1
 
-    def one_step(X, dY, ev=None):
+    def one_step(xs, dys, ev=None):
         st.t += 1
         rec = (lambda i: ev[i].record()) if ev is not None else (lambda i: None)
         rec(0)
-        st.cast_all([X], [dY]); rec(1)          # one launch: X, W -> E4M3, dY -> E5M2
-        st.gemm(0, 0); rec(2)
-        st.gemm(0, 1); rec(3)
-        st.gemm(0, 2); rec(4)
-        st.scale_update(); rec(5)
-        st.adamw(); rec(6)
+        for i, (name, kw) in enumerate(stages):
+            if name == "cast":
+                st.cast_all(xs, dys)              # grouped: X, W -> E4M3, dY -> E5M2
+            elif name == "scale update":
+                st.scale_update()
+            elif name == "adamw":
+                st.adamw()
+            else:
+                st.gemm(*kw)
+            rec(i + 1)
 
     for w in range(args.warmup):
         flush.zero_()
@@ -231,19 +238,21 @@ def run_ours(args, rank, world, local_rank):
                     for t in range(args.steps)]
         step_ms = [events[t][0].elapsed_time(events[t][NEV - 1]) for t in range(args.steps)]
     total_ms = reduce_max(sum(step_ms), world, dev)
-    flop_step = 3 * nums["gemm_flop"]
+    flop_step = 3 * sum(nums["gemm_flop"])
     value = throughput(flop_step, args.steps, world, total_ms)
 
     # per-kernel figures (this rank), averaged over the timed steps
-    avg = [statistics.mean(s[i] for s in stage_ms) for i in range(NEV - 1)]
-    gemm_ms = avg[1:4]
-    gemm_tflops = [nums["gemm_flop"] / (ms * 1e-3) / 1e12 for ms in gemm_ms]
-    cast_all_gbs = sum(nums["cast_bytes"]) / (avg[0] * 1e-3) / 1e9
-    adamw_gbs = nums["adamw_bytes"] / (avg[5] * 1e-3) / 1e9
+    avg = {name: statistics.mean(s[i] for s in stage_ms) for i, (name, _) in enumerate(stages)}
+    gemm_names = [n for n, kw in stages if kw is not None]
+    gemm_flop_of = {f"{r}/{lname}": nums["gemm_flop"][k]
+                    for k, (lname, _, _) in enumerate(wl.layers) for r in ("fprop", "dgrad", "wgrad")}
+    gemm_tflops = {n: round(gemm_flop_of[n] / (avg[n] * 1e-3) / 1e12, 1) for n in gemm_names}
+    gemm_ms_total = sum(avg[n] for n in gemm_names)
+    gemm_achieved = flop_step / (gemm_ms_total * 1e-3) / 1e12
+    cast_gbs = nums["cast_bytes"] / (avg["cast"] * 1e-3) / 1e9
+    adamw_gbs = nums["adamw_bytes"] / (avg["adamw"] * 1e-3) / 1e9
     fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
     hbm = peaks["hbm_gbs"]
-    gemm_avg_ms = statistics.mean(gemm_ms)
-    gemm_achieved = nums["gemm_flop"] / (gemm_avg_ms * 1e-3) / 1e12
     traffic = gemm_traffic_from_profile(wl.name)
 
     for g, _ in graphs:
@@ -254,63 +263,181 @@ def run_ours(args, rank, world, local_rank):
     # copy-in of step t+1 and the copy-out of step t-1 (separate streams and copy engines).
     from optimizer_fp8_cast_b200.host_stream import HostStreamedStep
     runner = HostStreamedStep(st)
-    hX = [b[0].cpu().pin_memory() for b in batches]
-    hdY = [b[1].cpu().pin_memory() for b in batches]
-    hY = [torch.empty(L.Y.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    hdX = [torch.empty(L.dX.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    hX = [[x.cpu().pin_memory() for x in b[0]] for b in batches]
+    hdY = [[d.cpu().pin_memory() for d in b[1]] for b in batches]
+    hY = [[torch.empty(l.Y.shape, dtype=torch.bfloat16).pin_memory() for l in st.layers] for _ in range(2)]
+    hdX = [[torch.empty(l.dX.shape, dtype=torch.bfloat16).pin_memory() for l in st.layers] for _ in range(2)]
     for t in range(2):                                   # warm the pinned paths
-        runner.step([hX[t]], [hdY[t]], [hY[t]], [hdX[t]])
+        runner.step(hX[t], hdY[t], hY[t], hdX[t])
     runner.finish()
     n_e2e = min(args.steps, 50)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(runner.s_in)
     for t in range(n_e2e):
-        runner.step([hX[t % 2]], [hdY[t % 2]], [hY[t % 2]], [hdX[t % 2]])
+        runner.step(hX[t % 2], hdY[t % 2], hY[t % 2], hdX[t % 2])
     e1.record(runner.s_out)
     runner.finish()
     fp8.fp8t_check_device_error()
     e2e_total = reduce_max(e0.elapsed_time(e1), world, dev)
     e2e_value = throughput(flop_step, n_e2e, world, e2e_total)
-    e2e_ms = [e2e_total / n_e2e] * n_e2e
 
+    shapes = {lname: [fin, fout] for lname, fin, fout in wl.layers}
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "fp8 (e4m3/e5m2 operands, f32 accumulate)",
         "data": "synthetic",
-        "config": {"workload": wl.name, "tokens": wl.tokens, "in_features": wl.layers[0][1],
-                   "out_features": wl.layers[0][2], "recipe": "HYBRID, delayed per-tensor scaling",
+        "config": {"workload": wl.name, "tokens": wl.tokens,
+                   "layers_in_out": shapes, "recipe": "HYBRID, delayed per-tensor scaling",
                    "history_len": wl.history_len, "amax_algo": wl.algo, "margin": wl.margin,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "launch": "eager" if args.eager else "CUDA graph per step (AdamW step counter on the device)",
                    "l2": "flushed before every timed step (256 MiB write)"},
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": nums["h2d"],
-                "d2h_bytes_per_step": nums["d2h"], "ms_per_step": round(e2e_total / len(e2e_ms), 4),
+                "d2h_bytes_per_step": nums["d2h"], "ms_per_step": round(e2e_total / n_e2e, 4),
                 "how": "pinned host X, dY in and Y, dX out every step; copies overlapped with "
                        "the previous/next step's kernels on separate streams"},
         "gpu_launches": args.steps * st.kernels_per_step(),
-        "roofline": {"kernel": "k_fp8_gemm (fprop, dgrad, wgrad)", "bound": "tensor",
+        "roofline": {"kernel": "k_fp8_gemm (all fprop, dgrad, wgrad launches)", "bound": "tensor",
                      "achieved": round(gemm_achieved, 1), "peak": round(fp8_peak, 1),
                      "unit": "TFLOP/s", "frac": round(gemm_achieved / fp8_peak, 4),
                      "traffic": traffic,
                      "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {FP8_OVER_BF16} (nominal FP8/BF16 ratio)"},
         "kernels": {
-            "stage_ms": {n: round(a, 4) for n, a in zip(stage_names, avg)},
-            "gemm_tflops": {"fprop": round(gemm_tflops[0], 1), "dgrad": round(gemm_tflops[1], 1),
-                            "wgrad": round(gemm_tflops[2], 1)},
-            "cast_gbs": round(cast_all_gbs, 1), "cast_frac_of_hbm": round(cast_all_gbs / hbm, 4),
-            "cast_bytes_per_step": sum(nums["cast_bytes"]),
+            "stage_ms": {n: round(a, 4) for n, a in avg.items()},
+            "gemm_tflops": gemm_tflops,
+            "cast_gbs": round(cast_gbs, 1), "cast_frac_of_hbm": round(cast_gbs / hbm, 4),
+            "cast_bytes_per_step": nums["cast_bytes"],
             "adamw_gbs": round(adamw_gbs, 1), "adamw_frac_of_hbm": round(adamw_gbs / hbm, 4),
             "hbm_peak_gbs": hbm, "peak_source": peaks["source"],
         },
         "clocks": clocks.summary(),
         "wall_s_timed_region": round(wall, 3),
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(st, wl, nums, batches[0], frac_rows=1024)
+    if rank == 0 and world == 1 and nl == 1 and not args.no_cpu_baseline:
+        b0 = (batches[0][0][0], batches[0][1][0])
+        result["cpu_baseline"] = cpu_baseline(st, wl, nums, b0, frac_rows=1024)
     return result
+
+
+def run_adamw_only(args):
+    """The standalone multi-tensor AdamW workload: 4.0e9 FP32 parameters in 512 tensors."""
+    import torch
+
+    import optimizer_fp8_cast_b200 as fp8
+    from optimizer_fp8_cast_b200 import synth
+    fp8.load()
+    dev = torch.device("cuda", 0)
+    cfg = synth.ADAMW4E9
+    sizes = [int(n) for n in synth.adamw_sizes(cfg["n_tensors"], cfg["total"], cfg["seed"],
+                                               cfg["min_bytes"] // 4, cfg["max_bytes"] // 4)]
+    free, _ = torch.cuda.mem_get_info()
+    need = 16 * sum(sizes) + (1 << 30)
+    if free < need:
+        return {"metric": METRIC, "workload": cfg["name"], "unavailable":
+                f"needs {need / 1e9:.0f} GB of free device memory, {free / 1e9:.0f} GB free"}
+    P = [synth.adamw_tensor("master", n, i, cfg, dev) for i, n in enumerate(sizes)]
+    M = [synth.adamw_tensor("m", n, i, cfg, dev) for i, n in enumerate(sizes)]
+    V = [synth.adamw_tensor("v", n, i, cfg, dev) for i, n in enumerate(sizes)]
+    G = [synth.adamw_tensor("grad", n, i, cfg, dev) for i, n in enumerate(sizes)]
+    W = [torch.empty(n, dtype=torch.bfloat16, device=dev) for n in sizes]
+    ws = torch.empty(fp8.fused_adamw_workspace_bytes(sizes), dtype=torch.uint8, device=dev)
+    counter = torch.tensor([cfg["hp"]["step"] - 1], dtype=torch.int64, device=dev)
+    hp = {k: v for k, v in cfg["hp"].items() if k != "step"}
+
+    def step():
+        fp8.fused_adamw_multi_tensor(P, M, V, G, W, step=0, step_counter=counter, workspace=ws, **hp)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    fp8.fp8t_check_device_error()
+    steps = min(args.steps, 20)
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    with ClockSampler(gpu_uuid(dev, 0)) as clocks:
+        e[0].record()
+        for t in range(steps):
+            step()
+            e[t + 1].record()
+        torch.cuda.synchronize()
+    fp8.fp8t_check_device_error()
+    ms = [e[t].elapsed_time(e[t + 1]) for t in range(steps)]
+    total = sum(sizes)
+    gbs = 30 * total * steps / (sum(ms) * 1e-3) / 1e9
+    hbm = load_peaks()["hbm_gbs"]
+    return {"metric": METRIC, "value": round(gbs, 1), "unit": "GB/s", "n_gpus": 1, "steps": steps,
+            "warmup": args.warmup, "ms_per_step": round(statistics.mean(ms), 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": cfg["name"], "params": total, "tensors": len(sizes),
+                       "bytes_per_param": "30 (2 norm pass + 28 update)",
+                       "l2": "inputs (64 GB) far larger than L2"},
+            "roofline": {"kernel": "k_adamw_sumsq + k_adamw_update", "bound": "hbm",
+                         "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(gbs / hbm, 4), "traffic": None},
+            "gpu_launches": steps * 4, "clocks": clocks.summary()}
+
+
+def run_stress_sweep(args):
+    """The 1024 x 1024 / 2048-token stress run, 50 steps with the x1000 X batch at step 20, swept
+    over history length, algorithm and margin: per-tensor saturation and zero fractions every
+    step, and the cast launch's share of the step time."""
+    import torch
+
+    import optimizer_fp8_cast_b200 as fp8
+    from optimizer_fp8_cast_b200 import synth
+    from optimizer_fp8_cast_b200.step import Fp8LinearStep
+    fp8.load()
+    dev = torch.device("cuda", 0)
+    wl = synth.STRESS1024
+    _, fin, fout = wl.layers[0]
+    n_el = [wl.tokens * fin, fin * fout, wl.tokens * fout]
+    table, summary = [], []
+    for H, algo, margin in synth.STRESS_SWEEP:
+        st = Fp8LinearStep([(fin, fout)], wl.tokens, H, algo, margin, wl.adamw,
+                           [synth.linear_weight(wl, 0, dev)], dev, counters=True)
+        cast_ms, step_ms = [], []
+        for t in range(wl.steps):
+            X, dY = synth.linear_inputs(wl, 0, t, dev)
+            st.counters.zero_()
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            st.t += 1
+            e[0].record()
+            st.cast_all([X], [dY])
+            e[1].record()
+            for which in (0, 1, 2):
+                st.gemm(0, which)
+            st.update()
+            e[2].record()
+            torch.cuda.synchronize()
+            cast_ms.append(e[0].elapsed_time(e[1]))
+            step_ms.append(e[0].elapsed_time(e[2]))
+            c = st.counters.cpu().numpy()
+            row = {"H": H, "algo": algo, "margin": margin, "step": t}
+            for r, name in enumerate(("X", "W", "dY")):
+                row[f"sat_{name}"] = float(c[r, 0]) / n_el[r]
+                row[f"zero_{name}"] = float(c[r, 1]) / n_el[r]
+            row["scale_X"] = float(st.scale[0].item())
+            table.append(row)
+        fp8.fp8t_check_device_error()
+        rows = table[-wl.steps:]
+        summary.append({"H": H, "algo": algo, "margin": margin,
+                        "sat_X_step19": rows[19]["sat_X"], "sat_X_step20": rows[20]["sat_X"],
+                        "sat_X_step21": rows[21]["sat_X"],
+                        "zero_X_step21": rows[21]["zero_X"], "zero_X_step49": rows[49]["zero_X"],
+                        "zero_W_step1": rows[1]["zero_W"], "zero_W_step49": rows[49]["zero_W"],
+                        "sat_dY_mean": statistics.mean(r["sat_dY"] for r in rows),
+                        "cast_overhead_frac": round(sum(cast_ms[5:]) / sum(step_ms[5:]), 4)})
+    if args.out:
+        with open(args.out, "w") as f:
+            json.dump(table, f)
+    return {"metric": METRIC, "workload": wl.name, "unit": "fractions",
+            "config": {"workload": wl.name, "tokens": wl.tokens, "in_features": fin,
+                       "out_features": fout, "steps": wl.steps, "spike_step": wl.x_spike_step,
+                       "launch": "eager, counters on, one synchronisation per step (not a throughput run)"},
+            "sweep": summary, "per_step_table": args.out}
 
 
 def gpu_uuid(dev, fallback):
@@ -379,7 +506,7 @@ def oracle_sample_step(oracle, host, wl, rows_div):
     w = [np.zeros(n, np.uint16)]
     oracle.fused_adamw(p, m, v, [host["dW"][:n]], w, dict(wl.adamw, step=1))
     dt = time.perf_counter() - t0
-    flop = 2 * (rt * fout * fin + rt * fin * fout + rw * fout * T)
+    flop = 2 * (rt * fout * fin + rt * fin * fout + rw * fout * T)   # the sampled GEMM rows
     return dt, flop
 
 
@@ -455,9 +582,12 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", default="linear4096_t8192")
+    ap.add_argument("--workload", default="linear4096_t8192",
+                    help="linear4096_t8192 (default), linear256_t512, block7b_t16384, "
+                         "adamw4e9_512t, stress1024_t2048")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager launches, not CUDA graphs")
+    ap.add_argument("--out", default=None, help="stress sweep: write the per-step table here")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         print("note: fewer than 3 warm-up steps", file=sys.stderr)
@@ -480,7 +610,12 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        result = run_ours(args, rank, world, local_rank)
+        if args.workload == "adamw4e9_512t":
+            result = run_adamw_only(args)
+        elif args.workload == "stress1024_t2048":
+            result = run_stress_sweep(args)
+        else:
+            result = run_ours(args, rank, world, local_rank)
         if rank == 0:
             print(json.dumps(result), flush=True)
     finally:
