@@ -317,15 +317,26 @@ fp8t_status fp8_gemm(const void* A, fp8t_format a_fmt, const void* B, fp8t_forma
   if (st != FP8T_OK) return st;
 
   using namespace fp8t::gemm;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, td;
   if ((st = encode_kmajor(&ta, A, M, K, kHalf)) != FP8T_OK) return st;
   if ((st = encode_kmajor(&tb, B, N, K, kHalf)) != FP8T_OK) return st;
+  {
+    // D (BF16 M x N): 32 x 32 boxes, 64-byte swizzle, written by the epilogue's TMA stores
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * 2};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = encode_fn()(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D_bf16, dims, strides, box,
+                             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(FP8T_ERR_CUDA, "cuTensorMapEncodeTiled (D) failed (%d)", (int)r);
+  }
   const int64_t tiles_n = (N + kBN - 1) / kBN;
   const int64_t tiles = ((M + kBM - 1) / kBM) * tiles_n;        // 256 x 256 tiles, one per pair
   if (tiles >= (int64_t(1) << 30)) return fail(FP8T_ERR_UNSUPPORTED_SHAPE, "fp8_gemm: too many tiles");
   const int64_t grid = 2 * std::min<int64_t>(tiles, dev->gemm_clusters);   // persistent pairs
   k_fp8_gemm<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, as_stream(stream)>>>(
-      ta, tb, static_cast<uint16_t*>(D_bf16), static_cast<int>(M), static_cast<int>(N),
+      ta, tb, td, static_cast<int>(M), static_cast<int>(N),
       static_cast<int>(K), d_a_scale_inv, d_b_scale_inv, make_idesc(a_fmt, b_fmt),
       static_cast<int>(tiles_n), static_cast<int>(tiles));
   return after_launch("fp8_gemm launch");

@@ -10,7 +10,7 @@
 // D[M x N] = bf16((A[M x K] . B[N x K]^T) * sa * sb), A and B K-major ("TN").
 // A cluster of two CTAs (one per SM) computes a 256 x 256 tile: CTA r loads A rows
 // [128r, 128r+128) and B rows (N columns) [128r, 128r+128) of the tile, 128-byte swizzled
-// 128 x 128-byte boxes, into its own 7-stage ring (32 KB per stage, 224 KB). Both CTAs' loads count on
+// 128 x 128-byte boxes, into its own 6-stage ring (32 KB per stage). Both CTAs' loads count on
 // the even CTA's "full" barrier; the even CTA's MMA thread issues tcgen05.mma.cta_group::2
 // (M=256, N=256, K=32), which reads A and B halves from both CTAs' shared memory, and releases
 // each stage in both CTAs with one multicast tcgen05.commit. Per SM that is 32 KB of operands per
@@ -21,8 +21,12 @@
 //   warp 0, lane 0  TMA producer (both CTAs)
 //   warp 1, lane 0  MMA issuer (even CTA only); warp 1 also owns the TMEM allocation
 //   warps 2-5       epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 of its own CTA (rows of
-//                   its half), scales by sa*sb, rounds to BF16, stores, and tells the even CTA
-//                   that the accumulator is free again (4 warps x 2 CTAs = 8 arrivals).
+//                   its half), 32 columns at a time, scales by sa*sb, rounds to BF16 and writes
+//                   the 32 x 32 chunk into a 64-byte-swizzled shared-memory buffer (double
+//                   buffered per warp), which one lane stores with a TMA bulk tensor store
+//                   (clipped at the M and N edges). Per-lane 16-byte stores to 32 different rows
+//                   cost ~15% of the GEMM's throughput. Once its TMEM reads are done the warp
+//                   tells the even CTA that the accumulator is free (4 warps x 2 CTAs arrive).
 // Every mbarrier wait is bounded (globaltimer). On expiry a CTA records kErrTimeout and stops
 // issuing; issued MMAs are awaited with a fixed bound, loads in flight are given time to land,
 // and both CTAs meet at a cluster barrier before TMEM is freed; D is then incomplete.
@@ -33,13 +37,17 @@
 namespace fp8t {
 namespace gemm {
 
-constexpr int kBM = 256, kBN = 256, kBK = 128, kStages = 7, kUmmaK = 32;
+constexpr int kBM = 256, kBN = 256, kBK = 128, kStages = 6, kUmmaK = 32;
 constexpr int kHalf = 128;                               // rows of A and of B per CTA
 constexpr int kThreads = 192;
 constexpr int kABytes = kHalf * kBK, kBBytes = kHalf * kBK, kStageBytes = kABytes + kBBytes;
 constexpr uint32_t kPairTxBytes = 2 * kStageBytes;       // both CTAs' boxes of one stage
 constexpr int kAccCols = 256, kTmemCols = 2 * kAccCols;
-constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*alignment slack*/ + 256 /*barriers*/;
+constexpr int kEpiWarps = 4;
+constexpr int kEpiChunkBytes = 32 * 32 * 2;              // 32 rows x 32 BF16 columns
+constexpr int kEpiBytes = kEpiWarps * 2 * kEpiChunkBytes; // double-buffered per epilogue warp
+constexpr int kSmemBytes =
+    kStages * kStageBytes + kEpiBytes + 1024 /*alignment slack*/ + 256 /*barriers*/;
 constexpr uint64_t kSettleNs = 200000;                   // let loads in flight land on abort
 constexpr uint64_t kPairDrainNs = 1000000;               // producer drain budget (1 ms)
 
@@ -80,14 +88,16 @@ struct Smem {
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     k_fp8_gemm(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
-               uint16_t* __restrict__ D, int M, int N, int K, const float* __restrict__ d_sa,
+               const __grid_constant__ CUtensorMap tma_d, int M, int N, int K,
+               const float* __restrict__ d_sa,
                const float* __restrict__ d_sb, uint32_t idesc, int n_tiles_n, int n_tiles) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   uint8_t* sA = smem;
   uint8_t* sB = smem + kStages * kABytes;
-  Smem* S = reinterpret_cast<Smem*>(smem + kStages * kStageBytes);
+  uint8_t* sEpi = smem + kStages * kStageBytes;              // 1024-byte aligned
+  Smem* S = reinterpret_cast<Smem*>(smem + kStages * kStageBytes + kEpiBytes);
   volatile int* abort_flag = &S->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -110,6 +120,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tma_a);
     tma_prefetch_desc(&tma_b);
+    tma_prefetch_desc(&tma_d);
   }
   if (warp == 1) {
     tmem_alloc_pair(smem_u32(&S->tmem_base), kTmemCols);
@@ -200,7 +211,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ---------------- epilogue warps 2..5 (both CTAs)
     const int quad = warp & 3;                       // TMEM lanes 32*quad .. 32*quad+31
     const float alpha = __fmul_rn(__ldg(d_sa), __ldg(d_sb));
-    uint32_t local = 0;
+    uint8_t* my_buf = sEpi + (warp - 2) * 2 * kEpiChunkBytes;
+    uint32_t local = 0, chunk_count = 0;
     for (int tile = cluster; tile < n_tiles; tile += n_clusters, ++local) {
       const uint32_t acc = local & 1, aph = (local >> 1) & 1;
       if (*abort_flag) break;
@@ -210,7 +222,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const int row = (tile / n_tiles_n) * kBM + static_cast<int>(rank) * kHalf + quad * 32 + lane;
+      const int row0 = (tile / n_tiles_n) * kBM + static_cast<int>(rank) * kHalf + quad * 32;
       const int n0 = (tile % n_tiles_n) * kBN;
       const uint32_t t_base = tmem + (static_cast<uint32_t>(quad * 32) << 16) + acc * kAccCols;
 #pragma unroll 1
@@ -218,25 +230,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         uint32_t r[32];
         tmem_ld_32x32b_x32(t_base + c * 32, r);
         tmem_ld_wait();
-        const int col = n0 + c * 32;
-        if (row < M && col < N) {
-          uint32_t packed[16];
+        if (n0 + c * 32 >= N || row0 >= M) continue;  // chunk entirely outside the matrix
+        uint8_t* buf = my_buf + (chunk_count & 1) * kEpiChunkBytes;
+        ++chunk_count;
+        if (lane == 0) bulk_wait_group_read<1>();    // the store that last used buf has read it
+        __syncwarp();
+        // row `lane` of the chunk: 64 bytes = four 16-byte pieces, 64-byte swizzle
+        // (piece p of row i lives at piece p ^ ((i >> 1) & 3)), matching the store's map
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            packed[j] = pack_bf16x2(__fmul_rn(__uint_as_float(r[2 * j]), alpha),
-                                    __fmul_rn(__uint_as_float(r[2 * j + 1]), alpha));
-          uint16_t* dst = D + static_cast<int64_t>(row) * N + col;
+        for (int p = 0; p < 4; ++p) {
+          uint32_t w[4];
 #pragma unroll
-          for (int qd = 0; qd < 4; ++qd)
-            if (col + 8 * qd < N)
-              *reinterpret_cast<uint4*>(dst + 8 * qd) = make_uint4(
-                  packed[4 * qd], packed[4 * qd + 1], packed[4 * qd + 2], packed[4 * qd + 3]);
+          for (int q = 0; q < 4; ++q) {
+            const int j = 4 * p + q;
+            w[q] = pack_bf16x2(__fmul_rn(__uint_as_float(r[2 * j]), alpha),
+                               __fmul_rn(__uint_as_float(r[2 * j + 1]), alpha));
+          }
+          const int pp = p ^ ((lane >> 1) & 3);
+          *reinterpret_cast<uint4*>(buf + lane * 64 + pp * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tma_d, smem_u32(buf), n0 + c * 32, row0);
+          bulk_commit_group();
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&S->acc_empty[acc]), 0));
     }
+    if (lane == 0) bulk_wait_group<0>();             // every store complete before exit
   }
   __syncwarp();
   __syncthreads();
