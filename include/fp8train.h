@@ -142,6 +142,28 @@ fp8t_status fp8_gemm(const void* A, fp8t_format a_fmt, const void* B, fp8t_forma
                      const float* d_a_scale_inv, const float* d_b_scale_inv,
                      void* D_bf16, void* stream);
 
+/* One GEMM of fp8_gemm_multi: the arguments of fp8_gemm. */
+typedef struct fp8t_gemm_desc {
+    const void* A;
+    fp8t_format a_fmt;
+    const void* B;
+    fp8t_format b_fmt;
+    int64_t M, N, K;
+    const float* d_a_scale_inv;
+    const float* d_b_scale_inv;
+    void* D_bf16;
+} fp8t_gemm_desc;
+
+/*
+ * fp8_gemm_multi — several independent fp8_gemm problems in one persistent launch (the fprop,
+ * dgrad and wgrad of a step, or those of several layers), same per-problem semantics and
+ * validation. One launch holds up to 24 problems; tiles are taken problem by problem, so the
+ * whole group shares one tile schedule (no gap between problems, balanced last wave).
+ *   gemms     HOST array of n_gemms descriptors (read during the call only).
+ *   n_gemms   1 .. 4096.
+ */
+fp8t_status fp8_gemm_multi(const fp8t_gemm_desc* gemms, int32_t n_gemms, void* stream);
+
 /*
  * fp8_scale_update — roll each tensor's amax history and compute the next scale
  * [P3 核心原理, Scale 决定数值是否进入可表示区间 (scale = (FP8_MAX / amax) / 2^margin) and

@@ -13,7 +13,7 @@ import torch
 
 from . import _abi
 
-__all__ = ["fp8_cast_transpose_amax", "fp8_cast_transpose_amax_multi", "fp8_gemm", "fp8_scale_update", "fused_adamw_multi_tensor",
+__all__ = ["fp8_cast_transpose_amax", "fp8_cast_transpose_amax_multi", "fp8_gemm", "fp8_gemm_multi", "fp8_scale_update", "fused_adamw_multi_tensor",
            "fused_adamw_workspace_bytes", "fused_adamw_multi_tensor_noalloc",
            "fp8t_check_device_error", "fp8t_debug_expire_waits", "fp8t_set_wait_timeout_ns",
            "Fp8TrainError", "E4M3", "E5M2", "AMAX_MAX", "AMAX_MOST_RECENT", "FP8_MAX", "load",
@@ -101,6 +101,20 @@ def fp8_gemm(A, a_fmt, B, b_fmt, a_scale_inv, b_scale_inv, D, stream=None):
     assert K == K2 and D.shape == (M, N) and D.dtype == torch.bfloat16
     _check(load().fp8_gemm(_ptr(A), int(a_fmt), _ptr(B), int(b_fmt), M, N, K, _ptr(a_scale_inv),
                            _ptr(b_scale_inv), _ptr(D), _stream(stream)), "fp8_gemm")
+
+
+def fp8_gemm_multi(gemms, stream=None):
+    """Several GEMMs in one persistent launch. ``gemms`` is a list of dicts with the arguments of
+    fp8_gemm: A, a_fmt, B, b_fmt, a_scale_inv, b_scale_inv, D."""
+    arr = (_abi.GemmDesc * len(gemms))()
+    for i, g in enumerate(gemms):
+        A, B, D = g["A"], g["B"], g["D"]
+        M, K = A.shape
+        N, K2 = B.shape
+        assert K == K2 and D.shape == (M, N) and D.dtype == torch.bfloat16
+        arr[i] = _abi.GemmDesc(_ptr(A), int(g["a_fmt"]), _ptr(B), int(g["b_fmt"]), M, N, K,
+                               _ptr(g["a_scale_inv"]), _ptr(g["b_scale_inv"]), _ptr(D))
+    _check(load().fp8_gemm_multi(arr, len(gemms), _stream(stream)), "fp8_gemm_multi")
 
 
 def fp8_scale_update(amax, history, fp8_max, algo, margin, scale, scale_inv, stream=None):

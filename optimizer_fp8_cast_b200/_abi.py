@@ -24,12 +24,21 @@ class CastTensor(C.Structure):
                 ("d_scale_inv_out", C.c_void_p), ("d_counters", C.c_void_p)]
 
 
+class GemmDesc(C.Structure):
+    """fp8t_gemm_desc."""
+    _fields_ = [("A", C.c_void_p), ("a_fmt", C.c_int), ("B", C.c_void_p), ("b_fmt", C.c_int),
+                ("M", C.c_int64), ("N", C.c_int64), ("K", C.c_int64),
+                ("d_a_scale_inv", C.c_void_p), ("d_b_scale_inv", C.c_void_p), ("D_bf16", C.c_void_p)]
+
+
 def declare(L):
     vp, i32, i64, f32 = C.c_void_p, C.c_int32, C.c_int64, C.c_float
     L.fp8_cast_transpose_amax.restype = C.c_int
     L.fp8_cast_transpose_amax.argtypes = [vp, i64, i64, C.c_int, vp, vp, vp, vp, vp, vp, vp]
     L.fp8_cast_transpose_amax_multi.restype = C.c_int
     L.fp8_cast_transpose_amax_multi.argtypes = [C.POINTER(CastTensor), i32, vp]
+    L.fp8_gemm_multi.restype = C.c_int
+    L.fp8_gemm_multi.argtypes = [C.POINTER(GemmDesc), i32, vp]
     L.fp8_gemm.restype = C.c_int
     L.fp8_gemm.argtypes = [vp, C.c_int, vp, C.c_int, i64, i64, i64, vp, vp, vp, vp]
     L.fp8_scale_update.restype = C.c_int

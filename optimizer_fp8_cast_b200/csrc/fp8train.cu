@@ -297,49 +297,77 @@ fp8t_status fp8_cast_transpose_amax(const void* x_bf16, int64_t rows, int64_t co
 }
 
 // ------------------------------------------------------------------ GEMM
-fp8t_status fp8_gemm(const void* A, fp8t_format a_fmt, const void* B, fp8t_format b_fmt, int64_t M,
-                     int64_t N, int64_t K, const float* d_a_scale_inv, const float* d_b_scale_inv,
-                     void* D_bf16, void* stream) {
+fp8t_status fp8_gemm_multi(const fp8t_gemm_desc* gemms, int32_t n_gemms, void* stream) {
   t_last_error.clear();
-  if (!A || !B || !D_bf16 || !d_a_scale_inv || !d_b_scale_inv)
-    return fail(FP8T_ERR_INVALID_ARG, "fp8_gemm: NULL pointer");
-  if ((a_fmt != FP8T_E4M3 && a_fmt != FP8T_E5M2) || (b_fmt != FP8T_E4M3 && b_fmt != FP8T_E5M2))
-    return fail(FP8T_ERR_INVALID_ARG, "fp8_gemm: unknown format");
-  if (M <= 0 || N <= 0 || K <= 0) return fail(FP8T_ERR_INVALID_ARG, "fp8_gemm: M, N, K must be > 0");
+  if (!gemms || n_gemms < 1 || n_gemms > 4096)
+    return fail(FP8T_ERR_INVALID_ARG, "fp8_gemm: gemms NULL or n_gemms out of range");
   const int64_t lim = int64_t(1) << 31;
-  if (M % 16 || N % 16 || K % 16 || M >= lim || N >= lim || K >= lim)
-    return fail(FP8T_ERR_UNSUPPORTED_SHAPE, "fp8_gemm: M, N, K must be multiples of 16 below 2^31");
-  if (!aligned(A, 16) || !aligned(B, 16) || !aligned(D_bf16, 16) || !aligned(d_a_scale_inv, 4) ||
-      !aligned(d_b_scale_inv, 4))
-    return fail(FP8T_ERR_MISALIGNED, "fp8_gemm: misaligned pointer");
+  for (int32_t i = 0; i < n_gemms; ++i) {
+    const fp8t_gemm_desc& d = gemms[i];
+    if (!d.A || !d.B || !d.D_bf16 || !d.d_a_scale_inv || !d.d_b_scale_inv)
+      return fail(FP8T_ERR_INVALID_ARG, "fp8_gemm: problem %d: NULL pointer", i);
+    if ((d.a_fmt != FP8T_E4M3 && d.a_fmt != FP8T_E5M2) || (d.b_fmt != FP8T_E4M3 && d.b_fmt != FP8T_E5M2))
+      return fail(FP8T_ERR_INVALID_ARG, "fp8_gemm: problem %d: unknown format", i);
+    if (d.M <= 0 || d.N <= 0 || d.K <= 0)
+      return fail(FP8T_ERR_INVALID_ARG, "fp8_gemm: problem %d: M, N, K must be > 0", i);
+    if (d.M % 16 || d.N % 16 || d.K % 16 || d.M >= lim || d.N >= lim || d.K >= lim)
+      return fail(FP8T_ERR_UNSUPPORTED_SHAPE, "fp8_gemm: problem %d: M, N, K must be multiples of 16 below 2^31", i);
+    if (!aligned(d.A, 16) || !aligned(d.B, 16) || !aligned(d.D_bf16, 16) ||
+        !aligned(d.d_a_scale_inv, 4) || !aligned(d.d_b_scale_inv, 4))
+      return fail(FP8T_ERR_MISALIGNED, "fp8_gemm: problem %d: misaligned pointer", i);
+  }
   DeviceInfo* dev = nullptr;
   fp8t_status st = current_device(&dev);
   if (st != FP8T_OK) return st;
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(FP8T_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
 
   using namespace fp8t::gemm;
-  CUtensorMap ta, tb, td;
-  if ((st = encode_kmajor(&ta, A, M, K, kHalf)) != FP8T_OK) return st;
-  if ((st = encode_kmajor(&tb, B, N, K, kHalf)) != FP8T_OK) return st;
-  {
-    // D (BF16 M x N): 32 x 32 boxes, 64-byte swizzle, written by the epilogue's TMA stores
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * 2};
-    cuuint32_t box[2] = {32, 32};
-    cuuint32_t es[2] = {1, 1};
-    CUresult r = encode_fn()(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D_bf16, dims, strides, box,
-                             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
-                             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return fail(FP8T_ERR_CUDA, "cuTensorMapEncodeTiled (D) failed (%d)", (int)r);
+  static thread_local Group group;
+  for (int32_t b0 = 0; b0 < n_gemms; b0 += kMaxProblems) {
+    const int32_t b1 = std::min<int32_t>(n_gemms, b0 + kMaxProblems);
+    std::memset(&group, 0, sizeof(group));
+    group.n = b1 - b0;
+    int64_t tiles = 0;
+    for (int32_t i = b0; i < b1; ++i) {
+      const fp8t_gemm_desc& d = gemms[i];
+      Problem& P = group.p[i - b0];
+      if ((st = encode_kmajor(&P.a, d.A, d.M, d.K, kHalf)) != FP8T_OK) return st;
+      if ((st = encode_kmajor(&P.b, d.B, d.N, d.K, kHalf)) != FP8T_OK) return st;
+      // D (BF16 M x N): 32 x 32 boxes, 64-byte swizzle, written by the epilogue's TMA stores
+      cuuint64_t dims[2] = {static_cast<cuuint64_t>(d.N), static_cast<cuuint64_t>(d.M)};
+      cuuint64_t strides[1] = {static_cast<cuuint64_t>(d.N) * 2};
+      cuuint32_t box[2] = {32, 32};
+      cuuint32_t es[2] = {1, 1};
+      CUresult r = fn(&P.d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.D_bf16, dims, strides, box, es,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                      CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (r != CUDA_SUCCESS) return fail(FP8T_ERR_CUDA, "cuTensorMapEncodeTiled (D) failed (%d)", (int)r);
+      P.sa = d.d_a_scale_inv;
+      P.sb = d.d_b_scale_inv;
+      P.M = static_cast<int32_t>(d.M);
+      P.N = static_cast<int32_t>(d.N);
+      P.K = static_cast<int32_t>(d.K);
+      P.idesc = make_idesc(d.a_fmt, d.b_fmt);
+      P.tiles_n = static_cast<int32_t>((d.N + kBN - 1) / kBN);
+      P.tile_start = static_cast<int32_t>(tiles);
+      tiles += ((d.M + kBM - 1) / kBM) * P.tiles_n;            // 256 x 256 tiles, one per pair
+      if (tiles >= (int64_t(1) << 30))
+        return fail(FP8T_ERR_UNSUPPORTED_SHAPE, "fp8_gemm: too many tiles in one launch");
+    }
+    group.total_tiles = static_cast<int32_t>(tiles);
+    const int64_t grid = 2 * std::min<int64_t>(tiles, dev->gemm_clusters);   // persistent pairs
+    k_fp8_gemm<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, as_stream(stream)>>>(group);
+    if ((st = after_launch("fp8_gemm launch")) != FP8T_OK) return st;
   }
-  const int64_t tiles_n = (N + kBN - 1) / kBN;
-  const int64_t tiles = ((M + kBM - 1) / kBM) * tiles_n;        // 256 x 256 tiles, one per pair
-  if (tiles >= (int64_t(1) << 30)) return fail(FP8T_ERR_UNSUPPORTED_SHAPE, "fp8_gemm: too many tiles");
-  const int64_t grid = 2 * std::min<int64_t>(tiles, dev->gemm_clusters);   // persistent pairs
-  k_fp8_gemm<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, as_stream(stream)>>>(
-      ta, tb, td, static_cast<int>(M), static_cast<int>(N),
-      static_cast<int>(K), d_a_scale_inv, d_b_scale_inv, make_idesc(a_fmt, b_fmt),
-      static_cast<int>(tiles_n), static_cast<int>(tiles));
-  return after_launch("fp8_gemm launch");
+  return FP8T_OK;
+}
+
+fp8t_status fp8_gemm(const void* A, fp8t_format a_fmt, const void* B, fp8t_format b_fmt, int64_t M,
+                     int64_t N, int64_t K, const float* d_a_scale_inv, const float* d_b_scale_inv,
+                     void* D_bf16, void* stream) {
+  const fp8t_gemm_desc d = {A, a_fmt, B, b_fmt, M, N, K, d_a_scale_inv, d_b_scale_inv, D_bf16};
+  return fp8_gemm_multi(&d, 1, stream);
 }
 
 // ------------------------------------------------------------------ scale update

@@ -76,6 +76,27 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// One GEMM of a grouped launch. Tiles are numbered problem by problem.
+constexpr int kMaxProblems = 24;
+struct alignas(64) Problem {
+  CUtensorMap a, b, d;           // A [M][K], B [N][K] (128 x 128-byte boxes), D [M][N] (32 x 32)
+  const float* sa;
+  const float* sb;
+  int32_t M, N, K;
+  uint32_t idesc;
+  int32_t tiles_n, tile_start;
+};
+struct alignas(64) Group {
+  Problem p[kMaxProblems];
+  int32_t n, total_tiles;
+};
+
+__device__ __forceinline__ int find_problem(const Group& g, int tile) {
+  int p = 0;
+  while (p + 1 < g.n && g.p[p + 1].tile_start <= tile) ++p;
+  return p;
+}
+
 struct Smem {
   uint64_t full[kStages];     // even CTA: both CTAs' loads of a stage have landed
   uint64_t empty[kStages];    // both CTAs: the pair MMA has consumed a stage
@@ -87,10 +108,7 @@ struct Smem {
 };
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    k_fp8_gemm(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
-               const __grid_constant__ CUtensorMap tma_d, int M, int N, int K,
-               const float* __restrict__ d_sa,
-               const float* __restrict__ d_sb, uint32_t idesc, int n_tiles_n, int n_tiles) {
+    k_fp8_gemm(const __grid_constant__ Group g) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -104,7 +122,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
   const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
-  const int num_kb = (K + kBK - 1) / kBK;
+  const int n_tiles = g.total_tiles;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -118,9 +136,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(smem_u32(&S->mma_done), 1);
     *abort_flag = 0;
     fence_mbar_init();
-    tma_prefetch_desc(&tma_a);
-    tma_prefetch_desc(&tma_b);
-    tma_prefetch_desc(&tma_d);
+    for (int p = 0; p < g.n && p < 8; ++p) {
+      tma_prefetch_desc(&g.p[p].a);
+      tma_prefetch_desc(&g.p[p].b);
+      tma_prefetch_desc(&g.p[p].d);
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(smem_u32(&S->tmem_base), kTmemCols);
@@ -140,8 +160,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // ---------------- TMA producer (both CTAs)
       uint32_t it = 0, issued = 0;
       for (int tile = cluster; tile < n_tiles && !*abort_flag; tile += n_clusters) {
-        const int m0 = (tile / n_tiles_n) * kBM + static_cast<int>(rank) * kHalf;
-        const int n0 = (tile % n_tiles_n) * kBN + static_cast<int>(rank) * kHalf;
+        const Problem& P = g.p[find_problem(g, tile)];
+        const int local = tile - P.tile_start;
+        const int m0 = (local / P.tiles_n) * kBM + static_cast<int>(rank) * kHalf;
+        const int n0 = (local % P.tiles_n) * kBN + static_cast<int>(rank) * kHalf;
+        const int num_kb = (P.K + kBK - 1) / kBK;
         for (int kb = 0; kb < num_kb; ++kb, ++it) {
           const uint32_t s = it % kStages, ph = (it / kStages) & 1;
           if (*abort_flag) break;
@@ -152,8 +175,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           const uint32_t full_leader = mapa_shared(smem_u32(&S->full[s]), 0);
           if (leader) mbar_arrive_expect_tx(smem_u32(&S->full[s]), kPairTxBytes);
-          tma_load_2d_pair(smem_u32(sA + s * kABytes), &tma_a, kb * kBK, m0, full_leader);
-          tma_load_2d_pair(smem_u32(sB + s * kBBytes), &tma_b, kb * kBK, n0, full_leader);
+          tma_load_2d_pair(smem_u32(sA + s * kABytes), &P.a, kb * kBK, m0, full_leader);
+          tma_load_2d_pair(smem_u32(sB + s * kBBytes), &P.b, kb * kBK, n0, full_leader);
           ++issued;
         }
       }
@@ -174,6 +197,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // ---------------- MMA issuer (even CTA)
       uint32_t it = 0, local = 0;
       for (int tile = cluster; tile < n_tiles && !*abort_flag; tile += n_clusters, ++local) {
+        const Problem& P = g.p[find_problem(g, tile)];
+        const int num_kb = (P.K + kBK - 1) / kBK;
+        const uint32_t idesc = P.idesc;
         const uint32_t acc = local & 1, aph = (local >> 1) & 1;
         if (!mbar_wait(smem_u32(&S->acc_empty[acc]), aph ^ 1, limit, expire_main)) {
           *abort_flag = 1;
@@ -210,7 +236,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else {
     // ---------------- epilogue warps 2..5 (both CTAs)
     const int quad = warp & 3;                       // TMEM lanes 32*quad .. 32*quad+31
-    const float alpha = __fmul_rn(__ldg(d_sa), __ldg(d_sb));
     uint8_t* my_buf = sEpi + (warp - 2) * 2 * kEpiChunkBytes;
     uint32_t local = 0, chunk_count = 0;
     for (int tile = cluster; tile < n_tiles; tile += n_clusters, ++local) {
@@ -222,8 +247,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const int row0 = (tile / n_tiles_n) * kBM + static_cast<int>(rank) * kHalf + quad * 32;
-      const int n0 = (tile % n_tiles_n) * kBN;
+      const Problem& P = g.p[find_problem(g, tile)];
+      const int M = P.M, N = P.N, local_tile = tile - P.tile_start;
+      const float alpha = __fmul_rn(__ldg(P.sa), __ldg(P.sb));
+      const int row0 = (local_tile / P.tiles_n) * kBM + static_cast<int>(rank) * kHalf + quad * 32;
+      const int n0 = (local_tile % P.tiles_n) * kBN;
       const uint32_t t_base = tmem + (static_cast<uint32_t>(quad * 32) << 16) + acc * kAccCols;
 #pragma unroll 1
       for (int c = 0; c < kBN / 32; ++c) {
@@ -252,7 +280,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&tma_d, smem_u32(buf), n0 + c * 32, row0);
+          tma_store_2d(&P.d, smem_u32(buf), n0 + c * 32, row0);
           bulk_commit_group();
         }
       }

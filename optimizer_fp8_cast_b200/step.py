@@ -14,7 +14,7 @@ All scalars stay on the device; nothing in a step synchronises with the host.
 import torch
 
 from . import (AMAX_MAX, AMAX_MOST_RECENT, E4M3, E5M2, FP8_MAX, fp8_cast_transpose_amax,
-               fp8_cast_transpose_amax_multi, fp8_gemm, fp8_scale_update,
+               fp8_cast_transpose_amax_multi, fp8_gemm, fp8_gemm_multi, fp8_scale_update,
                fused_adamw_multi_tensor, fused_adamw_workspace_bytes)
 
 ROLE_X, ROLE_W, ROLE_DY = 0, 1, 2
@@ -108,6 +108,20 @@ class Fp8LinearStep:
         else:
             fp8_gemm(L.XqT, E4M3, L.dYqT, E5M2, sx, sdy, L.dW, stream=stream)
 
+    def gemm_desc(self, k, which):
+        L = self.layers[k]
+        sx, sw, sdy = (self._slot(self.scale_inv, 3 * k + r) for r in (ROLE_X, ROLE_W, ROLE_DY))
+        if which == 0:
+            return dict(A=L.Xq, a_fmt=E4M3, B=L.WqT, b_fmt=E4M3, a_scale_inv=sx, b_scale_inv=sw, D=L.Y)
+        if which == 1:
+            return dict(A=L.dYq, a_fmt=E5M2, B=L.Wq, b_fmt=E4M3, a_scale_inv=sdy, b_scale_inv=sw, D=L.dX)
+        return dict(A=L.XqT, a_fmt=E4M3, B=L.dYqT, b_fmt=E5M2, a_scale_inv=sx, b_scale_inv=sdy, D=L.dW)
+
+    def gemm_all(self, stream=None):
+        """Every layer's fprop, dgrad and wgrad in one grouped launch (24 GEMMs per launch)."""
+        fp8_gemm_multi([self.gemm_desc(k, w) for k in range(len(self.layers)) for w in (0, 1, 2)],
+                       stream=stream)
+
     def layer_forward_backward(self, k, X, dY, stream=None):
         L = self.layers[k]
         self.cast(k, ROLE_X, X, L.Xq, L.XqT, stream)
@@ -139,13 +153,12 @@ class Fp8LinearStep:
         """One training step; xs[k] = X [tokens, in_k], dys[k] = dY [tokens, out_k] (BF16, device)."""
         self.t += 1
         self.cast_all(xs, dys, stream)
-        for k in range(len(self.layers)):
-            for which in (0, 1, 2):
-                self.gemm(k, which, stream)
+        self.gemm_all(stream)
         self.update(stream)
 
     # launches of the library's kernels per step (for the benchmark's launch count)
     def kernels_per_step(self):
         n_adamw_batches = (len(self.layers) + 255) // 256
         n_cast_launches = (3 * len(self.layers) + 7) // 8
-        return n_cast_launches + 3 * len(self.layers) + 1 + 2 * n_adamw_batches
+        n_gemm_launches = (3 * len(self.layers) + 23) // 24
+        return n_cast_launches + n_gemm_launches + 1 + 2 * n_adamw_batches

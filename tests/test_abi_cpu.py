@@ -68,6 +68,14 @@ def test_invalid_arguments_rejected_on_host(lib):
     assert lib.fp8_gemm(P, 0, P, 0, 16, 20, 16, P, P, P, z) == 2
     assert lib.fp8_gemm(P, 0, P, 0, 16, 16, 1 << 31, P, P, P, z) == 2
     assert lib.fp8_gemm(P, 0, U, 0, 16, 16, 16, P, P, P, z) == 3
+    # grouped gemm: validated per problem before anything runs
+    g = (_abi.GemmDesc * 2)()
+    g[0] = _abi.GemmDesc(P, 0, P, 0, 16, 16, 16, P, P, P)
+    g[1] = _abi.GemmDesc(P, 1, P, 0, 16, 16, 24, P, P, P)
+    assert lib.fp8_gemm_multi(g, 2, z) == 2 and b"problem 1" in lib.fp8t_last_error_message()
+    g[1] = _abi.GemmDesc(P, 1, P, 3, 16, 16, 16, P, P, P)
+    assert lib.fp8_gemm_multi(g, 2, z) == 1
+    assert lib.fp8_gemm_multi(g, 0, z) == 1
     # scale update
     assert lib.fp8_scale_update(0, P, P, 16, P, 0, 0, P, P, z) == 1
     assert lib.fp8_scale_update(3, P, P, 0, P, 0, 0, P, P, z) == 1

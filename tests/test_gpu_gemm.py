@@ -103,3 +103,25 @@ def test_full_size_sampled(cuda_lib, M, N, K, af, bf, label):
     R, ab = oracle.gemm_at(u8(A), af, u8(B), bf, sa, sb, ii, jj)
     ok = gemm_within_tolerance(Dh, R, ab)
     assert ok.all(), f"{label}: {(~ok).sum()} of {ok.size} samples outside tolerance"
+
+
+def test_grouped_launch_mixed_problems(cuda_lib):
+    """Problems of different shapes and formats in one launch (and more than one launch table)
+    each equal the oracle within the GEMM tolerance."""
+    rng = np.random.default_rng(42)
+    shapes = [(144, 272, 48), (512, 256, 256), (16, 16, 16), (400, 528, 1040), (256, 768, 128)]
+    probs = []
+    for i in range(26):                                  # 26 problems: two launch tables
+        M, N, K = shapes[i % len(shapes)]
+        af, bf = PAIRS[i % 4]
+        A = random_codes(M, K, af, 100 + i)
+        B = random_codes(N, K, bf, 200 + i)
+        sa, sb = float(rng.uniform(0.01, 1)), float(rng.uniform(0.01, 1))
+        probs.append(dict(A=A, a_fmt=af, B=B, b_fmt=bf, a_scale_inv=dev_scalar(sa),
+                          b_scale_inv=dev_scalar(sb), D=torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda"),
+                          sa=sa, sb=sb))
+    cuda_lib.fp8_gemm_multi([{k: v for k, v in p.items() if k not in ("sa", "sb")} for p in probs])
+    cuda_lib.fp8t_check_device_error()
+    for p in probs:
+        R, ab = oracle.gemm(u8(p["A"]), p["a_fmt"], u8(p["B"]), p["b_fmt"], p["sa"], p["sb"], want_abs=True)
+        assert gemm_within_tolerance(bf16_bits(p["D"]), R, ab).all()
