@@ -156,6 +156,32 @@ class Fp8LinearStep:
         self.gemm_all(stream)
         self.update(stream)
 
+    # ------------------------------------------------------------------ training state
+    def state_dict(self):
+        """Everything a resumed run needs to continue bit for bit: per layer the BF16 weight,
+        FP32 master, m and v; the FP8 scale state (amax slots, amax history, scales, scale
+        inverses); the step count (host and, when used, device counter). The pages' checkpoint
+        incident (a restore without the amax history re-warms the scales and drifts) is why the
+        scale state is part of it."""
+        out = {"t": self.t, "amax": self.amax.clone(), "history": self.history.clone(),
+               "scale": self.scale.clone(), "scale_inv": self.scale_inv.clone(),
+               "layers": [{"W": l.W.clone(), "master": l.master.clone(), "m": l.m.clone(),
+                           "v": l.v.clone()} for l in self.layers]}
+        if self.step_counter is not None:
+            out["step_counter"] = self.step_counter.clone()
+        return out
+
+    def load_state_dict(self, sd):
+        """Restore a state_dict into this step's buffers (shapes must match)."""
+        self.t = int(sd["t"])
+        for name in ("amax", "history", "scale", "scale_inv"):
+            getattr(self, name).copy_(sd[name])
+        for l, s in zip(self.layers, sd["layers"]):
+            for name in ("W", "master", "m", "v"):
+                getattr(l, name).copy_(s[name])
+        if self.step_counter is not None:
+            self.step_counter.copy_(sd.get("step_counter", torch.tensor([self.t])))
+
     # launches of the library's kernels per step (for the benchmark's launch count)
     def kernels_per_step(self):
         n_adamw_batches = (len(self.layers) + 255) // 256
