@@ -161,11 +161,16 @@ def run_ours(args, rank, world, local_rank):
 
     st = Fp8LinearStep([(i, o) for _, i, o in wl.layers], wl.tokens, wl.history_len, wl.algo,
                        wl.margin, wl.adamw, [synth.linear_weight(wl, k, dev) for k in range(nl)],
-                       dev, device_step=True)
+                       dev, device_step=True, fused_update=not args.separate_scale_update,
+                       fused_norm=not args.separate_norm_pass,
+                       fused_wcast=not args.separate_weight_cast)
     batches = [list(zip(*[synth.linear_inputs(wl, k, t, dev) for k in range(nl)])) for t in range(2)]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    # one timing window per kernel launch of the step
-    stages = [("cast", None), ("gemm", None), ("scale update", None), ("adamw", None)]
+    # one timing window per kernel launch of the step (the scale update runs in the last CTA of
+    # the cast launch unless --separate-scale-update)
+    stages = [("cast", None), ("gemm", None), ("adamw", None)]
+    if args.separate_scale_update:
+        stages.insert(2, ("scale update", None))
     NEV = len(stages) + 1
 
     def one_step(xs, dys, ev=None):
@@ -173,14 +178,14 @@ def run_ours(args, rank, world, local_rank):
         rec = (lambda i: ev[i].record()) if ev is not None else (lambda i: None)
         rec(0)
         for i, (name, kw) in enumerate(stages):
-            if name == "cast":
-                st.cast_all(xs, dys)              # grouped: X, W -> E4M3, dY -> E5M2
-            elif name == "gemm":
-                st.gemm_all()                     # grouped: every fprop, dgrad and wgrad
+            if name == "cast":                    # grouped: X, W -> E4M3, dY -> E5M2
+                st.cast_all(xs, dys, update=st.fused_update)
+            elif name == "gemm":                  # grouped: every fprop, dgrad and wgrad
+                st.gemm_all(sumsq=st.fused_norm)
             elif name == "scale update":
                 st.scale_update()
             elif name == "adamw":
-                st.adamw()
+                st.adamw(presummed=st.fused_norm)
             else:
                 st.gemm(*kw)
             rec(i + 1)
@@ -243,8 +248,13 @@ def run_ours(args, rank, world, local_rank):
     # per-kernel figures (this rank), averaged over the timed steps
     avg = {name: statistics.mean(s[i] for s in stage_ms) for i, (name, _) in enumerate(stages)}
     gemm_achieved = flop_step / (avg["gemm"] * 1e-3) / 1e12
-    cast_gbs = nums["cast_bytes"] / (avg["cast"] * 1e-3) / 1e9
-    adamw_gbs = nums["adamw_bytes"] / (avg["adamw"] * 1e-3) / 1e9
+    # algorithmic bytes of the launches as configured: the W cast (4 B/param) moves from the
+    # cast launch into AdamW as 2 B/param of codes (the weight it reads is already in registers)
+    cast_bytes = nums["cast_bytes"] - (4 * nums["params"] if st.fused_wcast else 0)
+    adamw_bytes = ((28 + (2 if st.fused_wcast else 0)) * nums["params"]
+                   + (0 if st.fused_norm else 2 * nums["params"]))
+    cast_gbs = cast_bytes / (avg["cast"] * 1e-3) / 1e9
+    adamw_gbs = adamw_bytes / (avg["adamw"] * 1e-3) / 1e9
     fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
     hbm = peaks["hbm_gbs"]
     traffic = gemm_traffic_from_profile(wl.name)
@@ -288,6 +298,12 @@ def run_ours(args, rank, world, local_rank):
                    "history_len": wl.history_len, "amax_algo": wl.algo, "margin": wl.margin,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "launch": "eager" if args.eager else "CUDA graph per step (AdamW step counter on the device)",
+                   "scale_update": "separate launch" if args.separate_scale_update
+                                   else "in the last CTA of the cast launch",
+                   "grad_sum_of_squares": "AdamW norm pass" if args.separate_norm_pass
+                                          else "in the wgrad GEMM epilogue",
+                   "weight_cast": "in AdamW (next step's codes)" if st.fused_wcast
+                                  else "in the cast launch",
                    "l2": "flushed before every timed step (256 MiB write)"},
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": nums["h2d"],
                 "d2h_bytes_per_step": nums["d2h"], "ms_per_step": round(e2e_total / n_e2e, 4),
@@ -303,7 +319,7 @@ def run_ours(args, rank, world, local_rank):
             "stage_ms": {n: round(a, 4) for n, a in avg.items()},
             "gemm_tflops": round(gemm_achieved, 1),
             "cast_gbs": round(cast_gbs, 1), "cast_frac_of_hbm": round(cast_gbs / hbm, 4),
-            "cast_bytes_per_step": nums["cast_bytes"],
+            "cast_bytes_per_step": cast_bytes, "adamw_bytes_per_step": adamw_bytes,
             "adamw_gbs": round(adamw_gbs, 1), "adamw_frac_of_hbm": round(adamw_gbs / hbm, 4),
             "hbm_peak_gbs": hbm, "peak_source": peaks["source"],
         },
@@ -581,6 +597,12 @@ def main(argv=None):
                          "adamw4e9_512t, stress1024_t2048")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager launches, not CUDA graphs")
+    ap.add_argument("--separate-weight-cast", action="store_true",
+                    help="cast W in the cast launch instead of inside AdamW")
+    ap.add_argument("--separate-norm-pass", action="store_true",
+                    help="run AdamW's own norm pass instead of summing dW^2 in the wgrad epilogue")
+    ap.add_argument("--separate-scale-update", action="store_true",
+                    help="run the scale update as its own launch instead of in the cast launch")
     ap.add_argument("--out", default=None, help="stress sweep: write the per-step table here")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":

@@ -116,6 +116,42 @@ typedef struct fp8t_cast_tensor {
 fp8t_status fp8_cast_transpose_amax_multi(const fp8t_cast_tensor* tensors, int32_t n_tensors,
                                           void* stream);
 
+/* The scale state fp8_cast_transpose_amax_update_multi updates for one tensor. */
+typedef struct fp8t_cast_update {
+    float* d_amax_history;     /* history_len floats of this tensor, entry 0 newest (in/out) */
+    float* d_scale_inv_next;   /* 1 float: receives 1 / next scale; must not be the cast's
+                                  d_scale_inv_out, which keeps 1 / the scale the cast used */
+} fp8t_cast_update;
+
+/*
+ * fp8_cast_transpose_amax_update_multi — the casts of fp8_cast_transpose_amax_multi followed,
+ * inside the same launch, by the delayed-scaling update of fp8_scale_update for the same
+ * tensors [P3 核心原理, Delayed Scaling: the scale for the next iteration comes from the amax
+ * history; the scale kernel is one of the extra launches 实践建议 warns about]. The CTA that
+ * finishes last rolls each tensor's history (amax pushed at entry 0), picks the representative
+ * amax (algo), writes the next scale IN PLACE into tensors[i].d_scale (declared const there
+ * because the cast only reads it; this call overwrites it after every read of it is done),
+ * writes 1/next scale to updates[i].d_scale_inv_next and resets tensors[i].d_amax_inout to 0.
+ * FP8 max is 448 for E4M3 tensors and 57344 for E5M2 ones. The result is bit-identical to
+ * fp8_cast_transpose_amax_multi then fp8_scale_update with the same arguments.
+ *   updates       HOST array of n_tensors entries.
+ *   history_len   1 .. 65536 (the same for every tensor of the call).
+ *   algo, margin  as in fp8_scale_update.
+ *   d_ticket      1 device uint32, zero before the first call; each launch leaves it zero.
+ *                 Calls that may run at the same time (other streams) need their own tickets.
+ * An entry with x_bf16 = NULL, rows = cols = 0 and no outputs or counters is UPDATE ONLY: its
+ * amax slot was filled by another call (the weight cast inside
+ * fused_adamw_multi_tensor_presummed of the previous step) and only the update runs for it.
+ * If a bounded wait of the launch expires (FP8T_ERR_TIMEOUT pending in the device error word),
+ * the scale state is left unchanged. Argument errors as in the two calls it combines, plus
+ * FP8T_ERR_INVALID_ARG for a NULL or shared scale-inverse pointer.
+ */
+fp8t_status fp8_cast_transpose_amax_update_multi(const fp8t_cast_tensor* tensors,
+                                                 const fp8t_cast_update* updates, int32_t n_tensors,
+                                                 int32_t history_len, fp8t_amax_algo algo,
+                                                 int32_t margin, unsigned int* d_ticket,
+                                                 void* stream);
+
 /*
  * fp8_gemm — per-tensor scaled FP8 GEMM, FP32 accumulation, BF16 output, "TN" layout:
  *
@@ -163,6 +199,30 @@ typedef struct fp8t_gemm_desc {
  *   n_gemms   1 .. 4096.
  */
 fp8t_status fp8_gemm_multi(const fp8t_gemm_desc* gemms, int32_t n_gemms, void* stream);
+
+/*
+ * fp8_gemm_multi_sumsq — fp8_gemm_multi that also returns, for the problems selected by
+ * sumsq_of, S = sum over their D elements of f32(D)^2, accumulated in FP64: the gradient
+ * sum of squares the AdamW global-norm clip needs [P1 FP8 训练主路径图 (unscale and clip before
+ * the optimizer); P1 Fused Optimizer 的意义 (read the gradient once)], formed while the wgrad
+ * output is still on chip. The summation order is fixed (per-warp partials in a workspace, then
+ * one pass in index order), so S is the same on every run; it may differ from a sequential
+ * FP64 sum in the last bits.
+ *   sumsq_of        HOST array of n_gemms int32: nonzero = include this problem's D.
+ *   d_sumsq_out     1 double (device), overwritten; NaN if a bounded wait of the call expired.
+ *   d_workspace     device scratch of fp8_gemm_sumsq_workspace_bytes() bytes, 256-byte aligned,
+ *                   ZERO-FILLED before its first use (it holds a ticket counter that every call
+ *                   leaves at zero). Calls that may run at the same time need their own.
+ * Errors as in fp8_gemm_multi, plus FP8T_ERR_INVALID_ARG for NULL/misaligned S or workspace,
+ * no selected problem, or a workspace that is too small.
+ */
+fp8t_status fp8_gemm_multi_sumsq(const fp8t_gemm_desc* gemms, int32_t n_gemms,
+                                 const int32_t* sumsq_of, double* d_sumsq_out, void* d_workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/* Scratch bytes fp8_gemm_multi_sumsq needs (0 on invalid input or no selected problem). */
+size_t fp8_gemm_sumsq_workspace_bytes(const fp8t_gemm_desc* gemms, int32_t n_gemms,
+                                      const int32_t* sumsq_of);
 
 /*
  * fp8_scale_update — roll each tensor's amax history and compute the next scale
@@ -244,6 +304,49 @@ fp8t_status fused_adamw_multi_tensor(const fp8t_adamw_tensor* tensors, int32_t n
 
 /* Scratch bytes fused_adamw_multi_tensor needs for these tensors (0 on invalid input). */
 size_t fused_adamw_workspace_bytes(const fp8t_adamw_tensor* tensors, int32_t n_tensors);
+
+/*
+ * The FP8 cast of a tensor's NEW BF16 weight, done by the AdamW update that produces it: the
+ * cast of fp8_cast_transpose_amax applied to weight_bf16 viewed as rows x cols (row-major),
+ * with the same element rule, outputs and amax accumulation. Under delayed scaling the scale
+ * for the next step's weight cast is known once the scale update of the current step has run,
+ * so the next step need not read the weight again [P1 优化器 kernel 的带宽账: every extra
+ * kernel re-reads the parameters; P3 核心原理: delayed scaling uses the previous scale].
+ * rows = cols = 0 means no cast for this tensor.
+ */
+typedef struct fp8t_adamw_cast {
+    int64_t rows, cols;             /* rows*cols == numel, multiples of 16 (or both 0)        */
+    fp8t_format fmt;
+    const float* d_scale;           /* 1 float: the scale of the next step's weight cast       */
+    void* q_rowmajor;               /* rows x cols FP8 bytes, or NULL                          */
+    void* q_transposed;             /* cols x rows FP8 bytes, or NULL                          */
+    float* d_amax_inout;            /* max-accumulated with max|new weight|                    */
+    float* d_scale_inv_out;         /* 1/scale, or NULL                                        */
+} fp8t_adamw_cast;
+
+/*
+ * fused_adamw_multi_tensor_presummed — fused_adamw_multi_tensor without its norm pass: the sum
+ * of f32(g)^2 over all gradients is read from *d_grad_sumsq (for example from
+ * fp8_gemm_multi_sumsq over the wgrad problems that produced them), so each gradient is read
+ * once, by the update itself [P1 Fused Optimizer 的意义; 优化器 kernel 的带宽账]. Everything else,
+ * including the skip on a non-finite norm, is as in fused_adamw_multi_tensor.
+ *   casts           NULL, or a HOST array of n_tensors fp8t_adamw_cast: the tensors with
+ *                   rows > 0 also get their new weight cast. On a skipped step their weight is
+ *                   left unchanged and cast again with the given scale, so codes, amax and
+ *                   scale inverse always describe the weight the next step uses.
+ *   d_grad_sumsq    1 double (device), read.
+ *   d_ticket        1 device uint32, zero before the first call and left zero; needed when
+ *                   d_step_inout is given (the counter is advanced by the CTA that finishes
+ *                   last), may be NULL otherwise. Concurrent calls need their own.
+ */
+fp8t_status fused_adamw_multi_tensor_presummed(const fp8t_adamw_tensor* tensors,
+                                               const fp8t_adamw_cast* casts, int32_t n_tensors,
+                                               float lr, float beta1, float beta2, float eps,
+                                               float weight_decay, int64_t step,
+                                               int64_t* d_step_inout, float loss_scale,
+                                               float max_grad_norm, const double* d_grad_sumsq,
+                                               float* d_grad_norm_out, int32_t* d_skipped_out,
+                                               unsigned int* d_ticket, void* stream);
 
 /* Size of the scratch array built into the library for fused_adamw_multi_tensor_noalloc. */
 #define FP8T_NOALLOC_SCRATCH_BYTES 65536

@@ -13,8 +13,11 @@ import torch
 
 from . import _abi
 
-__all__ = ["fp8_cast_transpose_amax", "fp8_cast_transpose_amax_multi", "fp8_gemm", "fp8_gemm_multi", "fp8_scale_update", "fused_adamw_multi_tensor",
+__all__ = ["fp8_cast_transpose_amax", "fp8_cast_transpose_amax_multi",
+           "fp8_cast_transpose_amax_update_multi", "fp8_gemm", "fp8_gemm_multi", "fp8_scale_update", "fused_adamw_multi_tensor",
            "fused_adamw_workspace_bytes", "fused_adamw_multi_tensor_noalloc",
+           "fp8_gemm_multi_sumsq", "fp8_gemm_sumsq_workspace_bytes",
+           "fused_adamw_multi_tensor_presummed",
            "fp8t_check_device_error", "fp8t_debug_expire_waits", "fp8t_set_wait_timeout_ns",
            "Fp8TrainError", "E4M3", "E5M2", "AMAX_MAX", "AMAX_MOST_RECENT", "FP8_MAX", "load",
            "LIB_PATH"]
@@ -80,18 +83,41 @@ def fp8_cast_transpose_amax(x, fmt, scale, q=None, qT=None, amax=None, scale_inv
                                           _stream(stream)), "fp8_cast_transpose_amax")
 
 
+def _cast_array(casts):
+    arr = (_abi.CastTensor * len(casts))()
+    for i, c in enumerate(casts):
+        x = c["x"]                  # None: a scale-update-only entry (update call only)
+        assert x is None or (x.dtype == torch.bfloat16 and x.dim() == 2)
+        rows, cols = (0, 0) if x is None else x.shape
+        arr[i] = _abi.CastTensor(_ptr(x), rows, cols, int(c["fmt"]), _ptr(c["scale"]),
+                                 _ptr(c.get("q")), _ptr(c.get("qT")), _ptr(c.get("amax")),
+                                 _ptr(c.get("scale_inv")), _ptr(c.get("counters")))
+    return arr
+
+
 def fp8_cast_transpose_amax_multi(casts, stream=None):
     """Several casts in one launch. ``casts`` is a list of dicts with the keyword arguments of
     fp8_cast_transpose_amax (x, fmt, scale and optionally q, qT, amax, scale_inv, counters)."""
-    arr = (_abi.CastTensor * len(casts))()
-    for i, c in enumerate(casts):
-        x = c["x"]
-        assert x.dtype == torch.bfloat16 and x.dim() == 2
-        arr[i] = _abi.CastTensor(_ptr(x), x.shape[0], x.shape[1], int(c["fmt"]), _ptr(c["scale"]),
-                                 _ptr(c.get("q")), _ptr(c.get("qT")), _ptr(c.get("amax")),
-                                 _ptr(c.get("scale_inv")), _ptr(c.get("counters")))
-    _check(load().fp8_cast_transpose_amax_multi(arr, len(casts), _stream(stream)),
+    _check(load().fp8_cast_transpose_amax_multi(_cast_array(casts), len(casts), _stream(stream)),
            "fp8_cast_transpose_amax_multi")
+
+
+def fp8_cast_transpose_amax_update_multi(casts, updates, algo, margin, ticket, stream=None):
+    """The casts of fp8_cast_transpose_amax_multi and, in the same launch, the scale update of
+    those tensors: ``updates[i]`` holds ``history`` (this tensor's [H] float32 row, entry 0
+    newest) and ``scale_inv_next`` (1 float32, distinct from the cast's ``scale_inv``); the next
+    scale is written into ``casts[i]["scale"]``. ``ticket``: one zeroed int32 on the device."""
+    assert len(updates) == len(casts) and ticket.dtype == torch.int32
+    H = updates[0]["history"].numel()
+    arr = (_abi.CastUpdate * len(updates))()
+    for i, u in enumerate(updates):
+        h = u["history"]
+        assert h.dtype == torch.float32 and h.numel() == H and h.is_contiguous()
+        arr[i] = _abi.CastUpdate(_ptr(h), _ptr(u["scale_inv_next"]))
+    _check(load().fp8_cast_transpose_amax_update_multi(_cast_array(casts), arr, len(casts), H,
+                                                       int(algo), int(margin), _ptr(ticket),
+                                                       _stream(stream)),
+           "fp8_cast_transpose_amax_update_multi")
 
 
 def fp8_gemm(A, a_fmt, B, b_fmt, a_scale_inv, b_scale_inv, D, stream=None):
@@ -103,9 +129,7 @@ def fp8_gemm(A, a_fmt, B, b_fmt, a_scale_inv, b_scale_inv, D, stream=None):
                            _ptr(b_scale_inv), _ptr(D), _stream(stream)), "fp8_gemm")
 
 
-def fp8_gemm_multi(gemms, stream=None):
-    """Several GEMMs in one persistent launch. ``gemms`` is a list of dicts with the arguments of
-    fp8_gemm: A, a_fmt, B, b_fmt, a_scale_inv, b_scale_inv, D."""
+def _gemm_array(gemms):
     arr = (_abi.GemmDesc * len(gemms))()
     for i, g in enumerate(gemms):
         A, B, D = g["A"], g["B"], g["D"]
@@ -114,7 +138,34 @@ def fp8_gemm_multi(gemms, stream=None):
         assert K == K2 and D.shape == (M, N) and D.dtype == torch.bfloat16
         arr[i] = _abi.GemmDesc(_ptr(A), int(g["a_fmt"]), _ptr(B), int(g["b_fmt"]), M, N, K,
                                _ptr(g["a_scale_inv"]), _ptr(g["b_scale_inv"]), _ptr(D))
-    _check(load().fp8_gemm_multi(arr, len(gemms), _stream(stream)), "fp8_gemm_multi")
+    return arr
+
+
+def fp8_gemm_sumsq_workspace_bytes(gemms):
+    """Scratch bytes of fp8_gemm_multi_sumsq for these problems (dicts with a ``sumsq`` flag)."""
+    flags = (C.c_int32 * len(gemms))(*[1 if g.get("sumsq") else 0 for g in gemms])
+    arr = (_abi.GemmDesc * len(gemms))()                 # only the shapes are read
+    for i, g in enumerate(gemms):
+        arr[i].M, arr[i].K = g["A"].shape
+        arr[i].N = g["B"].shape[0]
+    return int(load().fp8_gemm_sumsq_workspace_bytes(arr, len(gemms), flags))
+
+
+def fp8_gemm_multi_sumsq(gemms, sumsq_out, workspace, stream=None):
+    """fp8_gemm_multi that also writes into ``sumsq_out`` (float64 [1]) the FP64 sum of f32(D)^2
+    over the problems whose dict has ``sumsq=True``. ``workspace``: uint8 CUDA tensor of
+    fp8_gemm_sumsq_workspace_bytes, zero-filled once before its first use."""
+    flags = (C.c_int32 * len(gemms))(*[1 if g.get("sumsq") else 0 for g in gemms])
+    assert sumsq_out.dtype == torch.float64
+    _check(load().fp8_gemm_multi_sumsq(_gemm_array(gemms), len(gemms), flags, _ptr(sumsq_out),
+                                       _ptr(workspace), workspace.numel(), _stream(stream)),
+           "fp8_gemm_multi_sumsq")
+
+
+def fp8_gemm_multi(gemms, stream=None):
+    """Several GEMMs in one persistent launch. ``gemms`` is a list of dicts with the arguments of
+    fp8_gemm: A, a_fmt, B, b_fmt, a_scale_inv, b_scale_inv, D."""
+    _check(load().fp8_gemm_multi(_gemm_array(gemms), len(gemms), _stream(stream)), "fp8_gemm_multi")
 
 
 def fp8_scale_update(amax, history, fp8_max, algo, margin, scale, scale_inv, stream=None):
@@ -167,6 +218,34 @@ def fused_adamw_multi_tensor(master, m, v, grads, weights, *, lr, beta1, beta2, 
                                            _ptr(grad_norm), _ptr(skipped), _ptr(workspace),
                                            workspace.numel(), _stream(stream)),
            "fused_adamw_multi_tensor")
+
+
+def fused_adamw_multi_tensor_presummed(master, m, v, grads, weights, *, lr, beta1, beta2, eps,
+                                       weight_decay, step, loss_scale, max_grad_norm, grad_sumsq,
+                                       grad_norm=None, skipped=None, step_counter=None,
+                                       ticket=None, casts=None, stream=None):
+    """The AdamW step without its norm pass: ``grad_sumsq`` (float64 [1] on the device) holds
+    the FP64 sum of f32(g)^2 over all gradients. ``ticket`` (zeroed int32 [1]) is required with
+    ``step_counter``. ``casts``: None, or one entry per tensor, None or a dict (rows, cols, fmt,
+    scale, and optionally q, qT, amax, scale_inv) to cast that tensor's new BF16 weight."""
+    arr, n = _tensor_table(master, m, v, grads, weights)
+    assert grad_sumsq.dtype == torch.float64
+    carr = None
+    if casts is not None:
+        assert len(casts) == n
+        carr = (_abi.AdamWCast * n)()
+        for i, c in enumerate(casts):
+            if c is not None:
+                carr[i] = _abi.AdamWCast(int(c["rows"]), int(c["cols"]), int(c["fmt"]),
+                                         _ptr(c["scale"]), _ptr(c.get("q")), _ptr(c.get("qT")),
+                                         _ptr(c.get("amax")), _ptr(c.get("scale_inv")))
+    _check(load().fused_adamw_multi_tensor_presummed(arr, carr, n, float(lr), float(beta1), float(beta2),
+                                                     float(eps), float(weight_decay), int(step),
+                                                     _ptr(step_counter), float(loss_scale),
+                                                     float(max_grad_norm), _ptr(grad_sumsq),
+                                                     _ptr(grad_norm), _ptr(skipped), _ptr(ticket),
+                                                     _stream(stream)),
+           "fused_adamw_multi_tensor_presummed")
 
 
 def fused_adamw_multi_tensor_noalloc(master, m, v, grads, weights, *, lr, beta1, beta2, eps,

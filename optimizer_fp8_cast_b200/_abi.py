@@ -16,12 +16,24 @@ class AdamWTensor(C.Structure):
                 ("grad_bf16", C.c_void_p), ("weight_bf16", C.c_void_p), ("numel", C.c_int64)]
 
 
+class AdamWCast(C.Structure):
+    """fp8t_adamw_cast."""
+    _fields_ = [("rows", C.c_int64), ("cols", C.c_int64), ("fmt", C.c_int), ("d_scale", C.c_void_p),
+                ("q_rowmajor", C.c_void_p), ("q_transposed", C.c_void_p),
+                ("d_amax_inout", C.c_void_p), ("d_scale_inv_out", C.c_void_p)]
+
+
 class CastTensor(C.Structure):
     """fp8t_cast_tensor."""
     _fields_ = [("x_bf16", C.c_void_p), ("rows", C.c_int64), ("cols", C.c_int64),
                 ("fmt", C.c_int), ("d_scale", C.c_void_p), ("q_rowmajor", C.c_void_p),
                 ("q_transposed", C.c_void_p), ("d_amax_inout", C.c_void_p),
                 ("d_scale_inv_out", C.c_void_p), ("d_counters", C.c_void_p)]
+
+
+class CastUpdate(C.Structure):
+    """fp8t_cast_update."""
+    _fields_ = [("d_amax_history", C.c_void_p), ("d_scale_inv_next", C.c_void_p)]
 
 
 class GemmDesc(C.Structure):
@@ -37,8 +49,21 @@ def declare(L):
     L.fp8_cast_transpose_amax.argtypes = [vp, i64, i64, C.c_int, vp, vp, vp, vp, vp, vp, vp]
     L.fp8_cast_transpose_amax_multi.restype = C.c_int
     L.fp8_cast_transpose_amax_multi.argtypes = [C.POINTER(CastTensor), i32, vp]
+    L.fp8_cast_transpose_amax_update_multi.restype = C.c_int
+    L.fp8_cast_transpose_amax_update_multi.argtypes = [C.POINTER(CastTensor), C.POINTER(CastUpdate),
+                                                       i32, i32, C.c_int, i32, vp, vp]
     L.fp8_gemm_multi.restype = C.c_int
     L.fp8_gemm_multi.argtypes = [C.POINTER(GemmDesc), i32, vp]
+    L.fp8_gemm_multi_sumsq.restype = C.c_int
+    L.fp8_gemm_multi_sumsq.argtypes = [C.POINTER(GemmDesc), i32, C.POINTER(C.c_int32), vp, vp,
+                                       C.c_size_t, vp]
+    L.fp8_gemm_sumsq_workspace_bytes.restype = C.c_size_t
+    L.fp8_gemm_sumsq_workspace_bytes.argtypes = [C.POINTER(GemmDesc), i32, C.POINTER(C.c_int32)]
+    L.fused_adamw_multi_tensor_presummed.restype = C.c_int
+    L.fused_adamw_multi_tensor_presummed.argtypes = [C.POINTER(AdamWTensor), C.POINTER(AdamWCast),
+                                                     i32, f32, f32, f32,
+                                                     f32, f32, i64, vp, f32, f32, vp, vp, vp, vp,
+                                                     vp]
     L.fp8_gemm.restype = C.c_int
     L.fp8_gemm.argtypes = [vp, C.c_int, vp, C.c_int, i64, i64, i64, vp, vp, vp, vp]
     L.fp8_scale_update.restype = C.c_int

@@ -15,11 +15,16 @@
 //   * the transposing pass gathers 16 x 4-byte blocks from the staged tile (conflict-free),
 //     transposes 4 x 4 byte blocks with byte permutes and writes the 128 x 128 q^T tile to shared
 //     memory, which thread 0 stores with one TMA bulk tensor store (clipped at the tensor edge);
-//   * amax and counters are reduced per tile (warp reductions, one atomic per tile).
+//   * amax and counters are reduced per tile (warp reductions, one atomic per tile);
+//   * optionally the CTA that finishes last (a ticket counter) performs the delayed-scaling
+//     update of every tensor of the launch, one warp per tensor: history roll, next scale and
+//     its inverse, amax slot reset (the same arithmetic as the scale-update kernel). Every read
+//     of a tensor's scale and every amax atomic happened before the ticket was taken.
 // Algorithmic traffic: 2 B read + 2 B written per element.
 #pragma once
 
 #include "ptx.cuh"
+#include "scale_update.cuh"
 
 namespace fp8t {
 namespace cast {
@@ -34,9 +39,11 @@ constexpr int kSmemBytes = 2 * kInBytes + 2 * kQBytes + 1024 /*alignment*/ + 64 
 struct alignas(64) Tensor {
   CUtensorMap x_map;               // BF16 [rows][cols], 128 x 128 boxes
   CUtensorMap qt_map;              // FP8 [cols][rows] (q^T), 128 x 128 boxes
-  const float* scale;
+  float* scale;                    // read by the cast; replaced by the next scale when updating
   unsigned int* amax_bits;
   float* scale_inv;
+  float* hist;                     // update only: [H] history, entry 0 newest
+  float* scale_inv_next;           // update only: 1 / next scale
   unsigned long long* counters;    // may be null
   uint8_t* q;                      // row-major FP8 output, may be null
   int64_t rows, cols, tiles_c, tile_start;
@@ -47,6 +54,8 @@ struct alignas(64) Group {
   Tensor t[kMaxTensors];
   int32_t n;
   int64_t total_tiles;
+  unsigned int* ticket;            // update only: zero on entry, left zero
+  int32_t update, H, algo_max, margin;
 };
 
 __device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) { return __reduce_max_sync(0xffffffffu, v); }
@@ -275,6 +284,26 @@ __global__ void __launch_bounds__(kThreads, 2) k_cast_transpose_amax(const __gri
       if (pending & (1u << b)) mbar_wait(smem_u32(&full[b]), (pending_ph >> b) & 1u, kDrainLimitNs);
     bulk_wait_group<0>();                          // stores complete before the CTA exits
   }
+  if (!g.update) return;
+
+  // ---- the last CTA to finish updates the scale state of every tensor of the launch
+  __shared__ int s_last;
+  if (tid == 0) {
+    __threadfence();                               // this CTA's amax atomics before its ticket
+    s_last = atomicAdd(g.ticket, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // a launch whose waits expired leaves the scale state alone (its amax may be incomplete)
+  const bool ok = *reinterpret_cast<volatile unsigned int*>(&g_error_word) == 0u;
+  if (ok && warp < g.n) {
+    const Tensor& T = g.t[warp];
+    scale::warp_update(reinterpret_cast<float*>(T.amax_bits), T.hist, g.H,
+                       T.fmt == 0 ? 448.0f : 57344.0f, g.algo_max != 0, g.margin, T.scale,
+                       T.scale_inv_next);
+  }
+  if (tid == 0) atomicExch(g.ticket, 0u);
 }
 
 }  // namespace cast

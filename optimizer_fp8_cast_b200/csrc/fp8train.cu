@@ -41,6 +41,7 @@ struct DeviceInfo {
   int state = 0;               // 0 unknown, 1 sm_100, 2 other
   int sms = 0;
   int adamw_blocks_per_sm = 0;
+  int adamw_cast_blocks_per_sm = 0;
   int gemm_clusters = 0;       // co-resident 2-CTA clusters of the GEMM kernel
   int cast_blocks_per_sm = 0;
   void* noalloc_scratch = nullptr;   // device address of g_adamw_noalloc_scratch
@@ -66,9 +67,13 @@ fp8t_status current_device(DeviceInfo** out) {
     d.state = (major == 10 && minor == 0) ? 1 : 2;
     if (d.state == 1) {
       e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.adamw_blocks_per_sm,
-                                                        fp8t::adamw::k_adamw_update,
+                                                        fp8t::adamw::k_adamw_update<false>,
                                                         fp8t::adamw::kThreads, 0);
       if (e != cudaSuccess || d.adamw_blocks_per_sm < 1) d.adamw_blocks_per_sm = 1;
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.adamw_cast_blocks_per_sm,
+                                                        fp8t::adamw::k_adamw_update<true>,
+                                                        fp8t::adamw::kThreads, 0);
+      if (e != cudaSuccess || d.adamw_cast_blocks_per_sm < 1) d.adamw_cast_blocks_per_sm = 1;
       e = cudaFuncSetAttribute(fp8t::gemm::k_fp8_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                fp8t::gemm::kSmemBytes);
       if (e != cudaSuccess) {
@@ -202,13 +207,45 @@ const char* fp8t_status_string(fp8t_status s) {
 }
 
 // ------------------------------------------------------------------ cast / transpose / amax
-fp8t_status fp8_cast_transpose_amax_multi(const fp8t_cast_tensor* tensors, int32_t n_tensors,
-                                          void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Casts of n tensors in launches of up to eight; with `updates`, the last CTA of each launch also
+// performs the delayed-scaling update of that launch's tensors.
+fp8t_status cast_multi(const fp8t_cast_tensor* tensors, const fp8t_cast_update* updates,
+                       int32_t n_tensors, int32_t history_len, fp8t_amax_algo algo, int32_t margin,
+                       unsigned int* d_ticket, void* stream) {
   t_last_error.clear();
   if (!tensors || n_tensors < 1 || n_tensors > 4096)
     return fail(FP8T_ERR_INVALID_ARG, "fp8_cast_transpose_amax: tensors NULL or n_tensors out of range");
+  if (updates) {
+    if (!d_ticket || !aligned(d_ticket, 4))
+      return fail(FP8T_ERR_INVALID_ARG, "fp8_cast_transpose_amax_update: NULL or misaligned ticket");
+    if (history_len < 1 || history_len > 65536)
+      return fail(FP8T_ERR_INVALID_ARG, "fp8_cast_transpose_amax_update: history_len in 1..65536");
+    if (algo != FP8T_AMAX_MAX && algo != FP8T_AMAX_MOST_RECENT)
+      return fail(FP8T_ERR_INVALID_ARG, "fp8_cast_transpose_amax_update: unknown amax algorithm %d", (int)algo);
+    if (margin < 0 || margin > 126)
+      return fail(FP8T_ERR_INVALID_ARG, "fp8_cast_transpose_amax_update: margin in 0..126");
+    for (int32_t i = 0; i < n_tensors; ++i) {
+      const fp8t_cast_update& u = updates[i];
+      if (!u.d_amax_history || !u.d_scale_inv_next)
+        return fail(FP8T_ERR_INVALID_ARG, "fp8_cast_transpose_amax_update: tensor %d: NULL history or scale_inv_next", i);
+      if (!aligned(u.d_amax_history, 4) || !aligned(u.d_scale_inv_next, 4))
+        return fail(FP8T_ERR_MISALIGNED, "fp8_cast_transpose_amax_update: tensor %d: misaligned pointer", i);
+      if (u.d_scale_inv_next == tensors[i].d_scale_inv_out)
+        return fail(FP8T_ERR_INVALID_ARG,
+                    "fp8_cast_transpose_amax_update: tensor %d: scale_inv_next must differ from the cast's scale_inv_out", i);
+    }
+  }
   for (int32_t i = 0; i < n_tensors; ++i) {
     const fp8t_cast_tensor& t = tensors[i];
+    if (updates && !t.x_bf16 && t.rows == 0 && t.cols == 0 && !t.q_rowmajor && !t.q_transposed &&
+        !t.d_counters && t.d_scale && t.d_amax_inout && aligned(t.d_scale, 4) &&
+        aligned(t.d_amax_inout, 4) && aligned(t.d_scale_inv_out, 4) &&
+        (t.fmt == FP8T_E4M3 || t.fmt == FP8T_E5M2))
+      continue;                       // scale update only: the amax was accumulated elsewhere
     if (!t.x_bf16 || !t.d_scale || !t.d_amax_inout)
       return fail(FP8T_ERR_INVALID_ARG, "fp8_cast_transpose_amax: tensor %d: NULL input, scale or amax pointer", i);
     if (t.fmt != FP8T_E4M3 && t.fmt != FP8T_E5M2)
@@ -240,7 +277,7 @@ fp8t_status fp8_cast_transpose_amax_multi(const fp8t_cast_tensor* tensors, int32
     for (int32_t i = b0; i < b1; ++i) {
       const fp8t_cast_tensor& t = tensors[i];
       Tensor& T = group.t[i - b0];
-      {
+      if (t.x_bf16) {
         cuuint64_t dims[2] = {static_cast<cuuint64_t>(t.cols), static_cast<cuuint64_t>(t.rows)};
         cuuint64_t strides[1] = {static_cast<cuuint64_t>(t.cols) * 2};
         cuuint32_t box[2] = {kTile, kTile};
@@ -261,9 +298,13 @@ fp8t_status fp8_cast_transpose_amax_multi(const fp8t_cast_tensor* tensors, int32
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return fail(FP8T_ERR_CUDA, "cuTensorMapEncodeTiled (q^T store) failed (%d)", (int)r);
       }
-      T.scale = t.d_scale;
+      T.scale = const_cast<float*>(t.d_scale);      // written only by the update
       T.amax_bits = reinterpret_cast<unsigned int*>(t.d_amax_inout);
       T.scale_inv = t.d_scale_inv_out;
+      if (updates) {
+        T.hist = updates[i].d_amax_history;
+        T.scale_inv_next = updates[i].d_scale_inv_next;
+      }
       T.counters = t.d_counters;
       T.q = static_cast<uint8_t*>(t.q_rowmajor);
       T.rows = t.rows;
@@ -275,9 +316,17 @@ fp8t_status fp8_cast_transpose_amax_multi(const fp8t_cast_tensor* tensors, int32
       tiles += ((t.rows + kTile - 1) / kTile) * T.tiles_c;
     }
     group.total_tiles = tiles;
+    if (updates) {
+      group.update = 1;
+      group.ticket = d_ticket;
+      group.H = history_len;
+      group.algo_max = algo == FP8T_AMAX_MAX ? 1 : 0;
+      group.margin = margin;
+    }
     bool count = false;
     for (int32_t i = b0; i < b1; ++i) count |= tensors[i].d_counters != nullptr;
-    const int64_t grid = std::min<int64_t>(tiles, static_cast<int64_t>(dev->sms) * dev->cast_blocks_per_sm);
+    int64_t grid = std::min<int64_t>(tiles, static_cast<int64_t>(dev->sms) * dev->cast_blocks_per_sm);
+    if (grid < 1) grid = 1;           // update-only entries: one CTA does the update
     if (count)
       k_cast_transpose_amax<true><<<static_cast<unsigned>(grid), kThreads, kSmemBytes, as_stream(stream)>>>(group);
     else
@@ -285,6 +334,27 @@ fp8t_status fp8_cast_transpose_amax_multi(const fp8t_cast_tensor* tensors, int32
     if ((st = after_launch("fp8_cast_transpose_amax launch")) != FP8T_OK) return st;
   }
   return FP8T_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+fp8t_status fp8_cast_transpose_amax_multi(const fp8t_cast_tensor* tensors, int32_t n_tensors,
+                                          void* stream) {
+  return cast_multi(tensors, nullptr, n_tensors, 0, FP8T_AMAX_MAX, 0, nullptr, stream);
+}
+
+fp8t_status fp8_cast_transpose_amax_update_multi(const fp8t_cast_tensor* tensors,
+                                                 const fp8t_cast_update* updates, int32_t n_tensors,
+                                                 int32_t history_len, fp8t_amax_algo algo,
+                                                 int32_t margin, unsigned int* d_ticket,
+                                                 void* stream) {
+  if (!updates) {
+    t_last_error.clear();
+    return fail(FP8T_ERR_INVALID_ARG, "fp8_cast_transpose_amax_update: updates NULL");
+  }
+  return cast_multi(tensors, updates, n_tensors, history_len, algo, margin, d_ticket, stream);
 }
 
 fp8t_status fp8_cast_transpose_amax(const void* x_bf16, int64_t rows, int64_t cols, fp8t_format fmt,
@@ -297,7 +367,27 @@ fp8t_status fp8_cast_transpose_amax(const void* x_bf16, int64_t rows, int64_t co
 }
 
 // ------------------------------------------------------------------ GEMM
-fp8t_status fp8_gemm_multi(const fp8t_gemm_desc* gemms, int32_t n_gemms, void* stream) {
+}  // extern "C"
+
+namespace {
+
+constexpr size_t kSumsqHeader = 256;    // ticket, then the partial slots
+
+int64_t gemm_tiles(const fp8t_gemm_desc& d) {
+  using namespace fp8t::gemm;
+  return ((d.M + kBM - 1) / kBM) * ((d.N + kBN - 1) / kBN);
+}
+
+int64_t sumsq_slots(const fp8t_gemm_desc* gemms, int32_t n, const int32_t* sumsq_of) {
+  int64_t slots = 0;
+  for (int32_t i = 0; i < n; ++i)
+    if (sumsq_of[i]) slots += gemm_tiles(gemms[i]) * fp8t::gemm::kSumsqPerTile;
+  return slots;
+}
+
+fp8t_status gemm_multi(const fp8t_gemm_desc* gemms, int32_t n_gemms, const int32_t* sumsq_of,
+                       double* d_sumsq_out, void* d_workspace, size_t workspace_bytes,
+                       void* stream) {
   t_last_error.clear();
   if (!gemms || n_gemms < 1 || n_gemms > 4096)
     return fail(FP8T_ERR_INVALID_ARG, "fp8_gemm: gemms NULL or n_gemms out of range");
@@ -316,6 +406,17 @@ fp8t_status fp8_gemm_multi(const fp8t_gemm_desc* gemms, int32_t n_gemms, void* s
         !aligned(d.d_a_scale_inv, 4) || !aligned(d.d_b_scale_inv, 4))
       return fail(FP8T_ERR_MISALIGNED, "fp8_gemm: problem %d: misaligned pointer", i);
   }
+  int64_t n_slots = 0;
+  if (sumsq_of) {
+    if (!d_sumsq_out || !aligned(d_sumsq_out, 8) || !d_workspace || !aligned(d_workspace, 256))
+      return fail(FP8T_ERR_INVALID_ARG, "fp8_gemm_multi_sumsq: NULL or misaligned sumsq_out or workspace");
+    n_slots = sumsq_slots(gemms, n_gemms, sumsq_of);
+    if (n_slots < 1 || n_slots >= (int64_t(1) << 31))
+      return fail(FP8T_ERR_INVALID_ARG, "fp8_gemm_multi_sumsq: no problem (or too many tiles) selected");
+    const size_t need = kSumsqHeader + static_cast<size_t>(n_slots) * 8;
+    if (workspace_bytes < need)
+      return fail(FP8T_ERR_INVALID_ARG, "fp8_gemm_multi_sumsq: workspace of %zu bytes needed", need);
+  }
   DeviceInfo* dev = nullptr;
   fp8t_status st = current_device(&dev);
   if (st != FP8T_OK) return st;
@@ -324,10 +425,18 @@ fp8t_status fp8_gemm_multi(const fp8t_gemm_desc* gemms, int32_t n_gemms, void* s
 
   using namespace fp8t::gemm;
   static thread_local Group group;
+  int64_t slot = 0;
   for (int32_t b0 = 0; b0 < n_gemms; b0 += kMaxProblems) {
     const int32_t b1 = std::min<int32_t>(n_gemms, b0 + kMaxProblems);
     std::memset(&group, 0, sizeof(group));
     group.n = b1 - b0;
+    if (sumsq_of) {
+      group.ticket = static_cast<unsigned int*>(d_workspace);
+      group.partials = reinterpret_cast<double*>(static_cast<char*>(d_workspace) + kSumsqHeader);
+      group.sumsq_out = d_sumsq_out;
+      group.n_partials = static_cast<int32_t>(n_slots);
+      group.last_launch = b1 == n_gemms ? 1 : 0;
+    }
     int64_t tiles = 0;
     for (int32_t i = b0; i < b1; ++i) {
       const fp8t_gemm_desc& d = gemms[i];
@@ -351,6 +460,11 @@ fp8t_status fp8_gemm_multi(const fp8t_gemm_desc* gemms, int32_t n_gemms, void* s
       P.idesc = make_idesc(d.a_fmt, d.b_fmt);
       P.tiles_n = static_cast<int32_t>((d.N + kBN - 1) / kBN);
       P.tile_start = static_cast<int32_t>(tiles);
+      P.sumsq_slot = -1;
+      if (sumsq_of && sumsq_of[i]) {
+        P.sumsq_slot = static_cast<int32_t>(slot);
+        slot += gemm_tiles(d) * kSumsqPerTile;
+      }
       tiles += ((d.M + kBM - 1) / kBM) * P.tiles_n;            // 256 x 256 tiles, one per pair
       if (tiles >= (int64_t(1) << 30))
         return fail(FP8T_ERR_UNSUPPORTED_SHAPE, "fp8_gemm: too many tiles in one launch");
@@ -361,6 +475,34 @@ fp8t_status fp8_gemm_multi(const fp8t_gemm_desc* gemms, int32_t n_gemms, void* s
     if ((st = after_launch("fp8_gemm launch")) != FP8T_OK) return st;
   }
   return FP8T_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+fp8t_status fp8_gemm_multi(const fp8t_gemm_desc* gemms, int32_t n_gemms, void* stream) {
+  return gemm_multi(gemms, n_gemms, nullptr, nullptr, nullptr, 0, stream);
+}
+
+size_t fp8_gemm_sumsq_workspace_bytes(const fp8t_gemm_desc* gemms, int32_t n_gemms,
+                                      const int32_t* sumsq_of) {
+  if (!gemms || !sumsq_of || n_gemms < 1 || n_gemms > 4096) return 0;
+  for (int32_t i = 0; i < n_gemms; ++i)
+    if (gemms[i].M <= 0 || gemms[i].N <= 0) return 0;
+  const int64_t slots = sumsq_slots(gemms, n_gemms, sumsq_of);
+  if (slots < 1) return 0;
+  return kSumsqHeader + static_cast<size_t>(slots) * 8;
+}
+
+fp8t_status fp8_gemm_multi_sumsq(const fp8t_gemm_desc* gemms, int32_t n_gemms,
+                                 const int32_t* sumsq_of, double* d_sumsq_out, void* d_workspace,
+                                 size_t workspace_bytes, void* stream) {
+  if (!sumsq_of) {
+    t_last_error.clear();
+    return fail(FP8T_ERR_INVALID_ARG, "fp8_gemm_multi_sumsq: sumsq_of NULL");
+  }
+  return gemm_multi(gemms, n_gemms, sumsq_of, d_sumsq_out, d_workspace, workspace_bytes, stream);
 }
 
 fp8t_status fp8_gemm(const void* A, fp8t_format a_fmt, const void* B, fp8t_format b_fmt, int64_t M,
@@ -402,12 +544,18 @@ size_t fused_adamw_workspace_bytes(const fp8t_adamw_tensor* tensors, int32_t n_t
   return workspace_for(plan_adamw(tensors, n_tensors));
 }
 
-fp8t_status fused_adamw_multi_tensor(const fp8t_adamw_tensor* tensors, int32_t n_tensors, float lr,
-                                     float beta1, float beta2, float eps, float weight_decay,
-                                     int64_t step, int64_t* d_step_inout, float loss_scale,
-                                     float max_grad_norm, float* d_grad_norm_out,
-                                     int32_t* d_skipped_out, void* d_workspace,
-                                     size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The AdamW call; with d_presummed the norm pass is skipped and its sum of squares read there.
+fp8t_status adamw_call(const fp8t_adamw_tensor* tensors, const fp8t_adamw_cast* casts,
+                       int32_t n_tensors, float lr, float beta1,
+                       float beta2, float eps, float weight_decay, int64_t step,
+                       int64_t* d_step_inout, float loss_scale, float max_grad_norm,
+                       float* d_grad_norm_out, int32_t* d_skipped_out, void* d_workspace,
+                       size_t workspace_bytes, const double* d_presummed, unsigned int* d_ticket,
+                       void* stream) {
   t_last_error.clear();
   if (!tensors || n_tensors < 1 || n_tensors > (1 << 20))
     return fail(FP8T_ERR_INVALID_ARG, "fused_adamw_multi_tensor: tensors NULL or n_tensors out of range");
@@ -418,6 +566,23 @@ fp8t_status fused_adamw_multi_tensor(const fp8t_adamw_tensor* tensors, int32_t n
     if (!aligned(t.master, 16) || !aligned(t.m, 16) || !aligned(t.v, 16) ||
         !aligned(t.grad_bf16, 16) || !aligned(t.weight_bf16, 16))
       return fail(FP8T_ERR_MISALIGNED, "fused_adamw_multi_tensor: tensor %d is not 16-byte aligned", i);
+  }
+  if (casts) {
+    for (int32_t i = 0; i < n_tensors; ++i) {
+      const fp8t_adamw_cast& c = casts[i];
+      if (c.rows == 0 && c.cols == 0) continue;                     // no cast for this tensor
+      if (c.rows <= 0 || c.cols <= 0 || c.rows % 16 || c.cols % 16 || c.rows >= (int64_t(1) << 31) ||
+          c.cols >= (int64_t(1) << 31) || c.rows * c.cols != tensors[i].numel)
+        return fail(FP8T_ERR_UNSUPPORTED_SHAPE,
+                    "fused_adamw_multi_tensor_presummed: cast %d: rows x cols must equal numel, multiples of 16", i);
+      if (c.fmt != FP8T_E4M3 && c.fmt != FP8T_E5M2)
+        return fail(FP8T_ERR_INVALID_ARG, "fused_adamw_multi_tensor_presummed: cast %d: unknown format", i);
+      if (!c.d_scale || !c.d_amax_inout)
+        return fail(FP8T_ERR_INVALID_ARG, "fused_adamw_multi_tensor_presummed: cast %d: NULL scale or amax", i);
+      if (!aligned(c.d_scale, 4) || !aligned(c.d_amax_inout, 4) || !aligned(c.d_scale_inv_out, 4) ||
+          !aligned(c.q_rowmajor, 16) || !aligned(c.q_transposed, 16))
+        return fail(FP8T_ERR_MISALIGNED, "fused_adamw_multi_tensor_presummed: cast %d: misaligned pointer", i);
+    }
   }
   if (!d_step_inout && step < 1)
     return fail(FP8T_ERR_INVALID_ARG, "fused_adamw_multi_tensor: step must be >= 1");
@@ -430,8 +595,14 @@ fp8t_status fused_adamw_multi_tensor(const fp8t_adamw_tensor* tensors, int32_t n
     return fail(FP8T_ERR_MISALIGNED, "fused_adamw_multi_tensor: misaligned output or workspace");
   const AdamWPlan plan = plan_adamw(tensors, n_tensors);
   const size_t need = workspace_for(plan);
-  if (!d_workspace || workspace_bytes < need)
+  if (d_presummed) {
+    if (!aligned(d_presummed, 8))
+      return fail(FP8T_ERR_MISALIGNED, "fused_adamw_multi_tensor_presummed: misaligned sum of squares");
+    if (d_step_inout && (!d_ticket || !aligned(d_ticket, 4)))
+      return fail(FP8T_ERR_INVALID_ARG, "fused_adamw_multi_tensor_presummed: a device step counter needs a ticket");
+  } else if (!d_workspace || workspace_bytes < need) {
     return fail(FP8T_ERR_INVALID_ARG, "fused_adamw_multi_tensor: workspace of %zu bytes needed", need);
+  }
   DeviceInfo* dev = nullptr;
   fp8t_status st = current_device(&dev);
   if (st != FP8T_OK) return st;
@@ -444,7 +615,9 @@ fp8t_status fused_adamw_multi_tensor(const fp8t_adamw_tensor* tensors, int32_t n
   k.omb2 = static_cast<float>(1.0 - static_cast<double>(beta2));
   k.decay = static_cast<float>(1.0 - static_cast<double>(lr) * static_cast<double>(weight_decay));
   k.d_step = d_step_inout;
-  k.step_slot = reinterpret_cast<const int64_t*>(static_cast<double*>(d_workspace) + plan.nparts);
+  k.step_slot = d_presummed ? nullptr
+                            : reinterpret_cast<const int64_t*>(static_cast<double*>(d_workspace) + plan.nparts);
+  k.step_ticket = d_ticket;
   k.lr_d = lr;
   k.beta1_d = beta1;
   k.beta2_d = beta2;
@@ -463,19 +636,51 @@ fp8t_status fused_adamw_multi_tensor(const fp8t_adamw_tensor* tensors, int32_t n
 
   cudaStream_t s = as_stream(stream);
   double* partials = static_cast<double*>(d_workspace);
-  static thread_local Batch batch;   // ~14 KB: kept off the stack
+  static thread_local Batch batch;   // ~17 KB: kept off the stack
+  // a batch ends at kMaxTensors tensors or kMaxCasts casts
+  auto has_cast = [&](int32_t i) { return casts && casts[i].rows > 0; };
+  auto batch_end = [&](int32_t b0) {
+    int32_t b1 = b0, nc = 0;
+    while (b1 < n_tensors && b1 - b0 < kMaxTensors) {
+      if (has_cast(b1)) {
+        if (nc == kMaxCasts) break;
+        ++nc;
+      }
+      ++b1;
+    }
+    return b1;
+  };
   int64_t off = 0;
-  for (int pass = 0; pass < 2; ++pass) {
+  for (int pass = d_presummed ? 1 : 0; pass < 2; ++pass) {
     off = 0;
-    for (int32_t b0 = 0, bi = 0; b0 < n_tensors; b0 += kMaxTensors, ++bi) {
-      const int32_t b1 = std::min<int32_t>(n_tensors, b0 + kMaxTensors);
+    for (int32_t b0 = 0, bi = 0, b1 = 0; b0 < n_tensors; b0 = b1, ++bi) {
+      b1 = batch_end(b0);
       batch.n = b1 - b0;
       batch.first = bi == 0 ? 1 : 0;
+      batch.last = b1 == n_tensors ? 1 : 0;
       int64_t acc = 0;
+      int32_t nc = 0;
       for (int32_t i = b0; i < b1; ++i) {
         const int j = i - b0;
         batch.chunk_start[j] = acc;
-        acc += chunks_of(tensors[i].numel);
+        batch.cast_of[j] = -1;
+        if (has_cast(i)) {
+          const fp8t_adamw_cast& c = casts[i];
+          CastInfo& ci = batch.cast[nc];
+          ci.scale = c.d_scale;
+          ci.amax_bits = reinterpret_cast<unsigned int*>(c.d_amax_inout);
+          ci.scale_inv = c.d_scale_inv_out;
+          ci.q = static_cast<uint8_t*>(c.q_rowmajor);
+          ci.qt = static_cast<uint8_t*>(c.q_transposed);
+          ci.rows = c.rows;
+          ci.cols = c.cols;
+          ci.tiles_c = (c.cols + kTileCols - 1) / kTileCols;
+          ci.fmt = c.fmt;
+          batch.cast_of[j] = static_cast<int8_t>(nc++);
+          acc += ((c.rows + kTileRows - 1) / kTileRows) * ci.tiles_c;
+        } else {
+          acc += chunks_of(tensors[i].numel);
+        }
         batch.numel[j] = tensors[i].numel;
         batch.master[j] = tensors[i].master;
         batch.m[j] = tensors[i].m;
@@ -492,14 +697,54 @@ fp8t_status fused_adamw_multi_tensor(const fp8t_adamw_tensor* tensors, int32_t n
         off += grid;
         if ((st = after_launch("adamw norm pass launch")) != FP8T_OK) return st;
       } else {
-        const int64_t grid = std::min<int64_t>(acc, static_cast<int64_t>(dev->sms) * dev->adamw_blocks_per_sm);
-        k_adamw_update<<<static_cast<unsigned>(grid), kThreads, 0, s>>>(
-            batch, k, partials, static_cast<int>(plan.nparts), d_grad_norm_out, d_skipped_out);
+        const double* parts = d_presummed ? d_presummed : partials;
+        const int np = d_presummed ? 1 : static_cast<int>(plan.nparts);
+        if (nc) {
+          const int64_t grid = std::min<int64_t>(acc, static_cast<int64_t>(dev->sms) * dev->adamw_cast_blocks_per_sm);
+          k_adamw_update<true><<<static_cast<unsigned>(grid), kThreads, 0, s>>>(
+              batch, k, parts, np, d_grad_norm_out, d_skipped_out);
+        } else {
+          const int64_t grid = std::min<int64_t>(acc, static_cast<int64_t>(dev->sms) * dev->adamw_blocks_per_sm);
+          k_adamw_update<false><<<static_cast<unsigned>(grid), kThreads, 0, s>>>(
+              batch, k, parts, np, d_grad_norm_out, d_skipped_out);
+        }
         if ((st = after_launch("adamw update launch")) != FP8T_OK) return st;
       }
     }
   }
   return FP8T_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+fp8t_status fused_adamw_multi_tensor(const fp8t_adamw_tensor* tensors, int32_t n_tensors, float lr,
+                                     float beta1, float beta2, float eps, float weight_decay,
+                                     int64_t step, int64_t* d_step_inout, float loss_scale,
+                                     float max_grad_norm, float* d_grad_norm_out,
+                                     int32_t* d_skipped_out, void* d_workspace,
+                                     size_t workspace_bytes, void* stream) {
+  return adamw_call(tensors, nullptr, n_tensors, lr, beta1, beta2, eps, weight_decay, step,
+                    d_step_inout, loss_scale, max_grad_norm, d_grad_norm_out, d_skipped_out,
+                    d_workspace, workspace_bytes, nullptr, nullptr, stream);
+}
+
+fp8t_status fused_adamw_multi_tensor_presummed(const fp8t_adamw_tensor* tensors,
+                                               const fp8t_adamw_cast* casts, int32_t n_tensors,
+                                               float lr, float beta1, float beta2, float eps,
+                                               float weight_decay, int64_t step,
+                                               int64_t* d_step_inout, float loss_scale,
+                                               float max_grad_norm, const double* d_grad_sumsq,
+                                               float* d_grad_norm_out, int32_t* d_skipped_out,
+                                               unsigned int* d_ticket, void* stream) {
+  if (!d_grad_sumsq) {
+    t_last_error.clear();
+    return fail(FP8T_ERR_INVALID_ARG, "fused_adamw_multi_tensor_presummed: d_grad_sumsq NULL");
+  }
+  return adamw_call(tensors, casts, n_tensors, lr, beta1, beta2, eps, weight_decay, step,
+                    d_step_inout, loss_scale, max_grad_norm, d_grad_norm_out, d_skipped_out,
+                    nullptr, 0, d_grad_sumsq, d_ticket, stream);
 }
 
 // Same step as fused_adamw_multi_tensor, with the built-in scratch array as its workspace.

@@ -12,6 +12,15 @@
 //   k_adamw_update  persistent CTAs; each first reduces all workspace slots in a fixed order
 //                   (so every CTA derives the identical norm and clip factor), then streams its
 //                   chunks: 16-byte loads of g (8 BF16) and 2 x 16-byte loads of m, v, p.
+// When the sum of squares was formed elsewhere (the wgrad GEMM's epilogue), k_adamw_update runs
+// alone on that one value; a device step counter is then read by every CTA at its start and
+// advanced by the CTA of the last batch that finishes last (a ticket counter).
+// A tensor may also carry the FP8 cast of its new BF16 weight for the next step (delayed
+// scaling: that step's scale is already known). Such a tensor is walked in 64 x 128 tiles
+// instead of flat chunks: each thread updates 4 x 8 elements, quantises the 8 new BF16 weights
+// (f32 multiply by the scale, cvt.rn.satfinite), stores them row-major and into a shared tile,
+// from which 128 threads write the transposed codes (4 x 4 byte transposes, 16-byte stores);
+// the tile's amax is max-accumulated into the tensor's slot. Same codes as the cast kernel.
 // Traffic: 2 B/param for the norm pass, 28 B/param for the update (g 2 + m, v, p 4 each read,
 // m, v, p 4 each + BF16 weight 2 written).
 // Every f32 operation is an explicit round-to-nearest intrinsic, so no multiply-add is fused.
@@ -27,10 +36,23 @@ constexpr int kThreads = 256;
 constexpr int kVec = 8;                                  // elements per 16-byte BF16 vector
 constexpr int64_t kChunk = 4 * kThreads * kVec;          // 8192 elements per chunk
 constexpr int kSumsqBlocks = 592;
+constexpr int kMaxCasts = 32;                            // weight casts per launch
+constexpr int kTileRows = 64, kTileCols = 128;           // one cast tile = 8192 elements
+
+struct CastInfo {
+  const float* scale;
+  unsigned int* amax_bits;
+  float* scale_inv;                                       // may be null
+  uint8_t* q;                                             // row-major codes, may be null
+  uint8_t* qt;                                            // transposed codes, may be null
+  int64_t rows, cols, tiles_c;
+  int32_t fmt;
+};
 
 struct Batch {
   int32_t n;
   int32_t first;                                          // 1 for the batch that reports
+  int32_t last;                                           // 1 for the last batch of the call
   int64_t chunk_start[kMaxTensors + 1];                   // prefix sums of chunks per tensor
   int64_t numel[kMaxTensors];
   float* master[kMaxTensors];
@@ -38,6 +60,8 @@ struct Batch {
   float* v[kMaxTensors];
   const uint16_t* g[kMaxTensors];
   uint16_t* w[kMaxTensors];
+  int8_t cast_of[kMaxTensors];                            // index into cast, or -1
+  CastInfo cast[kMaxCasts];
 };
 
 struct Scalars {            // host-computed, rounded once to f32 (double where noted)
@@ -47,7 +71,8 @@ struct Scalars {            // host-computed, rounded once to f32 (double where 
   // the norm pass), step_size and bc2_sqrt are formed on the device, and the counter is advanced
   // by the first CTA of the first update launch unless the step is skipped
   int64_t* d_step;
-  const int64_t* step_slot;
+  const int64_t* step_slot;      // null: read the counter itself and advance it by ticket
+  unsigned int* step_ticket;
   double lr_d, beta1_d, beta2_d;
 };
 
@@ -124,6 +149,32 @@ __global__ void __launch_bounds__(kThreads)
   if (threadIdx.x == 0) partials[blockIdx.x] = total;
 }
 
+// 8 BF16 weights (4 words) -> 8 FP8 codes; `mag` receives their largest magnitude bit pattern.
+// NaN products (a NaN weight or a non-finite scale) give the byte 0x7F, as in the cast kernel.
+template <int FMT>
+__device__ __forceinline__ uint2 quant8(const uint32_t (&w)[4], float s, uint32_t& mag) {
+  uint32_t out[2] = {0u, 0u}, m2 = 0u;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    m2 = __vmaxu2(m2, w[j] & 0x7FFF7FFFu);
+    const float p0 = __fmul_rn(__uint_as_float(w[j] << 16), s);
+    const float p1 = __fmul_rn(__uint_as_float(w[j] & 0xFFFF0000u), s);
+    out[j >> 1] |= cvt_fp8x2<FMT>(p0, p1) << (16 * (j & 1));
+  }
+  mag = max(m2 & 0xFFFFu, m2 >> 16);
+  if (mag > 0x7F80u || !isfinite(s)) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float p0 = __fmul_rn(__uint_as_float(w[j] << 16), s);
+      const float p1 = __fmul_rn(__uint_as_float(w[j] & 0xFFFF0000u), s);
+      const int sh = 16 * (j & 1);
+      if (p0 != p0) out[j >> 1] = (out[j >> 1] & ~(0xFFu << sh)) | (0x7Fu << sh);
+      if (p1 != p1) out[j >> 1] = (out[j >> 1] & ~(0xFF00u << sh)) | (0x7F00u << sh);
+    }
+  }
+  return make_uint2(out[0], out[1]);
+}
+
 __device__ __forceinline__ void adam_one(float& p, float& m, float& v, float g, const Scalars& k,
                                          float f) {
   const float gg = __fmul_rn(g, f);
@@ -137,13 +188,111 @@ __device__ __forceinline__ void adam_one(float& p, float& m, float& v, float g, 
   v = vv;
 }
 
-__global__ void __launch_bounds__(kThreads)
+// One 64 x 128 tile of a tensor whose new weight is also cast (see the file comment).
+// With update = false (a skipped step) the weight is left alone and only cast again, so the
+// codes, scale inverse and amax still describe it.
+__device__ __forceinline__ void update_cast_tile(const Batch& b, const CastInfo& ci, int t,
+                                                 int64_t local, const Scalars& kk, float f,
+                                                 bool update, uint32_t* stage, uint32_t* red) {
+  const int tid = threadIdx.x;
+  const int64_t rows = ci.rows, cols = ci.cols;
+  const int64_t r0 = (local / ci.tiles_c) * kTileRows, c0 = (local % ci.tiles_c) * kTileCols;
+  const float s = __ldg(ci.scale);
+  float* __restrict__ P = b.master[t];
+  float* __restrict__ M = b.m[t];
+  float* __restrict__ V = b.v[t];
+  const uint16_t* __restrict__ G = b.g[t];
+  uint16_t* __restrict__ W = b.w[t];
+  uint32_t vmax = 0;
+#pragma unroll 1
+  for (int u = 0; u < 4; ++u) {                      // one 8-element vector at a time
+    const int vec = u * kThreads + tid;
+    const int64_t row = r0 + (vec >> 4), col = c0 + (vec & 15) * 8;
+    if (row >= rows || col >= cols) continue;
+    const int64_t e = row * cols + col;
+    uint32_t wout[4];
+    if (!update) {
+      const uint4 wv = *reinterpret_cast<const uint4*>(W + e);
+      wout[0] = wv.x; wout[1] = wv.y; wout[2] = wv.z; wout[3] = wv.w;
+    } else {
+    const uint4 gv = ld_stream_u4(G + e);
+    float4 mv[2], vv[2], pv[2];
+    mv[0] = __ldcs(reinterpret_cast<const float4*>(M + e));
+    mv[1] = __ldcs(reinterpret_cast<const float4*>(M + e + 4));
+    vv[0] = __ldcs(reinterpret_cast<const float4*>(V + e));
+    vv[1] = __ldcs(reinterpret_cast<const float4*>(V + e + 4));
+    pv[0] = __ldcs(reinterpret_cast<const float4*>(P + e));
+    pv[1] = __ldcs(reinterpret_cast<const float4*>(P + e + 4));
+    const uint32_t* gw = reinterpret_cast<const uint32_t*>(&gv);
+    float* pp = reinterpret_cast<float*>(&pv[0]);
+    float* mm = reinterpret_cast<float*>(&mv[0]);
+    float* vq = reinterpret_cast<float*>(&vv[0]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      adam_one(pp[2 * j], mm[2 * j], vq[2 * j], bf16_to_f32(gw[j] & 0xFFFFu), kk, f);
+      adam_one(pp[2 * j + 1], mm[2 * j + 1], vq[2 * j + 1], bf16_to_f32(gw[j] >> 16), kk, f);
+      wout[j] = f32_to_bf16_rne(pp[2 * j]) | (f32_to_bf16_rne(pp[2 * j + 1]) << 16);
+    }
+    __stcs(reinterpret_cast<float4*>(M + e), mv[0]);
+    __stcs(reinterpret_cast<float4*>(M + e + 4), mv[1]);
+    __stcs(reinterpret_cast<float4*>(V + e), vv[0]);
+    __stcs(reinterpret_cast<float4*>(V + e + 4), vv[1]);
+    __stcs(reinterpret_cast<float4*>(P + e), pv[0]);
+    __stcs(reinterpret_cast<float4*>(P + e + 4), pv[1]);
+    *reinterpret_cast<uint4*>(W + e) = make_uint4(wout[0], wout[1], wout[2], wout[3]);
+    }
+    uint32_t mag;
+    const uint2 q8 = ci.fmt == 0 ? quant8<0>(wout, s, mag) : quant8<1>(wout, s, mag);
+    vmax = max(vmax, mag);
+    if (ci.q) *reinterpret_cast<uint2*>(ci.q + e) = q8;
+    *reinterpret_cast<uint2*>(&stage[(vec >> 4) * 32 + (vec & 15) * 2]) = q8;
+  }
+  vmax = __reduce_max_sync(0xffffffffu, vmax);
+  if ((tid & 31) == 0) red[tid >> 5] = vmax;
+  __syncthreads();                                   // staged tile and warp maxima complete
+  if (tid == 0) {
+    uint32_t m = 0;
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) m = max(m, red[w]);
+    if (m > 0x7F80u) m = 0x7FC0u;                    // canonical NaN
+    atomicMax(ci.amax_bits, m << 16);
+    if (ci.scale_inv && local == 0) *ci.scale_inv = __fdiv_rn(1.0f, s);
+  }
+  if (ci.qt && tid < 128) {
+    const int rb = tid >> 5, cb = tid & 31;          // rows 16rb.., columns 4cb..
+    if (r0 + 16 * rb < rows && c0 + 4 * cb < cols) {
+      uint32_t v[16];
+#pragma unroll
+      for (int r = 0; r < 16; ++r) v[r] = stage[(16 * rb + r) * 32 + cb];
+      uint32_t o[4][4];
+#pragma unroll
+      for (int kq = 0; kq < 4; ++kq) {
+        const uint32_t a = v[4 * kq], bq = v[4 * kq + 1], cq = v[4 * kq + 2], d = v[4 * kq + 3];
+        const uint32_t t0 = __byte_perm(a, bq, 0x5140), t1 = __byte_perm(a, bq, 0x7362);
+        const uint32_t w0 = __byte_perm(cq, d, 0x5140), w1 = __byte_perm(cq, d, 0x7362);
+        o[0][kq] = __byte_perm(t0, w0, 0x5410);
+        o[1][kq] = __byte_perm(t0, w0, 0x7632);
+        o[2][kq] = __byte_perm(t1, w1, 0x5410);
+        o[3][kq] = __byte_perm(t1, w1, 0x7632);
+      }
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc)
+        *reinterpret_cast<uint4*>(ci.qt + (c0 + 4 * cb + cc) * rows + r0 + 16 * rb) =
+            make_uint4(o[cc][0], o[cc][1], o[cc][2], o[cc][3]);
+    }
+  }
+  __syncthreads();                                   // tile and maxima free for the next one
+}
+
+template <bool CAST>
+__global__ void __launch_bounds__(kThreads, 2)
     k_adamw_update(const __grid_constant__ Batch b, const Scalars k,
                    const double* __restrict__ partials, int nparts, float* __restrict__ norm_out,
                    int32_t* __restrict__ skipped_out) {
   __shared__ double sh[kThreads];
   __shared__ float s_f, s_step_size, s_bc2_sqrt;
   __shared__ int s_skip;
+  __shared__ int64_t s_step;
   {
     double acc = 0.0;
     for (int i = threadIdx.x; i < nparts; i += kThreads) acc = __dadd_rn(acc, partials[i]);
@@ -156,11 +305,14 @@ __global__ void __launch_bounds__(kThreads)
       s_f = __fmul_rn(coef, k.inv_s);
       s_skip = skip;
       if (k.d_step) {
-        const int64_t step = *k.step_slot;
+        const int64_t step = k.step_slot ? *k.step_slot
+                                         : *reinterpret_cast<volatile int64_t*>(k.d_step) + 1;
+        s_step = step;
         const double t = static_cast<double>(step);
         s_step_size = static_cast<float>(__ddiv_rn(k.lr_d, 1.0 - pow(k.beta1_d, t)));
         s_bc2_sqrt = static_cast<float>(__dsqrt_rn(1.0 - pow(k.beta2_d, t)));
-        if (b.first && blockIdx.x == 0 && !skip) *k.d_step = step;   // no CTA reads the counter
+        if (k.step_slot && b.first && blockIdx.x == 0 && !skip)
+          *k.d_step = step;                                   // no CTA reads the counter
       } else {
         s_step_size = k.step_size;
         s_bc2_sqrt = k.bc2_sqrt;
@@ -172,14 +324,22 @@ __global__ void __launch_bounds__(kThreads)
     }
     __syncthreads();
   }
-  if (s_skip) return;
+  if (s_skip && !CAST) return;          // a skipped step only re-casts weights that carry a cast
+  const bool skip = s_skip != 0;
   const float f = s_f;
   Scalars kk = k;
   kk.step_size = s_step_size;
   kk.bc2_sqrt = s_bc2_sqrt;
+  __shared__ uint32_t stage[CAST ? kTileRows * kTileCols / 4 : 1];   // one tile of codes
+  __shared__ uint32_t red[kThreads / 32];
   const int64_t nchunks = b.chunk_start[b.n];
   for (int64_t c = blockIdx.x; c < nchunks; c += gridDim.x) {
     const int t = find_tensor(b, c);
+    if (CAST && b.cast_of[t] >= 0) {
+      update_cast_tile(b, b.cast[b.cast_of[t]], t, c - b.chunk_start[t], kk, f, !skip, stage, red);
+      continue;
+    }
+    if (CAST && skip) continue;
     const int64_t base = (c - b.chunk_start[t]) * kChunk;
     const int64_t n = b.numel[t];
     float* __restrict__ P = b.master[t];
@@ -238,6 +398,19 @@ __global__ void __launch_bounds__(kThreads)
             W[i] = static_cast<uint16_t>(f32_to_bf16_rne(p));
           }
         }
+      }
+    }
+  }
+  // counter read by every CTA above: the last CTA of the last batch advances it
+  if (k.d_step && !k.step_slot && b.last && !skip) {
+    __shared__ int s_last;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      s_last = atomicAdd(k.step_ticket, 1u) == gridDim.x - 1;
+      if (s_last) {
+        *k.d_step = s_step;
+        atomicExch(k.step_ticket, 0u);
       }
     }
   }

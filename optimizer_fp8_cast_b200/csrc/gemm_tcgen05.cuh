@@ -27,6 +27,12 @@
 //                   (clipped at the M and N edges). Per-lane 16-byte stores to 32 different rows
 //                   cost ~15% of the GEMM's throughput. Once its TMEM reads are done the warp
 //                   tells the even CTA that the accumulator is free (4 warps x 2 CTAs arrive).
+// Optional sum of squares (the AdamW global norm's input, fused here so that the gradient is not
+// read again): for flagged problems each epilogue warp adds up f32(bf16(D))^2 of its rows of the
+// tile in FP64 (a fixed butterfly over the lanes) and stores one partial per (tile, CTA, warp)
+// into a workspace slot; the CTA that finishes the last launch last (a ticket counter) sums all
+// slots in index order, so the result does not depend on scheduling. Out-of-range rows and
+// columns hold exact zeros (TMA zero-fills the operands there) and add nothing.
 // Every mbarrier wait is bounded (globaltimer). On expiry a CTA records kErrTimeout and stops
 // issuing; issued MMAs are awaited with a fixed bound, loads in flight are given time to land,
 // and both CTAs meet at a cluster barrier before TMEM is freed; D is then incomplete.
@@ -85,11 +91,19 @@ struct alignas(64) Problem {
   int32_t M, N, K;
   uint32_t idesc;
   int32_t tiles_n, tile_start;
+  int32_t sumsq_slot;            // first partial slot of this problem, or -1 (not summed)
 };
 struct alignas(64) Group {
   Problem p[kMaxProblems];
   int32_t n, total_tiles;
+  // sum of squares (sumsq_out null: off)
+  double* partials;              // every launch's slots (8 per summed tile)
+  double* sumsq_out;
+  unsigned int* ticket;          // zero on entry, left zero
+  int32_t n_partials;            // slots of all launches of the call
+  int32_t last_launch;           // this launch reduces the slots
 };
+constexpr int kSumsqPerTile = 8; // 2 CTAs x 4 epilogue warps
 
 __device__ __forceinline__ int find_problem(const Group& g, int tile) {
   int p = 0;
@@ -253,6 +267,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int row0 = (local_tile / P.tiles_n) * kBM + static_cast<int>(rank) * kHalf + quad * 32;
       const int n0 = (local_tile % P.tiles_n) * kBN;
       const uint32_t t_base = tmem + (static_cast<uint32_t>(quad * 32) << 16) + acc * kAccCols;
+      const bool sumsq = P.sumsq_slot >= 0;
+      double ss = 0.0;
 #pragma unroll 1
       for (int c = 0; c < kBN / 32; ++c) {
         uint32_t r[32];
@@ -274,6 +290,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             w[q] = pack_bf16x2(__fmul_rn(__uint_as_float(r[2 * j]), alpha),
                                __fmul_rn(__uint_as_float(r[2 * j + 1]), alpha));
           }
+          if (sumsq) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const double lo = __uint_as_float(w[q] << 16), hi = __uint_as_float(w[q] & 0xFFFF0000u);
+              ss = __fma_rn(lo, lo, ss);                // squares of BF16 values are exact
+              ss = __fma_rn(hi, hi, ss);
+            }
+          }
           const int pp = p ^ ((lane >> 1) & 3);
           *reinterpret_cast<uint4*>(buf + lane * 64 + pp * 16) = make_uint4(w[0], w[1], w[2], w[3]);
         }
@@ -287,6 +311,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&S->acc_empty[acc]), 0));
+      if (sumsq) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, o));
+        if (lane == 0) {
+          g.partials[P.sumsq_slot + local_tile * kSumsqPerTile + static_cast<int>(rank) * 4 + quad] = ss;
+          __threadfence();                           // before this CTA's ticket
+        }
+      }
     }
     if (lane == 0) bulk_wait_group<0>();             // every store complete before exit
   }
@@ -301,6 +333,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   cluster_sync();                 // neither CTA leaves while the pair MMA may still read it
   tc_fence_after();
   if (warp == 1) tmem_dealloc_pair(tmem, kTmemCols);
+
+  // ---------------- sum of squares: the last CTA of the last launch adds the slots in order
+  if (!g.sumsq_out || !g.last_launch) return;
+  __shared__ int s_last;
+  __shared__ double s_part[kThreads];
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(g.ticket, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  double acc = 0.0;
+  for (int i = threadIdx.x; i < g.n_partials; i += kThreads) acc = __dadd_rn(acc, __ldcg(g.partials + i));
+  s_part[threadIdx.x] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double total = 0.0;
+    for (int i = 0; i < kThreads; ++i) total = __dadd_rn(total, s_part[i]);
+    // a launch whose waits expired has slots that were never written
+    if (*reinterpret_cast<volatile unsigned int*>(&g_error_word) != 0u) total = __longlong_as_double(0x7FF8000000000000LL);
+    *g.sumsq_out = total;
+    atomicExch(g.ticket, 0u);
+  }
 }
 
 }  // namespace gemm

@@ -17,6 +17,56 @@ namespace scale {
 
 constexpr int kThreads = 256;
 
+// Next scale from the representative amax (its magnitude bits): FP8_MAX / rep, times 2^-margin;
+// rep 0 gives 1; NaN or infinity keeps the previous scale; an overflow to infinity gives FLT_MAX.
+__device__ __forceinline__ float next_scale(uint32_t rep, float fmax, int margin, float prev) {
+  if (rep >= 0x7F800000u) return prev;
+  if (rep == 0u) return 1.0f;
+  const float pow2 = __uint_as_float(static_cast<uint32_t>(127 - margin) << 23);
+  float s = __fmul_rn(__fdiv_rn(fmax, __uint_as_float(rep)), pow2);
+  if (isinf(s)) s = 3.40282346638528859812e+38f;                // FLT_MAX
+  return s;
+}
+
+// The same update for one tensor, done by one warp (used inside other kernels once their amax
+// is complete). The roll goes from the top down in chunks of 32 x kPer entries: every lane
+// reads its kPer entries, the warp synchronises, then writes them one place higher.
+// amax is read with a volatile load: other CTAs of the calling kernel accumulated it.
+template <int kPer = 8>
+__device__ __forceinline__ void warp_update(float* amax, float* h, int H, float fmax, bool algo_max,
+                                            int margin, float* scale, float* scale_inv) {
+  const int lane = threadIdx.x & 31;
+  const float a = *reinterpret_cast<volatile float*>(amax);
+  uint32_t m = __float_as_uint(a) & 0x7FFFFFFFu;
+  for (int top = H - 1; top >= 1; top -= 32 * kPer) {
+    float v[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int i = top - lane - 32 * j;
+      v[j] = i >= 1 ? h[i - 1] : 0.0f;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int i = top - lane - 32 * j;
+      if (i >= 1) {
+        h[i] = v[j];
+        if (algo_max) m = max(m, __float_as_uint(v[j]) & 0x7FFFFFFFu);
+      }
+    }
+    __syncwarp();
+  }
+  m = __reduce_max_sync(0xffffffffu, m);
+  if (lane == 0) {
+    const uint32_t rep = algo_max ? m : (__float_as_uint(a) & 0x7FFFFFFFu);
+    h[0] = a;
+    const float s = next_scale(rep, fmax, margin, *reinterpret_cast<volatile float*>(scale));
+    *scale = s;
+    *scale_inv = __fdiv_rn(1.0f, s);
+    *amax = 0.0f;
+  }
+}
+
 __global__ void __launch_bounds__(kThreads)
     k_scale_update(float* __restrict__ amax, float* __restrict__ hist, int H,
                    const float* __restrict__ fp8_max, int algo_max, int margin,
@@ -47,17 +97,7 @@ __global__ void __launch_bounds__(kThreads)
     for (int i = 0; i < kThreads / 32; ++i) rep = max(rep, red[i]);
     if (!algo_max) rep = __float_as_uint(a) & 0x7FFFFFFFu;
     h[0] = a;
-    float s;
-    if (rep >= 0x7F800000u) {
-      s = scale[t];                                           // NaN or inf: keep
-    } else if (rep == 0u) {
-      s = 1.0f;
-    } else {
-      const float pow2 = __uint_as_float(static_cast<uint32_t>(127 - margin) << 23);
-      s = __fdiv_rn(fp8_max[t], __uint_as_float(rep));
-      s = __fmul_rn(s, pow2);
-      if (isinf(s)) s = 3.40282346638528859812e+38f;          // FLT_MAX
-    }
+    const float s = next_scale(rep, fp8_max[t], margin, scale[t]);
     scale[t] = s;
     scale_inv[t] = __fdiv_rn(1.0f, s);
     amax[t] = 0.0f;                                           // consumed: ready to accumulate

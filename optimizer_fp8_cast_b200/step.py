@@ -9,13 +9,23 @@ One step for each layer (W stored in x out, Y = X.W), following the precision fl
   dW = Xq^T . dYq   (wgrad,  A = Xq^T, B = dYq^T)
 then, for all layers at once, the amax-history roll and next scales, and one fused AdamW over
 every dW (loss-scale unscale, global-norm clip, FP32 master/m/v, BF16 weight for the next step).
-All scalars stay on the device; nothing in a step synchronises with the host.
+With fused_update (the default) the roll and next scales run in the last CTA of the cast launch,
+which is possible because the GEMMs read the inverse scales the casts used (sinv_used), not the
+next ones (scale_inv). With fused_norm (the default) the wgrad epilogues also form the gradient
+sum of squares, and AdamW runs without its norm pass, so each dW is read once. With fused_wcast
+(the default when both are on and no counters are kept) AdamW also casts each new BF16 weight
+for the next step with that step's scale, which the cast launch's update has already formed;
+the cast launch then carries only the scale update of W (its amax came from AdamW), and W is
+never read by a cast. The first step's W cast happens once, at construction (prime). All
+scalars stay on the device; nothing in a step synchronises with the host.
 """
 import torch
 
 from . import (AMAX_MAX, AMAX_MOST_RECENT, E4M3, E5M2, FP8_MAX, fp8_cast_transpose_amax,
-               fp8_cast_transpose_amax_multi, fp8_gemm, fp8_gemm_multi, fp8_scale_update,
-               fused_adamw_multi_tensor, fused_adamw_workspace_bytes)
+               fp8_cast_transpose_amax_multi, fp8_cast_transpose_amax_update_multi, fp8_gemm,
+               fp8_gemm_multi, fp8_gemm_multi_sumsq, fp8_gemm_sumsq_workspace_bytes,
+               fp8_scale_update, fused_adamw_multi_tensor, fused_adamw_multi_tensor_presummed,
+               fused_adamw_workspace_bytes)
 
 ROLE_X, ROLE_W, ROLE_DY = 0, 1, 2
 ROLE_FMT = (E4M3, E4M3, E5M2)
@@ -47,7 +57,8 @@ class Fp8LinearStep:
     Scale state is indexed 3*layer + role (role 0 = X, 1 = W, 2 = dY)."""
 
     def __init__(self, layer_shapes, tokens, history_len, algo="max", margin=0, adamw=None,
-                 w_init=None, device="cuda", counters=False, device_step=False):
+                 w_init=None, device="cuda", counters=False, device_step=False, fused_update=True,
+                 fused_norm=True, fused_wcast=True):
         self.device = torch.device(device)
         self.tokens = tokens
         self.algo = AMAX_MAX if algo == "max" else AMAX_MOST_RECENT
@@ -58,7 +69,10 @@ class Fp8LinearStep:
         self.amax = torch.zeros(n, **f32)
         self.history = torch.zeros(n, history_len, **f32)
         self.scale = torch.ones(n, **f32)
-        self.scale_inv = torch.ones(n, **f32)
+        self.scale_inv = torch.ones(n, **f32)          # 1 / next scale (scale update output)
+        self.sinv_used = torch.ones(n, **f32)          # 1 / scale the casts used (GEMM input)
+        self.fused_update = fused_update
+        self.ticket = torch.zeros(1, dtype=torch.int32, device=self.device)
         self.fp8_max = torch.tensor([FP8_MAX[ROLE_FMT[i % 3]] for i in range(n)], **f32)
         self.counters = torch.zeros(n, 3, dtype=torch.int64, device=self.device) if counters else None
         self.layers = [LinearLayerBuffers(fi, fo, tokens, w_init[k], self.device)
@@ -71,6 +85,24 @@ class Fp8LinearStep:
         # device_step: AdamW counts steps in device memory, so a captured graph can be replayed
         self.step_counter = (torch.zeros(1, dtype=torch.int64, device=self.device)
                              if device_step else None)
+        # gradient sum of squares from the wgrad epilogues (fused_norm)
+        self.fused_norm = fused_norm
+        self.sumsq = torch.zeros(1, dtype=torch.float64, device=self.device)
+        gws = fp8_gemm_sumsq_workspace_bytes(self._gemm_descs(sumsq=True))
+        self.gemm_workspace = torch.zeros(gws, dtype=torch.uint8, device=self.device)
+        self.adamw_ticket = torch.zeros(1, dtype=torch.int32, device=self.device)
+        # the W cast inside AdamW needs the in-launch scale update and the presummed AdamW; the
+        # saturation / zero counters of W are only kept by the separate cast
+        self.fused_wcast = fused_wcast and fused_update and fused_norm and not counters
+        if self.fused_wcast and self.device.type == "cuda":
+            self.prime()
+
+    def prime(self):
+        """Cast every W with its current scale (codes, transposed codes, amax, scale inverse), as
+        the AdamW of a previous step would have: needed before the first step, and after the
+        weights or the scale state were loaded."""
+        fp8_cast_transpose_amax_multi(
+            [self.cast_desc(k, ROLE_W, L.W, L.Wq, L.WqT) for k, L in enumerate(self.layers)])
 
     def _slot(self, t, i):
         return t[i:i + 1]
@@ -78,29 +110,39 @@ class Fp8LinearStep:
     def cast(self, k, role, src, q, qT, stream=None):
         i = 3 * k + role
         fp8_cast_transpose_amax(src, ROLE_FMT[role], self._slot(self.scale, i), q, qT,
-                                self._slot(self.amax, i), self._slot(self.scale_inv, i),
+                                self._slot(self.amax, i), self._slot(self.sinv_used, i),
                                 self.counters[i] if self.counters is not None else None,
                                 stream=stream)
 
     def cast_desc(self, k, role, src, q, qT):
         i = 3 * k + role
         return dict(x=src, fmt=ROLE_FMT[role], scale=self._slot(self.scale, i), q=q, qT=qT,
-                    amax=self._slot(self.amax, i), scale_inv=self._slot(self.scale_inv, i),
-                    counters=self.counters[i] if self.counters is not None else None)
+                    amax=self._slot(self.amax, i),
+                    scale_inv=self._slot(self.sinv_used, i) if src is not None else None,
+                    counters=self.counters[i] if self.counters is not None and src is not None
+                    else None)
 
-    def cast_all(self, xs, dys, stream=None):
-        """Every layer's X, W and dY casts, grouped into launches of up to 8 tensors."""
+    def cast_all(self, xs, dys, stream=None, update=False):
+        """Every layer's X, W and dY casts, grouped into launches of up to 8 tensors; with
+        update, each launch's last CTA also performs those tensors' scale update."""
         descs = []
         for k, L in enumerate(self.layers):
-            descs += [self.cast_desc(k, ROLE_X, xs[k], L.Xq, L.XqT),
-                      self.cast_desc(k, ROLE_W, L.W, L.Wq, L.WqT),
+            w = (self.cast_desc(k, ROLE_W, None, None, None) if update and self.fused_wcast
+                 else self.cast_desc(k, ROLE_W, L.W, L.Wq, L.WqT))   # None: scale update only
+            descs += [self.cast_desc(k, ROLE_X, xs[k], L.Xq, L.XqT), w,
                       self.cast_desc(k, ROLE_DY, dys[k], L.dYq, L.dYqT)]
-        fp8_cast_transpose_amax_multi(descs, stream=stream)
+        if update:
+            ups = [dict(history=self.history[i], scale_inv_next=self._slot(self.scale_inv, i))
+                   for i in range(len(descs))]
+            fp8_cast_transpose_amax_update_multi(descs, ups, self.algo, self.margin, self.ticket,
+                                                 stream=stream)
+        else:
+            fp8_cast_transpose_amax_multi(descs, stream=stream)
 
     def gemm(self, k, which, stream=None):
         """which: 0 = fprop Y = X.W, 1 = dgrad dX = dY.W^T, 2 = wgrad dW = X^T.dY."""
         L = self.layers[k]
-        sx, sw, sdy = (self._slot(self.scale_inv, 3 * k + r) for r in (ROLE_X, ROLE_W, ROLE_DY))
+        sx, sw, sdy = (self._slot(self.sinv_used, 3 * k + r) for r in (ROLE_X, ROLE_W, ROLE_DY))
         if which == 0:
             fp8_gemm(L.Xq, E4M3, L.WqT, E4M3, sx, sw, L.Y, stream=stream)
         elif which == 1:
@@ -110,17 +152,28 @@ class Fp8LinearStep:
 
     def gemm_desc(self, k, which):
         L = self.layers[k]
-        sx, sw, sdy = (self._slot(self.scale_inv, 3 * k + r) for r in (ROLE_X, ROLE_W, ROLE_DY))
+        sx, sw, sdy = (self._slot(self.sinv_used, 3 * k + r) for r in (ROLE_X, ROLE_W, ROLE_DY))
         if which == 0:
             return dict(A=L.Xq, a_fmt=E4M3, B=L.WqT, b_fmt=E4M3, a_scale_inv=sx, b_scale_inv=sw, D=L.Y)
         if which == 1:
             return dict(A=L.dYq, a_fmt=E5M2, B=L.Wq, b_fmt=E4M3, a_scale_inv=sdy, b_scale_inv=sw, D=L.dX)
         return dict(A=L.XqT, a_fmt=E4M3, B=L.dYqT, b_fmt=E5M2, a_scale_inv=sx, b_scale_inv=sdy, D=L.dW)
 
-    def gemm_all(self, stream=None):
-        """Every layer's fprop, dgrad and wgrad in one grouped launch (24 GEMMs per launch)."""
-        fp8_gemm_multi([self.gemm_desc(k, w) for k in range(len(self.layers)) for w in (0, 1, 2)],
-                       stream=stream)
+    def _gemm_descs(self, sumsq=False):
+        descs = [self.gemm_desc(k, w) for k in range(len(self.layers)) for w in (0, 1, 2)]
+        if sumsq:
+            for i in range(2, len(descs), 3):
+                descs[i]["sumsq"] = True                     # the wgrad outputs are the gradients
+        return descs
+
+    def gemm_all(self, stream=None, sumsq=False):
+        """Every layer's fprop, dgrad and wgrad in one grouped launch (24 GEMMs per launch); with
+        sumsq the wgrad epilogues also leave the FP64 sum of dW^2 in self.sumsq."""
+        if sumsq:
+            fp8_gemm_multi_sumsq(self._gemm_descs(sumsq=True), self.sumsq, self.gemm_workspace,
+                                 stream=stream)
+        else:
+            fp8_gemm_multi(self._gemm_descs(), stream=stream)
 
     def layer_forward_backward(self, k, X, dY, stream=None):
         L = self.layers[k]
@@ -138,8 +191,20 @@ class Fp8LinearStep:
         self.scale_update(stream)
         self.adamw(stream)
 
-    def adamw(self, stream=None):
+    def adamw(self, stream=None, presummed=False):
+        """One fused AdamW over every layer's dW; presummed: take the sum of squares the wgrad
+        epilogues left in self.sumsq instead of running the norm pass."""
         hp = self.hp
+        if presummed:
+            fused_adamw_multi_tensor_presummed(
+                [l.master for l in self.layers], [l.m for l in self.layers],
+                [l.v for l in self.layers], [l.dW for l in self.layers], [l.W for l in self.layers],
+                lr=hp["lr"], beta1=hp["beta1"], beta2=hp["beta2"], eps=hp["eps"],
+                weight_decay=hp["weight_decay"], step=self.t, loss_scale=hp["loss_scale"],
+                max_grad_norm=hp["max_grad_norm"], grad_sumsq=self.sumsq, grad_norm=self.grad_norm,
+                skipped=self.skipped, step_counter=self.step_counter, ticket=self.adamw_ticket,
+                casts=self._weight_casts() if self.fused_wcast else None, stream=stream)
+            return
         fused_adamw_multi_tensor([l.master for l in self.layers], [l.m for l in self.layers],
                                  [l.v for l in self.layers], [l.dW for l in self.layers],
                                  [l.W for l in self.layers], lr=hp["lr"], beta1=hp["beta1"],
@@ -149,12 +214,23 @@ class Fp8LinearStep:
                                  skipped=self.skipped, workspace=self.workspace,
                                  step_counter=self.step_counter, stream=stream)
 
+    def _weight_casts(self):
+        out = []
+        for k, L in enumerate(self.layers):
+            i = 3 * k + ROLE_W
+            out.append(dict(rows=L.fin, cols=L.fout, fmt=E4M3, scale=self._slot(self.scale, i),
+                            q=L.Wq, qT=L.WqT, amax=self._slot(self.amax, i),
+                            scale_inv=self._slot(self.sinv_used, i)))
+        return out
+
     def step(self, xs, dys, stream=None):
         """One training step; xs[k] = X [tokens, in_k], dys[k] = dY [tokens, out_k] (BF16, device)."""
         self.t += 1
-        self.cast_all(xs, dys, stream)
-        self.gemm_all(stream)
-        self.update(stream)
+        self.cast_all(xs, dys, stream, update=self.fused_update)
+        self.gemm_all(stream, sumsq=self.fused_norm)
+        if not self.fused_update:
+            self.scale_update(stream)
+        self.adamw(stream, presummed=self.fused_norm)
 
     # ------------------------------------------------------------------ training state
     def state_dict(self):
@@ -181,10 +257,14 @@ class Fp8LinearStep:
                 getattr(l, name).copy_(s[name])
         if self.step_counter is not None:
             self.step_counter.copy_(sd.get("step_counter", torch.tensor([self.t])))
+        if self.fused_wcast and self.device.type == "cuda":
+            self.prime()
 
     # launches of the library's kernels per step (for the benchmark's launch count)
     def kernels_per_step(self):
         n_adamw_batches = (len(self.layers) + 255) // 256
         n_cast_launches = (3 * len(self.layers) + 7) // 8
         n_gemm_launches = (3 * len(self.layers) + 23) // 24
-        return n_cast_launches + n_gemm_launches + 1 + 2 * n_adamw_batches
+        n_scale_launches = 0 if self.fused_update else 1
+        n_adamw_launches = (1 if self.fused_norm else 2) * n_adamw_batches
+        return n_cast_launches + n_gemm_launches + n_scale_launches + n_adamw_launches

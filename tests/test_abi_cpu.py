@@ -62,6 +62,29 @@ def test_invalid_arguments_rejected_on_host(lib):
     assert lib.fp8_cast_transpose_amax_multi(arr, 0, z) == 1
     arr[1] = _abi.CastTensor(P, 16, 16, 1, P, U, P, P, P, None)
     assert lib.fp8_cast_transpose_amax_multi(arr, 2, z) == 3
+    # cast with the scale update in the same launch
+    Q = C.c_void_p(32 * 1024)
+    arr[1] = _abi.CastTensor(P, 16, 16, 1, P, P, P, P, P, None)
+    ups = (_abi.CastUpdate * 2)()
+    ups[0] = _abi.CastUpdate(P, Q)
+    ups[1] = _abi.CastUpdate(P, Q)
+    upd = lambda u=ups, H=16, algo=0, margin=0, ticket=P: lib.fp8_cast_transpose_amax_update_multi(
+        arr, u, 2, H, algo, margin, ticket, z)
+    assert upd(u=None) == 1
+    assert upd(ticket=None) == 1 and upd(ticket=C.c_void_p(16 * 1024 + 2)) == 1
+    assert upd(H=0) == 1 and upd(H=65537) == 1
+    assert upd(algo=2) == 1 and upd(margin=127) == 1
+    ups[1] = _abi.CastUpdate(P, P)                 # the next inverse scale over the used one
+    assert upd() == 1 and b"scale_inv_next must differ" in lib.fp8t_last_error_message()
+    ups[1] = _abi.CastUpdate(None, Q)
+    assert upd() == 1
+    ups[1] = _abi.CastUpdate(C.c_void_p(16 * 1024 + 2), Q)
+    assert upd() == 3
+    ups[1] = _abi.CastUpdate(P, Q)
+    arr[1] = _abi.CastTensor(None, 0, 0, 0, P, P, None, P, None, None)   # update only: no outputs
+    assert upd() == 1
+    assert lib.fp8_cast_transpose_amax_multi(
+        (_abi.CastTensor * 1)(_abi.CastTensor(None, 0, 0, 0, P, None, None, P, None, None)), 1, z) == 1
     # gemm
     assert lib.fp8_gemm(z, 0, P, 0, 16, 16, 16, P, P, P, z) == 1
     assert lib.fp8_gemm(P, 0, P, 9, 16, 16, 16, P, P, P, z) == 1
@@ -76,6 +99,18 @@ def test_invalid_arguments_rejected_on_host(lib):
     g[1] = _abi.GemmDesc(P, 1, P, 3, 16, 16, 16, P, P, P)
     assert lib.fp8_gemm_multi(g, 2, z) == 1
     assert lib.fp8_gemm_multi(g, 0, z) == 1
+    # grouped gemm with the sum of squares
+    g[1] = _abi.GemmDesc(P, 1, P, 0, 16, 16, 16, P, P, P)
+    flags = (C.c_int32 * 2)(0, 1)
+    need = lib.fp8_gemm_sumsq_workspace_bytes(g, 2, flags)
+    assert need == 256 + 8 * 8                          # one 256 x 256 tile, 8 partial slots
+    W = C.c_void_p(64 * 1024)                           # 256-byte aligned
+    assert lib.fp8_gemm_multi_sumsq(g, 2, None, P, W, need, z) == 1
+    assert lib.fp8_gemm_multi_sumsq(g, 2, flags, None, W, need, z) == 1
+    assert lib.fp8_gemm_multi_sumsq(g, 2, flags, P, C.c_void_p(16 * 1024 + 16), need, z) == 1  # not 256-aligned
+    assert lib.fp8_gemm_multi_sumsq(g, 2, flags, P, W, need - 1, z) == 1
+    assert lib.fp8_gemm_sumsq_workspace_bytes(g, 2, (C.c_int32 * 2)(0, 0)) == 0
+    assert lib.fp8_gemm_multi_sumsq(g, 2, (C.c_int32 * 2)(0, 0), P, W, need, z) == 1
     # scale update
     assert lib.fp8_scale_update(0, P, P, 16, P, 0, 0, P, P, z) == 1
     assert lib.fp8_scale_update(3, P, P, 0, P, 0, 0, P, P, z) == 1
@@ -101,5 +136,23 @@ def test_invalid_arguments_rejected_on_host(lib):
     bad[0] = _abi.AdamWTensor(P, P, P, P, P, 0)
     assert call(bad) == 1
     assert lib.fused_adamw_workspace_bytes(bad, 1) == 0
-    assert b"numel" in lib.fp8t_last_error_message()
+    assert call(bad) == 1 and b"numel" in lib.fp8t_last_error_message()
+    pre = lambda a, sumsq=P, dstep=z, ticket=z, casts=None: lib.fused_adamw_multi_tensor_presummed(
+        a, casts, 1, 1e-3, 0.9, 0.999, 1e-8, 0.0, 1, dstep, 1.0, 1.0, sumsq, z, z, ticket, z)
+    assert pre(arr, sumsq=None) == 1
+    assert pre(arr, sumsq=C.c_void_p(16 * 1024 + 4)) == 3
+    assert pre(arr, dstep=P) == 1                       # a device counter needs a ticket
+    assert pre(bad) == 1
+    # weight casts inside AdamW: rows x cols must be numel, multiples of 16
+    w16 = (_abi.AdamWTensor * 1)()
+    w16[0] = _abi.AdamWTensor(P, P, P, P, P, 32 * 48)
+    cast = (_abi.AdamWCast * 1)()
+    cast[0] = _abi.AdamWCast(32, 40, 0, P, P, P, P, P)
+    assert pre(w16, casts=cast) == 2
+    cast[0] = _abi.AdamWCast(32, 48, 5, P, P, P, P, P)
+    assert pre(w16, casts=cast) == 1
+    cast[0] = _abi.AdamWCast(32, 48, 0, None, P, P, P, P)
+    assert pre(w16, casts=cast) == 1
+    cast[0] = _abi.AdamWCast(32, 48, 0, P, U, P, P, P)
+    assert pre(w16, casts=cast) == 3
     assert lib.fp8t_debug_expire_waits(3) == 1 and lib.fp8t_debug_expire_waits(-1) == 1

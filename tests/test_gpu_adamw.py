@@ -29,12 +29,23 @@ def make(sizes, seed, device="cuda", grad_std=1e-3):
     return P, M, V, G, W
 
 
-def run_both(fp8, P, M, V, G, W, hp, steps=1):
+def sumsq_of(G):
+    """FP64 sum of f32(g)^2 over all gradients: the input the presummed call expects (squares of
+    BF16 values are exact in FP64; numpy's pairwise sum rounds ~1e-16 relative)."""
+    return torch.tensor([sum(float(np.sum(np.square(f32(g.float()).astype(np.float64)))) for g in G)],
+                        dtype=torch.float64, device="cuda")
+
+
+def run_both(fp8, P, M, V, G, W, hp, steps=1, presummed=False):
     host = [[f32(t) for t in P], [f32(t) for t in M], [f32(t) for t in V]]
     for step in range(1, steps + 1):
         hpp = dict(hp, step=step + 999)
         norm = torch.zeros(1, device="cuda"); skipped = torch.full((1,), 7, dtype=torch.int32, device="cuda")
-        fp8.fused_adamw_multi_tensor(P, M, V, G, W, grad_norm=norm, skipped=skipped, **hpp)
+        if presummed:
+            fp8.fused_adamw_multi_tensor_presummed(P, M, V, G, W, grad_sumsq=sumsq_of(G),
+                                                   grad_norm=norm, skipped=skipped, **hpp)
+        else:
+            fp8.fused_adamw_multi_tensor(P, M, V, G, W, grad_norm=norm, skipped=skipped, **hpp)
         fp8.fp8t_check_device_error()
         gbits = [bf16_bits(g) for g in G]
         wref = [np.zeros(g.size, np.uint16) for g in gbits]
@@ -145,3 +156,109 @@ def test_adamw4e9_full_size_sampled(cuda_lib):
         for got, ref in ((P[i], p), (M[i], m), (V[i], v)):
             assert ulp_distance_f32(f32(got), ref).max() <= 4
         assert np.abs(bf16_bits(W[i]).astype(np.int32) - w.astype(np.int32)).max() <= 1
+
+
+def test_presummed_matches_oracle(cuda_lib):
+    """fused_adamw_multi_tensor_presummed (sum of squares given, no norm pass) against the oracle,
+    which forms the norm itself: ragged tensors, two steps, clip active."""
+    P, M, V, G, W = make([1, 7, 8193, 100003], seed=11)
+    run_both(cuda_lib, P, M, V, G, W, HP, steps=2, presummed=True)
+
+
+def test_presummed_device_counter_over_two_launch_tables(cuda_lib):
+    """300 tensors (two launches) with a device step counter: every call performs counter+1 in
+    both launches, the last CTA of the last launch advances the counter, the ticket returns to
+    zero; a NaN sum of squares skips the update and leaves the counter alone."""
+    rng = np.random.default_rng(12)
+    sizes = [int(x) for x in rng.integers(1, 5000, 300)]
+    P, M, V, G, W = make(sizes, seed=12)
+    counter = torch.tensor([99], dtype=torch.int64, device="cuda")
+    ticket = torch.zeros(1, dtype=torch.int32, device="cuda")
+    host = [[f32(t) for t in P], [f32(t) for t in M], [f32(t) for t in V]]
+    for k in range(3):
+        cuda_lib.fused_adamw_multi_tensor_presummed(P, M, V, G, W, grad_sumsq=sumsq_of(G), step=0,
+                                                    step_counter=counter, ticket=ticket, **HP)
+        cuda_lib.fp8t_check_device_error()
+        assert counter.item() == 100 + k and ticket.item() == 0
+        gbits = [bf16_bits(g) for g in G]
+        oracle.fused_adamw(host[0], host[1], host[2], gbits,
+                           [np.zeros(g.size, np.uint16) for g in gbits], dict(HP, step=100 + k))
+        for i in (0, 150, 299):
+            for got, ref in ((P[i], host[0][i]), (M[i], host[1][i]), (V[i], host[2][i])):
+                assert ulp_distance_f32(f32(got), ref).max() <= 4
+    before = [f32(t) for t in P[:3]]
+    skipped = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nan = torch.tensor([float("nan")], dtype=torch.float64, device="cuda")
+    cuda_lib.fused_adamw_multi_tensor_presummed(P, M, V, G, W, grad_sumsq=nan, skipped=skipped,
+                                                step=0, step_counter=counter, ticket=ticket, **HP)
+    cuda_lib.fp8t_check_device_error()
+    assert skipped.item() == 1 and counter.item() == 102 and ticket.item() == 0
+    assert all(np.array_equal(a, f32(b)) for a, b in zip(before, P[:3]))
+
+
+def _weight_casts(shapes, fmts, scales):
+    casts = []
+    for (r, c), f, s in zip(shapes, fmts, scales):
+        if r == 0:
+            casts.append(None)
+            continue
+        casts.append(dict(rows=r, cols=c, fmt=f, scale=torch.tensor([s], device="cuda"),
+                          q=torch.full((r, c), 0xAB, dtype=torch.uint8, device="cuda"),
+                          qT=torch.full((c, r), 0xAB, dtype=torch.uint8, device="cuda"),
+                          amax=torch.zeros(1, device="cuda"), scale_inv=torch.zeros(1, device="cuda")))
+    return casts
+
+
+def _check_weight_casts(W, casts, scales):
+    from tests._gpu import u8
+    for w, c, s in zip(W, casts, scales):
+        if c is None:
+            continue
+        bits = bf16_bits(w).reshape(c["rows"], c["cols"])
+        q, qT, a, si, _ = oracle.cast_transpose_amax(bits, c["fmt"], s)
+        assert np.array_equal(u8(c["q"]), q) and np.array_equal(u8(c["qT"]), qT)
+        assert np.float32(c["amax"].item()).view(np.uint32) == np.float32(a).view(np.uint32)
+        assert np.float32(c["scale_inv"].item()).view(np.uint32) == np.float32(si).view(np.uint32)
+
+
+def test_presummed_with_weight_casts(cuda_lib):
+    """The next step's weight cast inside AdamW ("算子与编译器" 优化器 kernel 的带宽账: one pass over
+    the parameters): the update matches the oracle, and the codes, transposed codes, amax and
+    scale inverse of each new BF16 weight match the oracle's cast of it. Ragged tile edges, both
+    formats, a tensor without a cast among them, and 40 casts (two launch tables). Then a skipped
+    step (NaN sum of squares): weights unchanged and cast again with a new scale."""
+    rng = np.random.default_rng(13)
+    shapes = [(272, 400), (16, 16), (0, 0), (4096 // 8, 128 * 3), (64, 2064)]
+    shapes += [(16 * int(rng.integers(1, 9)), 16 * int(rng.integers(1, 9))) for _ in range(38)]
+    sizes = [r * c if r else 7777 for r, c in shapes]
+    fmts = [oracle.E4M3 if i % 5 else oracle.E5M2 for i in range(len(shapes))]
+    scales = [float(np.float32(2.0 ** rng.uniform(2, 12))) for _ in shapes]
+    P, M, V, G, W = make(sizes, seed=13)
+    casts = _weight_casts(shapes, fmts, scales)
+    host = [[f32(t) for t in P], [f32(t) for t in M], [f32(t) for t in V]]
+    hp = dict(HP, step=7)
+    cuda_lib.fused_adamw_multi_tensor_presummed(P, M, V, G, W, grad_sumsq=sumsq_of(G), casts=casts, **hp)
+    cuda_lib.fp8t_check_device_error()
+    gbits = [bf16_bits(g) for g in G]
+    wref = [np.zeros(g.size, np.uint16) for g in gbits]
+    oracle.fused_adamw(host[0], host[1], host[2], gbits, wref, hp)
+    for i in range(len(P)):
+        assert ulp_distance_f32(f32(P[i]), host[0][i]).max() <= 4
+        assert np.array_equal(bf16_bits(W[i]), bf16_bits(P[i].to(torch.bfloat16)))
+    _check_weight_casts(W, casts, scales)
+
+    # skipped step: nothing updated, the unchanged weights cast again with new scales
+    before = [bf16_bits(w).copy() for w in W]
+    scales2 = [s * 0.5 for s in scales]
+    for c, s in zip(casts, scales2):
+        if c is not None:
+            c["scale"].fill_(s)
+            c["amax"].zero_()
+    skipped = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nan = torch.tensor([float("nan")], dtype=torch.float64, device="cuda")
+    cuda_lib.fused_adamw_multi_tensor_presummed(P, M, V, G, W, grad_sumsq=nan, casts=casts,
+                                                skipped=skipped, **dict(HP, step=8))
+    cuda_lib.fp8t_check_device_error()
+    assert skipped.item() == 1
+    assert all(np.array_equal(b, bf16_bits(w)) for b, w in zip(before, W))
+    _check_weight_casts(W, casts, scales2)

@@ -9,7 +9,7 @@ import torch
 
 import oracle
 from optimizer_fp8_cast_b200 import synth
-from tests._gpu import bf16_bits, bf16_from_bits, dev_scalar, u8
+from tests._gpu import bf16_bits, bf16_from_bits, dev_scalar, f32, u8
 
 pytestmark = pytest.mark.gpu
 
@@ -157,3 +157,93 @@ def test_multi_tensor_launch(cuda_lib):
         assert np.float32(c["amax"].item()).view(np.uint32) == np.float32(ramax).view(np.uint32)
         assert np.float32(c["scale_inv"].item()) == rsinv
         assert np.array_equal(c["counters"].cpu().numpy().astype(np.uint64), rcnt)
+
+
+@pytest.mark.parametrize("n,H,algo,margin", [(3, 1, oracle.AMAX_MAX, 0), (3, 16, oracle.AMAX_MAX, 1),
+                                             (21, 16, oracle.AMAX_MOST_RECENT, 0),
+                                             (5, 1024, oracle.AMAX_MAX, 0), (9, 3000, oracle.AMAX_MAX, 3)])
+def test_cast_with_fused_scale_update(cuda_lib, n, H, algo, margin):
+    """fp8_cast_transpose_amax_update_multi equals the oracle's cast followed by its scale
+    update ("LLM FP8 微调上线生产实战" 核心原理: history roll, representative amax, next scale), bit
+    for bit: codes, inverse of the scale used, history, next scale and its inverse, amax slots
+    reset, ticket left at zero. 21 tensors take three launches; H = 3000 needs several chunks of
+    the warp roll. One tensor carries a NaN (its scale is kept) and one is all zero."""
+    rng = np.random.default_rng(1000 + n + H)
+    shapes = [(16 * int(rng.integers(1, 20)), 16 * int(rng.integers(1, 20))) for _ in range(n)]
+    fmts = [oracle.E4M3 if i % 3 != 2 else oracle.E5M2 for i in range(n)]
+    xs = []
+    for i, (r, c) in enumerate(shapes):
+        x = (rng.standard_normal((r, c)) * 10.0 ** rng.uniform(-3, 3)).astype(np.float32)
+        if i == 1:
+            x[r // 2, c // 3] = np.nan
+        if i == n - 1:
+            x[:] = 0.0
+        xs.append(bf16_bits(torch.from_numpy(x).to(torch.bfloat16)))
+    scale0 = (2.0 ** rng.uniform(-8, 8, n)).astype(np.float32)
+    hist0 = np.abs(rng.standard_normal((n, H)) * 10.0 ** rng.uniform(-2, 2, (n, 1))).astype(np.float32)
+    fp8_max = np.array([448.0 if f == oracle.E4M3 else 57344.0 for f in fmts], np.float32)
+
+    scale = torch.from_numpy(scale0.copy()).cuda()
+    hist = torch.from_numpy(hist0.copy()).cuda()
+    amax = torch.zeros(n, device="cuda")
+    sinv_used = torch.zeros(n, device="cuda")
+    sinv_next = torch.zeros(n, device="cuda")
+    ticket = torch.zeros(1, dtype=torch.int32, device="cuda")
+    casts, ups = [], []
+    for i, ((r, c), f) in enumerate(zip(shapes, fmts)):
+        casts.append(dict(x=bf16_from_bits(xs[i]), fmt=f, scale=scale[i:i + 1],
+                          q=torch.empty(r, c, dtype=torch.uint8, device="cuda"),
+                          qT=torch.empty(c, r, dtype=torch.uint8, device="cuda"),
+                          amax=amax[i:i + 1], scale_inv=sinv_used[i:i + 1]))
+        ups.append(dict(history=hist[i], scale_inv_next=sinv_next[i:i + 1]))
+    cuda_lib.fp8_cast_transpose_amax_update_multi(casts, ups, algo, margin, ticket)
+    cuda_lib.fp8t_check_device_error()
+
+    amax_ref = np.zeros(n, np.float32)
+    for i, f in enumerate(fmts):
+        rq, rqT, ra, rsinv, _ = oracle.cast_transpose_amax(xs[i], f, scale0[i])
+        assert np.array_equal(u8(casts[i]["q"]), rq) and np.array_equal(u8(casts[i]["qT"]), rqT)
+        assert np.float32(sinv_used[i].item()).view(np.uint32) == np.float32(rsinv).view(np.uint32)
+        amax_ref[i] = ra
+    h_ref, s_ref, si_ref = hist0.copy(), scale0.copy(), np.zeros(n, np.float32)
+    oracle.scale_update(amax_ref, h_ref, fp8_max, algo, margin, s_ref, si_ref)
+    assert np.array_equal(f32(hist).view(np.uint32), h_ref.view(np.uint32))
+    assert np.array_equal(f32(scale).view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(f32(sinv_next).view(np.uint32), si_ref.view(np.uint32))
+    assert np.isnan(h_ref[1, 0]) and s_ref[1] == scale0[1]          # the NaN tensor kept its scale
+    assert not amax.any().item() and ticket.item() == 0
+
+
+def test_fused_scale_update_equals_separate_launch(cuda_lib):
+    """Ten consecutive steps of three tensors: the fused launch and cast + fp8_scale_update in
+    separate launches leave identical scale state and codes."""
+    rng = np.random.default_rng(77)
+    H, n = 16, 3
+    shapes = [(512, 256), (256, 256), (512, 256)]
+    fmts = [oracle.E4M3, oracle.E4M3, oracle.E5M2]
+    fp8_max = torch.tensor([448.0, 448.0, 57344.0], device="cuda")
+    state = [dict(scale=torch.ones(n, device="cuda"), hist=torch.zeros(n, H, device="cuda"),
+                  amax=torch.zeros(n, device="cuda"), used=torch.zeros(n, device="cuda"),
+                  nxt=torch.zeros(n, device="cuda")) for _ in range(2)]
+    ticket = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for t in range(10):
+        xs = [torch.from_numpy((rng.standard_normal(s) * 10.0 ** rng.uniform(-2, 2)).astype(np.float32))
+              .to(torch.bfloat16).cuda() for s in shapes]
+        outs = []
+        for k, S in enumerate(state):
+            casts = [dict(x=xs[i], fmt=fmts[i], scale=S["scale"][i:i + 1],
+                          q=torch.empty(shapes[i], dtype=torch.uint8, device="cuda"),
+                          amax=S["amax"][i:i + 1], scale_inv=S["used"][i:i + 1]) for i in range(n)]
+            if k == 0:
+                ups = [dict(history=S["hist"][i], scale_inv_next=S["nxt"][i:i + 1]) for i in range(n)]
+                cuda_lib.fp8_cast_transpose_amax_update_multi(casts, ups, oracle.AMAX_MAX, 0, ticket)
+            else:
+                cuda_lib.fp8_cast_transpose_amax_multi(casts)
+                cuda_lib.fp8_scale_update(S["amax"], S["hist"], fp8_max, oracle.AMAX_MAX, 0,
+                                          S["scale"], S["nxt"])
+            outs.append([c["q"] for c in casts])
+        cuda_lib.fp8t_check_device_error()
+        for a, b in zip(*outs):
+            assert torch.equal(a, b)
+        for key in ("scale", "hist", "amax", "used", "nxt"):
+            assert torch.equal(state[0][key], state[1][key]), (t, key)

@@ -9,7 +9,7 @@ import torch
 
 import oracle
 from optimizer_fp8_cast_b200 import synth
-from tests._gpu import bf16_bits, dev_scalar, sample_positions, u8
+from tests._gpu import bf16_bits, dev_scalar, f32, sample_positions, u8
 from tests._pins import gemm_within_tolerance
 
 pytestmark = pytest.mark.gpu
@@ -125,3 +125,40 @@ def test_grouped_launch_mixed_problems(cuda_lib):
     for p in probs:
         R, ab = oracle.gemm(u8(p["A"]), p["a_fmt"], u8(p["B"]), p["b_fmt"], p["sa"], p["sb"], want_abs=True)
         assert gemm_within_tolerance(bf16_bits(p["D"]), R, ab).all()
+
+
+def test_grouped_launch_with_sum_of_squares(cuda_lib):
+    """fp8_gemm_multi_sumsq: D as in fp8_gemm_multi, plus the FP64 sum of f32(D)^2 over the
+    flagged problems only (the AdamW global-norm input, "算子与编译器" FP8 训练主路径图), across two
+    launch tables and ragged tiles; a repeated call gives the identical bits and the workspace
+    ticket is left at zero."""
+    rng = np.random.default_rng(43)
+    shapes = [(144, 272, 48), (512, 256, 256), (16, 16, 16), (400, 528, 1040), (256, 768, 128)]
+    probs = []
+    for i in range(27):                                  # 27 problems: two launch tables
+        M, N, K = shapes[i % len(shapes)]
+        af, bf = PAIRS[i % 4]
+        A = random_codes(M, K, af, 300 + i)
+        B = random_codes(N, K, bf, 400 + i)
+        sa, sb = float(rng.uniform(0.01, 1)), float(rng.uniform(0.01, 1))
+        probs.append(dict(A=A, a_fmt=af, B=B, b_fmt=bf, a_scale_inv=dev_scalar(sa),
+                          b_scale_inv=dev_scalar(sb), sumsq=(i % 3 == 1) or i == 26,
+                          D=torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda"),
+                          sa=sa, sb=sb))
+    descs = [{k: v for k, v in p.items() if k not in ("sa", "sb")} for p in probs]
+    ws = torch.zeros(cuda_lib.fp8_gemm_sumsq_workspace_bytes(descs), dtype=torch.uint8, device="cuda")
+    out = torch.zeros(1, dtype=torch.float64, device="cuda")
+    cuda_lib.fp8_gemm_multi_sumsq(descs, out, ws)
+    cuda_lib.fp8t_check_device_error()
+    first = out.item()
+    for p in probs:
+        R, ab = oracle.gemm(u8(p["A"]), p["a_fmt"], u8(p["B"]), p["b_fmt"], p["sa"], p["sb"], want_abs=True)
+        assert gemm_within_tolerance(bf16_bits(p["D"]), R, ab).all()
+    squares = np.concatenate([np.square(f32(p["D"].float()).astype(np.float64)).reshape(-1)
+                              for p in probs if p["sumsq"]])
+    exact = float(np.sum(np.sort(squares)))
+    assert abs(first - exact) <= 1e-13 * exact
+    assert ws[:4].view(torch.int32).item() == 0
+    cuda_lib.fp8_gemm_multi_sumsq(descs, out, ws)
+    cuda_lib.fp8t_check_device_error()
+    assert np.float64(out.item()).view(np.uint64) == np.float64(first).view(np.uint64)

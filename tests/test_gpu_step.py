@@ -23,17 +23,20 @@ pytestmark = pytest.mark.gpu
 FMT = (oracle.E4M3, oracle.E4M3, oracle.E5M2)
 
 
-def make_step(wl, algo=None, margin=None, H=None, counters=True):
+def make_step(wl, algo=None, margin=None, H=None, counters=True, fused=True):
+    """fused: scale update in the cast launch, dW sum of squares in the wgrad epilogue and (when
+    no counters are kept) the next W cast inside AdamW; False: every stage its own launch."""
     w0 = [synth.linear_weight(wl, k, "cuda") for k in range(len(wl.layers))]
     return Fp8LinearStep([(i, o) for _, i, o in wl.layers], wl.tokens,
                          H or wl.history_len, algo or wl.algo,
                          wl.margin if margin is None else margin, wl.adamw, w0, "cuda",
-                         counters=counters)
+                         counters=counters, fused_update=fused, fused_norm=fused, fused_wcast=fused)
 
 
 def snapshot(st):
     return dict(scale=f32(st.scale), hist=f32(st.history),
                 W=[bf16_bits(l.W) for l in st.layers], master=[f32(l.master) for l in st.layers],
+                Wq=[u8(l.Wq) for l in st.layers], WqT=[u8(l.WqT) for l in st.layers],
                 m=[f32(l.m) for l in st.layers], v=[f32(l.v) for l in st.layers],
                 counters=st.counters.cpu().numpy().astype(np.uint64).copy() if st.counters is not None else None)
 
@@ -46,23 +49,26 @@ def check_step(st, pre, xs, dys, gemm_full=True, gemm_samples=2048, cast_check=T
     sinv_used = np.array([np.float32(1.0) / np.float32(s) for s in pre["scale"]], np.float32)
     for k, L in enumerate(st.layers):
         srcs = (bf16_bits(xs[k]), pre["W"][k], bf16_bits(dys[k]))
-        outs = ((L.Xq, L.XqT), (L.Wq, L.WqT), (L.dYq, L.dYqT))
+        # the W codes this step's GEMMs read: cast during the previous AdamW when fused
+        wq = (pre["Wq"][k], pre["WqT"][k]) if st.fused_wcast else (u8(L.Wq), u8(L.WqT))
+        outs = ((u8(L.Xq), u8(L.XqT)), wq, (u8(L.dYq), u8(L.dYqT)))
         for r in range(3):
             i = 3 * k + r
             if cast_check:
                 q, qT, a, si, c = oracle.cast_transpose_amax(srcs[r], FMT[r], pre["scale"][i])
-                assert np.array_equal(u8(outs[r][0]), q), f"layer {k} role {r} codes"
-                assert np.array_equal(u8(outs[r][1]), qT), f"layer {k} role {r} transposed"
+                assert np.array_equal(outs[r][0], q), f"layer {k} role {r} codes"
+                assert np.array_equal(outs[r][1], qT), f"layer {k} role {r} transposed"
                 if cnt_ref is not None:
                     cnt_ref[i] += c
             else:
                 _, _, a, si, _ = oracle.cast_transpose_amax(srcs[r], FMT[r], pre["scale"][i], False, False)
             amax_ref[i] = a
         sx, sw, sdy = sinv_used[3 * k], sinv_used[3 * k + 1], sinv_used[3 * k + 2]
-        gemms = ((L.Xq, 0, L.WqT, 0, sx, sw, L.Y), (L.dYq, 1, L.Wq, 0, sdy, sw, L.dX),
-                 (L.XqT, 0, L.dYqT, 1, sx, sdy, L.dW))
-        for A, af, B, bf, sa, sb, D in gemms:
-            Ah, Bh, Dh = u8(A), u8(B), bf16_bits(D)
+        (Xq, XqT), (Wq, WqT), (dYq, dYqT) = outs
+        gemms = ((Xq, 0, WqT, 0, sx, sw, L.Y), (dYq, 1, Wq, 0, sdy, sw, L.dX),
+                 (XqT, 0, dYqT, 1, sx, sdy, L.dW))
+        for Ah, af, Bh, bf, sa, sb, D in gemms:
+            Dh = bf16_bits(D)
             if gemm_full:
                 R, ab = oracle.gemm(Ah, af, Bh, bf, sa, sb, want_abs=True)
                 assert gemm_within_tolerance(Dh, R, ab).all()
@@ -72,13 +78,19 @@ def check_step(st, pre, xs, dys, gemm_full=True, gemm_samples=2048, cast_check=T
                 assert gemm_within_tolerance(Dh[ii, jj], R, ab).all()
     # amax (entry 0 of each history row) and the scale update; consumed amax slots are reset
     assert np.array_equal(f32(st.history)[:, 0].view(np.uint32), amax_ref.view(np.uint32))
-    assert not st.amax.any().item()
+    if not st.fused_wcast:
+        assert not st.amax.any().item()
     hist, scale = pre["hist"].copy(), pre["scale"].copy()
     sinv = np.zeros_like(scale)
     oracle.scale_update(amax_ref, hist, f32(st.fp8_max), st.algo, st.margin, scale, sinv)
     assert np.array_equal(f32(st.history).view(np.uint32), hist.view(np.uint32))
     assert np.array_equal(f32(st.scale).view(np.uint32), scale.view(np.uint32))
     assert np.array_equal(f32(st.scale_inv).view(np.uint32), sinv.view(np.uint32))
+    if st.fused_wcast:                     # W's inverse scale is already the next step's
+        for k in range(len(st.layers)):
+            sinv_used[3 * k + 1] = np.float32(1.0) / scale[3 * k + 1]
+    assert np.array_equal(f32(st.sinv_used).view(np.uint32), sinv_used.view(np.uint32))
+    assert st.ticket.item() == 0 and st.adamw_ticket.item() == 0
     if cnt_ref is not None and cast_check:
         assert np.array_equal(st.counters.cpu().numpy().astype(np.uint64), cnt_ref)
     # AdamW on the GPU's own dW
@@ -96,11 +108,26 @@ def check_step(st, pre, xs, dys, gemm_full=True, gemm_samples=2048, cast_check=T
             assert ulp_distance_f32(f32(got).reshape(-1), ref.reshape(-1)).max() <= 4
         wg = bf16_bits(L.W).reshape(-1)
         assert np.abs(wg.astype(np.int32) - Wref[k].astype(np.int32)).max() <= 1
+        if st.fused_wcast:
+            # AdamW cast the new weight with the next step's scale: codes, amax slot
+            i = 3 * k + 1
+            q, qT, a, _, _ = oracle.cast_transpose_amax(bf16_bits(L.W), oracle.E4M3, scale[i],
+                                                         cast_check, cast_check)
+            if cast_check:
+                assert np.array_equal(u8(L.Wq), q) and np.array_equal(u8(L.WqT), qT)
+            assert np.float32(st.amax[i].item()).view(np.uint32) == np.float32(a).view(np.uint32)
+            assert st.amax[3 * k].item() == 0 and st.amax[3 * k + 2].item() == 0
 
 
-def test_linear256_three_steps(cuda_lib):
+@pytest.mark.parametrize("fused,counters", [(True, False), (True, True), (False, True)],
+                         ids=["all-fused", "fused-with-counters", "separate-launches"])
+def test_linear256_three_steps(cuda_lib, fused, counters):
+    """Three steps in full. all-fused: scale update in the cast launch, dW sum of squares in the
+    wgrad epilogue, next W cast in AdamW (three launches per step); with counters the W cast
+    stays in the cast launch; separate-launches: every stage its own kernel."""
     wl = synth.LINEAR256
-    st = make_step(wl)
+    st = make_step(wl, fused=fused, counters=counters)
+    assert st.fused_wcast == (fused and not counters)
     for t in range(wl.steps):
         xs, dys = zip(*[synth.linear_inputs(wl, k, t, "cuda") for k in range(len(wl.layers))])
         pre = snapshot(st)
@@ -115,7 +142,7 @@ def test_linear256_step_in_cuda_graph(cuda_lib):
     AdamW tolerance (the graph forms the bias corrections on the device)."""
     wl = synth.LINEAR256
     xs, dys = zip(*[synth.linear_inputs(wl, k, 0, "cuda") for k in range(len(wl.layers))])
-    eager = make_step(wl)
+    eager = make_step(wl, counters=False)
     for _ in range(3):
         eager.step(xs, dys)
     graphed = Fp8LinearStep([(i, o) for _, i, o in wl.layers], wl.tokens, wl.history_len, wl.algo,
@@ -167,7 +194,7 @@ def test_block7b_one_step(cuda_lib):
     free, _ = torch.cuda.mem_get_info()
     if free < 40e9:
         pytest.skip("needs ~30 GB of free device memory")
-    st = make_step(wl, counters=True)
+    st = make_step(wl, counters=False)
     xs, dys = zip(*[synth.linear_inputs(wl, k, 0, "cuda") for k in range(len(wl.layers))])
     pre = snapshot(st)
     st.step(xs, dys)

@@ -62,3 +62,47 @@ def test_gemm_waits_expire_and_context_survives(cuda_lib, mode):
     ii = rng.integers(0, M, 512); jj = rng.integers(0, N, 512)
     R, ab = oracle.gemm_at(u8(A), 0, u8(B), 0, 1.0, 1.0, ii, jj)
     assert gemm_within_tolerance(bf16_bits(D)[ii, jj], R, ab).all()
+
+
+def test_expired_cast_leaves_scale_state_alone(cuda_lib):
+    """The cast launch that also updates the scales: when its waits expire, its amax may be
+    incomplete, so the last CTA leaves history, scale and amax slot as they were (and resets
+    its ticket); the next call performs the update normally."""
+    x = (torch.randn(4096, 2048) * 3).to(torch.bfloat16).cuda()
+    scale = torch.tensor([2.0], device="cuda")
+    hist = torch.full((16,), 5.0, device="cuda")
+    amax = torch.zeros(1, device="cuda")
+    used, nxt = torch.zeros(1, device="cuda"), torch.zeros(1, device="cuda")
+    ticket = torch.zeros(1, dtype=torch.int32, device="cuda")
+    casts = [dict(x=x, fmt=oracle.E4M3, scale=scale, q=torch.empty(4096, 2048, dtype=torch.uint8, device="cuda"),
+                  amax=amax, scale_inv=used)]
+    ups = [dict(history=hist, scale_inv_next=nxt)]
+    _run_expired(cuda_lib, 1, lambda: cuda_lib.fp8_cast_transpose_amax_update_multi(
+        casts, ups, oracle.AMAX_MAX, 0, ticket))
+    assert scale.item() == 2.0 and nxt.item() == 0.0 and ticket.item() == 0
+    assert torch.equal(hist, torch.full((16,), 5.0, device="cuda"))
+    amax.zero_()
+    cuda_lib.fp8_cast_transpose_amax_update_multi(casts, ups, oracle.AMAX_MAX, 0, ticket)
+    cuda_lib.fp8t_check_device_error()
+    a = float(x.float().abs().max())
+    assert hist[0].item() == a and hist[1].item() == 5.0 and amax.item() == 0.0
+    assert scale.item() == np.float32(448.0) / np.float32(max(a, 5.0))
+
+
+def test_expired_gemm_sum_of_squares_is_nan(cuda_lib):
+    """fp8_gemm_multi_sumsq with expired epilogue waits reports a NaN sum (so a following AdamW
+    skips its update) and leaves its workspace ticket at zero."""
+    rng = np.random.default_rng(9)
+    A = torch.from_numpy(rng.integers(0x20, 0x48, (1024, 2048)).astype(np.uint8)).cuda()
+    B = torch.from_numpy(rng.integers(0x20, 0x48, (1024, 2048)).astype(np.uint8)).cuda()
+    one = dev_scalar(1.0)
+    g = [dict(A=A, a_fmt=0, B=B, b_fmt=0, a_scale_inv=one, b_scale_inv=one, sumsq=True,
+              D=torch.empty(1024, 1024, dtype=torch.bfloat16, device="cuda"))]
+    ws = torch.zeros(cuda_lib.fp8_gemm_sumsq_workspace_bytes(g), dtype=torch.uint8, device="cuda")
+    out = torch.zeros(1, dtype=torch.float64, device="cuda")
+    _run_expired(cuda_lib, 2, lambda: cuda_lib.fp8_gemm_multi_sumsq(g, out, ws))
+    assert np.isnan(out.item()) and ws[:4].view(torch.int32).item() == 0
+    cuda_lib.fp8_gemm_multi_sumsq(g, out, ws)
+    cuda_lib.fp8t_check_device_error()
+    d = g[0]["D"].float().double()
+    assert abs(out.item() - float((d * d).sum())) <= 1e-12 * float((d * d).sum())
