@@ -163,13 +163,14 @@ def run_ours(args, rank, world, local_rank):
                        wl.margin, wl.adamw, [synth.linear_weight(wl, k, dev) for k in range(nl)],
                        dev, device_step=True, fused_update=not args.separate_scale_update,
                        fused_norm=not args.separate_norm_pass,
-                       fused_wcast=not args.separate_weight_cast)
+                       fused_wcast=not args.separate_weight_cast, transposes=args.transposes,
+                       recipe=args.recipe)
     batches = [list(zip(*[synth.linear_inputs(wl, k, t, dev) for k in range(nl)])) for t in range(2)]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     # one timing window per kernel launch of the step (the scale update runs in the last CTA of
     # the cast launch unless --separate-scale-update)
     stages = [("cast", None), ("gemm", None), ("adamw", None)]
-    if args.separate_scale_update:
+    if args.separate_scale_update and args.recipe == "delayed":
         stages.insert(2, ("scale update", None))
     NEV = len(stages) + 1
 
@@ -178,7 +179,10 @@ def run_ours(args, rank, world, local_rank):
         rec = (lambda i: ev[i].record()) if ev is not None else (lambda i: None)
         rec(0)
         for i, (name, kw) in enumerate(stages):
-            if name == "cast":                    # grouped: X, W -> E4M3, dY -> E5M2
+            if name == "cast" and st.recipe == "current":
+                st.amax.zero_()
+                st.cast_all_current(xs, dys)      # amax launch, then the grouped cast
+            elif name == "cast":                  # grouped: X, W -> E4M3, dY -> E5M2
                 st.cast_all(xs, dys, update=st.fused_update)
             elif name == "gemm":                  # grouped: every fprop, dgrad and wgrad
                 st.gemm_all(sumsq=st.fused_norm)
@@ -248,10 +252,12 @@ def run_ours(args, rank, world, local_rank):
     # per-kernel figures (this rank), averaged over the timed steps
     avg = {name: statistics.mean(s[i] for s in stage_ms) for i, (name, _) in enumerate(stages)}
     gemm_achieved = flop_step / (avg["gemm"] * 1e-3) / 1e12
-    # algorithmic bytes of the launches as configured: the W cast (4 B/param) moves from the
-    # cast launch into AdamW as 2 B/param of codes (the weight it reads is already in registers)
-    cast_bytes = nums["cast_bytes"] - (4 * nums["params"] if st.fused_wcast else 0)
-    adamw_bytes = ((28 + (2 if st.fused_wcast else 0)) * nums["params"]
+    # algorithmic bytes of the launches as configured: a cast moves 2 B in and 1 B of codes out
+    # per element (+1 B with the transposed copy); the W cast moves from the cast launch into
+    # AdamW as 1 B/param of codes (the new weight is already in registers there)
+    per_el = (4 if st.transposes else 3) + (2 if st.recipe == "current" else 0)
+    cast_bytes = nums["cast_bytes"] // 4 * per_el - (per_el * nums["params"] if st.fused_wcast else 0)
+    adamw_bytes = ((28 + (1 if st.fused_wcast else 0)) * nums["params"]
                    + (0 if st.fused_norm else 2 * nums["params"]))
     cast_gbs = cast_bytes / (avg["cast"] * 1e-3) / 1e9
     adamw_gbs = adamw_bytes / (avg["adamw"] * 1e-3) / 1e9
@@ -294,16 +300,21 @@ def run_ours(args, rank, world, local_rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "fp8 (e4m3/e5m2 operands, f32 accumulate)",
         "data": "synthetic",
         "config": {"workload": wl.name, "tokens": wl.tokens,
-                   "layers_in_out": shapes, "recipe": "HYBRID, delayed per-tensor scaling",
+                   "layers_in_out": shapes,
+                   "recipe": f"HYBRID, {args.recipe} per-tensor scaling",
                    "history_len": wl.history_len, "amax_algo": wl.algo, "margin": wl.margin,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "launch": "eager" if args.eager else "CUDA graph per step (AdamW step counter on the device)",
-                   "scale_update": "separate launch" if args.separate_scale_update
+                   "scale_update": "none (current scaling)" if args.recipe == "current"
+                                   else "separate launch" if args.separate_scale_update
                                    else "in the last CTA of the cast launch",
                    "grad_sum_of_squares": "AdamW norm pass" if args.separate_norm_pass
                                           else "in the wgrad GEMM epilogue",
                    "weight_cast": "in AdamW (next step's codes)" if st.fused_wcast
                                   else "in the cast launch",
+                   "operands": "K-major only (transposed FP8 copies written by the casts)"
+                               if st.transposes else "no transposed copies (wgrad A, B and fprop B "
+                                                     "read MN-major by tcgen05)",
                    "l2": "flushed before every timed step (256 MiB write)"},
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": nums["h2d"],
                 "d2h_bytes_per_step": nums["d2h"], "ms_per_step": round(e2e_total / n_e2e, 4),
@@ -522,9 +533,12 @@ def oracle_sample_step(oracle, host, wl, rows_div):
 
 def host_copies(st, batch):
     from optimizer_fp8_cast_b200.synth import bf16_bits, u8
+    import numpy as np
     L = st.layers[0]
+    t = lambda q, qT: u8(qT) if qT is not None else np.ascontiguousarray(u8(q).T)
     return dict(X=bf16_bits(batch[0]), dY=bf16_bits(batch[1]), W=bf16_bits(L.W), Xq=u8(L.Xq),
-                XqT=u8(L.XqT), Wq=u8(L.Wq), WqT=u8(L.WqT), dYq=u8(L.dYq), dYqT=u8(L.dYqT),
+                XqT=t(L.Xq, L.XqT), Wq=u8(L.Wq), WqT=t(L.Wq, L.WqT), dYq=u8(L.dYq),
+                dYqT=t(L.dYq, L.dYqT),
                 master=L.master.detach().cpu().numpy().reshape(-1),
                 dW=bf16_bits(L.dW).reshape(-1))
 
@@ -597,6 +611,10 @@ def main(argv=None):
                          "adamw4e9_512t, stress1024_t2048")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager launches, not CUDA graphs")
+    ap.add_argument("--recipe", choices=("delayed", "current"), default="delayed",
+                    help="current: each scale from its own tensor's amax (an extra read)")
+    ap.add_argument("--transposes", action="store_true",
+                    help="casts also write q^T and every GEMM reads K-major operands")
     ap.add_argument("--separate-weight-cast", action="store_true",
                     help="cast W in the cast launch instead of inside AdamW")
     ap.add_argument("--separate-norm-pass", action="store_true",

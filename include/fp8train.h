@@ -116,6 +116,27 @@ typedef struct fp8t_cast_tensor {
 fp8t_status fp8_cast_transpose_amax_multi(const fp8t_cast_tensor* tensors, int32_t n_tensors,
                                           void* stream);
 
+/*
+ * fp8_cast_transpose_amax_current_multi — current ("just-in-time") scaling: each tensor's scale
+ * is derived from its own amax before it is cast, instead of from the history of earlier steps
+ * [P2 §四 FP8Tensor.quantize measures amax = max|x| of the tensor it quantises; P3 核心原理 gives
+ * scale = (FP8_MAX / amax) / 2^margin]. Per group of up to 8 tensors one amax launch reads the
+ * tensors, and its last CTA writes scale = (FP8_MAX / amax) * 2^-margin IN PLACE into
+ * tensors[i].d_scale (amax 0 gives 1; a NaN or infinite amax keeps the previous scale; an
+ * overflow gives FLT_MAX; FP8_MAX 448 for E4M3, 57344 for E5M2); then the cast of
+ * fp8_cast_transpose_amax_multi runs with that scale, with all its outputs (the amax slot
+ * max-accumulates as usual).
+ *   margin        0 .. 126.
+ *   d_workspace   FP8T_CURRENT_WORKSPACE_BYTES of device memory, 4-byte aligned, ZERO-FILLED
+ *                 before its first use and left zero by every call; concurrent calls need
+ *                 their own.
+ * Traffic: 2 B/element more than the delayed cast (the amax read).
+ */
+#define FP8T_CURRENT_WORKSPACE_BYTES 64
+fp8t_status fp8_cast_transpose_amax_current_multi(const fp8t_cast_tensor* tensors,
+                                                  int32_t n_tensors, int32_t margin,
+                                                  unsigned int* d_workspace, void* stream);
+
 /* The scale state fp8_cast_transpose_amax_update_multi updates for one tensor. */
 typedef struct fp8t_cast_update {
     float* d_amax_history;     /* history_len floats of this tensor, entry 0 newest (in/out) */
@@ -178,7 +199,15 @@ fp8t_status fp8_gemm(const void* A, fp8t_format a_fmt, const void* B, fp8t_forma
                      const float* d_a_scale_inv, const float* d_b_scale_inv,
                      void* D_bf16, void* stream);
 
-/* One GEMM of fp8_gemm_multi: the arguments of fp8_gemm. */
+/* How an operand of fp8_gemm_multi is stored. The 5th-generation tensor cores read 8-bit
+ * operands in either order, so no transposed copy is needed for the wgrad or fprop operands. */
+typedef enum fp8t_layout {
+    FP8T_K_MAJOR = 0,   /* A stored M x K row-major (B: N x K), the layout of fp8_gemm        */
+    FP8T_MN_MAJOR = 1   /* A stored K x M row-major (B: K x N): e.g. Xq itself for wgrad     */
+} fp8t_layout;
+
+/* One GEMM of fp8_gemm_multi: the arguments of fp8_gemm plus the operands' layouts (zero =
+ * K-major, so a descriptor filled like fp8_gemm's arguments computes the same product). */
 typedef struct fp8t_gemm_desc {
     const void* A;
     fp8t_format a_fmt;
@@ -188,6 +217,8 @@ typedef struct fp8t_gemm_desc {
     const float* d_a_scale_inv;
     const float* d_b_scale_inv;
     void* D_bf16;
+    fp8t_layout a_layout;
+    fp8t_layout b_layout;
 } fp8t_gemm_desc;
 
 /*
@@ -223,6 +254,61 @@ fp8t_status fp8_gemm_multi_sumsq(const fp8t_gemm_desc* gemms, int32_t n_gemms,
 /* Scratch bytes fp8_gemm_multi_sumsq needs (0 on invalid input or no selected problem). */
 size_t fp8_gemm_sumsq_workspace_bytes(const fp8t_gemm_desc* gemms, int32_t n_gemms,
                                       const int32_t* sumsq_of);
+
+/*
+ * MXFP8 block scaling [P2 §九, Blackwell microscaling: 32 values share one 8-bit E8M0 scale,
+ * each stored as FP8; P2 §三: micro scaling with E4M3 elements]. For every block of 32 values
+ * the shared exponent is X = floor(log2(amax)) - emax, emax = 8 for E4M3 (448 = 1.75 * 2^8)
+ * and 15 for E5M2, clamped to [-127, 127] (amax 0: -127; infinite amax: 127); the scale code is
+ * X + 127 (0xFF if the block holds a NaN, whose elements are then encoded at unit scale), and
+ * every element is q = encode_fmt(f32(x) * 2^-X) with the rounding and saturation of
+ * fp8_cast_transpose_amax.
+ *
+ * Scale layout ("atoms"): for an operand with MN rows (M for A, N for B) and K columns of the
+ * contraction, the scales are stored as [MN/128][K/128] atoms of 512 bytes; inside an atom,
+ * byte (i % 32) * 16 + (i / 32) * 4 + kb holds the scale of row i (0..127) and K-block kb
+ * (0..3, 32 values each). This is the order in which the tensor cores' scale copy reads them.
+ */
+typedef struct fp8t_mx_cast_tensor {
+    const void* x_bf16;      /* rows x cols BF16, row-major; rows, cols multiples of 128     */
+    int64_t rows, cols;
+    fp8t_format fmt;
+    void* q_row;             /* rows x cols codes, blocks along each row (K = cols), or NULL  */
+    void* scales_row;        /* atoms [rows/128][cols/128] (MN = rows, K = cols)              */
+    void* q_col;             /* rows x cols codes, blocks down each column (K = rows), or NULL */
+    void* scales_col;        /* atoms [cols/128][rows/128] (MN = cols, K = rows)              */
+} fp8t_mx_cast_tensor;
+
+/*
+ * fp8_mx_cast_multi — MX quantisation of several BF16 matrices, each into its row-wise copy
+ * (the K-major GEMM operand: Xq for fprop, dYq for dgrad, W for dgrad's B) and/or its
+ * column-wise copy (the MN-major operand: W for fprop's B, X and dY for wgrad), both in x's own
+ * row-major layout with their scale atoms. At least one copy per tensor. Up to 8 tensors share
+ * a launch. All pointers 16-byte aligned. Errors: INVALID_ARG, UNSUPPORTED_SHAPE (dimensions
+ * not multiples of 128), MISALIGNED, CUDA.
+ */
+fp8t_status fp8_mx_cast_multi(const fp8t_mx_cast_tensor* tensors, int32_t n_tensors, void* stream);
+
+/* One block-scaled GEMM of fp8_mx_gemm_multi: D = bf16(sum_k a_k b_k 2^(Xa + Xb)). */
+typedef struct fp8t_mx_gemm_desc {
+    const void* A;           /* M x K (K-major) or K x M (MN-major) codes                       */
+    const void* A_scales;    /* atoms [M/128][K/128]                                            */
+    fp8t_format a_fmt;
+    fp8t_layout a_layout;
+    const void* B;           /* N x K (K-major) or K x N (MN-major) codes                       */
+    const void* B_scales;    /* atoms [N/128][K/128]                                            */
+    fp8t_format b_fmt;
+    fp8t_layout b_layout;
+    int64_t M, N, K;         /* positive multiples of 128                                       */
+    void* D_bf16;            /* M x N BF16, row-major                                           */
+} fp8t_mx_gemm_desc;
+
+/*
+ * fp8_mx_gemm_multi — several MXFP8 GEMMs in one persistent launch on the block-scaled tensor
+ * cores (FP32 accumulation, BF16 output, no per-tensor scale). HOST array of n_gemms (1..4096)
+ * descriptors. Errors as fp8_gemm_multi; dimensions must be multiples of 128.
+ */
+fp8t_status fp8_mx_gemm_multi(const fp8t_mx_gemm_desc* gemms, int32_t n_gemms, void* stream);
 
 /*
  * fp8_scale_update — roll each tensor's amax history and compute the next scale
@@ -308,10 +394,11 @@ size_t fused_adamw_workspace_bytes(const fp8t_adamw_tensor* tensors, int32_t n_t
 /*
  * The FP8 cast of a tensor's NEW BF16 weight, done by the AdamW update that produces it: the
  * cast of fp8_cast_transpose_amax applied to weight_bf16 viewed as rows x cols (row-major),
- * with the same element rule, outputs and amax accumulation. Under delayed scaling the scale
- * for the next step's weight cast is known once the scale update of the current step has run,
- * so the next step need not read the weight again [P1 优化器 kernel 的带宽账: every extra
- * kernel re-reads the parameters; P3 核心原理: delayed scaling uses the previous scale].
+ * with the same element rule, row-major codes and amax accumulation (no transposed copy: the
+ * GEMMs read the weight codes MN-major where they need the transpose). Under delayed scaling
+ * the scale for the next step's weight cast is known once the scale update of the current step
+ * has run, so the next step need not read the weight again [P1 优化器 kernel 的带宽账: every
+ * extra kernel re-reads the parameters; P3 核心原理: delayed scaling uses the previous scale].
  * rows = cols = 0 means no cast for this tensor.
  */
 typedef struct fp8t_adamw_cast {
@@ -319,7 +406,6 @@ typedef struct fp8t_adamw_cast {
     fp8t_format fmt;
     const float* d_scale;           /* 1 float: the scale of the next step's weight cast       */
     void* q_rowmajor;               /* rows x cols FP8 bytes, or NULL                          */
-    void* q_transposed;             /* cols x rows FP8 bytes, or NULL                          */
     float* d_amax_inout;            /* max-accumulated with max|new weight|                    */
     float* d_scale_inv_out;         /* 1/scale, or NULL                                        */
 } fp8t_adamw_cast;
@@ -401,7 +487,7 @@ const char* fp8t_status_string(fp8t_status status);
 /* Message describing the last failure on the calling thread ("" if none). */
 const char* fp8t_last_error_message(void);
 
-/* ABI version of this header: 1. */
+/* ABI version of this header: 2 (fp8t_gemm_desc carries the operand layouts). */
 int32_t fp8t_abi_version(void);
 
 #ifdef __cplusplus

@@ -14,16 +14,19 @@ import torch
 from . import _abi
 
 __all__ = ["fp8_cast_transpose_amax", "fp8_cast_transpose_amax_multi",
-           "fp8_cast_transpose_amax_update_multi", "fp8_gemm", "fp8_gemm_multi", "fp8_scale_update", "fused_adamw_multi_tensor",
+           "fp8_cast_transpose_amax_update_multi", "fp8_cast_transpose_amax_current_multi",
+           "CURRENT_WORKSPACE_BYTES", "fp8_gemm", "fp8_gemm_multi", "fp8_scale_update", "fused_adamw_multi_tensor",
            "fused_adamw_workspace_bytes", "fused_adamw_multi_tensor_noalloc",
            "fp8_gemm_multi_sumsq", "fp8_gemm_sumsq_workspace_bytes",
-           "fused_adamw_multi_tensor_presummed",
+           "fused_adamw_multi_tensor_presummed", "fp8_mx_cast_multi", "fp8_mx_gemm_multi",
+           "mx_scale_bytes",
            "fp8t_check_device_error", "fp8t_debug_expire_waits", "fp8t_set_wait_timeout_ns",
-           "Fp8TrainError", "E4M3", "E5M2", "AMAX_MAX", "AMAX_MOST_RECENT", "FP8_MAX", "load",
+           "Fp8TrainError", "E4M3", "E5M2", "K_MAJOR", "MN_MAJOR", "AMAX_MAX", "AMAX_MOST_RECENT", "FP8_MAX", "load",
            "LIB_PATH"]
 
 E4M3, E5M2 = 0, 1
 AMAX_MAX, AMAX_MOST_RECENT = 0, 1
+K_MAJOR, MN_MAJOR = 0, 1
 FP8_MAX = {E4M3: 448.0, E5M2: 57344.0}
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8train.so")
 
@@ -102,6 +105,19 @@ def fp8_cast_transpose_amax_multi(casts, stream=None):
            "fp8_cast_transpose_amax_multi")
 
 
+CURRENT_WORKSPACE_BYTES = 64
+
+
+def fp8_cast_transpose_amax_current_multi(casts, margin, workspace, stream=None):
+    """Current scaling: each tensor's scale (written into ``casts[i]["scale"]``) comes from its
+    own amax, then the casts of fp8_cast_transpose_amax_multi run with it. ``workspace``: a
+    zero-filled uint8 CUDA tensor of CURRENT_WORKSPACE_BYTES, left zero."""
+    assert workspace.numel() >= CURRENT_WORKSPACE_BYTES
+    _check(load().fp8_cast_transpose_amax_current_multi(_cast_array(casts), len(casts), int(margin),
+                                                        _ptr(workspace), _stream(stream)),
+           "fp8_cast_transpose_amax_current_multi")
+
+
 def fp8_cast_transpose_amax_update_multi(casts, updates, algo, margin, ticket, stream=None):
     """The casts of fp8_cast_transpose_amax_multi and, in the same launch, the scale update of
     those tensors: ``updates[i]`` holds ``history`` (this tensor's [H] float32 row, entry 0
@@ -129,15 +145,26 @@ def fp8_gemm(A, a_fmt, B, b_fmt, a_scale_inv, b_scale_inv, D, stream=None):
                            _ptr(b_scale_inv), _ptr(D), _stream(stream)), "fp8_gemm")
 
 
+def _gemm_shape(g):
+    """(M, N, K) of a descriptor dict; ``a_mn`` / ``b_mn`` mark operands stored MN-major
+    (A as [K, M], B as [K, N])."""
+    a_mn, b_mn = bool(g.get("a_mn")), bool(g.get("b_mn"))
+    K, M = g["A"].shape if a_mn else g["A"].shape[::-1]
+    K2, N = g["B"].shape if b_mn else g["B"].shape[::-1]
+    assert K == K2, "inner dimensions differ"
+    return M, N, K
+
+
 def _gemm_array(gemms):
     arr = (_abi.GemmDesc * len(gemms))()
     for i, g in enumerate(gemms):
-        A, B, D = g["A"], g["B"], g["D"]
-        M, K = A.shape
-        N, K2 = B.shape
-        assert K == K2 and D.shape == (M, N) and D.dtype == torch.bfloat16
-        arr[i] = _abi.GemmDesc(_ptr(A), int(g["a_fmt"]), _ptr(B), int(g["b_fmt"]), M, N, K,
-                               _ptr(g["a_scale_inv"]), _ptr(g["b_scale_inv"]), _ptr(D))
+        M, N, K = _gemm_shape(g)
+        D = g["D"]
+        assert D.shape == (M, N) and D.dtype == torch.bfloat16
+        arr[i] = _abi.GemmDesc(_ptr(g["A"]), int(g["a_fmt"]), _ptr(g["B"]), int(g["b_fmt"]), M, N, K,
+                               _ptr(g["a_scale_inv"]), _ptr(g["b_scale_inv"]), _ptr(D),
+                               MN_MAJOR if g.get("a_mn") else K_MAJOR,
+                               MN_MAJOR if g.get("b_mn") else K_MAJOR)
     return arr
 
 
@@ -146,8 +173,7 @@ def fp8_gemm_sumsq_workspace_bytes(gemms):
     flags = (C.c_int32 * len(gemms))(*[1 if g.get("sumsq") else 0 for g in gemms])
     arr = (_abi.GemmDesc * len(gemms))()                 # only the shapes are read
     for i, g in enumerate(gemms):
-        arr[i].M, arr[i].K = g["A"].shape
-        arr[i].N = g["B"].shape[0]
+        arr[i].M, arr[i].N, arr[i].K = _gemm_shape(g)
     return int(load().fp8_gemm_sumsq_workspace_bytes(arr, len(gemms), flags))
 
 
@@ -166,6 +192,40 @@ def fp8_gemm_multi(gemms, stream=None):
     """Several GEMMs in one persistent launch. ``gemms`` is a list of dicts with the arguments of
     fp8_gemm: A, a_fmt, B, b_fmt, a_scale_inv, b_scale_inv, D."""
     _check(load().fp8_gemm_multi(_gemm_array(gemms), len(gemms), _stream(stream)), "fp8_gemm_multi")
+
+
+def mx_scale_bytes(mn, k):
+    """Bytes of the scale atoms of an MX operand with mn rows (M or N) and contraction k."""
+    return (mn // 128) * (k // 128) * 512
+
+
+def fp8_mx_cast_multi(casts, stream=None):
+    """MXFP8 quantisation. ``casts``: dicts with x (BF16 [rows, cols]), fmt and q_row / sf_row
+    (row-wise copy: blocks of 32 along rows) and/or q_col / sf_col (column-wise copy: blocks of
+    32 down columns); codes are uint8 [rows, cols], scales uint8 tensors of mx_scale_bytes."""
+    arr = (_abi.MxCastTensor * len(casts))()
+    for i, c in enumerate(casts):
+        x = c["x"]
+        assert x.dtype == torch.bfloat16 and x.dim() == 2
+        rows, cols = x.shape
+        arr[i] = _abi.MxCastTensor(_ptr(x), rows, cols, int(c["fmt"]), _ptr(c.get("q_row")),
+                                   _ptr(c.get("sf_row")), _ptr(c.get("q_col")), _ptr(c.get("sf_col")))
+    _check(load().fp8_mx_cast_multi(arr, len(casts), _stream(stream)), "fp8_mx_cast_multi")
+
+
+def fp8_mx_gemm_multi(gemms, stream=None):
+    """Block-scaled FP8 GEMMs in one launch: dicts with A, a_sf, a_fmt, (a_mn), B, b_sf, b_fmt,
+    (b_mn), D; D = bf16(A . B^T) with the operands' block scales (no per-tensor scale)."""
+    arr = (_abi.MxGemmDesc * len(gemms))()
+    for i, g in enumerate(gemms):
+        M, N, K = _gemm_shape(g)
+        D = g["D"]
+        assert D.shape == (M, N) and D.dtype == torch.bfloat16
+        arr[i] = _abi.MxGemmDesc(_ptr(g["A"]), _ptr(g["a_sf"]), int(g["a_fmt"]),
+                                 MN_MAJOR if g.get("a_mn") else K_MAJOR, _ptr(g["B"]), _ptr(g["b_sf"]),
+                                 int(g["b_fmt"]), MN_MAJOR if g.get("b_mn") else K_MAJOR, M, N, K,
+                                 _ptr(D))
+    _check(load().fp8_mx_gemm_multi(arr, len(gemms), _stream(stream)), "fp8_mx_gemm_multi")
 
 
 def fp8_scale_update(amax, history, fp8_max, algo, margin, scale, scale_inv, stream=None):
@@ -227,7 +287,8 @@ def fused_adamw_multi_tensor_presummed(master, m, v, grads, weights, *, lr, beta
     """The AdamW step without its norm pass: ``grad_sumsq`` (float64 [1] on the device) holds
     the FP64 sum of f32(g)^2 over all gradients. ``ticket`` (zeroed int32 [1]) is required with
     ``step_counter``. ``casts``: None, or one entry per tensor, None or a dict (rows, cols, fmt,
-    scale, and optionally q, qT, amax, scale_inv) to cast that tensor's new BF16 weight."""
+    scale, and optionally q, amax, scale_inv) to cast that tensor's new BF16 weight (row-major
+    codes)."""
     arr, n = _tensor_table(master, m, v, grads, weights)
     assert grad_sumsq.dtype == torch.float64
     carr = None
@@ -236,8 +297,9 @@ def fused_adamw_multi_tensor_presummed(master, m, v, grads, weights, *, lr, beta
         carr = (_abi.AdamWCast * n)()
         for i, c in enumerate(casts):
             if c is not None:
+                assert c.get("qT") is None, "weight casts inside AdamW write row-major codes only"
                 carr[i] = _abi.AdamWCast(int(c["rows"]), int(c["cols"]), int(c["fmt"]),
-                                         _ptr(c["scale"]), _ptr(c.get("q")), _ptr(c.get("qT")),
+                                         _ptr(c["scale"]), _ptr(c.get("q")),
                                          _ptr(c.get("amax")), _ptr(c.get("scale_inv")))
     _check(load().fused_adamw_multi_tensor_presummed(arr, carr, n, float(lr), float(beta1), float(beta2),
                                                      float(eps), float(weight_decay), int(step),

@@ -19,8 +19,8 @@ class AdamWTensor(C.Structure):
 class AdamWCast(C.Structure):
     """fp8t_adamw_cast."""
     _fields_ = [("rows", C.c_int64), ("cols", C.c_int64), ("fmt", C.c_int), ("d_scale", C.c_void_p),
-                ("q_rowmajor", C.c_void_p), ("q_transposed", C.c_void_p),
-                ("d_amax_inout", C.c_void_p), ("d_scale_inv_out", C.c_void_p)]
+                ("q_rowmajor", C.c_void_p), ("d_amax_inout", C.c_void_p),
+                ("d_scale_inv_out", C.c_void_p)]
 
 
 class CastTensor(C.Structure):
@@ -40,7 +40,22 @@ class GemmDesc(C.Structure):
     """fp8t_gemm_desc."""
     _fields_ = [("A", C.c_void_p), ("a_fmt", C.c_int), ("B", C.c_void_p), ("b_fmt", C.c_int),
                 ("M", C.c_int64), ("N", C.c_int64), ("K", C.c_int64),
-                ("d_a_scale_inv", C.c_void_p), ("d_b_scale_inv", C.c_void_p), ("D_bf16", C.c_void_p)]
+                ("d_a_scale_inv", C.c_void_p), ("d_b_scale_inv", C.c_void_p), ("D_bf16", C.c_void_p),
+                ("a_layout", C.c_int), ("b_layout", C.c_int)]
+
+
+class MxCastTensor(C.Structure):
+    """fp8t_mx_cast_tensor."""
+    _fields_ = [("x_bf16", C.c_void_p), ("rows", C.c_int64), ("cols", C.c_int64), ("fmt", C.c_int),
+                ("q_row", C.c_void_p), ("scales_row", C.c_void_p), ("q_col", C.c_void_p),
+                ("scales_col", C.c_void_p)]
+
+
+class MxGemmDesc(C.Structure):
+    """fp8t_mx_gemm_desc."""
+    _fields_ = [("A", C.c_void_p), ("A_scales", C.c_void_p), ("a_fmt", C.c_int), ("a_layout", C.c_int),
+                ("B", C.c_void_p), ("B_scales", C.c_void_p), ("b_fmt", C.c_int), ("b_layout", C.c_int),
+                ("M", C.c_int64), ("N", C.c_int64), ("K", C.c_int64), ("D_bf16", C.c_void_p)]
 
 
 def declare(L):
@@ -54,6 +69,8 @@ def declare(L):
                                                        i32, i32, C.c_int, i32, vp, vp]
     L.fp8_gemm_multi.restype = C.c_int
     L.fp8_gemm_multi.argtypes = [C.POINTER(GemmDesc), i32, vp]
+    L.fp8_cast_transpose_amax_current_multi.restype = C.c_int
+    L.fp8_cast_transpose_amax_current_multi.argtypes = [C.POINTER(CastTensor), i32, i32, vp, vp]
     L.fp8_gemm_multi_sumsq.restype = C.c_int
     L.fp8_gemm_multi_sumsq.argtypes = [C.POINTER(GemmDesc), i32, C.POINTER(C.c_int32), vp, vp,
                                        C.c_size_t, vp]
@@ -64,6 +81,10 @@ def declare(L):
                                                      i32, f32, f32, f32,
                                                      f32, f32, i64, vp, f32, f32, vp, vp, vp, vp,
                                                      vp]
+    L.fp8_mx_cast_multi.restype = C.c_int
+    L.fp8_mx_cast_multi.argtypes = [C.POINTER(MxCastTensor), i32, vp]
+    L.fp8_mx_gemm_multi.restype = C.c_int
+    L.fp8_mx_gemm_multi.argtypes = [C.POINTER(MxGemmDesc), i32, vp]
     L.fp8_gemm.restype = C.c_int
     L.fp8_gemm.argtypes = [vp, C.c_int, vp, C.c_int, i64, i64, i64, vp, vp, vp, vp]
     L.fp8_scale_update.restype = C.c_int

@@ -39,6 +39,7 @@ constexpr int kSmemBytes = 2 * kInBytes + 2 * kQBytes + 1024 /*alignment*/ + 64 
 struct alignas(64) Tensor {
   CUtensorMap x_map;               // BF16 [rows][cols], 128 x 128 boxes
   CUtensorMap qt_map;              // FP8 [cols][rows] (q^T), 128 x 128 boxes
+  const uint4* x;                  // the same BF16 data (row-major kernel), null: update only
   float* scale;                    // read by the cast; replaced by the next scale when updating
   unsigned int* amax_bits;
   float* scale_inv;
@@ -129,6 +130,29 @@ __device__ __forceinline__ uint32_t quantise_segment(const Tensor& T, const uint
   return m;
 }
 
+// The last CTA of a launch to finish (ticket counter) updates the scale state of every tensor of
+// the launch, one warp per tensor. Called by every thread of every CTA once its own work, amax
+// atomics included, is issued.
+__device__ __forceinline__ void last_cta_update(const Group& g) {
+  __shared__ int s_last;
+  __threadfence();                                 // this CTA's amax atomics before its ticket
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(g.ticket, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // a launch whose waits expired leaves the scale state alone (its amax may be incomplete)
+  const bool ok = *reinterpret_cast<volatile unsigned int*>(&g_error_word) == 0u;
+  const int warp = threadIdx.x >> 5;
+  if (ok && warp < g.n) {
+    const Tensor& T = g.t[warp];
+    scale::warp_update(reinterpret_cast<float*>(T.amax_bits), T.hist, g.H,
+                       T.fmt == 0 ? 448.0f : 57344.0f, g.algo_max != 0, g.margin, T.scale,
+                       T.scale_inv_next);
+  }
+  if (threadIdx.x == 0) atomicExch(g.ticket, 0u);
+}
+
 template <bool COUNT>
 __global__ void __launch_bounds__(kThreads, 2) k_cast_transpose_amax(const __grid_constant__ Group g) {
   extern __shared__ uint8_t smem_raw[];
@@ -201,9 +225,11 @@ __global__ void __launch_bounds__(kThreads, 2) k_cast_transpose_amax(const __gri
           *reinterpret_cast<uint4*>(T.q + gr * T.cols + gc) =
               make_uint4(packed[0], packed[1], packed[2], packed[3]);
       }
-      const int pchunk = c16 ^ ((row >> 4) & 7);
-      *reinterpret_cast<uint4*>(&stage[row * 32 + pchunk * 4]) =
-          make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      if (T.has_qt) {
+        const int pchunk = c16 ^ ((row >> 4) & 7);
+        *reinterpret_cast<uint4*>(&stage[row * 32 + pchunk * 4]) =
+            make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      }
     }
     vmax = warp_max_u32(vmax);
     nsat = warp_add_u32(nsat);
@@ -270,11 +296,11 @@ __global__ void __launch_bounds__(kThreads, 2) k_cast_transpose_amax(const __gri
         *reinterpret_cast<uint4*>(qt_tile + (4 * jg + c) * kTile + 16 * ig) =
             make_uint4(o[c][0], o[c][1], o[c][2], o[c][3]);
       fence_proxy_async_smem();                    // visible to the TMA store
-    }
-    __syncthreads();                               // q^T tile complete; staged tile free again
-    if (tid == 0 && T.has_qt) {
-      tma_store_2d(&T.qt_map, smem_u32(qt_tile), static_cast<int32_t>(r0), static_cast<int32_t>(c0));
-      bulk_commit_group();
+      __syncthreads();                             // q^T tile complete; staged tile free again
+      if (tid == 0) {
+        tma_store_2d(&T.qt_map, smem_u32(qt_tile), static_cast<int32_t>(r0), static_cast<int32_t>(c0));
+        bulk_commit_group();
+      }
     }
   }
 
@@ -284,26 +310,66 @@ __global__ void __launch_bounds__(kThreads, 2) k_cast_transpose_amax(const __gri
       if (pending & (1u << b)) mbar_wait(smem_u32(&full[b]), (pending_ph >> b) & 1u, kDrainLimitNs);
     bulk_wait_group<0>();                          // stores complete before the CTA exits
   }
-  if (!g.update) return;
+  if (g.update) last_cta_update(g);
+}
 
-  // ---- the last CTA to finish updates the scale state of every tensor of the launch
-  __shared__ int s_last;
-  if (tid == 0) {
-    __threadfence();                               // this CTA's amax atomics before its ticket
-    s_last = atomicAdd(g.ticket, 1u) == gridDim.x - 1;
+// Row-major-only casts (no tensor of the launch wants q^T): a plain streaming kernel. Each
+// thread converts 16-element segments (two 16-byte loads, one 16-byte store), two segments in
+// flight, grid-striding over one tensor after another; amax and counters are reduced per warp
+// (one atomic per warp and tensor).
+template <bool COUNT>
+__global__ void __launch_bounds__(kThreads, 4) k_cast_rowmajor(const __grid_constant__ Group g) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
+  for (int t = 0; t < g.n; ++t) {
+    const Tensor& T = g.t[t];
+    if (!T.x) continue;                            // scale update only
+    const uint4* __restrict__ x = T.x;
+    uint4* __restrict__ q = reinterpret_cast<uint4*>(T.q);
+    const int64_t nseg = T.rows * T.cols / 16;
+    const float s = __ldg(T.scale);
+    uint32_t vmax = 0, nsat = 0, nzero = 0, nnonfinite = 0;
+    int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + tid;
+    for (; i + stride < nseg; i += 2 * stride) {
+      uint4 in0[2], in1[2];
+      in0[0] = ld_stream_u4(x + 2 * i);
+      in0[1] = ld_stream_u4(x + 2 * i + 1);
+      in1[0] = ld_stream_u4(x + 2 * (i + stride));
+      in1[1] = ld_stream_u4(x + 2 * (i + stride) + 1);
+      uint32_t p0[4] = {0u, 0u, 0u, 0u}, p1[4] = {0u, 0u, 0u, 0u};
+      vmax = max(vmax, quantise_segment<COUNT>(T, in0, s, p0, nsat, nzero, nnonfinite));
+      vmax = max(vmax, quantise_segment<COUNT>(T, in1, s, p1, nsat, nzero, nnonfinite));
+      if (q) {
+        q[i] = make_uint4(p0[0], p0[1], p0[2], p0[3]);
+        q[i + stride] = make_uint4(p1[0], p1[1], p1[2], p1[3]);
+      }
+    }
+    for (; i < nseg; i += stride) {
+      uint4 in[2];
+      in[0] = ld_stream_u4(x + 2 * i);
+      in[1] = ld_stream_u4(x + 2 * i + 1);
+      uint32_t p[4] = {0u, 0u, 0u, 0u};
+      vmax = max(vmax, quantise_segment<COUNT>(T, in, s, p, nsat, nzero, nnonfinite));
+      if (q) q[i] = make_uint4(p[0], p[1], p[2], p[3]);
+    }
+    vmax = warp_max_u32(vmax);
+    if (COUNT) {
+      nsat = warp_add_u32(nsat);
+      nzero = warp_add_u32(nzero);
+      nnonfinite = warp_add_u32(nnonfinite);
+    }
+    if (lane == 0) {
+      if (vmax > 0x7F80u) vmax = 0x7FC0u;          // canonical NaN
+      if (vmax) atomicMax(T.amax_bits, vmax << 16);
+      if (COUNT && T.counters) {
+        if (nsat) atomicAdd(T.counters + 0, static_cast<unsigned long long>(nsat));
+        if (nzero) atomicAdd(T.counters + 1, static_cast<unsigned long long>(nzero));
+        if (nnonfinite) atomicAdd(T.counters + 2, static_cast<unsigned long long>(nnonfinite));
+      }
+    }
+    if (T.scale_inv && blockIdx.x == 0 && tid == 0) *T.scale_inv = __fdiv_rn(1.0f, s);
   }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  // a launch whose waits expired leaves the scale state alone (its amax may be incomplete)
-  const bool ok = *reinterpret_cast<volatile unsigned int*>(&g_error_word) == 0u;
-  if (ok && warp < g.n) {
-    const Tensor& T = g.t[warp];
-    scale::warp_update(reinterpret_cast<float*>(T.amax_bits), T.hist, g.H,
-                       T.fmt == 0 ? 448.0f : 57344.0f, g.algo_max != 0, g.margin, T.scale,
-                       T.scale_inv_next);
-  }
-  if (tid == 0) atomicExch(g.ticket, 0u);
+  if (g.update) last_cta_update(g);
 }
 
 }  // namespace cast

@@ -14,8 +14,10 @@
 
 #include "fp8train.h"
 #include "cast_transpose_amax.cuh"
+#include "current_scaling.cuh"
 #include "fused_adamw.cuh"
 #include "gemm_tcgen05.cuh"
+#include "mx_cast.cuh"
 #include "scale_update.cuh"
 
 namespace {
@@ -43,7 +45,10 @@ struct DeviceInfo {
   int adamw_blocks_per_sm = 0;
   int adamw_cast_blocks_per_sm = 0;
   int gemm_clusters = 0;       // co-resident 2-CTA clusters of the GEMM kernel
+  int gemm_mx_clusters = 0;    // ... of its MXFP8 variant
+  int mx_cast_blocks_per_sm = 0;
   int cast_blocks_per_sm = 0;
+  int cast_rowmajor_blocks_per_sm = 0;
   void* noalloc_scratch = nullptr;   // device address of g_adamw_noalloc_scratch
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -74,8 +79,14 @@ fp8t_status current_device(DeviceInfo** out) {
                                                         fp8t::adamw::k_adamw_update<true>,
                                                         fp8t::adamw::kThreads, 0);
       if (e != cudaSuccess || d.adamw_cast_blocks_per_sm < 1) d.adamw_cast_blocks_per_sm = 1;
-      e = cudaFuncSetAttribute(fp8t::gemm::k_fp8_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      e = cudaFuncSetAttribute(fp8t::gemm::k_fp8_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                fp8t::gemm::kSmemBytes);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(fp8t::gemm::k_fp8_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 fp8t::gemm::kSmemBytesMX);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(fp8t::mx::k_mx_cast, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 fp8t::mx::kSmemBytes);
       if (e != cudaSuccess) {
         d.state = 0;
         return fail(FP8T_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
@@ -85,12 +96,26 @@ fp8t_status current_device(DeviceInfo** out) {
       cfg.blockDim = dim3(fp8t::gemm::kThreads, 1, 1);
       cfg.dynamicSmemBytes = fp8t::gemm::kSmemBytes;
       int clusters = 0;
-      e = cudaOccupancyMaxActiveClusters(&clusters, fp8t::gemm::k_fp8_gemm, &cfg);
+      e = cudaOccupancyMaxActiveClusters(&clusters, fp8t::gemm::k_fp8_gemm<false>, &cfg);
       if (e != cudaSuccess || clusters < 1) {
         (void)cudaGetLastError();
         clusters = sms / 2;
       }
       d.gemm_clusters = clusters;
+      cfg.dynamicSmemBytes = fp8t::gemm::kSmemBytesMX;
+      clusters = 0;
+      e = cudaOccupancyMaxActiveClusters(&clusters, fp8t::gemm::k_fp8_gemm<true>, &cfg);
+      if (e != cudaSuccess || clusters < 1) {
+        (void)cudaGetLastError();
+        clusters = sms / 2;
+      }
+      d.gemm_mx_clusters = clusters;
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.mx_cast_blocks_per_sm, fp8t::mx::k_mx_cast,
+                                                        fp8t::mx::kThreads, fp8t::mx::kSmemBytes);
+      if (e != cudaSuccess || d.mx_cast_blocks_per_sm < 1) {
+        (void)cudaGetLastError();
+        d.mx_cast_blocks_per_sm = 1;
+      }
       e = cudaFuncSetAttribute(fp8t::cast::k_cast_transpose_amax<false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, fp8t::cast::kSmemBytes);
       if (e == cudaSuccess)
@@ -99,6 +124,13 @@ fp8t_status current_device(DeviceInfo** out) {
       if (e != cudaSuccess) {
         d.state = 0;
         return fail(FP8T_ERR_CUDA, "cudaFuncSetAttribute(cast): %s", cudaGetErrorString(e));
+      }
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.cast_rowmajor_blocks_per_sm,
+                                                        fp8t::cast::k_cast_rowmajor<true>,
+                                                        fp8t::cast::kThreads, 0);
+      if (e != cudaSuccess || d.cast_rowmajor_blocks_per_sm < 1) {
+        (void)cudaGetLastError();
+        d.cast_rowmajor_blocks_per_sm = 1;
       }
       e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.cast_blocks_per_sm,
                                                         fp8t::cast::k_cast_transpose_amax<true>,
@@ -189,7 +221,7 @@ static __device__ __align__(256) unsigned char g_adamw_noalloc_scratch[FP8T_NOAL
 
 extern "C" {
 
-int32_t fp8t_abi_version(void) { return 1; }
+int32_t fp8t_abi_version(void) { return 2; }
 
 const char* fp8t_last_error_message(void) { return t_last_error.c_str(); }
 
@@ -212,13 +244,16 @@ const char* fp8t_status_string(fp8t_status s) {
 namespace {
 
 // Casts of n tensors in launches of up to eight; with `updates`, the last CTA of each launch also
-// performs the delayed-scaling update of that launch's tensors.
+// performs the delayed-scaling update of that launch's tensors; with `current_ws`, each launch
+// is preceded by the current-scaling amax pass that sets the scales it uses.
 fp8t_status cast_multi(const fp8t_cast_tensor* tensors, const fp8t_cast_update* updates,
                        int32_t n_tensors, int32_t history_len, fp8t_amax_algo algo, int32_t margin,
-                       unsigned int* d_ticket, void* stream) {
+                       unsigned int* d_ticket, unsigned int* current_ws, void* stream) {
   t_last_error.clear();
   if (!tensors || n_tensors < 1 || n_tensors > 4096)
     return fail(FP8T_ERR_INVALID_ARG, "fp8_cast_transpose_amax: tensors NULL or n_tensors out of range");
+  if (current_ws && (!aligned(current_ws, 4) || margin < 0 || margin > 126))
+    return fail(FP8T_ERR_INVALID_ARG, "fp8_cast_transpose_amax_current: misaligned workspace or margin outside 0..126");
   if (updates) {
     if (!d_ticket || !aligned(d_ticket, 4))
       return fail(FP8T_ERR_INVALID_ARG, "fp8_cast_transpose_amax_update: NULL or misaligned ticket");
@@ -299,6 +334,7 @@ fp8t_status cast_multi(const fp8t_cast_tensor* tensors, const fp8t_cast_update* 
         if (r != CUDA_SUCCESS) return fail(FP8T_ERR_CUDA, "cuTensorMapEncodeTiled (q^T store) failed (%d)", (int)r);
       }
       T.scale = const_cast<float*>(t.d_scale);      // written only by the update
+      T.x = static_cast<const uint4*>(t.x_bf16);
       T.amax_bits = reinterpret_cast<unsigned int*>(t.d_amax_inout);
       T.scale_inv = t.d_scale_inv_out;
       if (updates) {
@@ -323,14 +359,47 @@ fp8t_status cast_multi(const fp8t_cast_tensor* tensors, const fp8t_cast_update* 
       group.algo_max = algo == FP8T_AMAX_MAX ? 1 : 0;
       group.margin = margin;
     }
-    bool count = false;
-    for (int32_t i = b0; i < b1; ++i) count |= tensors[i].d_counters != nullptr;
+    bool count = false, any_qt = false;
+    for (int32_t i = b0; i < b1; ++i) {
+      count |= tensors[i].d_counters != nullptr;
+      any_qt |= tensors[i].q_transposed != nullptr;
+    }
     int64_t grid = std::min<int64_t>(tiles, static_cast<int64_t>(dev->sms) * dev->cast_blocks_per_sm);
     if (grid < 1) grid = 1;           // update-only entries: one CTA does the update
-    if (count)
+    if (current_ws) {                  // the scales of this group, from its own amax
+      fp8t::current::Group cg;
+      std::memset(&cg, 0, sizeof(cg));
+      cg.n = b1 - b0;
+      cg.margin = margin;
+      cg.ws = current_ws;
+      int64_t vecs = 0;
+      for (int32_t i = b0; i < b1; ++i) {
+        cg.x[i - b0] = static_cast<const uint4*>(tensors[i].x_bf16);
+        cg.nvec[i - b0] = tensors[i].rows * tensors[i].cols / 8;
+        cg.scale[i - b0] = const_cast<float*>(tensors[i].d_scale);
+        cg.fp8_max[i - b0] = tensors[i].fmt == FP8T_E4M3 ? 448.0f : 57344.0f;
+        vecs += cg.nvec[i - b0];
+      }
+      const int64_t cgrid = std::max<int64_t>(1, std::min<int64_t>(
+          (vecs + fp8t::current::kThreads - 1) / fp8t::current::kThreads, 4 * static_cast<int64_t>(dev->sms)));
+      fp8t::current::k_current_amax<<<static_cast<unsigned>(cgrid), fp8t::current::kThreads, 0,
+                                      as_stream(stream)>>>(cg);
+      if ((st = after_launch("current-scaling amax launch")) != FP8T_OK) return st;
+    }
+    if (!any_qt) {                     // row-major codes only: the streaming kernel
+      int64_t segs = 0;
+      for (int32_t i = b0; i < b1; ++i) segs += tensors[i].rows * tensors[i].cols / 16;
+      const int64_t rgrid = std::max<int64_t>(1, std::min<int64_t>(
+          (segs + kThreads - 1) / kThreads, static_cast<int64_t>(dev->sms) * dev->cast_rowmajor_blocks_per_sm));
+      if (count)
+        k_cast_rowmajor<true><<<static_cast<unsigned>(rgrid), kThreads, 0, as_stream(stream)>>>(group);
+      else
+        k_cast_rowmajor<false><<<static_cast<unsigned>(rgrid), kThreads, 0, as_stream(stream)>>>(group);
+    } else if (count) {
       k_cast_transpose_amax<true><<<static_cast<unsigned>(grid), kThreads, kSmemBytes, as_stream(stream)>>>(group);
-    else
+    } else {
       k_cast_transpose_amax<false><<<static_cast<unsigned>(grid), kThreads, kSmemBytes, as_stream(stream)>>>(group);
+    }
     if ((st = after_launch("fp8_cast_transpose_amax launch")) != FP8T_OK) return st;
   }
   return FP8T_OK;
@@ -342,7 +411,7 @@ extern "C" {
 
 fp8t_status fp8_cast_transpose_amax_multi(const fp8t_cast_tensor* tensors, int32_t n_tensors,
                                           void* stream) {
-  return cast_multi(tensors, nullptr, n_tensors, 0, FP8T_AMAX_MAX, 0, nullptr, stream);
+  return cast_multi(tensors, nullptr, n_tensors, 0, FP8T_AMAX_MAX, 0, nullptr, nullptr, stream);
 }
 
 fp8t_status fp8_cast_transpose_amax_update_multi(const fp8t_cast_tensor* tensors,
@@ -354,7 +423,19 @@ fp8t_status fp8_cast_transpose_amax_update_multi(const fp8t_cast_tensor* tensors
     t_last_error.clear();
     return fail(FP8T_ERR_INVALID_ARG, "fp8_cast_transpose_amax_update: updates NULL");
   }
-  return cast_multi(tensors, updates, n_tensors, history_len, algo, margin, d_ticket, stream);
+  return cast_multi(tensors, updates, n_tensors, history_len, algo, margin, d_ticket, nullptr,
+                    stream);
+}
+
+fp8t_status fp8_cast_transpose_amax_current_multi(const fp8t_cast_tensor* tensors,
+                                                  int32_t n_tensors, int32_t margin,
+                                                  unsigned int* d_workspace, void* stream) {
+  if (!d_workspace) {
+    t_last_error.clear();
+    return fail(FP8T_ERR_INVALID_ARG, "fp8_cast_transpose_amax_current: workspace NULL");
+  }
+  return cast_multi(tensors, nullptr, n_tensors, 0, FP8T_AMAX_MAX, margin, nullptr, d_workspace,
+                    stream);
 }
 
 fp8t_status fp8_cast_transpose_amax(const void* x_bf16, int64_t rows, int64_t cols, fp8t_format fmt,
@@ -398,6 +479,9 @@ fp8t_status gemm_multi(const fp8t_gemm_desc* gemms, int32_t n_gemms, const int32
       return fail(FP8T_ERR_INVALID_ARG, "fp8_gemm: problem %d: NULL pointer", i);
     if ((d.a_fmt != FP8T_E4M3 && d.a_fmt != FP8T_E5M2) || (d.b_fmt != FP8T_E4M3 && d.b_fmt != FP8T_E5M2))
       return fail(FP8T_ERR_INVALID_ARG, "fp8_gemm: problem %d: unknown format", i);
+    if ((d.a_layout != FP8T_K_MAJOR && d.a_layout != FP8T_MN_MAJOR) ||
+        (d.b_layout != FP8T_K_MAJOR && d.b_layout != FP8T_MN_MAJOR))
+      return fail(FP8T_ERR_INVALID_ARG, "fp8_gemm: problem %d: unknown operand layout", i);
     if (d.M <= 0 || d.N <= 0 || d.K <= 0)
       return fail(FP8T_ERR_INVALID_ARG, "fp8_gemm: problem %d: M, N, K must be > 0", i);
     if (d.M % 16 || d.N % 16 || d.K % 16 || d.M >= lim || d.N >= lim || d.K >= lim)
@@ -441,8 +525,14 @@ fp8t_status gemm_multi(const fp8t_gemm_desc* gemms, int32_t n_gemms, const int32
     for (int32_t i = b0; i < b1; ++i) {
       const fp8t_gemm_desc& d = gemms[i];
       Problem& P = group.p[i - b0];
-      if ((st = encode_kmajor(&P.a, d.A, d.M, d.K, kHalf)) != FP8T_OK) return st;
-      if ((st = encode_kmajor(&P.b, d.B, d.N, d.K, kHalf)) != FP8T_OK) return st;
+      // 128 x 128-byte boxes either way: [rows][K] (K-major) or [K][rows] (MN-major)
+      const bool a_mn = d.a_layout == FP8T_MN_MAJOR, b_mn = d.b_layout == FP8T_MN_MAJOR;
+      if ((st = a_mn ? encode_kmajor(&P.a, d.A, d.K, d.M, kBK)
+                     : encode_kmajor(&P.a, d.A, d.M, d.K, kHalf)) != FP8T_OK) return st;
+      if ((st = b_mn ? encode_kmajor(&P.b, d.B, d.K, d.N, kBK)
+                     : encode_kmajor(&P.b, d.B, d.N, d.K, kHalf)) != FP8T_OK) return st;
+      P.a_mn = a_mn ? 1 : 0;
+      P.b_mn = b_mn ? 1 : 0;
       // D (BF16 M x N): 32 x 32 boxes, 64-byte swizzle, written by the epilogue's TMA stores
       cuuint64_t dims[2] = {static_cast<cuuint64_t>(d.N), static_cast<cuuint64_t>(d.M)};
       cuuint64_t strides[1] = {static_cast<cuuint64_t>(d.N) * 2};
@@ -457,7 +547,7 @@ fp8t_status gemm_multi(const fp8t_gemm_desc* gemms, int32_t n_gemms, const int32
       P.M = static_cast<int32_t>(d.M);
       P.N = static_cast<int32_t>(d.N);
       P.K = static_cast<int32_t>(d.K);
-      P.idesc = make_idesc(d.a_fmt, d.b_fmt);
+      P.idesc = make_idesc(d.a_fmt, d.b_fmt, P.a_mn, P.b_mn);
       P.tiles_n = static_cast<int32_t>((d.N + kBN - 1) / kBN);
       P.tile_start = static_cast<int32_t>(tiles);
       P.sumsq_slot = -1;
@@ -471,7 +561,7 @@ fp8t_status gemm_multi(const fp8t_gemm_desc* gemms, int32_t n_gemms, const int32
     }
     group.total_tiles = static_cast<int32_t>(tiles);
     const int64_t grid = 2 * std::min<int64_t>(tiles, dev->gemm_clusters);   // persistent pairs
-    k_fp8_gemm<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, as_stream(stream)>>>(group);
+    k_fp8_gemm<false><<<static_cast<unsigned>(grid), kThreads, kSmemBytes, as_stream(stream)>>>(group);
     if ((st = after_launch("fp8_gemm launch")) != FP8T_OK) return st;
   }
   return FP8T_OK;
@@ -503,6 +593,144 @@ fp8t_status fp8_gemm_multi_sumsq(const fp8t_gemm_desc* gemms, int32_t n_gemms,
     return fail(FP8T_ERR_INVALID_ARG, "fp8_gemm_multi_sumsq: sumsq_of NULL");
   }
   return gemm_multi(gemms, n_gemms, sumsq_of, d_sumsq_out, d_workspace, workspace_bytes, stream);
+}
+
+// ------------------------------------------------------------------ MXFP8
+fp8t_status fp8_mx_cast_multi(const fp8t_mx_cast_tensor* tensors, int32_t n_tensors, void* stream) {
+  t_last_error.clear();
+  if (!tensors || n_tensors < 1 || n_tensors > 4096)
+    return fail(FP8T_ERR_INVALID_ARG, "fp8_mx_cast: tensors NULL or n_tensors out of range");
+  for (int32_t i = 0; i < n_tensors; ++i) {
+    const fp8t_mx_cast_tensor& t = tensors[i];
+    if (!t.x_bf16 || (!t.q_row && !t.q_col) || (t.q_row && !t.scales_row) || (t.q_col && !t.scales_col))
+      return fail(FP8T_ERR_INVALID_ARG, "fp8_mx_cast: tensor %d: NULL input, or an output without its scales", i);
+    if (t.fmt != FP8T_E4M3 && t.fmt != FP8T_E5M2)
+      return fail(FP8T_ERR_INVALID_ARG, "fp8_mx_cast: tensor %d: unknown format", i);
+    if (t.rows <= 0 || t.cols <= 0 || t.rows % 128 || t.cols % 128 || t.rows >= (int64_t(1) << 31) ||
+        t.cols >= (int64_t(1) << 31))
+      return fail(FP8T_ERR_UNSUPPORTED_SHAPE, "fp8_mx_cast: tensor %d: rows and cols must be positive multiples of 128", i);
+    if (!aligned(t.x_bf16, 16) || !aligned(t.q_row, 16) || !aligned(t.q_col, 16) ||
+        !aligned(t.scales_row, 16) || !aligned(t.scales_col, 16))
+      return fail(FP8T_ERR_MISALIGNED, "fp8_mx_cast: tensor %d: pointers must be 16-byte aligned", i);
+  }
+  DeviceInfo* dev = nullptr;
+  fp8t_status st = current_device(&dev);
+  if (st != FP8T_OK) return st;
+  using namespace fp8t::mx;
+  static thread_local Group group;
+  for (int32_t b0 = 0; b0 < n_tensors; b0 += kMaxTensors) {
+    const int32_t b1 = std::min<int32_t>(n_tensors, b0 + kMaxTensors);
+    std::memset(&group, 0, sizeof(group));
+    group.n = b1 - b0;
+    int64_t tiles = 0;
+    for (int32_t i = b0; i < b1; ++i) {
+      const fp8t_mx_cast_tensor& t = tensors[i];
+      Tensor& T = group.t[i - b0];
+      T.x = static_cast<const uint4*>(t.x_bf16);
+      T.q_row = static_cast<uint8_t*>(t.q_row);
+      T.sf_row = static_cast<uint8_t*>(t.scales_row);
+      T.q_col = static_cast<uint8_t*>(t.q_col);
+      T.sf_col = static_cast<uint8_t*>(t.scales_col);
+      T.rows = t.rows;
+      T.cols = t.cols;
+      T.tiles_c = t.cols / kTile;
+      T.tile_start = tiles;
+      T.fmt = t.fmt;
+      tiles += (t.rows / kTile) * T.tiles_c;
+    }
+    group.total_tiles = tiles;
+    const int64_t grid = std::min<int64_t>(tiles, static_cast<int64_t>(dev->sms) * dev->mx_cast_blocks_per_sm);
+    k_mx_cast<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, as_stream(stream)>>>(group);
+    if ((st = after_launch("fp8_mx_cast launch")) != FP8T_OK) return st;
+  }
+  return FP8T_OK;
+}
+
+fp8t_status fp8_mx_gemm_multi(const fp8t_mx_gemm_desc* gemms, int32_t n_gemms, void* stream) {
+  t_last_error.clear();
+  if (!gemms || n_gemms < 1 || n_gemms > 4096)
+    return fail(FP8T_ERR_INVALID_ARG, "fp8_mx_gemm: gemms NULL or n_gemms out of range");
+  const int64_t lim = int64_t(1) << 31;
+  for (int32_t i = 0; i < n_gemms; ++i) {
+    const fp8t_mx_gemm_desc& d = gemms[i];
+    if (!d.A || !d.B || !d.A_scales || !d.B_scales || !d.D_bf16)
+      return fail(FP8T_ERR_INVALID_ARG, "fp8_mx_gemm: problem %d: NULL pointer", i);
+    if ((d.a_fmt != FP8T_E4M3 && d.a_fmt != FP8T_E5M2) || (d.b_fmt != FP8T_E4M3 && d.b_fmt != FP8T_E5M2) ||
+        (d.a_layout != FP8T_K_MAJOR && d.a_layout != FP8T_MN_MAJOR) ||
+        (d.b_layout != FP8T_K_MAJOR && d.b_layout != FP8T_MN_MAJOR))
+      return fail(FP8T_ERR_INVALID_ARG, "fp8_mx_gemm: problem %d: unknown format or layout", i);
+    if (d.M <= 0 || d.N <= 0 || d.K <= 0 || d.M % 128 || d.N % 128 || d.K % 128 || d.M >= lim ||
+        d.N >= lim || d.K >= lim)
+      return fail(FP8T_ERR_UNSUPPORTED_SHAPE, "fp8_mx_gemm: problem %d: M, N, K must be positive multiples of 128", i);
+    if (!aligned(d.A, 16) || !aligned(d.B, 16) || !aligned(d.D_bf16, 16) || !aligned(d.A_scales, 16) ||
+        !aligned(d.B_scales, 16))
+      return fail(FP8T_ERR_MISALIGNED, "fp8_mx_gemm: problem %d: pointers must be 16-byte aligned", i);
+  }
+  DeviceInfo* dev = nullptr;
+  fp8t_status st = current_device(&dev);
+  if (st != FP8T_OK) return st;
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(FP8T_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  using namespace fp8t::gemm;
+  // scale atoms viewed as [atoms * 2][256] bytes, read 512 bytes (one atom) at a time
+  auto encode_sf = [&](CUtensorMap* map, const void* ptr, int64_t atoms) -> fp8t_status {
+    cuuint64_t dims[2] = {256, static_cast<cuuint64_t>(atoms * 2)};
+    cuuint64_t strides[1] = {256};
+    cuuint32_t box[2] = {256, 2};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(FP8T_ERR_CUDA, "cuTensorMapEncodeTiled (scales) failed (%d)", (int)r);
+    return FP8T_OK;
+  };
+  static thread_local Group group;
+  for (int32_t b0 = 0; b0 < n_gemms; b0 += kMaxProblems) {
+    const int32_t b1 = std::min<int32_t>(n_gemms, b0 + kMaxProblems);
+    std::memset(&group, 0, sizeof(group));
+    group.n = b1 - b0;
+    int64_t tiles = 0;
+    for (int32_t i = b0; i < b1; ++i) {
+      const fp8t_mx_gemm_desc& d = gemms[i];
+      Problem& P = group.p[i - b0];
+      const bool a_mn = d.a_layout == FP8T_MN_MAJOR, b_mn = d.b_layout == FP8T_MN_MAJOR;
+      if ((st = a_mn ? encode_kmajor(&P.a, d.A, d.K, d.M, kBK)
+                     : encode_kmajor(&P.a, d.A, d.M, d.K, kHalf)) != FP8T_OK) return st;
+      if ((st = b_mn ? encode_kmajor(&P.b, d.B, d.K, d.N, kBK)
+                     : encode_kmajor(&P.b, d.B, d.N, d.K, kHalf)) != FP8T_OK) return st;
+      if ((st = encode_sf(&P.sfa, d.A_scales, (d.M / 128) * (d.K / 128))) != FP8T_OK) return st;
+      if ((st = encode_sf(&P.sfb, d.B_scales, (d.N / 128) * (d.K / 128))) != FP8T_OK) return st;
+      cuuint64_t dims[2] = {static_cast<cuuint64_t>(d.N), static_cast<cuuint64_t>(d.M)};
+      cuuint64_t strides[1] = {static_cast<cuuint64_t>(d.N) * 2};
+      cuuint32_t box[2] = {32, 32};
+      cuuint32_t es[2] = {1, 1};
+      CUresult r = fn(&P.d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.D_bf16, dims, strides, box, es,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                      CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (r != CUDA_SUCCESS) return fail(FP8T_ERR_CUDA, "cuTensorMapEncodeTiled (D) failed (%d)", (int)r);
+      P.sa = nullptr;                          // block scales only: alpha = 1
+      P.sb = nullptr;
+      P.M = static_cast<int32_t>(d.M);
+      P.N = static_cast<int32_t>(d.N);
+      P.K = static_cast<int32_t>(d.K);
+      P.a_mn = a_mn ? 1 : 0;
+      P.b_mn = b_mn ? 1 : 0;
+      P.a_fmt = d.a_fmt;
+      P.b_fmt = d.b_fmt;
+      P.kb128 = static_cast<int32_t>(d.K / 128);
+      P.sumsq_slot = -1;
+      P.tiles_n = static_cast<int32_t>((d.N + kBN - 1) / kBN);
+      P.tile_start = static_cast<int32_t>(tiles);
+      tiles += ((d.M + kBM - 1) / kBM) * P.tiles_n;
+      if (tiles >= (int64_t(1) << 30))
+        return fail(FP8T_ERR_UNSUPPORTED_SHAPE, "fp8_mx_gemm: too many tiles in one launch");
+    }
+    group.total_tiles = static_cast<int32_t>(tiles);
+    const int64_t grid = 2 * std::min<int64_t>(tiles, dev->gemm_mx_clusters);
+    k_fp8_gemm<true><<<static_cast<unsigned>(grid), kThreads, kSmemBytesMX, as_stream(stream)>>>(group);
+    if ((st = after_launch("fp8_mx_gemm launch")) != FP8T_OK) return st;
+  }
+  return FP8T_OK;
 }
 
 fp8t_status fp8_gemm(const void* A, fp8t_format a_fmt, const void* B, fp8t_format b_fmt, int64_t M,
@@ -580,7 +808,7 @@ fp8t_status adamw_call(const fp8t_adamw_tensor* tensors, const fp8t_adamw_cast* 
       if (!c.d_scale || !c.d_amax_inout)
         return fail(FP8T_ERR_INVALID_ARG, "fused_adamw_multi_tensor_presummed: cast %d: NULL scale or amax", i);
       if (!aligned(c.d_scale, 4) || !aligned(c.d_amax_inout, 4) || !aligned(c.d_scale_inv_out, 4) ||
-          !aligned(c.q_rowmajor, 16) || !aligned(c.q_transposed, 16))
+          !aligned(c.q_rowmajor, 16))
         return fail(FP8T_ERR_MISALIGNED, "fused_adamw_multi_tensor_presummed: cast %d: misaligned pointer", i);
     }
   }
@@ -671,16 +899,10 @@ fp8t_status adamw_call(const fp8t_adamw_tensor* tensors, const fp8t_adamw_cast* 
           ci.amax_bits = reinterpret_cast<unsigned int*>(c.d_amax_inout);
           ci.scale_inv = c.d_scale_inv_out;
           ci.q = static_cast<uint8_t*>(c.q_rowmajor);
-          ci.qt = static_cast<uint8_t*>(c.q_transposed);
-          ci.rows = c.rows;
-          ci.cols = c.cols;
-          ci.tiles_c = (c.cols + kTileCols - 1) / kTileCols;
           ci.fmt = c.fmt;
           batch.cast_of[j] = static_cast<int8_t>(nc++);
-          acc += ((c.rows + kTileRows - 1) / kTileRows) * ci.tiles_c;
-        } else {
-          acc += chunks_of(tensors[i].numel);
         }
+        acc += chunks_of(tensors[i].numel);
         batch.numel[j] = tensors[i].numel;
         batch.master[j] = tensors[i].master;
         batch.m[j] = tensors[i].m;

@@ -16,11 +16,11 @@
 // alone on that one value; a device step counter is then read by every CTA at its start and
 // advanced by the CTA of the last batch that finishes last (a ticket counter).
 // A tensor may also carry the FP8 cast of its new BF16 weight for the next step (delayed
-// scaling: that step's scale is already known). Such a tensor is walked in 64 x 128 tiles
-// instead of flat chunks: each thread updates 4 x 8 elements, quantises the 8 new BF16 weights
-// (f32 multiply by the scale, cvt.rn.satfinite), stores them row-major and into a shared tile,
-// from which 128 threads write the transposed codes (4 x 4 byte transposes, 16-byte stores);
-// the tile's amax is max-accumulated into the tensor's slot. Same codes as the cast kernel.
+// scaling: that step's scale is already known): each 8-element vector of new BF16 weights is
+// quantised where it is produced (f32 multiply by the scale, cvt.rn.satfinite, the cast kernel's
+// codes) and stored row-major as 8 bytes; each warp keeps the amax of the weights it cast and
+// max-accumulates it into the tensor's slot when it moves on. The GEMMs read these codes
+// MN-major where they need the transpose, so none is written.
 // Traffic: 2 B/param for the norm pass, 28 B/param for the update (g 2 + m, v, p 4 each read,
 // m, v, p 4 each + BF16 weight 2 written).
 // Every f32 operation is an explicit round-to-nearest intrinsic, so no multiply-add is fused.
@@ -37,15 +37,12 @@ constexpr int kVec = 8;                                  // elements per 16-byte
 constexpr int64_t kChunk = 4 * kThreads * kVec;          // 8192 elements per chunk
 constexpr int kSumsqBlocks = 592;
 constexpr int kMaxCasts = 32;                            // weight casts per launch
-constexpr int kTileRows = 64, kTileCols = 128;           // one cast tile = 8192 elements
 
 struct CastInfo {
   const float* scale;
   unsigned int* amax_bits;
   float* scale_inv;                                       // may be null
   uint8_t* q;                                             // row-major codes, may be null
-  uint8_t* qt;                                            // transposed codes, may be null
-  int64_t rows, cols, tiles_c;
   int32_t fmt;
 };
 
@@ -188,100 +185,13 @@ __device__ __forceinline__ void adam_one(float& p, float& m, float& v, float g, 
   v = vv;
 }
 
-// One 64 x 128 tile of a tensor whose new weight is also cast (see the file comment).
-// With update = false (a skipped step) the weight is left alone and only cast again, so the
-// codes, scale inverse and amax still describe it.
-__device__ __forceinline__ void update_cast_tile(const Batch& b, const CastInfo& ci, int t,
-                                                 int64_t local, const Scalars& kk, float f,
-                                                 bool update, uint32_t* stage, uint32_t* red) {
-  const int tid = threadIdx.x;
-  const int64_t rows = ci.rows, cols = ci.cols;
-  const int64_t r0 = (local / ci.tiles_c) * kTileRows, c0 = (local % ci.tiles_c) * kTileCols;
-  const float s = __ldg(ci.scale);
-  float* __restrict__ P = b.master[t];
-  float* __restrict__ M = b.m[t];
-  float* __restrict__ V = b.v[t];
-  const uint16_t* __restrict__ G = b.g[t];
-  uint16_t* __restrict__ W = b.w[t];
-  uint32_t vmax = 0;
-#pragma unroll 1
-  for (int u = 0; u < 4; ++u) {                      // one 8-element vector at a time
-    const int vec = u * kThreads + tid;
-    const int64_t row = r0 + (vec >> 4), col = c0 + (vec & 15) * 8;
-    if (row >= rows || col >= cols) continue;
-    const int64_t e = row * cols + col;
-    uint32_t wout[4];
-    if (!update) {
-      const uint4 wv = *reinterpret_cast<const uint4*>(W + e);
-      wout[0] = wv.x; wout[1] = wv.y; wout[2] = wv.z; wout[3] = wv.w;
-    } else {
-    const uint4 gv = ld_stream_u4(G + e);
-    float4 mv[2], vv[2], pv[2];
-    mv[0] = __ldcs(reinterpret_cast<const float4*>(M + e));
-    mv[1] = __ldcs(reinterpret_cast<const float4*>(M + e + 4));
-    vv[0] = __ldcs(reinterpret_cast<const float4*>(V + e));
-    vv[1] = __ldcs(reinterpret_cast<const float4*>(V + e + 4));
-    pv[0] = __ldcs(reinterpret_cast<const float4*>(P + e));
-    pv[1] = __ldcs(reinterpret_cast<const float4*>(P + e + 4));
-    const uint32_t* gw = reinterpret_cast<const uint32_t*>(&gv);
-    float* pp = reinterpret_cast<float*>(&pv[0]);
-    float* mm = reinterpret_cast<float*>(&mv[0]);
-    float* vq = reinterpret_cast<float*>(&vv[0]);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      adam_one(pp[2 * j], mm[2 * j], vq[2 * j], bf16_to_f32(gw[j] & 0xFFFFu), kk, f);
-      adam_one(pp[2 * j + 1], mm[2 * j + 1], vq[2 * j + 1], bf16_to_f32(gw[j] >> 16), kk, f);
-      wout[j] = f32_to_bf16_rne(pp[2 * j]) | (f32_to_bf16_rne(pp[2 * j + 1]) << 16);
-    }
-    __stcs(reinterpret_cast<float4*>(M + e), mv[0]);
-    __stcs(reinterpret_cast<float4*>(M + e + 4), mv[1]);
-    __stcs(reinterpret_cast<float4*>(V + e), vv[0]);
-    __stcs(reinterpret_cast<float4*>(V + e + 4), vv[1]);
-    __stcs(reinterpret_cast<float4*>(P + e), pv[0]);
-    __stcs(reinterpret_cast<float4*>(P + e + 4), pv[1]);
-    *reinterpret_cast<uint4*>(W + e) = make_uint4(wout[0], wout[1], wout[2], wout[3]);
-    }
-    uint32_t mag;
-    const uint2 q8 = ci.fmt == 0 ? quant8<0>(wout, s, mag) : quant8<1>(wout, s, mag);
-    vmax = max(vmax, mag);
-    if (ci.q) *reinterpret_cast<uint2*>(ci.q + e) = q8;
-    *reinterpret_cast<uint2*>(&stage[(vec >> 4) * 32 + (vec & 15) * 2]) = q8;
+// amax of the new weights a warp cast, max-accumulated into the tensor's slot (all lanes).
+__device__ __forceinline__ void flush_amax(unsigned int* amax_bits, uint32_t vmax) {
+  uint32_t m = __reduce_max_sync(0xffffffffu, vmax);
+  if ((threadIdx.x & 31) == 0) {
+    if (m > 0x7F80u) m = 0x7FC0u;                  // canonical NaN
+    atomicMax(amax_bits, m << 16);
   }
-  vmax = __reduce_max_sync(0xffffffffu, vmax);
-  if ((tid & 31) == 0) red[tid >> 5] = vmax;
-  __syncthreads();                                   // staged tile and warp maxima complete
-  if (tid == 0) {
-    uint32_t m = 0;
-#pragma unroll
-    for (int w = 0; w < kThreads / 32; ++w) m = max(m, red[w]);
-    if (m > 0x7F80u) m = 0x7FC0u;                    // canonical NaN
-    atomicMax(ci.amax_bits, m << 16);
-    if (ci.scale_inv && local == 0) *ci.scale_inv = __fdiv_rn(1.0f, s);
-  }
-  if (ci.qt && tid < 128) {
-    const int rb = tid >> 5, cb = tid & 31;          // rows 16rb.., columns 4cb..
-    if (r0 + 16 * rb < rows && c0 + 4 * cb < cols) {
-      uint32_t v[16];
-#pragma unroll
-      for (int r = 0; r < 16; ++r) v[r] = stage[(16 * rb + r) * 32 + cb];
-      uint32_t o[4][4];
-#pragma unroll
-      for (int kq = 0; kq < 4; ++kq) {
-        const uint32_t a = v[4 * kq], bq = v[4 * kq + 1], cq = v[4 * kq + 2], d = v[4 * kq + 3];
-        const uint32_t t0 = __byte_perm(a, bq, 0x5140), t1 = __byte_perm(a, bq, 0x7362);
-        const uint32_t w0 = __byte_perm(cq, d, 0x5140), w1 = __byte_perm(cq, d, 0x7362);
-        o[0][kq] = __byte_perm(t0, w0, 0x5410);
-        o[1][kq] = __byte_perm(t0, w0, 0x7632);
-        o[2][kq] = __byte_perm(t1, w1, 0x5410);
-        o[3][kq] = __byte_perm(t1, w1, 0x7632);
-      }
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc)
-        *reinterpret_cast<uint4*>(ci.qt + (c0 + 4 * cb + cc) * rows + r0 + 16 * rb) =
-            make_uint4(o[cc][0], o[cc][1], o[cc][2], o[cc][3]);
-    }
-  }
-  __syncthreads();                                   // tile and maxima free for the next one
 }
 
 template <bool CAST>
@@ -330,16 +240,21 @@ __global__ void __launch_bounds__(kThreads, 2)
   Scalars kk = k;
   kk.step_size = s_step_size;
   kk.bc2_sqrt = s_bc2_sqrt;
-  __shared__ uint32_t stage[CAST ? kTileRows * kTileCols / 4 : 1];   // one tile of codes
-  __shared__ uint32_t red[kThreads / 32];
+  int cur = -1;                          // cast this CTA's warps are accumulating an amax for
+  uint32_t vmax = 0;
   const int64_t nchunks = b.chunk_start[b.n];
   for (int64_t c = blockIdx.x; c < nchunks; c += gridDim.x) {
     const int t = find_tensor(b, c);
-    if (CAST && b.cast_of[t] >= 0) {
-      update_cast_tile(b, b.cast[b.cast_of[t]], t, c - b.chunk_start[t], kk, f, !skip, stage, red);
-      continue;
+    const int cj = CAST ? b.cast_of[t] : -1;
+    if (CAST && cj != cur) {
+      if (cur >= 0) flush_amax(b.cast[cur].amax_bits, vmax);
+      cur = cj;
+      vmax = 0;
     }
-    if (CAST && skip) continue;
+    if (CAST && skip && cj < 0) continue;
+    const float s = CAST && cj >= 0 ? __ldg(b.cast[cj].scale) : 0.0f;
+    if (CAST && cj >= 0 && c == b.chunk_start[t] && threadIdx.x == 0 && b.cast[cj].scale_inv)
+      *b.cast[cj].scale_inv = __fdiv_rn(1.0f, s);
     const int64_t base = (c - b.chunk_start[t]) * kChunk;
     const int64_t n = b.numel[t];
     float* __restrict__ P = b.master[t];
@@ -356,7 +271,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int u = 0; u < 2; ++u) {
         const int64_t e = base + static_cast<int64_t>((u0 + u) * kThreads + threadIdx.x) * kVec;
         full[u] = e + kVec <= n;
-        if (full[u]) {
+        if (CAST && skip) {                  // skipped step: the unchanged weight, cast again
+          if (full[u]) gv[u] = *reinterpret_cast<const uint4*>(W + e);
+        } else if (full[u]) {
           gv[u] = ld_stream_u4(G + e);
           mv[u][0] = __ldcs(reinterpret_cast<const float4*>(M + e));
           mv[u][1] = __ldcs(reinterpret_cast<const float4*>(M + e + 4));
@@ -369,7 +286,15 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int64_t e = base + static_cast<int64_t>((u0 + u) * kThreads + threadIdx.x) * kVec;
-        if (full[u]) {
+        if (CAST && skip) {
+          if (full[u]) {
+            const uint32_t wout[4] = {gv[u].x, gv[u].y, gv[u].z, gv[u].w};
+            uint32_t mag;
+            const uint2 q8 = b.cast[cj].fmt == 0 ? quant8<0>(wout, s, mag) : quant8<1>(wout, s, mag);
+            vmax = max(vmax, mag);
+            if (b.cast[cj].q) *reinterpret_cast<uint2*>(b.cast[cj].q + e) = q8;
+          }
+        } else if (full[u]) {
           const uint32_t* gw = reinterpret_cast<const uint32_t*>(&gv[u]);
           float* pp = reinterpret_cast<float*>(&pv[u][0]);
           float* mm = reinterpret_cast<float*>(&mv[u][0]);
@@ -388,6 +313,12 @@ __global__ void __launch_bounds__(kThreads, 2)
           __stcs(reinterpret_cast<float4*>(P + e), pv[u][0]);
           __stcs(reinterpret_cast<float4*>(P + e + 4), pv[u][1]);
           *reinterpret_cast<uint4*>(W + e) = make_uint4(wout[0], wout[1], wout[2], wout[3]);
+          if (CAST && cj >= 0) {
+            uint32_t mag;
+            const uint2 q8 = b.cast[cj].fmt == 0 ? quant8<0>(wout, s, mag) : quant8<1>(wout, s, mag);
+            vmax = max(vmax, mag);
+            if (b.cast[cj].q) *reinterpret_cast<uint2*>(b.cast[cj].q + e) = q8;
+          }
         } else {
           for (int64_t i = e; i < n && i < e + kVec; ++i) {
             float p = P[i], mq = M[i], vq1 = V[i];
@@ -401,6 +332,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
   }
+  if (CAST && cur >= 0) flush_amax(b.cast[cur].amax_bits, vmax);
   // counter read by every CTA above: the last CTA of the last batch advances it
   if (k.d_step && !k.step_slot && b.last && !skip) {
     __shared__ int s_last;

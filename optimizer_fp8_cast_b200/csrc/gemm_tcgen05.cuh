@@ -7,7 +7,11 @@
 // as tcgen05.mma.kind::f8f6f4 issued by one thread for a PAIR of SMs, with the accumulator in
 // tensor memory.
 //
-// D[M x N] = bf16((A[M x K] . B[N x K]^T) * sa * sb), A and B K-major ("TN").
+// D[M x N] = bf16((A[M x K] . B[N x K]^T) * sa * sb). Each operand is either K-major (stored
+// [M or N rows][K], "TN") or MN-major (stored [K rows][M or N]): tcgen05 reads 8-bit operands in
+// both orders, so the transposed FP8 copies that a K-major-only tensor core needs (the pages'
+// Hopper design) are optional here. An MN-major operand is loaded as 128 K-rows x 128 bytes
+// boxes with the same 128-byte swizzle; its descriptor steps 32 K-rows (4 KB) per MMA.
 // A cluster of two CTAs (one per SM) computes a 256 x 256 tile: CTA r loads A rows
 // [128r, 128r+128) and B rows (N columns) [128r, 128r+128) of the tile, 128-byte swizzled
 // 128 x 128-byte boxes, into its own 6-stage ring (32 KB per stage). Both CTAs' loads count on
@@ -33,6 +37,15 @@
 // into a workspace slot; the CTA that finishes the last launch last (a ticket counter) sums all
 // slots in index order, so the result does not depend on scheduling. Out-of-range rows and
 // columns hold exact zeros (TMA zero-fills the operands there) and add nothing.
+// MXFP8 variant (template MX): block-scaled MMAs (tcgen05.mma.kind::mxf8f6f4.block_scale) with
+// one E8M0 scale per 32 K values of every row of A and B. Per stage each CTA also loads, by TMA,
+// the 512-byte scale atom of its 128 A rows and the two atoms of the tile's 256 B rows (the 4
+// K-blocks of the stage); the MMA thread copies them into tensor memory (tcgen05.cp 32x128b,
+// replicated into the four lane quarters: A scales in 4 columns, B scales in 8) right before
+// the stage's four MMAs, which pick the byte of their K-block through the descriptor's
+// scale-factor ids. The copies and MMAs run in issue order, so one set of scale columns serves
+// every stage. The scale columns take the place of the second accumulator: the MX kernel keeps
+// a single 256-column accumulator.
 // Every mbarrier wait is bounded (globaltimer). On expiry a CTA records kErrTimeout and stops
 // issuing; issued MMAs are awaited with a fixed bound, loads in flight are given time to land,
 // and both CTAs meet at a cluster barrier before TMEM is freed; D is then incomplete.
@@ -54,8 +67,26 @@ constexpr int kEpiChunkBytes = 32 * 32 * 2;              // 32 rows x 32 BF16 co
 constexpr int kEpiBytes = kEpiWarps * 2 * kEpiChunkBytes; // double-buffered per epilogue warp
 constexpr int kSmemBytes =
     kStages * kStageBytes + kEpiBytes + 1024 /*alignment slack*/ + 256 /*barriers*/;
+constexpr int kSfaBytes = 512, kSfbBytes = 1024;         // MX scale atoms per stage and CTA
+constexpr int kSfStageBytes = kSfaBytes + kSfbBytes;
+constexpr int kSmemBytesMX = kSmemBytes + kStages * kSfStageBytes;
+constexpr uint32_t kSfaCol = kAccCols, kSfbCol = kAccCols + 4;   // MX: scale columns in TMEM
 constexpr uint64_t kSettleNs = 200000;                   // let loads in flight land on abort
 constexpr uint64_t kPairDrainNs = 1000000;               // producer drain budget (1 ms)
+
+// Shared-memory matrix descriptor, MN-major operand, 128-byte swizzle: 128 MN-elements per
+// swizzle row, 8 K-rows (1024 B) per swizzle atom, atoms along K 1024 B apart (stride byte
+// offset); the 128 rows (M or N) a CTA holds are a single atom wide, so the leading byte offset
+// (distance between atoms along MN) is never stepped over.
+__device__ __forceinline__ uint64_t make_sw128_desc_mn(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);        // start address
+  d |= static_cast<uint64_t>(16384 >> 4) << 16;              // leading byte offset
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;               // stride byte offset
+  d |= static_cast<uint64_t>(1) << 46;                       // descriptor version (sm_100)
+  d |= static_cast<uint64_t>(2) << 61;                       // 128-byte swizzle
+  return d;
+}
 
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, 8-row groups 1024 B apart.
 __device__ __forceinline__ uint64_t make_sw128_desc(uint32_t saddr) {
@@ -68,11 +99,32 @@ __device__ __forceinline__ uint64_t make_sw128_desc(uint32_t saddr) {
   return d;
 }
 
-// Instruction descriptor: FP32 accumulator, FP8 A/B formats (0 = E4M3, 1 = E5M2), both K-major,
-// M = 256 (pair), N = 256.
-__host__ __device__ constexpr uint32_t make_idesc(int a_fmt, int b_fmt) {
+// Instruction descriptor: FP32 accumulator, FP8 A/B formats (0 = E4M3, 1 = E5M2), A and B
+// major-ness (0 = K-major, 1 = MN-major), M = 256 (pair), N = 256.
+__host__ __device__ constexpr uint32_t make_idesc(int a_fmt, int b_fmt, int a_mn = 0, int b_mn = 0) {
   return (1u << 4) | (static_cast<uint32_t>(a_fmt) << 7) | (static_cast<uint32_t>(b_fmt) << 10) |
+         (static_cast<uint32_t>(a_mn) << 15) | (static_cast<uint32_t>(b_mn) << 16) |
          (static_cast<uint32_t>(kBN >> 3) << 17) | (static_cast<uint32_t>(kBM >> 4) << 24);
+}
+
+// Block-scaled instruction descriptor (MXFP8): A/B formats and major-ness as above, E8M0 scales
+// (bit 23), scale-factor byte `sf_id` for A (bits 29-30) and B (bits 4-5), M = 256, N = 256.
+__host__ __device__ constexpr uint32_t make_idesc_mx(int a_fmt, int b_fmt, int a_mn, int b_mn, int sf_id) {
+  return (static_cast<uint32_t>(sf_id) << 4) | (static_cast<uint32_t>(a_fmt) << 7) |
+         (static_cast<uint32_t>(b_fmt) << 10) | (static_cast<uint32_t>(a_mn) << 15) |
+         (static_cast<uint32_t>(b_mn) << 16) | (static_cast<uint32_t>(kBN >> 3) << 17) | (1u << 23) |
+         (static_cast<uint32_t>(kBM >> 4) << 24) | (static_cast<uint32_t>(sf_id) << 29);
+}
+
+// Shared-memory descriptor of a 32-row x 16-byte scale atom (no swizzle, K-major): rows 16 B
+// apart, 8-row groups 128 B apart.
+__device__ __forceinline__ uint64_t make_sf_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);        // start address
+  d |= static_cast<uint64_t>(1) << 16;                       // leading byte offset (unused)
+  d |= static_cast<uint64_t>(128 >> 4) << 32;                // stride byte offset
+  d |= static_cast<uint64_t>(1) << 46;                       // descriptor version (sm_100)
+  return d;                                                  // layout type 0: no swizzle
 }
 
 // Two f32 -> two BF16 (round to nearest even); `lo` in the low half.
@@ -85,13 +137,18 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // One GEMM of a grouped launch. Tiles are numbered problem by problem.
 constexpr int kMaxProblems = 24;
 struct alignas(64) Problem {
-  CUtensorMap a, b, d;           // A [M][K], B [N][K] (128 x 128-byte boxes), D [M][N] (32 x 32)
+  CUtensorMap a, b, d;           // A [M][K] or [K][M], B [N][K] or [K][N] (128 x 128-byte boxes),
+                                 // D [M][N] (32 x 32)
+  CUtensorMap sfa, sfb;          // MX: scale atoms as [atoms * 2][256] bytes, 512-byte boxes
   const float* sa;
   const float* sb;
   int32_t M, N, K;
   uint32_t idesc;
   int32_t tiles_n, tile_start;
   int32_t sumsq_slot;            // first partial slot of this problem, or -1 (not summed)
+  int32_t a_mn, b_mn;            // 1: operand stored MN-major ([K][M], [K][N])
+  int32_t kb128;                 // MX: K / 128, atoms per 128 rows
+  int32_t a_fmt, b_fmt;          // MX: element formats (the descriptor is formed per K-block)
 };
 struct alignas(64) Group {
   Problem p[kMaxProblems];
@@ -121,6 +178,7 @@ struct Smem {
   int abort;
 };
 
+template <bool MX>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     k_fp8_gemm(const __grid_constant__ Group g) {
   extern __shared__ uint8_t smem_raw[];
@@ -129,7 +187,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint8_t* sA = smem;
   uint8_t* sB = smem + kStages * kABytes;
   uint8_t* sEpi = smem + kStages * kStageBytes;              // 1024-byte aligned
-  Smem* S = reinterpret_cast<Smem*>(smem + kStages * kStageBytes + kEpiBytes);
+  uint8_t* sSF = sEpi + kEpiBytes;                           // MX: [stage][SFA 512 | SFB 1024]
+  Smem* S = reinterpret_cast<Smem*>(sSF + (MX ? kStages * kSfStageBytes : 0));
+  constexpr uint32_t kTx = kPairTxBytes + (MX ? 2 * kSfStageBytes : 0);
   volatile int* abort_flag = &S->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -188,9 +248,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             break;
           }
           const uint32_t full_leader = mapa_shared(smem_u32(&S->full[s]), 0);
-          if (leader) mbar_arrive_expect_tx(smem_u32(&S->full[s]), kPairTxBytes);
-          tma_load_2d_pair(smem_u32(sA + s * kABytes), &P.a, kb * kBK, m0, full_leader);
-          tma_load_2d_pair(smem_u32(sB + s * kBBytes), &P.b, kb * kBK, n0, full_leader);
+          if (leader) mbar_arrive_expect_tx(smem_u32(&S->full[s]), kTx);
+          if (MX) {                    // scale atoms: this CTA's 128 A rows, the tile's 256 B rows
+            const int mt = (local / P.tiles_n), nt = (local % P.tiles_n);
+            uint8_t* sf = sSF + s * kSfStageBytes;
+            tma_load_2d_pair(smem_u32(sf), &P.sfa, 0,
+                             2 * ((2 * mt + static_cast<int>(rank)) * P.kb128 + kb), full_leader);
+            tma_load_2d_pair(smem_u32(sf + kSfaBytes), &P.sfb, 0, 2 * ((2 * nt) * P.kb128 + kb),
+                             full_leader);
+            tma_load_2d_pair(smem_u32(sf + kSfaBytes + 512), &P.sfb, 0,
+                             2 * ((2 * nt + 1) * P.kb128 + kb), full_leader);
+          }
+          if (P.a_mn) tma_load_2d_pair(smem_u32(sA + s * kABytes), &P.a, m0, kb * kBK, full_leader);
+          else        tma_load_2d_pair(smem_u32(sA + s * kABytes), &P.a, kb * kBK, m0, full_leader);
+          if (P.b_mn) tma_load_2d_pair(smem_u32(sB + s * kBBytes), &P.b, n0, kb * kBK, full_leader);
+          else        tma_load_2d_pair(smem_u32(sB + s * kBBytes), &P.b, kb * kBK, n0, full_leader);
           ++issued;
         }
       }
@@ -214,7 +286,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const Problem& P = g.p[find_problem(g, tile)];
         const int num_kb = (P.K + kBK - 1) / kBK;
         const uint32_t idesc = P.idesc;
-        const uint32_t acc = local & 1, aph = (local >> 1) & 1;
+        const bool a_mn = P.a_mn != 0, b_mn = P.b_mn != 0;
+        const uint32_t acc = MX ? 0u : (local & 1), aph = MX ? (local & 1) : ((local >> 1) & 1);
         if (!mbar_wait(smem_u32(&S->acc_empty[acc]), aph ^ 1, limit, expire_main)) {
           *abort_flag = 1;
           record_error(kErrTimeout);
@@ -234,10 +307,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t a_base = smem_u32(sA + s * kABytes);
           const uint32_t b_base = smem_u32(sB + s * kBBytes);
+          if (MX) {                    // this stage's scales into tensor memory, then 4 MMAs
+            const uint32_t sf = smem_u32(sSF + s * kSfStageBytes);
+            tc_cp_32x128b_warpx4_pair(tmem + kSfaCol, make_sf_desc(sf));
+            tc_cp_32x128b_warpx4_pair(tmem + kSfbCol, make_sf_desc(sf + kSfaBytes));
+            tc_cp_32x128b_warpx4_pair(tmem + kSfbCol + 4, make_sf_desc(sf + kSfaBytes + 512));
+#pragma unroll
+            for (int k = 0; k < kBK / kUmmaK; ++k)
+              tc_mma_mxf8_pair(d_tmem,
+                               a_mn ? make_sw128_desc_mn(a_base + k * kUmmaK * 128)
+                                    : make_sw128_desc(a_base + k * kUmmaK),
+                               b_mn ? make_sw128_desc_mn(b_base + k * kUmmaK * 128)
+                                    : make_sw128_desc(b_base + k * kUmmaK),
+                               make_idesc_mx(P.a_fmt, P.b_fmt, P.a_mn, P.b_mn, k),
+                               (tmem + kSfaCol) | (static_cast<uint32_t>(k) << 30),
+                               (tmem + kSfbCol) | (static_cast<uint32_t>(k) << 30),
+                               (kb | k) != 0 ? 1u : 0u);
+          } else {
 #pragma unroll
           for (int k = 0; k < kBK / kUmmaK; ++k)
-            tc_mma_f8_pair(d_tmem, make_sw128_desc(a_base + k * kUmmaK),
-                           make_sw128_desc(b_base + k * kUmmaK), idesc, (kb | k) != 0 ? 1u : 0u);
+            tc_mma_f8_pair(d_tmem,
+                           a_mn ? make_sw128_desc_mn(a_base + k * kUmmaK * 128)
+                                : make_sw128_desc(a_base + k * kUmmaK),
+                           b_mn ? make_sw128_desc_mn(b_base + k * kUmmaK * 128)
+                                : make_sw128_desc(b_base + k * kUmmaK),
+                           idesc, (kb | k) != 0 ? 1u : 0u);
+          }
           tc_commit_pair_mc(smem_u32(&S->empty[s]), 0x3);
         }
         if (!ok) break;
@@ -253,7 +348,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint8_t* my_buf = sEpi + (warp - 2) * 2 * kEpiChunkBytes;
     uint32_t local = 0, chunk_count = 0;
     for (int tile = cluster; tile < n_tiles; tile += n_clusters, ++local) {
-      const uint32_t acc = local & 1, aph = (local >> 1) & 1;
+      const uint32_t acc = MX ? 0u : (local & 1), aph = MX ? (local & 1) : ((local >> 1) & 1);
       if (*abort_flag) break;
       if (!mbar_wait(smem_u32(&S->acc_full[acc]), aph, limit, expire_epi)) {
         *abort_flag = 1;
@@ -263,7 +358,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const Problem& P = g.p[find_problem(g, tile)];
       const int M = P.M, N = P.N, local_tile = tile - P.tile_start;
-      const float alpha = __fmul_rn(__ldg(P.sa), __ldg(P.sb));
+      const float alpha = P.sa ? __fmul_rn(__ldg(P.sa), __ldg(P.sb)) : 1.0f;
       const int row0 = (local_tile / P.tiles_n) * kBM + static_cast<int>(rank) * kHalf + quad * 32;
       const int n0 = (local_tile % P.tiles_n) * kBN;
       const uint32_t t_base = tmem + (static_cast<uint32_t>(quad * 32) << 16) + acc * kAccCols;

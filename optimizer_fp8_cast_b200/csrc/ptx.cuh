@@ -228,6 +228,26 @@ __device__ __forceinline__ void tc_mma_f8_pair(uint32_t d_tmem, uint64_t adesc, 
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// Block-scaled pair MMA (MXFP8): as tc_mma_f8_pair, with one E8M0 scale per 32 K values of
+// every row of A and of B read from tensor memory at sfa_tmem / sfb_tmem (the byte of each
+// 32-bit scale column selected by the descriptor's scale-factor ids).
+__device__ __forceinline__ void tc_mma_mxf8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                 uint32_t idesc, uint32_t sfa_tmem,
+                                                 uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+      : "memory");
+}
+// Copy a 32-row x 16-byte matrix (described by a shared-memory descriptor) into 4 tensor-memory
+// columns at taddr, replicated into all four 32-lane quarters, in both CTAs of the pair (each
+// from its own shared memory). Ordered with the pair MMAs issued after it by the same thread.
+__device__ __forceinline__ void tc_cp_32x128b_warpx4_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
 // Arrive on the mbarrier at the same offset in every CTA of cta_mask once the pair MMAs issued
 // so far by this thread have completed.
 __device__ __forceinline__ void tc_commit_pair_mc(uint32_t bar, uint16_t cta_mask) {

@@ -30,9 +30,10 @@ __device__ __forceinline__ float next_scale(uint32_t rep, float fmax, int margin
 
 // The same update for one tensor, done by one warp (used inside other kernels once their amax
 // is complete). The roll goes from the top down in chunks of 32 x kPer entries: every lane
-// reads its kPer entries, the warp synchronises, then writes them one place higher.
+// reads its kPer entries (all loads in flight at once), the warp synchronises, then writes them
+// one place higher; a history of up to 1025 entries takes a single round trip to memory.
 // amax is read with a volatile load: other CTAs of the calling kernel accumulated it.
-template <int kPer = 8>
+template <int kPer = 32>
 __device__ __forceinline__ void warp_update(float* amax, float* h, int H, float fmax, bool algo_max,
                                             int margin, float* scale, float* scale_inv) {
   const int lane = threadIdx.x & 31;

@@ -4,9 +4,12 @@ One step for each layer (W stored in x out, Y = X.W), following the precision fl
 "FP8 混合精度训练工程实践" §四 and the HYBRID recipe of "LLM FP8 微调上线生产实战":
 
   cast X, W -> E4M3 and dY -> E5M2 with the scales of the previous step (delayed scaling)
-  Y  = Xq . Wq      (fprop,  A = Xq,   B = Wq^T)
-  dX = dYq . Wq^T   (dgrad,  A = dYq,  B = Wq)
-  dW = Xq^T . dYq   (wgrad,  A = Xq^T, B = dYq^T)
+  Y  = Xq . Wq      (fprop,  A = Xq K-major,  B = Wq MN-major)
+  dX = dYq . Wq^T   (dgrad,  A = dYq K-major, B = Wq K-major)
+  dW = Xq^T . dYq   (wgrad,  A = Xq MN-major, B = dYq MN-major)
+The tensor cores read 8-bit operands MN-major, so by default no transposed FP8 copy is made;
+with transposes=True the casts also write Xq^T, Wq^T, dYq^T and every GEMM reads K-major
+operands (the layout a K-major-only tensor core needs).
 then, for all layers at once, the amax-history roll and next scales, and one fused AdamW over
 every dW (loss-scale unscale, global-norm clip, FP32 master/m/v, BF16 weight for the next step).
 With fused_update (the default) the roll and next scales run in the last CTA of the cast launch,
@@ -21,8 +24,9 @@ scalars stay on the device; nothing in a step synchronises with the host.
 """
 import torch
 
-from . import (AMAX_MAX, AMAX_MOST_RECENT, E4M3, E5M2, FP8_MAX, fp8_cast_transpose_amax,
-               fp8_cast_transpose_amax_multi, fp8_cast_transpose_amax_update_multi, fp8_gemm,
+from . import (AMAX_MAX, AMAX_MOST_RECENT, CURRENT_WORKSPACE_BYTES, E4M3, E5M2, FP8_MAX,
+               fp8_cast_transpose_amax, fp8_cast_transpose_amax_current_multi,
+               fp8_cast_transpose_amax_multi, fp8_cast_transpose_amax_update_multi,
                fp8_gemm_multi, fp8_gemm_multi_sumsq, fp8_gemm_sumsq_workspace_bytes,
                fp8_scale_update, fused_adamw_multi_tensor, fused_adamw_multi_tensor_presummed,
                fused_adamw_workspace_bytes)
@@ -32,7 +36,7 @@ ROLE_FMT = (E4M3, E4M3, E5M2)
 
 
 class LinearLayerBuffers:
-    def __init__(self, fin, fout, tokens, w_init, device):
+    def __init__(self, fin, fout, tokens, w_init, device, transposes=False):
         u8 = dict(dtype=torch.uint8, device=device)
         bf = dict(dtype=torch.bfloat16, device=device)
         self.fin, self.fout, self.tokens = fin, fout, tokens
@@ -41,11 +45,11 @@ class LinearLayerBuffers:
         self.m = torch.zeros_like(self.master)
         self.v = torch.zeros_like(self.master)
         self.Xq = torch.empty(tokens, fin, **u8)
-        self.XqT = torch.empty(fin, tokens, **u8)
         self.Wq = torch.empty(fin, fout, **u8)
-        self.WqT = torch.empty(fout, fin, **u8)
         self.dYq = torch.empty(tokens, fout, **u8)
-        self.dYqT = torch.empty(fout, tokens, **u8)
+        self.XqT = torch.empty(fin, tokens, **u8) if transposes else None
+        self.WqT = torch.empty(fout, fin, **u8) if transposes else None
+        self.dYqT = torch.empty(fout, tokens, **u8) if transposes else None
         self.Y = torch.empty(tokens, fout, **bf)
         self.dX = torch.empty(tokens, fin, **bf)
         self.dW = torch.empty(fin, fout, **bf)
@@ -58,7 +62,7 @@ class Fp8LinearStep:
 
     def __init__(self, layer_shapes, tokens, history_len, algo="max", margin=0, adamw=None,
                  w_init=None, device="cuda", counters=False, device_step=False, fused_update=True,
-                 fused_norm=True, fused_wcast=True):
+                 fused_norm=True, fused_wcast=True, transposes=False, recipe="delayed"):
         self.device = torch.device(device)
         self.tokens = tokens
         self.algo = AMAX_MAX if algo == "max" else AMAX_MOST_RECENT
@@ -75,7 +79,8 @@ class Fp8LinearStep:
         self.ticket = torch.zeros(1, dtype=torch.int32, device=self.device)
         self.fp8_max = torch.tensor([FP8_MAX[ROLE_FMT[i % 3]] for i in range(n)], **f32)
         self.counters = torch.zeros(n, 3, dtype=torch.int64, device=self.device) if counters else None
-        self.layers = [LinearLayerBuffers(fi, fo, tokens, w_init[k], self.device)
+        self.transposes = transposes
+        self.layers = [LinearLayerBuffers(fi, fo, tokens, w_init[k], self.device, transposes)
                        for k, (fi, fo) in enumerate(layer_shapes)]
         self.grad_norm = torch.zeros(1, **f32)
         self.skipped = torch.zeros(1, dtype=torch.int32, device=self.device)
@@ -91,9 +96,17 @@ class Fp8LinearStep:
         gws = fp8_gemm_sumsq_workspace_bytes(self._gemm_descs(sumsq=True))
         self.gemm_workspace = torch.zeros(gws, dtype=torch.uint8, device=self.device)
         self.adamw_ticket = torch.zeros(1, dtype=torch.int32, device=self.device)
-        # the W cast inside AdamW needs the in-launch scale update and the presummed AdamW; the
-        # saturation / zero counters of W are only kept by the separate cast
-        self.fused_wcast = fused_wcast and fused_update and fused_norm and not counters
+        # current scaling: every scale from the tensor's own amax (no history, no delayed update)
+        assert recipe in ("delayed", "current")
+        self.recipe = recipe
+        self.current_ws = torch.zeros(CURRENT_WORKSPACE_BYTES, dtype=torch.uint8, device=self.device)
+        if recipe == "current":
+            fused_update = fused_wcast = False
+            self.fused_update = False
+        # the W cast inside AdamW needs the in-launch scale update and the presummed AdamW, and
+        # writes row-major codes only; the saturation / zero counters of W are only kept by the
+        # separate cast
+        self.fused_wcast = fused_wcast and fused_update and fused_norm and not counters and not transposes
         if self.fused_wcast and self.device.type == "cuda":
             self.prime()
 
@@ -139,25 +152,30 @@ class Fp8LinearStep:
         else:
             fp8_cast_transpose_amax_multi(descs, stream=stream)
 
+    def cast_all_current(self, xs, dys, stream=None):
+        """Current scaling: the X, W and dY scales from their own amax, then the casts."""
+        descs = []
+        for k, L in enumerate(self.layers):
+            descs += [self.cast_desc(k, ROLE_X, xs[k], L.Xq, L.XqT),
+                      self.cast_desc(k, ROLE_W, L.W, L.Wq, L.WqT),
+                      self.cast_desc(k, ROLE_DY, dys[k], L.dYq, L.dYqT)]
+        fp8_cast_transpose_amax_current_multi(descs, self.margin, self.current_ws, stream=stream)
+
     def gemm(self, k, which, stream=None):
         """which: 0 = fprop Y = X.W, 1 = dgrad dX = dY.W^T, 2 = wgrad dW = X^T.dY."""
-        L = self.layers[k]
-        sx, sw, sdy = (self._slot(self.sinv_used, 3 * k + r) for r in (ROLE_X, ROLE_W, ROLE_DY))
-        if which == 0:
-            fp8_gemm(L.Xq, E4M3, L.WqT, E4M3, sx, sw, L.Y, stream=stream)
-        elif which == 1:
-            fp8_gemm(L.dYq, E5M2, L.Wq, E4M3, sdy, sw, L.dX, stream=stream)
-        else:
-            fp8_gemm(L.XqT, E4M3, L.dYqT, E5M2, sx, sdy, L.dW, stream=stream)
+        fp8_gemm_multi([self.gemm_desc(k, which)], stream=stream)
 
     def gemm_desc(self, k, which):
         L = self.layers[k]
         sx, sw, sdy = (self._slot(self.sinv_used, 3 * k + r) for r in (ROLE_X, ROLE_W, ROLE_DY))
+        t = self.transposes
         if which == 0:
-            return dict(A=L.Xq, a_fmt=E4M3, B=L.WqT, b_fmt=E4M3, a_scale_inv=sx, b_scale_inv=sw, D=L.Y)
+            return dict(A=L.Xq, a_fmt=E4M3, B=L.WqT if t else L.Wq, b_mn=not t, b_fmt=E4M3,
+                        a_scale_inv=sx, b_scale_inv=sw, D=L.Y)
         if which == 1:
             return dict(A=L.dYq, a_fmt=E5M2, B=L.Wq, b_fmt=E4M3, a_scale_inv=sdy, b_scale_inv=sw, D=L.dX)
-        return dict(A=L.XqT, a_fmt=E4M3, B=L.dYqT, b_fmt=E5M2, a_scale_inv=sx, b_scale_inv=sdy, D=L.dW)
+        return dict(A=L.XqT if t else L.Xq, a_mn=not t, a_fmt=E4M3, B=L.dYqT if t else L.dYq,
+                    b_mn=not t, b_fmt=E5M2, a_scale_inv=sx, b_scale_inv=sdy, D=L.dW)
 
     def _gemm_descs(self, sumsq=False):
         descs = [self.gemm_desc(k, w) for k in range(len(self.layers)) for w in (0, 1, 2)]
@@ -219,16 +237,20 @@ class Fp8LinearStep:
         for k, L in enumerate(self.layers):
             i = 3 * k + ROLE_W
             out.append(dict(rows=L.fin, cols=L.fout, fmt=E4M3, scale=self._slot(self.scale, i),
-                            q=L.Wq, qT=L.WqT, amax=self._slot(self.amax, i),
+                            q=L.Wq, amax=self._slot(self.amax, i),
                             scale_inv=self._slot(self.sinv_used, i)))
         return out
 
     def step(self, xs, dys, stream=None):
         """One training step; xs[k] = X [tokens, in_k], dys[k] = dY [tokens, out_k] (BF16, device)."""
         self.t += 1
-        self.cast_all(xs, dys, stream, update=self.fused_update)
+        if self.recipe == "current":
+            self.amax.zero_()                  # amax slots report this step's tensors only
+            self.cast_all_current(xs, dys, stream)
+        else:
+            self.cast_all(xs, dys, stream, update=self.fused_update)
         self.gemm_all(stream, sumsq=self.fused_norm)
-        if not self.fused_update:
+        if not self.fused_update and self.recipe == "delayed":
             self.scale_update(stream)
         self.adamw(stream, presummed=self.fused_norm)
 
@@ -265,6 +287,8 @@ class Fp8LinearStep:
         n_adamw_batches = (len(self.layers) + 255) // 256
         n_cast_launches = (3 * len(self.layers) + 7) // 8
         n_gemm_launches = (3 * len(self.layers) + 23) // 24
-        n_scale_launches = 0 if self.fused_update else 1
+        n_scale_launches = 0 if self.fused_update or self.recipe == "current" else 1
+        if self.recipe == "current":
+            n_cast_launches *= 2                   # an amax launch before each cast launch
         n_adamw_launches = (1 if self.fused_norm else 2) * n_adamw_batches
         return n_cast_launches + n_gemm_launches + n_scale_launches + n_adamw_launches

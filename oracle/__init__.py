@@ -68,6 +68,16 @@ def lib():
         L.orc_fused_adamw.argtypes = [C.c_int32, pp, pp, pp, pp, pp, i64p, C.c_float,
                                       C.c_float, C.c_float, C.c_float, C.c_float, C.c_int64,
                                       C.c_float, C.c_float, f32p]
+        L.orc_e8m0_decode.restype = C.c_double
+        L.orc_e8m0_decode.argtypes = [C.c_uint8]
+        L.orc_mx_quantise.restype = None
+        L.orc_mx_quantise.argtypes = [u16p, C.c_int64, C.c_int64, C.c_int, C.c_int, u8p, u8p]
+        L.orc_mx_gemm.restype = None
+        L.orc_mx_gemm.argtypes = [u8p, u8p, C.c_int, u8p, u8p, C.c_int, C.c_int64, C.c_int64,
+                                  C.c_int64, u16p, f64p]
+        L.orc_mx_gemm_at.restype = None
+        L.orc_mx_gemm_at.argtypes = [u8p, u8p, C.c_int, u8p, u8p, C.c_int, C.c_int64, C.c_int64,
+                                     i64p, i64p, u16p, f64p]
         _lib = L
     return _lib
 
@@ -131,6 +141,25 @@ def cast_transpose_amax(x_bf16: np.ndarray, fmt: int, scale: float, want_q=True,
     return q, qT, amax[0], sinv[0], cnt
 
 
+def cast_current(x_bf16, fmt, margin, prev_scale, want_q=True, want_qT=True):
+    """Oracle of fp8_cast_transpose_amax_current_multi for one tensor: current scaling.
+
+    "FP8 混合精度训练工程实践" §四 (FP8Tensor.quantize measures amax = max|x| of the tensor it is
+    about to quantise) with the scale rule of "LLM FP8 微调上线生产实战" 核心原理
+    (scale = (FP8_MAX / amax) / 2^margin), applied without delay: the amax of x, the scale that
+    the scale update forms from a one-entry history holding it (its zero / non-finite / overflow
+    readings included), then the cast with that scale.
+    Returns (q, qT, amax, scale, scale_inv, counters)."""
+    _, _, amax, _, _ = cast_transpose_amax(x_bf16, fmt, 1.0, False, False)
+    hist = np.zeros((1, 1), np.float32)
+    scale = np.array([prev_scale], np.float32)
+    sinv = np.zeros(1, np.float32)
+    scale_update(np.array([amax], np.float32), hist, [FP8_MAX[fmt]], AMAX_MOST_RECENT, margin,
+                 scale, sinv)
+    q, qT, a, si, cnt = cast_transpose_amax(x_bf16, fmt, scale[0], want_q, want_qT)
+    return q, qT, a, scale[0], si, cnt
+
+
 # ----------------------------------------------------------------------------- scale update
 def scale_update(amax, hist, fp8_max, algo, margin, scale, scale_inv):
     """Oracle of fp8_scale_update. hist [n, H], scale and scale_inv [n] are updated in place;
@@ -178,6 +207,58 @@ def gemm_at(A, afmt, B, bfmt, a_scale_inv, b_scale_inv, ii, jj):
                       float(np.float32(a_scale_inv)), float(np.float32(b_scale_inv)), ii.size,
                       _ptr(ii, C.c_int64), _ptr(jj, C.c_int64), _ptr(out, C.c_uint16),
                       _ptr(ab, C.c_double))
+    return out, ab
+
+
+# ----------------------------------------------------------------------------- MXFP8
+def e8m0_decode(code):
+    """Value of an E8M0 block-scale code: 2^(code - 127), 0xFF = NaN ("FP8 混合精度训练工程实践" §九)."""
+    return lib().orc_e8m0_decode(int(code))
+
+
+def mx_quantise(x_bf16, axis, fmt):
+    """MX block quantisation (blocks of 32 along a row for axis 0, down a column for axis 1) of
+    a 2-D uint16 (BF16 bits) array; returns (q [rows, cols], sf) with sf [rows, cols/32] for
+    axis 0 and [rows/32, cols] for axis 1."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    rows, cols = x.shape
+    assert (cols if axis == 0 else rows) % 32 == 0
+    q = np.empty((rows, cols), np.uint8)
+    sf = np.empty((rows, cols // 32) if axis == 0 else (rows // 32, cols), np.uint8)
+    lib().orc_mx_quantise(_ptr(x, C.c_uint16), rows, cols, int(axis), int(fmt), _ptr(q, C.c_uint8),
+                          _ptr(sf, C.c_uint8))
+    return q, sf
+
+
+def mx_gemm(A, sfa, afmt, B, sfb, bfmt, want_abs=False):
+    """MX GEMM oracle: D = bf16(sum over K of a * b * 2^(Xa + Xb)); A [M, K], B [N, K] codes,
+    sfa [M, K/32], sfb [N, K/32] E8M0 codes (all K-contiguous)."""
+    A, B = np.ascontiguousarray(A, np.uint8), np.ascontiguousarray(B, np.uint8)
+    sfa, sfb = np.ascontiguousarray(sfa, np.uint8), np.ascontiguousarray(sfb, np.uint8)
+    M, K = A.shape
+    N = B.shape[0]
+    assert B.shape[1] == K and K % 32 == 0 and sfa.shape == (M, K // 32) and sfb.shape == (N, K // 32)
+    D = np.empty((M, N), np.uint16)
+    ab = np.empty((M, N), np.float64) if want_abs else None
+    lib().orc_mx_gemm(_ptr(A, C.c_uint8), _ptr(sfa, C.c_uint8), int(afmt), _ptr(B, C.c_uint8),
+                      _ptr(sfb, C.c_uint8), int(bfmt), M, N, K, _ptr(D, C.c_uint16),
+                      _ptr(ab, C.c_double))
+    return (D, ab) if want_abs else D
+
+
+def mx_gemm_at(A, sfa, afmt, B, sfb, bfmt, ii, jj):
+    """The MX GEMM oracle at output positions (ii[s], jj[s]); returns (D bits, abs_sum)."""
+    A, B = np.ascontiguousarray(A, np.uint8), np.ascontiguousarray(B, np.uint8)
+    sfa, sfb = np.ascontiguousarray(sfa, np.uint8), np.ascontiguousarray(sfb, np.uint8)
+    K = A.shape[1]
+    ii = np.ascontiguousarray(ii, np.int64)
+    jj = np.ascontiguousarray(jj, np.int64)
+    assert (ii >= 0).all() and (ii < A.shape[0]).all() and (jj >= 0).all() and (jj < B.shape[0]).all()
+    out = np.empty(ii.shape, np.uint16)
+    ab = np.empty(ii.shape, np.float64)
+    lib().orc_mx_gemm_at(_ptr(A, C.c_uint8), _ptr(sfa, C.c_uint8), int(afmt), _ptr(B, C.c_uint8),
+                         _ptr(sfb, C.c_uint8), int(bfmt), K, ii.size, _ptr(ii, C.c_int64),
+                         _ptr(jj, C.c_int64), _ptr(out, C.c_uint16), _ptr(ab, C.c_double))
     return out, ab
 
 

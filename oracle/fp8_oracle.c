@@ -387,3 +387,144 @@ int orc_fused_adamw(int32_t n, float* const* master, float* const* m, float* con
     return orc_adamw_update(n, master, m, v, g, w, numel, lr, beta1, beta2, eps, wd, step,
                             loss_scale, max_norm, norm);
 }
+
+/* ---------------------------------------------------------------------------------------
+ * MXFP8 block scaling [P2 §九, Blackwell Microscaling: groups of 32 values share one 8-bit
+ * E8M0 scale, each value stored as FP8; P2 §三, "为什么权重梯度用 E5M2": micro scaling with
+ * E4M3 elements is the Blackwell direction for gradients too].
+ *
+ * Readings (the pages fix the block size, the scale type and the element type only):
+ *   - E8M0 (8 exponent bits, no sign or mantissa) is 2^(code - 127); code 0xFF is NaN. (The
+ *     page's "FP32 scale per 32 elements" line contradicts its own E8M0 diagram; the diagram is
+ *     taken.)
+ *   - A block is 32 consecutive values along the contraction dimension: along a row for the
+ *     row-wise copy, down a column for the column-wise copy (the 32 x 32 "sub-block" wording of
+ *     §三 is read as this 1 x 32 grouping, which is what the diagram shows).
+ *   - The shared exponent follows the published MX rule: X = floor(log2(amax)) - emax, emax the
+ *     exponent of the element format's largest value (8 for E4M3, 448 = 1.75 * 2^8; 15 for
+ *     E5M2), clamped to [-127, 127]; elements are encode(f32(x) * 2^-X) with the same
+ *     round-to-nearest-even and saturation as the per-tensor cast, so the top of a block may
+ *     saturate (values in [448, 512) * 2^X become 448 * 2^X).
+ *   - amax = 0: X = -127 (all elements are zero). amax = +inf: X = 127. A NaN in the block:
+ *     scale code 0xFF and the elements encoded with X = 0.
+ * ------------------------------------------------------------------------------------- */
+double orc_e8m0_decode(uint8_t code)
+{
+    if (code == 0xFF) return NAN;
+    return ldexp(1.0, (int)code - 127);
+}
+
+/* floor(log2(|v|)) of a non-zero finite BF16 magnitude pattern (normal or subnormal). */
+static int bf16_floor_log2(uint16_t mag)
+{
+    const int e = (mag >> 7) & 0xFF;
+    if (e) return e - 127;
+    int top = 6;                                   /* subnormal: m * 2^-133, m < 128 */
+    while (!((mag >> top) & 1)) --top;
+    return top - 133;
+}
+
+static uint8_t mx_block(const uint16_t* x, int64_t stride, int fmt, uint8_t* q, int64_t qstride)
+{
+    uint16_t amax = 0;
+    for (int i = 0; i < 32; ++i) {
+        const uint16_t m = x[i * stride] & 0x7FFF;
+        if (m > amax) amax = m;                    /* NaN patterns sort above infinity */
+    }
+    int X;
+    uint8_t code;
+    if (amax > 0x7F80) {                           /* NaN in the block */
+        X = 0;
+        code = 0xFF;
+    } else {
+        if (amax == 0) X = -127;
+        else if (amax == 0x7F80) X = 127;
+        else {
+            X = bf16_floor_log2(amax) - (fmt == ORC_E4M3 ? 8 : 15);
+            if (X < -127) X = -127;
+            if (X > 127) X = 127;
+        }
+        code = (uint8_t)(X + 127);
+    }
+    const float inv = (float)ldexp(1.0, -X);      /* exact power of two in f32 */
+    for (int i = 0; i < 32; ++i)
+        q[i * qstride] = orc_fp8_encode(orc_bf16_to_f32(x[i * stride]) * inv, fmt);
+    return code;
+}
+
+/* MX quantisation of a BF16 matrix x [rows x cols]. axis 0: blocks of 32 consecutive columns
+ * of a row, sf [rows x cols/32]; axis 1: blocks of 32 consecutive rows of a column, sf
+ * [rows/32 x cols]. q [rows x cols] in the same layout as x either way. */
+void orc_mx_quantise(const uint16_t* x, int64_t rows, int64_t cols, int axis, int fmt,
+                     uint8_t* q, uint8_t* sf)
+{
+    if (axis == 0) {
+        for (int64_t r = 0; r < rows; ++r)
+            for (int64_t b = 0; b < cols / 32; ++b)
+                sf[r * (cols / 32) + b] = mx_block(x + r * cols + 32 * b, 1, fmt, q + r * cols + 32 * b, 1);
+    } else {
+        for (int64_t b = 0; b < rows / 32; ++b)
+            for (int64_t c = 0; c < cols; ++c)
+                sf[b * cols + c] = mx_block(x + 32 * b * cols + c, cols, fmt, q + 32 * b * cols + c, cols);
+    }
+}
+
+/* One output of the MX GEMM: sum over K-blocks of 2^(Xa + Xb) * sum_k a_k b_k. Each block sum
+ * is exact in __int128 (FP8 values times 2^16 are integers); blocks are combined in 64-bit-
+ * mantissa long double (relative error below 2^-55 of the sum of magnitudes, far inside the
+ * GEMM tolerance), then rounded to f32 and BF16. NaN scales or non-finite codes fall back to a
+ * plain sum with IEEE propagation. abs_out: sum |a_k b_k| 2^(Xa + Xb). */
+static void mx_element(const uint8_t* a, const uint8_t* sa, int afmt, const uint8_t* b,
+                       const uint8_t* sb, int bfmt, int64_t K, uint16_t* d_out, double* abs_out)
+{
+    long double acc = 0.0L, absacc = 0.0L;
+    for (int64_t kb = 0; kb < K / 32; ++kb) {
+        const double s = orc_e8m0_decode(sa[kb]) * orc_e8m0_decode(sb[kb]);
+        __int128 blk = 0, babs = 0;
+        int plain = isnan(s);
+        for (int k = 0; k < 32 && !plain; ++k)
+            if (!orc_fp8_is_finite(a[32 * kb + k], afmt) || !orc_fp8_is_finite(b[32 * kb + k], bfmt))
+                plain = 1;
+        if (plain) {
+            for (int k = 0; k < 32; ++k) {
+                const double p = orc_fp8_decode(a[32 * kb + k], afmt) * orc_fp8_decode(b[32 * kb + k], bfmt);
+                acc += (long double)p * s;
+                absacc += fabsl((long double)p * s);
+            }
+            continue;
+        }
+        for (int k = 0; k < 32; ++k) {
+            const __int128 p = (__int128)fp8_times_2p16(a[32 * kb + k], afmt) *
+                               fp8_times_2p16(b[32 * kb + k], bfmt);
+            blk += p;
+            babs += p < 0 ? -p : p;
+        }
+        const int e = ((int)sa[kb] - 127) + ((int)sb[kb] - 127) - 32;
+        acc += ldexpl((long double)blk, e);
+        absacc += ldexpl((long double)babs, e);
+    }
+    *d_out = orc_f32_to_bf16((float)(double)acc);
+    if (abs_out) *abs_out = (double)absacc;
+}
+
+/* D [M x N] = bf16(A . B^T) with block scales: A [M x K] and B [N x K] codes (K contiguous),
+ * sfa [M x K/32], sfb [N x K/32]. */
+void orc_mx_gemm(const uint8_t* A, const uint8_t* sfa, int afmt, const uint8_t* B,
+                 const uint8_t* sfb, int bfmt, int64_t M, int64_t N, int64_t K, uint16_t* D,
+                 double* abs_out)
+{
+    for (int64_t i = 0; i < M; ++i)
+        for (int64_t j = 0; j < N; ++j)
+            mx_element(A + i * K, sfa + i * (K / 32), afmt, B + j * K, sfb + j * (K / 32), bfmt, K,
+                       D + i * N + j, abs_out ? abs_out + i * N + j : NULL);
+}
+
+/* The MX GEMM at chosen output positions (ii[s], jj[s]). */
+void orc_mx_gemm_at(const uint8_t* A, const uint8_t* sfa, int afmt, const uint8_t* B,
+                    const uint8_t* sfb, int bfmt, int64_t K, int64_t n, const int64_t* ii,
+                    const int64_t* jj, uint16_t* out, double* abs_out)
+{
+    for (int64_t s = 0; s < n; ++s)
+        mx_element(A + ii[s] * K, sfa + ii[s] * (K / 32), afmt, B + jj[s] * K, sfb + jj[s] * (K / 32),
+                   bfmt, K, out + s, abs_out ? abs_out + s : NULL);
+}

@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(lib):
     raw = C.CDLL(fp8.LIB_PATH)
     for name in declared_functions():
         assert hasattr(raw, name), name
-    assert lib.fp8t_abi_version() == 1
+    assert lib.fp8t_abi_version() == 2
     for s in range(7):
         assert lib.fp8t_status_string(s).decode() == _abi.status_name(s)
 
@@ -98,6 +98,8 @@ def test_invalid_arguments_rejected_on_host(lib):
     assert lib.fp8_gemm_multi(g, 2, z) == 2 and b"problem 1" in lib.fp8t_last_error_message()
     g[1] = _abi.GemmDesc(P, 1, P, 3, 16, 16, 16, P, P, P)
     assert lib.fp8_gemm_multi(g, 2, z) == 1
+    g[1] = _abi.GemmDesc(P, 1, P, 0, 16, 16, 16, P, P, P, 0, 2)     # unknown operand layout
+    assert lib.fp8_gemm_multi(g, 2, z) == 1 and b"layout" in lib.fp8t_last_error_message()
     assert lib.fp8_gemm_multi(g, 0, z) == 1
     # grouped gemm with the sum of squares
     g[1] = _abi.GemmDesc(P, 1, P, 0, 16, 16, 16, P, P, P)
@@ -147,12 +149,12 @@ def test_invalid_arguments_rejected_on_host(lib):
     w16 = (_abi.AdamWTensor * 1)()
     w16[0] = _abi.AdamWTensor(P, P, P, P, P, 32 * 48)
     cast = (_abi.AdamWCast * 1)()
-    cast[0] = _abi.AdamWCast(32, 40, 0, P, P, P, P, P)
+    cast[0] = _abi.AdamWCast(32, 40, 0, P, P, P, P)
     assert pre(w16, casts=cast) == 2
-    cast[0] = _abi.AdamWCast(32, 48, 5, P, P, P, P, P)
+    cast[0] = _abi.AdamWCast(32, 48, 5, P, P, P, P)
     assert pre(w16, casts=cast) == 1
-    cast[0] = _abi.AdamWCast(32, 48, 0, None, P, P, P, P)
+    cast[0] = _abi.AdamWCast(32, 48, 0, None, P, P, P)
     assert pre(w16, casts=cast) == 1
-    cast[0] = _abi.AdamWCast(32, 48, 0, P, U, P, P, P)
+    cast[0] = _abi.AdamWCast(32, 48, 0, P, U, P, P)
     assert pre(w16, casts=cast) == 3
     assert lib.fp8t_debug_expire_waits(3) == 1 and lib.fp8t_debug_expire_waits(-1) == 1

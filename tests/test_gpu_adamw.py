@@ -204,7 +204,6 @@ def _weight_casts(shapes, fmts, scales):
             continue
         casts.append(dict(rows=r, cols=c, fmt=f, scale=torch.tensor([s], device="cuda"),
                           q=torch.full((r, c), 0xAB, dtype=torch.uint8, device="cuda"),
-                          qT=torch.full((c, r), 0xAB, dtype=torch.uint8, device="cuda"),
                           amax=torch.zeros(1, device="cuda"), scale_inv=torch.zeros(1, device="cuda")))
     return casts
 
@@ -215,18 +214,18 @@ def _check_weight_casts(W, casts, scales):
         if c is None:
             continue
         bits = bf16_bits(w).reshape(c["rows"], c["cols"])
-        q, qT, a, si, _ = oracle.cast_transpose_amax(bits, c["fmt"], s)
-        assert np.array_equal(u8(c["q"]), q) and np.array_equal(u8(c["qT"]), qT)
+        q, _, a, si, _ = oracle.cast_transpose_amax(bits, c["fmt"], s, True, False)
+        assert np.array_equal(u8(c["q"]), q)
         assert np.float32(c["amax"].item()).view(np.uint32) == np.float32(a).view(np.uint32)
         assert np.float32(c["scale_inv"].item()).view(np.uint32) == np.float32(si).view(np.uint32)
 
 
 def test_presummed_with_weight_casts(cuda_lib):
     """The next step's weight cast inside AdamW ("算子与编译器" 优化器 kernel 的带宽账: one pass over
-    the parameters): the update matches the oracle, and the codes, transposed codes, amax and
-    scale inverse of each new BF16 weight match the oracle's cast of it. Ragged tile edges, both
-    formats, a tensor without a cast among them, and 40 casts (two launch tables). Then a skipped
-    step (NaN sum of squares): weights unchanged and cast again with a new scale."""
+    the parameters): the update matches the oracle, and the row-major codes, amax and scale
+    inverse of each new BF16 weight match the oracle's cast of it. Both formats, a tensor
+    without a cast among them, and 40 casts (two launch tables). Then a skipped step (NaN sum of
+    squares): weights unchanged and cast again with a new scale."""
     rng = np.random.default_rng(13)
     shapes = [(272, 400), (16, 16), (0, 0), (4096 // 8, 128 * 3), (64, 2064)]
     shapes += [(16 * int(rng.integers(1, 9)), 16 * int(rng.integers(1, 9))) for _ in range(38)]

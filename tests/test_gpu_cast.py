@@ -31,14 +31,16 @@ def run_gpu(fp8, x, fmt, scale, want_q=True, want_qT=True, counters=True):
 
 
 def check(fp8, x_bits, fmt, scale):
+    """Both kernels: the tiled one (q and q^T) and the streaming one (q only)."""
     x = bf16_from_bits(x_bits)
-    q, qT, amax, sinv, cnt = run_gpu(fp8, x, fmt, scale)
     rq, rqT, ramax, rsinv, rcnt = oracle.cast_transpose_amax(x_bits, fmt, scale)
-    assert np.array_equal(q, rq), "row-major codes differ"
-    assert np.array_equal(qT, rqT), "transposed codes differ"
-    assert amax.view(np.uint32) == np.float32(ramax).view(np.uint32), (amax, ramax)
-    assert sinv.view(np.uint32) == np.float32(rsinv).view(np.uint32)
-    assert np.array_equal(cnt, rcnt), (cnt, rcnt)
+    for want_qT in (True, False):
+        q, qT, amax, sinv, cnt = run_gpu(fp8, x, fmt, scale, want_qT=want_qT)
+        assert np.array_equal(q, rq), "row-major codes differ"
+        assert not want_qT or np.array_equal(qT, rqT), "transposed codes differ"
+        assert amax.view(np.uint32) == np.float32(ramax).view(np.uint32), (amax, ramax)
+        assert sinv.view(np.uint32) == np.float32(rsinv).view(np.uint32)
+        assert np.array_equal(cnt, rcnt), (cnt, rcnt)
 
 
 @pytest.mark.parametrize("fmt", [oracle.E4M3, oracle.E5M2])
@@ -162,7 +164,8 @@ def test_multi_tensor_launch(cuda_lib):
 @pytest.mark.parametrize("n,H,algo,margin", [(3, 1, oracle.AMAX_MAX, 0), (3, 16, oracle.AMAX_MAX, 1),
                                              (21, 16, oracle.AMAX_MOST_RECENT, 0),
                                              (5, 1024, oracle.AMAX_MAX, 0), (9, 3000, oracle.AMAX_MAX, 3)])
-def test_cast_with_fused_scale_update(cuda_lib, n, H, algo, margin):
+@pytest.mark.parametrize("with_qT", [True, False], ids=["tiled", "streaming"])
+def test_cast_with_fused_scale_update(cuda_lib, n, H, algo, margin, with_qT):
     """fp8_cast_transpose_amax_update_multi equals the oracle's cast followed by its scale
     update ("LLM FP8 微调上线生产实战" 核心原理: history roll, representative amax, next scale), bit
     for bit: codes, inverse of the scale used, history, next scale and its inverse, amax slots
@@ -193,7 +196,7 @@ def test_cast_with_fused_scale_update(cuda_lib, n, H, algo, margin):
     for i, ((r, c), f) in enumerate(zip(shapes, fmts)):
         casts.append(dict(x=bf16_from_bits(xs[i]), fmt=f, scale=scale[i:i + 1],
                           q=torch.empty(r, c, dtype=torch.uint8, device="cuda"),
-                          qT=torch.empty(c, r, dtype=torch.uint8, device="cuda"),
+                          qT=torch.empty(c, r, dtype=torch.uint8, device="cuda") if with_qT else None,
                           amax=amax[i:i + 1], scale_inv=sinv_used[i:i + 1]))
         ups.append(dict(history=hist[i], scale_inv_next=sinv_next[i:i + 1]))
     cuda_lib.fp8_cast_transpose_amax_update_multi(casts, ups, algo, margin, ticket)
@@ -202,7 +205,8 @@ def test_cast_with_fused_scale_update(cuda_lib, n, H, algo, margin):
     amax_ref = np.zeros(n, np.float32)
     for i, f in enumerate(fmts):
         rq, rqT, ra, rsinv, _ = oracle.cast_transpose_amax(xs[i], f, scale0[i])
-        assert np.array_equal(u8(casts[i]["q"]), rq) and np.array_equal(u8(casts[i]["qT"]), rqT)
+        assert np.array_equal(u8(casts[i]["q"]), rq)
+        assert not with_qT or np.array_equal(u8(casts[i]["qT"]), rqT)
         assert np.float32(sinv_used[i].item()).view(np.uint32) == np.float32(rsinv).view(np.uint32)
         amax_ref[i] = ra
     h_ref, s_ref, si_ref = hist0.copy(), scale0.copy(), np.zeros(n, np.float32)
@@ -247,3 +251,42 @@ def test_fused_scale_update_equals_separate_launch(cuda_lib):
             assert torch.equal(a, b)
         for key in ("scale", "hist", "amax", "used", "nxt"):
             assert torch.equal(state[0][key], state[1][key]), (t, key)
+
+
+def test_current_scaling_multi(cuda_lib):
+    """fp8_cast_transpose_amax_current_multi against the oracle's current scaling (amax of the
+    tensor itself, then scale = (FP8_MAX / amax) / 2^margin, then the cast), bit for bit: scale
+    written in place, codes, transposed codes, inverse scale, amax slot; 11 tensors (two amax
+    launches), an all-zero tensor (scale 1) and one with an infinity (previous scale kept); the
+    workspace is left zeroed."""
+    rng = np.random.default_rng(31)
+    n, margin = 11, 1
+    shapes = [(16 * int(rng.integers(1, 40)), 16 * int(rng.integers(1, 40))) for _ in range(n)]
+    shapes[0] = (4096, 2048)                             # a tensor large enough for many CTAs
+    fmts = [oracle.E4M3 if i % 2 else oracle.E5M2 for i in range(n)]
+    xs = []
+    for i, (r, c) in enumerate(shapes):
+        x = (rng.standard_normal((r, c)) * 10.0 ** rng.uniform(-3, 3)).astype(np.float32)
+        if i == 3:
+            x[:] = 0.0
+        if i == 5:
+            x[r - 1, c - 1] = np.inf
+        xs.append(bf16_bits(torch.from_numpy(x).to(torch.bfloat16)))
+    prev = [float(np.float32(2.0 ** rng.uniform(-4, 4))) for _ in range(n)]
+    ws = torch.zeros(cuda_lib.CURRENT_WORKSPACE_BYTES, dtype=torch.uint8, device="cuda")
+    casts = []
+    for i, ((r, c), f) in enumerate(zip(shapes, fmts)):
+        casts.append(dict(x=bf16_from_bits(xs[i]), fmt=f, scale=dev_scalar(prev[i]),
+                          q=torch.empty(r, c, dtype=torch.uint8, device="cuda"),
+                          qT=torch.empty(c, r, dtype=torch.uint8, device="cuda"),
+                          amax=torch.zeros(1, device="cuda"), scale_inv=torch.zeros(1, device="cuda")))
+    cuda_lib.fp8_cast_transpose_amax_current_multi(casts, margin, ws)
+    cuda_lib.fp8t_check_device_error()
+    for i, c in enumerate(casts):
+        rq, rqT, ra, rs, rsinv, _ = oracle.cast_current(xs[i], fmts[i], margin, prev[i])
+        assert np.float32(c["scale"].item()).view(np.uint32) == np.float32(rs).view(np.uint32), i
+        assert np.array_equal(u8(c["q"]), rq) and np.array_equal(u8(c["qT"]), rqT), i
+        assert np.float32(c["scale_inv"].item()).view(np.uint32) == np.float32(rsinv).view(np.uint32)
+        assert np.float32(c["amax"].item()).view(np.uint32) == np.float32(ra).view(np.uint32)
+    assert casts[3]["scale"].item() == 1.0 and casts[5]["scale"].item() == np.float32(prev[5])
+    assert not ws.any().item()

@@ -162,3 +162,51 @@ def test_grouped_launch_with_sum_of_squares(cuda_lib):
     cuda_lib.fp8_gemm_multi_sumsq(descs, out, ws)
     cuda_lib.fp8t_check_device_error()
     assert np.float64(out.item()).view(np.uint64) == np.float64(first).view(np.uint64)
+
+
+@pytest.mark.parametrize("a_mn,b_mn", [(False, True), (True, False), (True, True)],
+                         ids=["B-MN-major", "A-MN-major", "both-MN-major"])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 128), (144, 272, 48), (400, 528, 1040),
+                                   (256, 768, 4096), (16, 16, 16)])
+def test_mn_major_operands(cuda_lib, a_mn, b_mn, M, N, K):
+    """Operands stored MN-major (A as K x M, B as K x N, row-major) give the product of the same
+    logical matrices: the tensor cores read 8-bit operands in either order, which is what lets
+    the step skip the transposed FP8 copies. All four format pairs, ragged tiles."""
+    for i, (af, bf) in enumerate(PAIRS):
+        A = random_codes(M, K, af, 1000 + M + K + i)
+        B = random_codes(N, K, bf, 2000 + N + K + i)
+        sa, sb = 0.021, 0.37
+        D = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        cuda_lib.fp8_gemm_multi([dict(A=A.t().contiguous() if a_mn else A, a_mn=a_mn, a_fmt=af,
+                                      B=B.t().contiguous() if b_mn else B, b_mn=b_mn, b_fmt=bf,
+                                      a_scale_inv=dev_scalar(sa), b_scale_inv=dev_scalar(sb), D=D)])
+        cuda_lib.fp8t_check_device_error()
+        R, ab = oracle.gemm(u8(A), af, u8(B), bf, sa, sb, want_abs=True)
+        ok = gemm_within_tolerance(bf16_bits(D), R, ab)
+        assert ok.all(), f"pair {i}: {(~ok).sum()} of {ok.size} outside tolerance"
+
+
+def test_step_layouts_full_size_sampled(cuda_lib):
+    """The 4096-class step's GEMMs exactly as the step issues them, in one grouped launch: fprop
+    (Xq K-major, Wq MN-major), dgrad (dYq, Wq both K-major), wgrad (Xq, dYq both MN-major, K =
+    8192 tokens), each on 4096 sampled outputs against the oracle's transposed operands."""
+    T, fin, fout = 8192, 4096, 4096
+    Xq = random_codes(T, fin, oracle.E4M3, 1)
+    Wq = random_codes(fin, fout, oracle.E4M3, 2)
+    dYq = random_codes(T, fout, oracle.E5M2, 3)
+    s = [dev_scalar(v) for v in (0.011, 0.023, 0.5)]
+    Y = torch.empty(T, fout, dtype=torch.bfloat16, device="cuda")
+    dX = torch.empty(T, fin, dtype=torch.bfloat16, device="cuda")
+    dW = torch.empty(fin, fout, dtype=torch.bfloat16, device="cuda")
+    cuda_lib.fp8_gemm_multi([
+        dict(A=Xq, a_fmt=0, B=Wq, b_mn=True, b_fmt=0, a_scale_inv=s[0], b_scale_inv=s[1], D=Y),
+        dict(A=dYq, a_fmt=1, B=Wq, b_fmt=0, a_scale_inv=s[2], b_scale_inv=s[1], D=dX),
+        dict(A=Xq, a_mn=True, a_fmt=0, B=dYq, b_mn=True, b_fmt=1, a_scale_inv=s[0],
+             b_scale_inv=s[2], D=dW)])
+    cuda_lib.fp8t_check_device_error()
+    hX, hW, hdY = u8(Xq), u8(Wq), u8(dYq)
+    for D, A, af, B, bf, sa, sb in ((Y, hX, 0, hW.T, 0, 0.011, 0.023), (dX, hdY, 1, hW, 0, 0.5, 0.023),
+                                    (dW, hX.T, 0, hdY.T, 1, 0.011, 0.5)):
+        ii, jj = sample_positions(D.shape[0], D.shape[1], 4096, seed=D.shape[1])
+        R, ab = oracle.gemm_at(np.ascontiguousarray(A), af, np.ascontiguousarray(B), bf, sa, sb, ii, jj)
+        assert gemm_within_tolerance(bf16_bits(D)[ii, jj], R, ab).all()

@@ -23,20 +23,27 @@ pytestmark = pytest.mark.gpu
 FMT = (oracle.E4M3, oracle.E4M3, oracle.E5M2)
 
 
-def make_step(wl, algo=None, margin=None, H=None, counters=True, fused=True):
+def make_step(wl, algo=None, margin=None, H=None, counters=True, fused=True, transposes=False):
     """fused: scale update in the cast launch, dW sum of squares in the wgrad epilogue and (when
-    no counters are kept) the next W cast inside AdamW; False: every stage its own launch."""
+    no counters are kept) the next W cast inside AdamW; False: every stage its own launch.
+    transposes: the casts also write q^T and the GEMMs read K-major operands only."""
     w0 = [synth.linear_weight(wl, k, "cuda") for k in range(len(wl.layers))]
     return Fp8LinearStep([(i, o) for _, i, o in wl.layers], wl.tokens,
                          H or wl.history_len, algo or wl.algo,
                          wl.margin if margin is None else margin, wl.adamw, w0, "cuda",
-                         counters=counters, fused_update=fused, fused_norm=fused, fused_wcast=fused)
+                         counters=counters, fused_update=fused, fused_norm=fused, fused_wcast=fused,
+                         transposes=transposes)
+
+
+def tr(q):
+    return np.ascontiguousarray(q.T)
 
 
 def snapshot(st):
     return dict(scale=f32(st.scale), hist=f32(st.history),
                 W=[bf16_bits(l.W) for l in st.layers], master=[f32(l.master) for l in st.layers],
-                Wq=[u8(l.Wq) for l in st.layers], WqT=[u8(l.WqT) for l in st.layers],
+                Wq=[u8(l.Wq) for l in st.layers],
+                WqT=[u8(l.WqT) if l.WqT is not None else tr(u8(l.Wq)) for l in st.layers],
                 m=[f32(l.m) for l in st.layers], v=[f32(l.v) for l in st.layers],
                 counters=st.counters.cpu().numpy().astype(np.uint64).copy() if st.counters is not None else None)
 
@@ -50,8 +57,11 @@ def check_step(st, pre, xs, dys, gemm_full=True, gemm_samples=2048, cast_check=T
     for k, L in enumerate(st.layers):
         srcs = (bf16_bits(xs[k]), pre["W"][k], bf16_bits(dys[k]))
         # the W codes this step's GEMMs read: cast during the previous AdamW when fused
-        wq = (pre["Wq"][k], pre["WqT"][k]) if st.fused_wcast else (u8(L.Wq), u8(L.WqT))
-        outs = ((u8(L.Xq), u8(L.XqT)), wq, (u8(L.dYq), u8(L.dYqT)))
+        # (without transposed copies on the device, q^T below is the host transpose of q; the
+        # GEMMs then read q MN-major)
+        both = lambda q, qT: (u8(q), u8(qT) if qT is not None else tr(u8(q)))
+        wq = (pre["Wq"][k], pre["WqT"][k]) if st.fused_wcast else both(L.Wq, L.WqT)
+        outs = (both(L.Xq, L.XqT), wq, both(L.dYq, L.dYqT))
         for r in range(3):
             i = 3 * k + r
             if cast_check:
@@ -114,20 +124,25 @@ def check_step(st, pre, xs, dys, gemm_full=True, gemm_samples=2048, cast_check=T
             q, qT, a, _, _ = oracle.cast_transpose_amax(bf16_bits(L.W), oracle.E4M3, scale[i],
                                                          cast_check, cast_check)
             if cast_check:
-                assert np.array_equal(u8(L.Wq), q) and np.array_equal(u8(L.WqT), qT)
+                assert np.array_equal(u8(L.Wq), q)
+                assert L.WqT is None or np.array_equal(u8(L.WqT), qT)
             assert np.float32(st.amax[i].item()).view(np.uint32) == np.float32(a).view(np.uint32)
             assert st.amax[3 * k].item() == 0 and st.amax[3 * k + 2].item() == 0
 
 
-@pytest.mark.parametrize("fused,counters", [(True, False), (True, True), (False, True)],
-                         ids=["all-fused", "fused-with-counters", "separate-launches"])
-def test_linear256_three_steps(cuda_lib, fused, counters):
+@pytest.mark.parametrize("fused,counters,transposes",
+                         [(True, False, False), (True, True, False), (False, True, False),
+                          (True, False, True), (False, True, True)],
+                         ids=["all-fused", "fused-with-counters", "separate-launches",
+                              "all-fused-transposes", "separate-launches-transposes"])
+def test_linear256_three_steps(cuda_lib, fused, counters, transposes):
     """Three steps in full. all-fused: scale update in the cast launch, dW sum of squares in the
     wgrad epilogue, next W cast in AdamW (three launches per step); with counters the W cast
-    stays in the cast launch; separate-launches: every stage its own kernel."""
+    stays in the cast launch; separate-launches: every stage its own kernel. Without transposes
+    the GEMMs read Xq, Wq, dYq MN-major where needed; with them, the K-major transposed copies."""
     wl = synth.LINEAR256
-    st = make_step(wl, fused=fused, counters=counters)
-    assert st.fused_wcast == (fused and not counters)
+    st = make_step(wl, fused=fused, counters=counters, transposes=transposes)
+    assert st.fused_wcast == (fused and not counters and not transposes)
     for t in range(wl.steps):
         xs, dys = zip(*[synth.linear_inputs(wl, k, t, "cuda") for k in range(len(wl.layers))])
         pre = snapshot(st)
@@ -158,7 +173,7 @@ def test_linear256_step_in_cuda_graph(cuda_lib):
     cuda_lib.fp8t_check_device_error()
     assert graphed.step_counter.item() == 3
     e, q = eager.layers[0], graphed.layers[0]
-    for a, b in ((e.Xq, q.Xq), (e.WqT, q.WqT), (e.dYqT, q.dYqT)):
+    for a, b in ((e.Xq, q.Xq), (e.Wq, q.Wq), (e.dYq, q.dYq)):
         assert torch.equal(a, b)
     assert torch.equal(eager.scale, graphed.scale) and torch.equal(eager.history, graphed.history)
     assert ulp_distance_f32(f32(e.master).reshape(-1), f32(q.master).reshape(-1)).max() <= 8
@@ -278,3 +293,28 @@ def test_monitor_flags_the_stress_spike(cuda_lib):
         flagged += [(s, msg) for kind, s, msg in mon.maybe_check(st) if kind == "amax_spike"]
     x_flags = [s for s, msg in flagged if msg.startswith("tensor 0:")]
     assert x_flags == [21]          # the batch of loop index 20 is the step counted t = 21
+
+
+def test_current_scaling_steps(cuda_lib):
+    """Three steps with current scaling: every cast uses the scale its own tensor's amax gives
+    (oracle cast_current), the GEMMs and AdamW as in the delayed recipe (the dW sum of squares
+    from the wgrad epilogue)."""
+    wl = synth.LINEAR256
+    st = Fp8LinearStep([(256, 256)], wl.tokens, wl.history_len, wl.algo, 1, wl.adamw,
+                       [synth.linear_weight(wl, 0, "cuda")], "cuda", recipe="current")
+    assert not st.fused_wcast and st.kernels_per_step() == 4
+    for t in range(3):
+        X, dY = synth.linear_inputs(wl, 0, t, "cuda")
+        W0 = bf16_bits(st.layers[0].W)
+        scale0 = f32(st.scale).copy()
+        st.step([X], [dY])
+        cuda_lib.fp8t_check_device_error()
+        L = st.layers[0]
+        srcs = (bf16_bits(X), W0, bf16_bits(dY))
+        for r, (q, src) in enumerate(zip((L.Xq, L.Wq, L.dYq), srcs)):
+            rq, _, ra, rs, rsinv, _ = oracle.cast_current(src, FMT[r], 1, scale0[r], True, False)
+            assert np.array_equal(u8(q), rq) and np.float32(st.scale[r].item()) == rs
+            assert np.float32(st.sinv_used[r].item()) == rsinv and np.float32(st.amax[r].item()) == ra
+        R, ab = oracle.gemm(u8(L.Xq), 0, tr(u8(L.Wq)), 0, f32(st.sinv_used)[0], f32(st.sinv_used)[1],
+                            want_abs=True)
+        assert gemm_within_tolerance(bf16_bits(L.Y), R, ab).all()

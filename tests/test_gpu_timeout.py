@@ -74,8 +74,9 @@ def test_expired_cast_leaves_scale_state_alone(cuda_lib):
     amax = torch.zeros(1, device="cuda")
     used, nxt = torch.zeros(1, device="cuda"), torch.zeros(1, device="cuda")
     ticket = torch.zeros(1, dtype=torch.int32, device="cuda")
+    # with q^T requested the tiled kernel runs (the streaming one has no waits to expire)
     casts = [dict(x=x, fmt=oracle.E4M3, scale=scale, q=torch.empty(4096, 2048, dtype=torch.uint8, device="cuda"),
-                  amax=amax, scale_inv=used)]
+                  qT=torch.empty(2048, 4096, dtype=torch.uint8, device="cuda"), amax=amax, scale_inv=used)]
     ups = [dict(history=hist, scale_inv_next=nxt)]
     _run_expired(cuda_lib, 1, lambda: cuda_lib.fp8_cast_transpose_amax_update_multi(
         casts, ups, oracle.AMAX_MAX, 0, ticket))

@@ -1,0 +1,108 @@
+"""Pins of the MXFP8 oracle ("FP8 混合精度训练工程实践" §九: 32 values share one E8M0 scale,
+each stored as FP8; §三: micro scaling with E4M3 elements), independent of its own code:
+
+* E8M0 decodes as 2^(code - 127) with 0xFF = NaN (the format's definition), checked on all codes;
+* the shared exponent is the published MX rule X = floor(log2 amax) - emax (emax 8 for E4M3,
+  15 for E5M2: 448 = 1.75 * 2^8, 57344 = 1.75 * 2^15, page values): for every block amax / 2^X
+  lies in [2^emax, 2^(emax+1)), checked by brute force on random blocks and on every power of two;
+* with every scale at 2^0 the MX quantisation reduces to the per-tensor cast at scale 1 and the MX
+  GEMM to the per-tensor GEMM at unit scales (special cases, both pinned elsewhere);
+* exact rational sums (fractions) on small GEMMs with mixed block scales;
+* all-ones and power-of-two closed forms."""
+from fractions import Fraction
+
+import numpy as np
+import torch
+
+import oracle
+from optimizer_fp8_cast_b200.synth import bf16_bits
+
+EMAX = {oracle.E4M3: 8, oracle.E5M2: 15}
+
+
+def test_e8m0_decode_every_code():
+    for c in range(255):
+        assert oracle.e8m0_decode(c) == 2.0 ** (c - 127)
+    assert np.isnan(oracle.e8m0_decode(255))
+
+
+def test_shared_exponent_rule_by_brute_force():
+    rng = np.random.default_rng(5)
+    for fmt in (oracle.E4M3, oracle.E5M2):
+        x = (rng.standard_normal((64, 256)) * 10.0 ** rng.uniform(-20, 20, (64, 1))).astype(np.float32)
+        bits = bf16_bits(torch.from_numpy(x).to(torch.bfloat16))
+        vals = (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        for axis in (0, 1):
+            q, sf = oracle.mx_quantise(bits, axis, fmt)
+            blocks = vals.reshape(64, 8, 32) if axis == 0 else vals.T.reshape(256, 2, 32)
+            scales = sf if axis == 0 else sf.T
+            for idx in np.ndindex(blocks.shape[:2]):
+                amax = np.abs(blocks[idx]).max()
+                X = int(scales[idx]) - 127
+                assert 2.0 ** EMAX[fmt] <= amax / 2.0 ** X < 2.0 ** (EMAX[fmt] + 1)
+            # decode(q) * 2^X is the element rounded to the format (within half a step of x)
+            dec = np.vectorize(lambda c: oracle.fp8_decode(int(c), fmt))(q).astype(np.float64)
+            rep = np.repeat(sf.astype(np.int64) - 127, 32, axis=1) if axis == 0 else \
+                np.repeat(sf.astype(np.int64) - 127, 32, axis=0)
+            back = dec * np.exp2(rep)
+            top = 448.0 if fmt == oracle.E4M3 else 57344.0
+            rel_step = 2.0 ** -(3 if fmt == oracle.E4M3 else 2)
+            unsat = np.abs(vals) <= top * np.exp2(rep)
+            err = np.abs(back - vals)[unsat]
+            assert (err <= np.abs(vals)[unsat] * rel_step / 2 + np.exp2(rep)[unsat] * 2.0 ** -10).all()
+
+
+def test_powers_of_two_and_zero_blocks():
+    for fmt in (oracle.E4M3, oracle.E5M2):
+        for k in range(-100, 101, 7):
+            x = np.full((1, 32), 2.0 ** k, np.float32)
+            q, sf = oracle.mx_quantise(bf16_bits(torch.from_numpy(x).to(torch.bfloat16)), 0, fmt)
+            assert sf[0, 0] == k - EMAX[fmt] + 127
+            # 2^emax is exponent field emax + bias, mantissa 0
+            assert q[0, 0] == ((EMAX[fmt] + (7 if fmt == oracle.E4M3 else 15)) << (3 if fmt == oracle.E4M3 else 2))
+        q, sf = oracle.mx_quantise(np.zeros((32, 32), np.uint16), 1, fmt)
+        assert (sf == 0).all() and not q.any()
+
+
+def test_unit_scales_reduce_to_the_per_tensor_cast_and_gemm():
+    rng = np.random.default_rng(6)
+    # blocks whose amax lies in [2^8, 2^9): the shared exponent is 0 for E4M3
+    x = rng.uniform(-300, 300, (32, 64)).astype(np.float32)
+    x[:, ::32] = 300.0
+    bits = bf16_bits(torch.from_numpy(x).to(torch.bfloat16))
+    q, sf = oracle.mx_quantise(bits, 0, oracle.E4M3)
+    assert (sf == 127).all()
+    rq, _, _, _, _ = oracle.cast_transpose_amax(bits, oracle.E4M3, 1.0)
+    assert np.array_equal(q, rq)
+    B = rng.integers(0, 0x7E, (48, 64)).astype(np.uint8)
+    D = oracle.mx_gemm(q, sf, oracle.E4M3, B, np.full((48, 2), 127, np.uint8), oracle.E4M3)
+    assert np.array_equal(D, oracle.gemm(q, oracle.E4M3, B, oracle.E4M3, 1.0, 1.0))
+
+
+def test_exact_rational_sums_with_block_scales():
+    rng = np.random.default_rng(7)
+    M, N, K = 3, 4, 96
+    A = rng.integers(0, 0x7E, (M, K)).astype(np.uint8) | (rng.integers(0, 2, (M, K)) << 7).astype(np.uint8)
+    B = rng.integers(0, 0x7B, (N, K)).astype(np.uint8)
+    sfa = rng.integers(100, 150, (M, K // 32)).astype(np.uint8)
+    sfb = rng.integers(110, 140, (N, K // 32)).astype(np.uint8)
+    D = oracle.mx_gemm(A, sfa, oracle.E4M3, B, sfb, oracle.E5M2)
+    for i in range(M):
+        for j in range(N):
+            s = sum(Fraction(oracle.fp8_decode(int(A[i, k]), oracle.E4M3)) *
+                    Fraction(oracle.fp8_decode(int(B[j, k]), oracle.E5M2)) *
+                    Fraction(2) ** (int(sfa[i, k // 32]) + int(sfb[j, k // 32]) - 254)
+                    for k in range(K))
+            ref = oracle.f32_to_bf16(np.float32(float(s)))
+            assert abs(int(D[i, j]) - int(ref)) <= 1 or D[i, j] == ref
+
+
+def test_all_ones_closed_form():
+    one = 0x38                                        # 1.0 in E4M3: exponent 7 (bias 7), mantissa 0
+    A = np.full((2, 128), one, np.uint8)
+    B = np.full((3, 128), one, np.uint8)
+    sfa = np.array([[127, 128, 126, 127]] * 2, np.uint8)
+    sfb = np.array([[130, 127, 127, 125]] * 3, np.uint8)
+    D = oracle.mx_gemm(A, sfa, oracle.E4M3, B, sfb, oracle.E4M3)
+    want = 32 * (2.0 ** 3 + 2.0 ** 1 + 2.0 ** -1 + 2.0 ** -2)
+    assert (D == oracle.f32_to_bf16(np.float32(want))).all()
