@@ -179,7 +179,11 @@ def run_ours(args, rank, world, local_rank):
         rec = (lambda i: ev[i].record()) if ev is not None else (lambda i: None)
         rec(0)
         for i, (name, kw) in enumerate(stages):
-            if name == "cast" and st.recipe == "current":
+            if name == "cast" and st.recipe == "mxfp8":
+                st.mx_cast_all(xs, dys)           # X, W, dY: both orientations + block scales
+            elif name == "gemm" and st.recipe == "mxfp8":
+                st.mx_gemm_all()                  # grouped block-scaled fprop, dgrad, wgrad
+            elif name == "cast" and st.recipe == "current":
                 st.amax.zero_()
                 st.cast_all_current(xs, dys)      # amax launch, then the grouped cast
             elif name == "cast":                  # grouped: X, W -> E4M3, dY -> E5M2
@@ -257,13 +261,17 @@ def run_ours(args, rank, world, local_rank):
     # AdamW as 1 B/param of codes (the new weight is already in registers there)
     per_el = (4 if st.transposes else 3) + (2 if st.recipe == "current" else 0)
     cast_bytes = nums["cast_bytes"] // 4 * per_el - (per_el * nums["params"] if st.fused_wcast else 0)
+    if st.recipe == "mxfp8":                # 2 B in, 2 x 1 B of codes, 2 x 1/32 B of scales
+        cast_bytes = nums["cast_bytes"] // 4 * 65 // 16
     adamw_bytes = ((28 + (1 if st.fused_wcast else 0)) * nums["params"]
                    + (0 if st.fused_norm else 2 * nums["params"]))
     cast_gbs = cast_bytes / (avg["cast"] * 1e-3) / 1e9
     adamw_gbs = adamw_bytes / (avg["adamw"] * 1e-3) / 1e9
     fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
     hbm = peaks["hbm_gbs"]
-    traffic = gemm_traffic_from_profile(wl.name)
+    # the committed counters are of the default configuration's GEMM launch
+    default_cfg = (args.recipe == "delayed" and not args.transposes and not args.separate_norm_pass)
+    traffic = gemm_traffic_from_profile(wl.name) if default_cfg else None
 
     for g, _ in graphs:
         del g
@@ -301,11 +309,13 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic",
         "config": {"workload": wl.name, "tokens": wl.tokens,
                    "layers_in_out": shapes,
-                   "recipe": f"HYBRID, {args.recipe} per-tensor scaling",
+                   "recipe": "MXFP8 (E4M3, E8M0 scale per 32 values)" if args.recipe == "mxfp8"
+                             else f"HYBRID, {args.recipe} per-tensor scaling",
                    "history_len": wl.history_len, "amax_algo": wl.algo, "margin": wl.margin,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "launch": "eager" if args.eager else "CUDA graph per step (AdamW step counter on the device)",
-                   "scale_update": "none (current scaling)" if args.recipe == "current"
+                   "scale_update": "none (MX block scales)" if args.recipe == "mxfp8"
+                                   else "none (current scaling)" if args.recipe == "current"
                                    else "separate launch" if args.separate_scale_update
                                    else "in the last CTA of the cast launch",
                    "grad_sum_of_squares": "AdamW norm pass" if args.separate_norm_pass
@@ -611,8 +621,9 @@ def main(argv=None):
                          "adamw4e9_512t, stress1024_t2048")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager launches, not CUDA graphs")
-    ap.add_argument("--recipe", choices=("delayed", "current"), default="delayed",
-                    help="current: each scale from its own tensor's amax (an extra read)")
+    ap.add_argument("--recipe", choices=("delayed", "current", "mxfp8"), default="delayed",
+                    help="current: each scale from its own tensor's amax (an extra read); "
+                         "mxfp8: E4M3 with one E8M0 scale per 32 values, block-scaled GEMMs")
     ap.add_argument("--transposes", action="store_true",
                     help="casts also write q^T and every GEMM reads K-major operands")
     ap.add_argument("--separate-weight-cast", action="store_true",

@@ -28,6 +28,7 @@ from . import (AMAX_MAX, AMAX_MOST_RECENT, CURRENT_WORKSPACE_BYTES, E4M3, E5M2, 
                fp8_cast_transpose_amax, fp8_cast_transpose_amax_current_multi,
                fp8_cast_transpose_amax_multi, fp8_cast_transpose_amax_update_multi,
                fp8_gemm_multi, fp8_gemm_multi_sumsq, fp8_gemm_sumsq_workspace_bytes,
+               fp8_mx_cast_multi, fp8_mx_gemm_multi, mx_scale_bytes,
                fp8_scale_update, fused_adamw_multi_tensor, fused_adamw_multi_tensor_presummed,
                fused_adamw_workspace_bytes)
 
@@ -97,12 +98,23 @@ class Fp8LinearStep:
         self.gemm_workspace = torch.zeros(gws, dtype=torch.uint8, device=self.device)
         self.adamw_ticket = torch.zeros(1, dtype=torch.int32, device=self.device)
         # current scaling: every scale from the tensor's own amax (no history, no delayed update)
-        assert recipe in ("delayed", "current")
+        # mxfp8: E4M3 codes with a scale per 32 values, both orientations, block-scaled GEMMs
+        assert recipe in ("delayed", "current", "mxfp8")
         self.recipe = recipe
         self.current_ws = torch.zeros(CURRENT_WORKSPACE_BYTES, dtype=torch.uint8, device=self.device)
-        if recipe == "current":
+        if recipe != "delayed":
             fused_update = fused_wcast = False
             self.fused_update = False
+        if recipe == "mxfp8":
+            self.fused_norm = fused_norm = False
+            u8 = dict(dtype=torch.uint8, device=self.device)
+            for L in self.layers:
+                shapes = dict(X=(tokens, L.fin), W=(L.fin, L.fout), dY=(tokens, L.fout))
+                L.mx = {}
+                for name, (r, c) in shapes.items():
+                    L.mx[name] = dict(q_row=torch.empty(r, c, **u8), q_col=torch.empty(r, c, **u8),
+                                      sf_row=torch.empty(mx_scale_bytes(r, c), **u8),
+                                      sf_col=torch.empty(mx_scale_bytes(c, r), **u8))
         # the W cast inside AdamW needs the in-launch scale update and the presummed AdamW, and
         # writes row-major codes only; the saturation / zero counters of W are only kept by the
         # separate cast
@@ -151,6 +163,31 @@ class Fp8LinearStep:
                                                  stream=stream)
         else:
             fp8_cast_transpose_amax_multi(descs, stream=stream)
+
+    def mx_cast_all(self, xs, dys, stream=None):
+        """MXFP8: X, W and dY quantised with E4M3 codes and one E8M0 scale per 32 values, in
+        both orientations (row-wise for K-major use, column-wise for MN-major use)."""
+        casts = []
+        for k, L in enumerate(self.layers):
+            for name, src in (("X", xs[k]), ("W", L.W), ("dY", dys[k])):
+                casts.append(dict(x=src, fmt=E4M3, **L.mx[name]))
+        fp8_mx_cast_multi(casts, stream=stream)
+
+    def mx_gemm_descs(self):
+        out = []
+        for L in self.layers:
+            X, W, dY = L.mx["X"], L.mx["W"], L.mx["dY"]
+            out += [dict(A=X["q_row"], a_sf=X["sf_row"], a_fmt=E4M3, B=W["q_col"], b_sf=W["sf_col"],
+                         b_mn=True, b_fmt=E4M3, D=L.Y),
+                    dict(A=dY["q_row"], a_sf=dY["sf_row"], a_fmt=E4M3, B=W["q_row"], b_sf=W["sf_row"],
+                         b_fmt=E4M3, D=L.dX),
+                    dict(A=X["q_col"], a_sf=X["sf_col"], a_mn=True, a_fmt=E4M3, B=dY["q_col"],
+                         b_sf=dY["sf_col"], b_mn=True, b_fmt=E4M3, D=L.dW)]
+        return out
+
+    def mx_gemm_all(self, stream=None):
+        """The block-scaled fprop, dgrad and wgrad of every layer in one grouped launch."""
+        fp8_mx_gemm_multi(self.mx_gemm_descs(), stream=stream)
 
     def cast_all_current(self, xs, dys, stream=None):
         """Current scaling: the X, W and dY scales from their own amax, then the casts."""
@@ -244,6 +281,11 @@ class Fp8LinearStep:
     def step(self, xs, dys, stream=None):
         """One training step; xs[k] = X [tokens, in_k], dys[k] = dY [tokens, out_k] (BF16, device)."""
         self.t += 1
+        if self.recipe == "mxfp8":
+            self.mx_cast_all(xs, dys, stream)
+            self.mx_gemm_all(stream)
+            self.adamw(stream)
+            return
         if self.recipe == "current":
             self.amax.zero_()                  # amax slots report this step's tensors only
             self.cast_all_current(xs, dys, stream)
@@ -287,6 +329,8 @@ class Fp8LinearStep:
         n_adamw_batches = (len(self.layers) + 255) // 256
         n_cast_launches = (3 * len(self.layers) + 7) // 8
         n_gemm_launches = (3 * len(self.layers) + 23) // 24
+        if self.recipe == "mxfp8":
+            return (3 * len(self.layers) + 7) // 8 + (3 * len(self.layers) + 23) // 24 + 2 * n_adamw_batches
         n_scale_launches = 0 if self.fused_update or self.recipe == "current" else 1
         if self.recipe == "current":
             n_cast_launches *= 2                   # an amax launch before each cast launch

@@ -318,3 +318,38 @@ def test_current_scaling_steps(cuda_lib):
         R, ab = oracle.gemm(u8(L.Xq), 0, tr(u8(L.Wq)), 0, f32(st.sinv_used)[0], f32(st.sinv_used)[1],
                             want_abs=True)
         assert gemm_within_tolerance(bf16_bits(L.Y), R, ab).all()
+
+
+def test_mxfp8_steps(cuda_lib):
+    """Two steps of the 256 x 256 / 512-token Linear with the MXFP8 recipe: X, W, dY quantised
+    with E4M3 codes and E8M0 block scales in both orientations (oracle mx_quantise, bit for bit),
+    the three block-scaled GEMMs in one launch (oracle mx_gemm on every output) and AdamW."""
+    from tests.test_gpu_mx import from_atoms
+    wl = synth.LINEAR256
+    st = Fp8LinearStep([(256, 256)], wl.tokens, wl.history_len, wl.algo, 0, wl.adamw,
+                       [synth.linear_weight(wl, 0, "cuda")], "cuda", recipe="mxfp8")
+    assert st.kernels_per_step() == 4 and not st.fused_norm
+    E = oracle.E4M3
+    T = wl.tokens
+    for t in range(2):
+        X, dY = synth.linear_inputs(wl, 0, t, "cuda")
+        L = st.layers[0]
+        W0 = bf16_bits(L.W)
+        st.step([X], [dY])
+        cuda_lib.fp8t_check_device_error()
+        host = {}
+        for name, bits in (("X", bf16_bits(X)), ("W", W0), ("dY", bf16_bits(dY))):
+            b = L.mx[name]
+            r, c = bits.shape
+            rq, rs = oracle.mx_quantise(bits, 0, E)
+            cq, cs = oracle.mx_quantise(bits, 1, E)
+            assert np.array_equal(u8(b["q_row"]), rq) and np.array_equal(from_atoms(b["sf_row"], r, c), rs)
+            assert np.array_equal(u8(b["q_col"]), cq) and np.array_equal(from_atoms(b["sf_col"], c, r), cs.T)
+            host[name] = (rq, rs, cq, cs)
+        xr, xs_, xc, xcs = host["X"]
+        wr, ws_, wc, wcs = host["W"]
+        dr, ds_, dc, dcs = host["dY"]
+        for D, A, sa, B, sb in ((L.Y, xr, xs_, tr(wc), tr(wcs)), (L.dX, dr, ds_, wr, ws_),
+                                (L.dW, tr(xc), tr(xcs), tr(dc), tr(dcs))):
+            R, ab = oracle.mx_gemm(A, sa, E, B, sb, E, want_abs=True)
+            assert gemm_within_tolerance(bf16_bits(D), R, ab).all()
