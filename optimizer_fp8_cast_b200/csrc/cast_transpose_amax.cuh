@@ -314,11 +314,11 @@ __global__ void __launch_bounds__(kThreads, 2) k_cast_transpose_amax(const __gri
 }
 
 // Row-major-only casts (no tensor of the launch wants q^T): a plain streaming kernel. Each
-// thread converts 16-element segments (two 16-byte loads, one 16-byte store), two segments in
-// flight, grid-striding over one tensor after another; amax and counters are reduced per warp
-// (one atomic per warp and tensor).
+// thread converts 16-element segments (two 16-byte loads, one 16-byte store), four segments
+// (128 bytes) in flight, grid-striding over one tensor after another; amax and counters are
+// reduced per warp (one atomic per warp and tensor).
 template <bool COUNT>
-__global__ void __launch_bounds__(kThreads, 4) k_cast_rowmajor(const __grid_constant__ Group g) {
+__global__ void __launch_bounds__(kThreads, 3) k_cast_rowmajor(const __grid_constant__ Group g) {
   const int tid = threadIdx.x, lane = tid & 31;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
   for (int t = 0; t < g.n; ++t) {
@@ -330,18 +330,18 @@ __global__ void __launch_bounds__(kThreads, 4) k_cast_rowmajor(const __grid_cons
     const float s = __ldg(T.scale);
     uint32_t vmax = 0, nsat = 0, nzero = 0, nnonfinite = 0;
     int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + tid;
-    for (; i + stride < nseg; i += 2 * stride) {
-      uint4 in0[2], in1[2];
-      in0[0] = ld_stream_u4(x + 2 * i);
-      in0[1] = ld_stream_u4(x + 2 * i + 1);
-      in1[0] = ld_stream_u4(x + 2 * (i + stride));
-      in1[1] = ld_stream_u4(x + 2 * (i + stride) + 1);
-      uint32_t p0[4] = {0u, 0u, 0u, 0u}, p1[4] = {0u, 0u, 0u, 0u};
-      vmax = max(vmax, quantise_segment<COUNT>(T, in0, s, p0, nsat, nzero, nnonfinite));
-      vmax = max(vmax, quantise_segment<COUNT>(T, in1, s, p1, nsat, nzero, nnonfinite));
-      if (q) {
-        q[i] = make_uint4(p0[0], p0[1], p0[2], p0[3]);
-        q[i + stride] = make_uint4(p1[0], p1[1], p1[2], p1[3]);
+    for (; i + 3 * stride < nseg; i += 4 * stride) {
+      uint4 in[4][2];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        in[u][0] = ld_stream_u4(x + 2 * (i + u * stride));
+        in[u][1] = ld_stream_u4(x + 2 * (i + u * stride) + 1);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        uint32_t p[4] = {0u, 0u, 0u, 0u};
+        vmax = max(vmax, quantise_segment<COUNT>(T, in[u], s, p, nsat, nzero, nnonfinite));
+        if (q) q[i + u * stride] = make_uint4(p[0], p[1], p[2], p[3]);
       }
     }
     for (; i < nseg; i += stride) {

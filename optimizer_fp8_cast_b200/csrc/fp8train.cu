@@ -9,8 +9,11 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 #include <string>
+#include <utility>
+#include <vector>
 
 #include "fp8train.h"
 #include "cast_transpose_amax.cuh"
@@ -454,6 +457,42 @@ namespace {
 
 constexpr size_t kSumsqHeader = 256;    // ticket, then the partial slots
 
+// Tile lists of a grouped GEMM launch: every tile costs its problem's K / 128 k-blocks; tiles are
+// handed out longest first, each to the least-loaded cluster, and every cluster then runs its
+// tiles in index order. Launches with more tiles than the table holds keep round-robin (with
+// thousands of tiles it is balanced already).
+void build_schedule(fp8t::gemm::Group& g, int clusters) {
+  using namespace fp8t::gemm;
+  g.scheduled = 0;
+  if (g.total_tiles > kMaxSchedTiles || clusters > kMaxClusters || clusters < 2) return;
+  std::vector<std::pair<int, int>> tiles;                  // (-cost, tile)
+  tiles.reserve(g.total_tiles);
+  for (int p = 0; p < g.n; ++p) {
+    const int end = p + 1 < g.n ? g.p[p + 1].tile_start : g.total_tiles;
+    const int cost = (g.p[p].K + kBK - 1) / kBK;
+    for (int t = g.p[p].tile_start; t < end; ++t) tiles.emplace_back(-cost, t);
+  }
+  std::stable_sort(tiles.begin(), tiles.end(),
+                   [](const std::pair<int, int>& a, const std::pair<int, int>& b) { return a.first < b.first; });
+  std::vector<int64_t> load(clusters, 0);
+  std::vector<std::vector<int>> own(clusters);
+  for (const auto& t : tiles) {
+    int best = 0;
+    for (int c = 1; c < clusters; ++c)
+      if (load[c] < load[best]) best = c;
+    load[best] -= t.first;
+    own[best].push_back(t.second);
+  }
+  int k = 0;
+  for (int c = 0; c < clusters; ++c) {
+    std::sort(own[c].begin(), own[c].end());
+    g.start[c] = static_cast<uint16_t>(k);
+    for (int t : own[c]) g.order[k++] = static_cast<uint16_t>(t);
+  }
+  g.start[clusters] = static_cast<uint16_t>(k);
+  g.scheduled = 1;
+}
+
 int64_t gemm_tiles(const fp8t_gemm_desc& d) {
   using namespace fp8t::gemm;
   return ((d.M + kBM - 1) / kBM) * ((d.N + kBN - 1) / kBN);
@@ -561,6 +600,7 @@ fp8t_status gemm_multi(const fp8t_gemm_desc* gemms, int32_t n_gemms, const int32
     }
     group.total_tiles = static_cast<int32_t>(tiles);
     const int64_t grid = 2 * std::min<int64_t>(tiles, dev->gemm_clusters);   // persistent pairs
+    build_schedule(group, static_cast<int>(grid / 2));
     k_fp8_gemm<false><<<static_cast<unsigned>(grid), kThreads, kSmemBytes, as_stream(stream)>>>(group);
     if ((st = after_launch("fp8_gemm launch")) != FP8T_OK) return st;
   }
@@ -727,6 +767,7 @@ fp8t_status fp8_mx_gemm_multi(const fp8t_mx_gemm_desc* gemms, int32_t n_gemms, v
     }
     group.total_tiles = static_cast<int32_t>(tiles);
     const int64_t grid = 2 * std::min<int64_t>(tiles, dev->gemm_mx_clusters);
+    build_schedule(group, static_cast<int>(grid / 2));
     k_fp8_gemm<true><<<static_cast<unsigned>(grid), kThreads, kSmemBytesMX, as_stream(stream)>>>(group);
     if ((st = after_launch("fp8_mx_gemm launch")) != FP8T_OK) return st;
   }

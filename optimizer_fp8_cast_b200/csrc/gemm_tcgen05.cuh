@@ -19,8 +19,11 @@
 // (M=256, N=256, K=32), which reads A and B halves from both CTAs' shared memory, and releases
 // each stage in both CTAs with one multicast tcgen05.commit. Per SM that is 32 KB of operands per
 // 512 tensor-core cycles, two thirds of what a single-SM 128 x 256 tile needs.
-// Persistent: cluster c walks the tiles c, c + clusters, ...; two TMEM accumulators (2 x 256
-// columns) let the epilogue of one tile overlap the main loop of the next.
+// Persistent: cluster c walks the tiles c, c + clusters, ... or, for launches of up to
+// kMaxSchedTiles tiles, the list the host built for it: tiles cost K / 128 k-blocks each, and a
+// longest-first greedy assignment balances the clusters (a grouped step mixes K = T wgrad tiles
+// with K = features fprop/dgrad tiles, which round-robin leaves several percent apart). Two TMEM
+// accumulators (2 x 256 columns) let the epilogue of one tile overlap the main loop of the next.
 // Warp roles (192 threads per CTA):
 //   warp 0, lane 0  TMA producer (both CTAs)
 //   warp 1, lane 0  MMA issuer (even CTA only); warp 1 also owns the TMEM allocation
@@ -150,9 +153,13 @@ struct alignas(64) Problem {
   int32_t kb128;                 // MX: K / 128, atoms per 128 rows
   int32_t a_fmt, b_fmt;          // MX: element formats (the descriptor is formed per K-block)
 };
+constexpr int kMaxSchedTiles = 4096, kMaxClusters = 128;
 struct alignas(64) Group {
   Problem p[kMaxProblems];
   int32_t n, total_tiles;
+  int32_t scheduled;             // 1: cluster c runs order[start[c] .. start[c+1])
+  uint16_t start[kMaxClusters + 1];
+  uint16_t order[kMaxSchedTiles];
   // sum of squares (sumsq_out null: off)
   double* partials;              // every launch's slots (8 per summed tile)
   double* sumsq_out;
@@ -161,6 +168,15 @@ struct alignas(64) Group {
   int32_t last_launch;           // this launch reduces the slots
 };
 constexpr int kSumsqPerTile = 8; // 2 CTAs x 4 epilogue warps
+
+// Number of tiles cluster c runs, and its i-th tile.
+__device__ __forceinline__ int tiles_of(const Group& g, int c, int n_clusters) {
+  return g.scheduled ? g.start[c + 1] - g.start[c]
+                     : (g.total_tiles > c ? (g.total_tiles - c + n_clusters - 1) / n_clusters : 0);
+}
+__device__ __forceinline__ int tile_at(const Group& g, int c, int n_clusters, int i) {
+  return g.scheduled ? g.order[g.start[c] + i] : c + i * n_clusters;
+}
 
 __device__ __forceinline__ int find_problem(const Group& g, int tile) {
   int p = 0;
@@ -196,7 +212,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
   const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
-  const int n_tiles = g.total_tiles;
+  const int my_tiles = tiles_of(g, cluster, n_clusters);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -233,7 +249,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       // ---------------- TMA producer (both CTAs)
       uint32_t it = 0, issued = 0;
-      for (int tile = cluster; tile < n_tiles && !*abort_flag; tile += n_clusters) {
+      for (int i = 0; i < my_tiles && !*abort_flag; ++i) {
+        const int tile = tile_at(g, cluster, n_clusters, i);
         const Problem& P = g.p[find_problem(g, tile)];
         const int local = tile - P.tile_start;
         const int m0 = (local / P.tiles_n) * kBM + static_cast<int>(rank) * kHalf;
@@ -282,7 +299,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (lane == 0 && leader) {
       // ---------------- MMA issuer (even CTA)
       uint32_t it = 0, local = 0;
-      for (int tile = cluster; tile < n_tiles && !*abort_flag; tile += n_clusters, ++local) {
+      for (int i = 0; i < my_tiles && !*abort_flag; ++i, ++local) {
+        const int tile = tile_at(g, cluster, n_clusters, i);
         const Problem& P = g.p[find_problem(g, tile)];
         const int num_kb = (P.K + kBK - 1) / kBK;
         const uint32_t idesc = P.idesc;
@@ -347,7 +365,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int quad = warp & 3;                       // TMEM lanes 32*quad .. 32*quad+31
     uint8_t* my_buf = sEpi + (warp - 2) * 2 * kEpiChunkBytes;
     uint32_t local = 0, chunk_count = 0;
-    for (int tile = cluster; tile < n_tiles; tile += n_clusters, ++local) {
+    for (int i = 0; i < my_tiles; ++i, ++local) {
+      const int tile = tile_at(g, cluster, n_clusters, i);
       const uint32_t acc = MX ? 0u : (local & 1), aph = MX ? (local & 1) : ((local >> 1) & 1);
       if (*abort_flag) break;
       if (!mbar_wait(smem_u32(&S->acc_full[acc]), aph, limit, expire_epi)) {
@@ -364,12 +383,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const uint32_t t_base = tmem + (static_cast<uint32_t>(quad * 32) << 16) + acc * kAccCols;
       const bool sumsq = P.sumsq_slot >= 0;
       double ss = 0.0;
-#pragma unroll 1
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(t_base + c * 32, r);
-        tmem_ld_wait();
-        if (n0 + c * 32 >= N || row0 >= M) continue;  // chunk entirely outside the matrix
+      // one 32 x 32 chunk of packed BF16 (16 words per lane) into the swizzled staging buffer
+      // and out with a TMA store; the sum of squares of the stored values when asked
+      auto store_chunk = [&](int c, const uint32_t (&w16)[16]) {
         uint8_t* buf = my_buf + (chunk_count & 1) * kEpiChunkBytes;
         ++chunk_count;
         if (lane == 0) bulk_wait_group_read<1>();    // the store that last used buf has read it
@@ -378,23 +394,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // (piece p of row i lives at piece p ^ ((i >> 1) & 3)), matching the store's map
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
-          uint32_t w[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int j = 4 * p + q;
-            w[q] = pack_bf16x2(__fmul_rn(__uint_as_float(r[2 * j]), alpha),
-                               __fmul_rn(__uint_as_float(r[2 * j + 1]), alpha));
-          }
           if (sumsq) {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              const double lo = __uint_as_float(w[q] << 16), hi = __uint_as_float(w[q] & 0xFFFF0000u);
+              const uint32_t w = w16[4 * p + q];
+              const double lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xFFFF0000u);
               ss = __fma_rn(lo, lo, ss);                // squares of BF16 values are exact
               ss = __fma_rn(hi, hi, ss);
             }
           }
           const int pp = p ^ ((lane >> 1) & 3);
-          *reinterpret_cast<uint4*>(buf + lane * 64 + pp * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(buf + lane * 64 + pp * 16) =
+              make_uint4(w16[4 * p], w16[4 * p + 1], w16[4 * p + 2], w16[4 * p + 3]);
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -402,10 +413,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tma_store_2d(&P.d, smem_u32(buf), n0 + c * 32, row0);
           bulk_commit_group();
         }
+      };
+      if (MX) {
+        // single accumulator: read all of it into registers (packed BF16, 128 words per lane),
+        // release it so that the next tile's MMAs start, then store
+        uint32_t packed[kBN / 32][16];
+#pragma unroll
+        for (int c = 0; c < kBN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(t_base + c * 32, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            packed[c][j] = pack_bf16x2(__fmul_rn(__uint_as_float(r[2 * j]), alpha),
+                                       __fmul_rn(__uint_as_float(r[2 * j + 1]), alpha));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&S->acc_empty[acc]), 0));
+#pragma unroll
+        for (int c = 0; c < kBN / 32; ++c)
+          if (n0 + c * 32 < N && row0 < M) store_chunk(c, packed[c]);
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < kBN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(t_base + c * 32, r);
+          tmem_ld_wait();
+          if (n0 + c * 32 >= N || row0 >= M) continue;  // chunk entirely outside the matrix
+          uint32_t w16[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            w16[j] = pack_bf16x2(__fmul_rn(__uint_as_float(r[2 * j]), alpha),
+                                 __fmul_rn(__uint_as_float(r[2 * j + 1]), alpha));
+          store_chunk(c, w16);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&S->acc_empty[acc]), 0));
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&S->acc_empty[acc]), 0));
       if (sumsq) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, o));

@@ -13,8 +13,10 @@
 // rows (M or N) x 4 blocks (128 K values): byte (i % 32) * 16 + (i / 32) * 4 + kb holds row i,
 // block kb, which is the order the tensor-core scale copy (tcgen05.cp 32x128b, replicated to
 // the four lane quarters) expects; atoms are stored [MN / 128][K / 128].
-// A CTA reads its tile into shared memory with 16-byte loads (16-byte chunk c of row r stored at
-// c ^ (r % 8), so that both the row-wise and the column-wise reads are free of bank conflicts),
+// A CTA reads its tiles into a double-buffered shared tile with 16-byte asynchronous copies (the
+// next tile's copies are in flight while the current one is quantised; 16-byte chunk c of row r
+// is stored at c ^ (r % 8), so that the row-wise and the column-wise reads are free of bank
+// conflicts),
 // quantises the row-wise blocks
 // straight to global memory, the column-wise blocks into a staged tile that it then writes out
 // row by row, and writes each atom with 16-byte stores.
@@ -28,7 +30,7 @@ namespace mx {
 constexpr int kTile = 128;
 constexpr int kThreads = 256;
 constexpr int kMaxTensors = 8;
-constexpr int kSmemBytes = kTile * kTile * 2 + kTile * kTile + 2 * 512 + 128;
+constexpr int kSmemBytes = 2 * kTile * kTile * 2 + kTile * kTile + 2 * 512 + 128;
 
 struct Tensor {
   const uint4* x;                  // BF16 [rows][cols]
@@ -78,29 +80,50 @@ __device__ __forceinline__ int xchunk(int row, int c16) { return row * 16 + (c16
 // position of BF16 element (row, col) of the tile (uint16 units)
 __device__ __forceinline__ int xelem(int row, int col) { return xchunk(row, col >> 3) * 8 + (col & 7); }
 
+__device__ __forceinline__ int tensor_of(const Group& g, int64_t tile) {
+  int ti = 0;
+  while (ti + 1 < g.n && g.t[ti + 1].tile_start <= tile) ++ti;
+  return ti;
+}
+
+// Issue the 16-byte copies of one 128 x 128 BF16 tile (128 rows x 256 bytes) into xs.
+__device__ __forceinline__ void prefetch_tile(const Group& g, int64_t tile, uint16_t* xs) {
+  const Tensor& T = g.t[tensor_of(g, tile)];
+  const int64_t local = tile - T.tile_start;
+  const int64_t r0 = (local / T.tiles_c) * kTile, c0 = (local % T.tiles_c) * kTile;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int v = u * kThreads + threadIdx.x, row = v >> 4, c16 = v & 15;
+    cp_async_16(smem_u32(reinterpret_cast<uint4*>(xs) + xchunk(row, c16)),
+                T.x + ((r0 + row) * T.cols + c0) / 8 + c16);
+  }
+}
+
 __global__ void __launch_bounds__(kThreads) k_mx_cast(const __grid_constant__ Group g) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);
-  uint16_t* xs = reinterpret_cast<uint16_t*>(smem);                 // [128][128] BF16
-  uint8_t* qs = smem + kTile * kTile * 2;                           // [128][128] column-wise codes
+  // [2][128][128] BF16 tiles at smem and smem + kXBytes
+  constexpr int kXBytes = kTile * kTile * 2;
+  auto xbuf = [&](int b) { return reinterpret_cast<uint16_t*>(smem + b * kXBytes); };
+  uint8_t* qs = smem + 2 * kTile * kTile * 2;                       // [128][128] column-wise codes
   uint8_t* atom_r = qs + kTile * kTile;                             // 512 B
   uint8_t* atom_c = atom_r + 512;                                   // 512 B
   const int tid = threadIdx.x;
 
-  for (int64_t tile = blockIdx.x; tile < g.total_tiles; tile += gridDim.x) {
-    int ti = 0;
-    while (ti + 1 < g.n && g.t[ti + 1].tile_start <= tile) ++ti;
-    const Tensor& T = g.t[ti];
+  if (static_cast<int64_t>(blockIdx.x) < g.total_tiles) prefetch_tile(g, blockIdx.x, xbuf(0));
+  cp_async_commit();
+  int k = 0;
+  for (int64_t tile = blockIdx.x; tile < g.total_tiles; tile += gridDim.x, ++k) {
+    const Tensor& T = g.t[tensor_of(g, tile)];
     const int64_t local = tile - T.tile_start;
     const int64_t r0 = (local / T.tiles_c) * kTile, c0 = (local % T.tiles_c) * kTile;
     const int emax = T.fmt == 0 ? 8 : 15;
+    uint16_t* xs = xbuf(k & 1);
 
-    // ---- load the tile: 128 rows x 256 bytes, 16 bytes per load
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int v = u * kThreads + tid, row = v >> 4, c16 = v & 15;
-      reinterpret_cast<uint4*>(xs)[xchunk(row, c16)] = ld_stream_u4(T.x + ((r0 + row) * T.cols + c0) / 8 + c16);
-    }
+    // ---- the next tile's copies go out; this tile's have landed
+    if (tile + gridDim.x < g.total_tiles) prefetch_tile(g, tile + gridDim.x, xbuf((k + 1) & 1));
+    cp_async_commit();
+    cp_async_wait<1>();
     __syncthreads();
 
     // ---- row-wise blocks: 128 rows x 4 blocks, two per thread

@@ -280,6 +280,14 @@ __device__ __forceinline__ uint32_t cvt_fp8x2(float lo, float hi) {
 }
 
 // Streaming 16-byte load (read once; do not keep in L1).
+// 16-byte asynchronous copy global -> shared (bypassing L1), grouped by commit/wait.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 __device__ __forceinline__ uint4 ld_stream_u4(const void* p) {
   return __ldcs(reinterpret_cast<const uint4*>(p));
 }
