@@ -155,30 +155,33 @@ __global__ void __launch_bounds__(kThreads) k_mx_cast(const __grid_constant__ Gr
         atom_r[(row & 31) * 16 + (row >> 5) * 4 + b] = m > 0x7F80u ? 0xFF : static_cast<uint8_t>(X + 127);
       }
     }
-    // ---- column-wise blocks: 128 columns x 4 blocks of 32 rows, two per thread
+    // ---- column-wise blocks: 128 columns x 4 blocks of 32 rows; each thread takes a column
+    //      pair of one block: 32 four-byte reads (two BF16 each) and 32 two-byte code stores
     if (T.q_col) {
-#pragma unroll 1
-      for (int u = 0; u < 2; ++u) {
-        const int j = u * kThreads + tid, col = j & 127, rb = j >> 7;
-        uint32_t m = 0;
-#pragma unroll 8
-        for (int i = 0; i < 32; ++i) m = max(m, static_cast<uint32_t>(xs[xelem(32 * rb + i, col)] & 0x7FFFu));
-        const int X = m > 0x7F80u ? 0 : block_exponent(m, emax);
-        const float inv = pow2_neg(X);
-#pragma unroll 8
-        for (int i = 0; i < 32; i += 2) {
-          const uint32_t pair = static_cast<uint32_t>(xs[xelem(32 * rb + i, col)]) |
-                                (static_cast<uint32_t>(xs[xelem(32 * rb + i + 1, col)]) << 16);
-          const float p0 = __fmul_rn(__uint_as_float(pair << 16), inv);
-          const float p1 = __fmul_rn(__uint_as_float(pair & 0xFFFF0000u), inv);
-          uint32_t c = T.fmt == 0 ? cvt_fp8x2<0>(p0, p1) : cvt_fp8x2<1>(p0, p1);
-          if (p0 != p0) c = (c & 0xFF00u) | 0x7Fu;
-          if (p1 != p1) c = (c & 0x00FFu) | 0x7F00u;
-          qs[(32 * rb + i) * kTile + col] = static_cast<uint8_t>(c);
-          qs[(32 * rb + i + 1) * kTile + col] = static_cast<uint8_t>(c >> 8);
-        }
-        atom_c[(col & 31) * 16 + (col >> 5) * 4 + rb] = m > 0x7F80u ? 0xFF : static_cast<uint8_t>(X + 127);
+      const int cp = tid & 63, rb = tid >> 6, col = 2 * cp;
+      uint32_t v[32];
+      uint32_t m2 = 0;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        v[i] = *reinterpret_cast<const uint32_t*>(xs + xelem(32 * rb + i, col));
+        m2 = __vmaxu2(m2, v[i] & 0x7FFF7FFFu);
       }
+      const uint32_t m0 = m2 & 0xFFFFu, m1 = m2 >> 16;   // column col, column col + 1
+      const int X0 = m0 > 0x7F80u ? 0 : block_exponent(m0, emax);
+      const int X1 = m1 > 0x7F80u ? 0 : block_exponent(m1, emax);
+      const float inv0 = pow2_neg(X0), inv1 = pow2_neg(X1);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float p0 = __fmul_rn(__uint_as_float(v[i] << 16), inv0);
+        const float p1 = __fmul_rn(__uint_as_float(v[i] & 0xFFFF0000u), inv1);
+        uint32_t c = T.fmt == 0 ? cvt_fp8x2<0>(p0, p1) : cvt_fp8x2<1>(p0, p1);
+        if (p0 != p0) c = (c & 0xFF00u) | 0x7Fu;
+        if (p1 != p1) c = (c & 0x00FFu) | 0x7F00u;
+        *reinterpret_cast<uint16_t*>(qs + (32 * rb + i) * kTile + col) = static_cast<uint16_t>(c);
+      }
+      atom_c[(col & 31) * 16 + (col >> 5) * 4 + rb] = m0 > 0x7F80u ? 0xFF : static_cast<uint8_t>(X0 + 127);
+      atom_c[((col + 1) & 31) * 16 + ((col + 1) >> 5) * 4 + rb] =
+          m1 > 0x7F80u ? 0xFF : static_cast<uint8_t>(X1 + 127);
     }
     __syncthreads();                                   // staged codes and both atoms complete
     if (T.q_col) {
