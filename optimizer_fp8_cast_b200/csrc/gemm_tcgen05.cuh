@@ -47,8 +47,12 @@
 // replicated into the four lane quarters: A scales in 4 columns, B scales in 8) right before
 // the stage's four MMAs, which pick the byte of their K-block through the descriptor's
 // scale-factor ids. The copies and MMAs run in issue order, so one set of scale columns serves
-// every stage. The scale columns take the place of the second accumulator: the MX kernel keeps
-// a single 256-column accumulator.
+// every stage. Two full accumulators and the 12 scale columns do not fit the 512 TMEM columns,
+// so the MX kernel overlaps its accumulators by one 32-column chunk: accumulator 0 at columns
+// 0..255, accumulator 1 at 224..479, scales at 480..491. The epilogue reads the shared chunk
+// first (accumulator 0 backwards from its last chunk, accumulator 1 forwards) and releases it
+// through its own barrier, so the next tile's MMAs, which overwrite that chunk, can start while
+// the rest of the accumulator is being stored.
 // Every mbarrier wait is bounded (globaltimer). On expiry a CTA records kErrTimeout and stops
 // issuing; issued MMAs are awaited with a fixed bound, loads in flight are given time to land,
 // and both CTAs meet at a cluster barrier before TMEM is freed; D is then incomplete.
@@ -73,7 +77,8 @@ constexpr int kSmemBytes =
 constexpr int kSfaBytes = 512, kSfbBytes = 1024;         // MX scale atoms per stage and CTA
 constexpr int kSfStageBytes = kSfaBytes + kSfbBytes;
 constexpr int kSmemBytesMX = kSmemBytes + kStages * kSfStageBytes;
-constexpr uint32_t kSfaCol = kAccCols, kSfbCol = kAccCols + 4;   // MX: scale columns in TMEM
+constexpr uint32_t kMxAcc1Col = kAccCols - 32;           // MX: second accumulator, overlapping
+constexpr uint32_t kSfaCol = kMxAcc1Col + kAccCols, kSfbCol = kSfaCol + 4;   // MX: scale columns
 constexpr uint64_t kSettleNs = 200000;                   // let loads in flight land on abort
 constexpr uint64_t kPairDrainNs = 1000000;               // producer drain budget (1 ms)
 
@@ -189,6 +194,7 @@ struct Smem {
   uint64_t empty[kStages];    // both CTAs: the pair MMA has consumed a stage
   uint64_t acc_full[2];       // both CTAs: an accumulator holds a finished tile
   uint64_t acc_empty[2];      // even CTA: both epilogues have drained an accumulator
+  uint64_t acc_shared_free;   // even CTA (MX): both epilogues have read the overlapping chunk
   uint64_t mma_done;          // even CTA: every issued MMA has completed
   uint32_t tmem_base;
   int abort;
@@ -223,6 +229,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&S->acc_full[a]), 1);
       mbar_init(smem_u32(&S->acc_empty[a]), 8);      // 4 epilogue warps x 2 CTAs
     }
+    mbar_init(smem_u32(&S->acc_shared_free), 8);
     mbar_init(smem_u32(&S->mma_done), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -305,14 +312,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int num_kb = (P.K + kBK - 1) / kBK;
         const uint32_t idesc = P.idesc;
         const bool a_mn = P.a_mn != 0, b_mn = P.b_mn != 0;
-        const uint32_t acc = MX ? 0u : (local & 1), aph = MX ? (local & 1) : ((local >> 1) & 1);
+        const uint32_t acc = local & 1, aph = (local >> 1) & 1;
         if (!mbar_wait(smem_u32(&S->acc_empty[acc]), aph ^ 1, limit, expire_main)) {
           *abort_flag = 1;
           record_error(kErrTimeout);
           break;
         }
+        // MX: the previous tile (other accumulator) must have handed back the shared chunk
+        if (MX && local > 0 &&
+            !mbar_wait(smem_u32(&S->acc_shared_free), (local - 1) & 1, limit, expire_main)) {
+          *abort_flag = 1;
+          record_error(kErrTimeout);
+          break;
+        }
         tc_fence_after();
-        const uint32_t d_tmem = tmem + acc * kAccCols;
+        const uint32_t d_tmem = tmem + acc * (MX ? kMxAcc1Col : kAccCols);
         bool ok = true;
         for (int kb = 0; kb < num_kb; ++kb, ++it) {
           const uint32_t s = it % kStages, ph = (it / kStages) & 1;
@@ -367,7 +381,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint32_t local = 0, chunk_count = 0;
     for (int i = 0; i < my_tiles; ++i, ++local) {
       const int tile = tile_at(g, cluster, n_clusters, i);
-      const uint32_t acc = MX ? 0u : (local & 1), aph = MX ? (local & 1) : ((local >> 1) & 1);
+      const uint32_t acc = local & 1, aph = (local >> 1) & 1;
       if (*abort_flag) break;
       if (!mbar_wait(smem_u32(&S->acc_full[acc]), aph, limit, expire_epi)) {
         *abort_flag = 1;
@@ -380,7 +394,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const float alpha = P.sa ? __fmul_rn(__ldg(P.sa), __ldg(P.sb)) : 1.0f;
       const int row0 = (local_tile / P.tiles_n) * kBM + static_cast<int>(rank) * kHalf + quad * 32;
       const int n0 = (local_tile % P.tiles_n) * kBN;
-      const uint32_t t_base = tmem + (static_cast<uint32_t>(quad * 32) << 16) + acc * kAccCols;
+      const uint32_t t_base =
+          tmem + (static_cast<uint32_t>(quad * 32) << 16) + acc * (MX ? kMxAcc1Col : kAccCols);
       const bool sumsq = P.sumsq_slot >= 0;
       double ss = 0.0;
       // one 32 x 32 chunk of packed BF16 (16 words per lane) into the swizzled staging buffer
@@ -415,25 +430,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
       };
       if (MX) {
-        // single accumulator: read all of it into registers (packed BF16, 128 words per lane),
-        // release it so that the next tile's MMAs start, then store
-        uint32_t packed[kBN / 32][16];
-#pragma unroll
-        for (int c = 0; c < kBN / 32; ++c) {
+        // the chunk the two accumulators share comes first (accumulator 0: chunk 7, walking
+        // down; accumulator 1: chunk 0, walking up); once it is in registers it is released
+#pragma unroll 1
+        for (int step = 0; step < kBN / 32; ++step) {
+          const int c = acc == 0 ? kBN / 32 - 1 - step : step;
           uint32_t r[32];
           tmem_ld_32x32b_x32(t_base + c * 32, r);
           tmem_ld_wait();
+          if (step == 0) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&S->acc_shared_free), 0));
+          }
+          if (n0 + c * 32 >= N || row0 >= M) continue;  // chunk entirely outside the matrix
+          uint32_t w16[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j)
-            packed[c][j] = pack_bf16x2(__fmul_rn(__uint_as_float(r[2 * j]), alpha),
-                                       __fmul_rn(__uint_as_float(r[2 * j + 1]), alpha));
+            w16[j] = pack_bf16x2(__fmul_rn(__uint_as_float(r[2 * j]), alpha),
+                                 __fmul_rn(__uint_as_float(r[2 * j + 1]), alpha));
+          store_chunk(c, w16);
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&S->acc_empty[acc]), 0));
-#pragma unroll
-        for (int c = 0; c < kBN / 32; ++c)
-          if (n0 + c * 32 < N && row0 < M) store_chunk(c, packed[c]);
       } else {
 #pragma unroll 1
         for (int c = 0; c < kBN / 32; ++c) {
