@@ -62,12 +62,15 @@ __device__ __forceinline__ float pow2_neg(int X) {
   return X == 127 ? __uint_as_float(0x00400000u) : __uint_as_float(static_cast<uint32_t>(127 - X) << 23);
 }
 
-template <int FMT>
+// Four BF16 values (two words) -> four codes; with NAN_CHECK, NaN products become 0x7F. Only a
+// block whose amax is NaN can hold a NaN product (2^-X is finite and an infinite input
+// saturates), so the check runs for those blocks only.
+template <int FMT, bool NAN_CHECK>
 __device__ __forceinline__ uint32_t q4(uint32_t w0, uint32_t w1, float inv) {
-  // four BF16 values (two words) -> four codes, NaN products -> 0x7F
   const float p0 = __fmul_rn(__uint_as_float(w0 << 16), inv), p1 = __fmul_rn(__uint_as_float(w0 & 0xFFFF0000u), inv);
   const float p2 = __fmul_rn(__uint_as_float(w1 << 16), inv), p3 = __fmul_rn(__uint_as_float(w1 & 0xFFFF0000u), inv);
   uint32_t r = cvt_fp8x2<FMT>(p0, p1) | (cvt_fp8x2<FMT>(p2, p3) << 16);
+  if (!NAN_CHECK) return r;
   if (p0 != p0) r = (r & 0xFFFFFF00u) | 0x7Fu;
   if (p1 != p1) r = (r & 0xFFFF00FFu) | 0x7F00u;
   if (p2 != p2) r = (r & 0xFF00FFFFu) | 0x7F0000u;
@@ -144,10 +147,24 @@ __global__ void __launch_bounds__(kThreads) k_mx_cast(const __grid_constant__ Gr
         const int X = m > 0x7F80u ? 0 : block_exponent(m, emax);
         const float inv = pow2_neg(X);
         uint32_t out[8];
+        if (m > 0x7F80u) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          out[2 * k] = T.fmt == 0 ? q4<0>(w[k].x, w[k].y, inv) : q4<1>(w[k].x, w[k].y, inv);
-          out[2 * k + 1] = T.fmt == 0 ? q4<0>(w[k].z, w[k].w, inv) : q4<1>(w[k].z, w[k].w, inv);
+          for (int k = 0; k < 4; ++k) {
+            out[2 * k] = T.fmt == 0 ? q4<0, true>(w[k].x, w[k].y, inv) : q4<1, true>(w[k].x, w[k].y, inv);
+            out[2 * k + 1] = T.fmt == 0 ? q4<0, true>(w[k].z, w[k].w, inv) : q4<1, true>(w[k].z, w[k].w, inv);
+          }
+        } else if (T.fmt == 0) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            out[2 * k] = q4<0, false>(w[k].x, w[k].y, inv);
+            out[2 * k + 1] = q4<0, false>(w[k].z, w[k].w, inv);
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            out[2 * k] = q4<1, false>(w[k].x, w[k].y, inv);
+            out[2 * k + 1] = q4<1, false>(w[k].z, w[k].w, inv);
+          }
         }
         uint4* dst = reinterpret_cast<uint4*>(T.q_row + (r0 + row) * T.cols + c0 + 32 * b);
         dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
@@ -170,13 +187,16 @@ __global__ void __launch_bounds__(kThreads) k_mx_cast(const __grid_constant__ Gr
       const int X0 = m0 > 0x7F80u ? 0 : block_exponent(m0, emax);
       const int X1 = m1 > 0x7F80u ? 0 : block_exponent(m1, emax);
       const float inv0 = pow2_neg(X0), inv1 = pow2_neg(X1);
+      const bool nan_block = max(m0, m1) > 0x7F80u;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const float p0 = __fmul_rn(__uint_as_float(v[i] << 16), inv0);
         const float p1 = __fmul_rn(__uint_as_float(v[i] & 0xFFFF0000u), inv1);
         uint32_t c = T.fmt == 0 ? cvt_fp8x2<0>(p0, p1) : cvt_fp8x2<1>(p0, p1);
-        if (p0 != p0) c = (c & 0xFF00u) | 0x7Fu;
-        if (p1 != p1) c = (c & 0x00FFu) | 0x7F00u;
+        if (nan_block) {                       // only a NaN input gives a NaN product
+          if (p0 != p0) c = (c & 0xFF00u) | 0x7Fu;
+          if (p1 != p1) c = (c & 0x00FFu) | 0x7F00u;
+        }
         *reinterpret_cast<uint16_t*>(qs + (32 * rb + i) * kTile + col) = static_cast<uint16_t>(c);
       }
       atom_c[(col & 31) * 16 + (col >> 5) * 4 + rb] = m0 > 0x7F80u ? 0xFF : static_cast<uint8_t>(X0 + 127);
