@@ -331,7 +331,8 @@ def run_ours(args, rank, world, local_rank):
                 "how": "pinned host X, dY in and Y, dX out every step; copies overlapped with "
                        "the previous/next step's kernels on separate streams"},
         "gpu_launches": args.steps * st.kernels_per_step(),
-        "roofline": {"kernel": "k_fp8_gemm (one grouped launch: every fprop, dgrad, wgrad)", "bound": "tensor",
+        "roofline": {"kernel": ("k_fp8_gemm<true> block-scaled" if st.recipe == "mxfp8" else "k_fp8_gemm")
+                               + " (one grouped launch: every fprop, dgrad, wgrad)", "bound": "tensor",
                      "achieved": round(gemm_achieved, 1), "peak": round(fp8_peak, 1),
                      "unit": "TFLOP/s", "frac": round(gemm_achieved / fp8_peak, 4),
                      "traffic": traffic,
