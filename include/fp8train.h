@@ -10,6 +10,15 @@
  *   amax history roll + next scales     fp8_scale_update
  *   unscale, clip, AdamW, BF16 weight   fused_adamw_multi_tensor
  *
+ * and the same step in three launches:
+ *
+ *   casts of X and dY + the scale update of X, W, dY    fp8_cast_transpose_amax_update_multi
+ *   fprop, dgrad, wgrad (+ sum of dW^2)                 fp8_gemm_multi_sumsq
+ *   AdamW on that sum + cast of the next step's W       fused_adamw_multi_tensor_presummed
+ *
+ * plus current scaling (fp8_cast_transpose_amax_current_multi) and MXFP8 block scaling
+ * (fp8_mx_cast_multi, fp8_mx_gemm_multi).
+ *
  * Sources, cited by page title and section:
  *   [P1] "算子与编译器：FP8 训练与优化器 Kernel" (charles2530.github.io)
  *   [P2] "FP8 混合精度训练工程实践：从 H100 到大模型训练的范式跃迁" (ybb.press)
@@ -44,7 +53,7 @@ extern "C" {
 typedef enum fp8t_status {
     FP8T_OK = 0,
     FP8T_ERR_INVALID_ARG = 1,       /* NULL pointer, non-positive size, unknown enum value     */
-    FP8T_ERR_UNSUPPORTED_SHAPE = 2, /* a dimension is not a multiple of 16, or is too large    */
+    FP8T_ERR_UNSUPPORTED_SHAPE = 2, /* a dimension is not a multiple of 16 (128 for MX) or too big */
     FP8T_ERR_MISALIGNED = 3,        /* a pointer is not 16-byte aligned                          */
     FP8T_ERR_UNSUPPORTED_DEVICE = 4,/* the current device is not sm_100                         */
     FP8T_ERR_CUDA = 5,              /* a CUDA runtime or driver call failed                      */
