@@ -542,6 +542,34 @@ def oracle_sample_step(oracle, host, wl, rows_div):
     return dt, flop
 
 
+def oracle_output_sample_step(oracle, host, wl, n_out, rng):
+    """One step of the path with every stage on a small sample: casts of one row of X, W and dY,
+    the three GEMMs at n_out seeded output positions each (oracle.gemm_at), the scale update
+    and AdamW on 16 * n_out parameters. Returns (seconds, GEMM FLOP of the sample)."""
+    import numpy as np
+    _, fin, fout = wl.layers[0]
+    T = wl.tokens
+    t0 = time.perf_counter()
+    oracle.cast_transpose_amax(host["X"][:1], oracle.E4M3, 1.0)
+    oracle.cast_transpose_amax(host["W"][:1], oracle.E4M3, 1.0)
+    oracle.cast_transpose_amax(host["dY"][:1], oracle.E5M2, 1.0)
+    flop = 0
+    for A, af, B, bf, K in ((host["Xq"], 0, host["WqT"], 0, fin), (host["dYq"], 1, host["Wq"], 0, fout),
+                            (host["XqT"], 0, host["dYqT"], 1, T)):
+        ii = rng.integers(0, A.shape[0], n_out)
+        jj = rng.integers(0, B.shape[0], n_out)
+        oracle.gemm_at(A, af, B, bf, 1.0, 1.0, ii, jj)
+        flop += 2 * n_out * K
+    hist = np.zeros((3, wl.history_len), np.float32)
+    sc = np.ones(3, np.float32)
+    si = np.ones(3, np.float32)
+    oracle.scale_update(np.ones(3, np.float32), hist, [448.0, 448.0, 57344.0], 0, 0, sc, si)
+    n = 16 * n_out
+    oracle.fused_adamw([host["master"][:n].copy()], [np.zeros(n, np.float32)], [np.zeros(n, np.float32)],
+                       [host["dW"][:n]], [np.zeros(n, np.uint16)], dict(wl.adamw, step=1))
+    return time.perf_counter() - t0, flop
+
+
 def host_copies(st, batch):
     from optimizer_fp8_cast_b200.synth import bf16_bits, u8
     import numpy as np
@@ -563,15 +591,18 @@ def cpu_baseline(st, wl, nums, batch, frac_rows):
                       f"work, {dt:.1f} s), single-threaded C oracle on the host"}
 
 
+REFERENCE_BUDGET_S = 90.0       # the reference arm's warm-up plus timed steps, about
+
+
 def run_reference(args):
     """The CPU oracle as the reference arm: bounded samples, same metric and unit."""
     import torch
 
     import oracle
     from optimizer_fp8_cast_b200 import synth
+    import numpy as np
     wl = synth.WORKLOADS[args.workload]
     _, fin, fout = wl.layers[0]
-    rows_div = 4096
     # inputs: seeded CPU draws of the workload's shapes, quantised by the oracle itself
     X, dY = synth.linear_inputs(wl, 0, 0, "cpu")
     W = synth.linear_weight(wl, 0, "cpu")
@@ -584,17 +615,24 @@ def run_reference(args):
     host["dYq"], host["dYqT"] = q, qT
     host["master"] = W.float().numpy().reshape(-1)
     host["dW"] = synth.bf16_bits(torch.randn(fin * fout, generator=torch.Generator().manual_seed(1)).to(torch.bfloat16))
+    host = {k: np.ascontiguousarray(v) for k, v in host.items()}
+    # size each step's sample so that warm-up plus timed steps take about REFERENCE_BUDGET_S
+    rng = np.random.default_rng(0)
+    probe, _ = oracle_output_sample_step(oracle, host, wl, 64, rng)
+    per_step = REFERENCE_BUDGET_S / max(1, args.steps + args.warmup)
+    n_out = int(min(16384, max(8, 64 * per_step / max(probe, 1e-6))))
     for _ in range(args.warmup):
-        oracle_sample_step(oracle, host, wl, rows_div)
+        oracle_output_sample_step(oracle, host, wl, n_out, rng)
     times, flops = [], []
     for _ in range(args.steps):
-        dt, fl = oracle_sample_step(oracle, host, wl, rows_div)
+        dt, fl = oracle_output_sample_step(oracle, host, wl, n_out, rng)
         times.append(dt)
         flops.append(fl)
     total = sum(times)
     value = sum(flops) / total / 1e12
-    sample = (f"every stage on 1/{rows_div} of its rows per step ({flops[0] / 1e9:.3f} GFLOP of "
-              f"GEMM work), single-threaded C oracle")
+    sample = (f"every stage on a sample per step: casts of one row of X, W, dY; each GEMM at {n_out} "
+              f"seeded outputs ({flops[0] / 1e9:.3f} GFLOP); scale update; AdamW on {16 * n_out} "
+              f"parameters; single-threaded C oracle")
     return {
         "metric": METRIC, "value": round(value, 9), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 3),
