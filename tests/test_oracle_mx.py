@@ -106,3 +106,17 @@ def test_all_ones_closed_form():
     D = oracle.mx_gemm(A, sfa, oracle.E4M3, B, sfb, oracle.E4M3)
     want = 32 * (2.0 ** 3 + 2.0 ** 1 + 2.0 ** -1 + 2.0 ** -2)
     assert (D == oracle.f32_to_bf16(np.float32(want))).all()
+
+
+def test_subnormal_blocks_clamp_the_exponent():
+    """A block whose amax is a BF16 subnormal: floor(log2) is taken from the mantissa's top bit
+    (2^-130 = 8 * 2^-133), X = -130 - 8 clamps to -127 (scale code 0), and the elements come out
+    as 2^-130 * 2^127 = 2^-3, the E4M3 code 0x20 (exponent field 4, bias 7)."""
+    v = np.uint16(8)                                   # BF16 bits of 2^-130 (subnormal)
+    bits = np.full((1, 32), v, np.uint16)
+    q, sf = oracle.mx_quantise(bits, 0, oracle.E4M3)
+    assert sf[0, 0] == 0 and (q == 0x20).all()
+    bits[0, 0] = 0x0001                                # 2^-133, the smallest subnormal
+    q, sf = oracle.mx_quantise(bits, 0, oracle.E5M2)   # X = -130 - 15 clamps to -127 as well
+    assert sf[0, 0] == 0
+    assert oracle.fp8_decode(int(q[0, 0]), oracle.E5M2) == 2.0 ** -6   # 2^-133 * 2^127
