@@ -250,10 +250,13 @@ def mx_gemm_at(A, sfa, afmt, B, sfb, bfmt, ii, jj):
     """The MX GEMM oracle at output positions (ii[s], jj[s]); returns (D bits, abs_sum)."""
     A, B = np.ascontiguousarray(A, np.uint8), np.ascontiguousarray(B, np.uint8)
     sfa, sfb = np.ascontiguousarray(sfa, np.uint8), np.ascontiguousarray(sfb, np.uint8)
-    K = A.shape[1]
+    M, K = A.shape
+    N = B.shape[0]
+    assert B.shape[1] == K and K % 32 == 0 and sfa.shape == (M, K // 32) and sfb.shape == (N, K // 32)
     ii = np.ascontiguousarray(ii, np.int64)
     jj = np.ascontiguousarray(jj, np.int64)
-    assert (ii >= 0).all() and (ii < A.shape[0]).all() and (jj >= 0).all() and (jj < B.shape[0]).all()
+    assert ii.shape == jj.shape
+    assert (ii >= 0).all() and (ii < M).all() and (jj >= 0).all() and (jj < N).all()
     out = np.empty(ii.shape, np.uint16)
     ab = np.empty(ii.shape, np.float64)
     lib().orc_mx_gemm_at(_ptr(A, C.c_uint8), _ptr(sfa, C.c_uint8), int(afmt), _ptr(B, C.c_uint8),

@@ -120,3 +120,83 @@ def test_subnormal_blocks_clamp_the_exponent():
     q, sf = oracle.mx_quantise(bits, 0, oracle.E5M2)   # X = -130 - 15 clamps to -127 as well
     assert sf[0, 0] == 0
     assert oracle.fp8_decode(int(q[0, 0]), oracle.E5M2) == 2.0 ** -6   # 2^-133 * 2^127
+
+
+def _exact_mx(A, sfa, afmt, B, sfb, bfmt, i, j):
+    """sum_k a_ik b_jk 2^(Xa + Xb) as an exact rational, operands decoded from the code tables."""
+    K = A.shape[1]
+    return sum(Fraction(oracle.fp8_decode(int(A[i, k]), afmt)) *
+               Fraction(oracle.fp8_decode(int(B[j, k]), bfmt)) *
+               Fraction(2) ** (int(sfa[i, k // 32]) + int(sfb[j, k // 32]) - 254)
+               for k in range(K))
+
+
+def test_mx_gemm_at_matches_full_gemm_and_exact_sums():
+    """The sampled MX GEMM (the oracle behind the full-size MX GEMM checks) against the full one
+    at random positions, with M != N, a distinct scale row for every row of A and of B and mixed
+    E4M3 x E5M2 operands, so that swapping the row and column indices, or taking one operand's
+    scale row for the other's, gives different values; a few positions also against the exact
+    rational sum."""
+    rng = np.random.default_rng(8)
+    M, N, K = 37, 53, 160
+    ta, tb = oracle.decode_table(oracle.E4M3), oracle.decode_table(oracle.E5M2)
+    A = rng.choice(np.flatnonzero(np.isfinite(ta)).astype(np.uint8), (M, K))
+    B = rng.choice(np.flatnonzero(np.isfinite(tb)).astype(np.uint8), (N, K))
+    sfa = rng.integers(110, 145, (M, K // 32)).astype(np.uint8)
+    sfb = rng.integers(115, 140, (N, K // 32)).astype(np.uint8)
+    D, ab = oracle.mx_gemm(A, sfa, oracle.E4M3, B, sfb, oracle.E5M2, want_abs=True)
+    ii = rng.integers(0, M, 400)
+    jj = rng.integers(0, N, 400)
+    got, gab = oracle.mx_gemm_at(A, sfa, oracle.E4M3, B, sfb, oracle.E5M2, ii, jj)
+    assert np.array_equal(got, D[ii, jj]) and np.array_equal(gab, ab[ii, jj])
+    # the sampled values are not those of transposed indices or of swapped scale rows
+    Dsw = oracle.mx_gemm(A, np.roll(sfa, 1, axis=0), oracle.E4M3, B, sfb, oracle.E5M2)
+    assert (Dsw[ii, jj] != got).mean() > 0.5
+    for s in range(12):
+        ref = oracle.f32_to_bf16(np.float32(float(_exact_mx(A, sfa, oracle.E4M3, B, sfb,
+                                                            oracle.E5M2, ii[s], jj[s]))))
+        assert abs(int(got[s]) - int(ref)) <= 1
+
+
+def test_nan_block_keeps_unit_scale_and_nan_code():
+    """A block holding a NaN has no finite amax: its E8M0 scale is the NaN code 0xFF (the only
+    non-numeric E8M0 code), and its other elements are encoded at unit scale, X = 0. Hand-worked
+    values: 1.0 -> 0x38 and -2.0 -> 0xC0 in E4M3 (bias 7), 1.0 -> 0x3C and 3.0 -> 0x42 in E5M2
+    (bias 15), 1000.0 saturates to 448 (0x7E) in E4M3; the NaN itself is the byte 0x7F."""
+    nan = np.uint16(0x7FC1)                                  # a NaN with a payload
+    for fmt, vals, codes in ((oracle.E4M3, [1.0, -2.0, 1000.0], [0x38, 0xC0, 0x7E]),
+                             (oracle.E5M2, [1.0, 3.0, -0.0], [0x3C, 0x42, 0x80])):
+        x = np.zeros((1, 32), np.float32)
+        x[0, 1:4] = vals
+        bits = bf16_bits(torch.from_numpy(x).to(torch.bfloat16))
+        bits[0, 17] = nan
+        q, sf = oracle.mx_quantise(bits, 0, fmt)
+        assert sf[0, 0] == 0xFF
+        assert list(q[0, 1:4]) == codes and q[0, 17] == 0x7F
+        assert q[0, 0] == 0x00 and (q[0, 4:17] == 0).all() and (q[0, 18:] == 0).all()
+        # column-wise blocks follow the same rule: only the column holding the NaN
+        cols = np.zeros((32, 4), np.uint16)
+        cols[:, 2] = bits[0]
+        cols[:, 0] = bits[0, 1]                               # a column of 1.0 / 1.0
+        qc, sfc = oracle.mx_quantise(cols, 1, fmt)
+        assert sfc[0, 2] == 0xFF and list(qc[1:4, 2]) == codes and qc[17, 2] == 0x7F
+        assert sfc[0, 0] == 127 - (8 if fmt == oracle.E4M3 else 15) and sfc[0, 1] == 0
+
+
+def test_infinite_amax_takes_the_largest_exponent():
+    """A block whose amax is +-inf: X = 127, the largest finite E8M0 exponent (code 254). The
+    infinity then saturates to the format's largest code (0x7E = 448 in E4M3, 0x7B = 57344 in
+    E5M2; sign kept), and finite elements times 2^-127 fall below the smallest subnormal and
+    encode as signed zeros."""
+    for fmt, top in ((oracle.E4M3, 0x7E), (oracle.E5M2, 0x7B)):
+        x = np.full((2, 32), 3.5, np.float32)
+        x[0, 5] = np.inf
+        x[1, 9] = -np.inf
+        x[1, 0] = -1.0e30
+        bits = bf16_bits(torch.from_numpy(x).to(torch.bfloat16))
+        q, sf = oracle.mx_quantise(bits, 0, fmt)
+        assert (sf[:, 0] == 254).all()
+        assert q[0, 5] == top and q[1, 9] == 0x80 | top
+        assert (np.delete(q[0], 5) == 0x00).all()
+        # -1e30 * 2^-127 ~ -5.9e-9: far below the smallest subnormal, a negative zero
+        assert q[1, 0] == 0x80 and (np.delete(q[1], [0, 9]) == 0x00).all()
