@@ -38,7 +38,10 @@
  *     returns an error status and launches nothing. A launch failure returns FP8T_ERR_CUDA;
  *     fp8t_last_error_message() describes the last failure on the calling thread.
  *   - Waits inside kernels are bounded in time. When one expires the kernel records it in a
- *     device error word and returns early; fp8t_check_device_error() reports it.
+ *     device error word and returns early; fp8t_check_device_error() reports it. The word is
+ *     for reporting only: what a fused call does about an expired wait (keep the scales, report
+ *     a NaN sum of squares) depends on that call's own launches, never on the word, so a stale
+ *     entry from an unrelated call changes nothing.
  */
 #ifndef FP8TRAIN_H
 #define FP8TRAIN_H
@@ -172,8 +175,8 @@ typedef struct fp8t_cast_update {
  * An entry with x_bf16 = NULL, rows = cols = 0 and no outputs or counters is UPDATE ONLY: its
  * amax slot was filled by another call (the weight cast inside
  * fused_adamw_multi_tensor_presummed of the previous step) and only the update runs for it.
- * If a bounded wait of the launch expires (FP8T_ERR_TIMEOUT pending in the device error word),
- * the scale state is left unchanged. Argument errors as in the two calls it combines, plus
+ * If a bounded wait of this launch expires (FP8T_ERR_TIMEOUT pending in the device error word),
+ * the scale state is left unchanged; the CTAs report it to the last one through the ticket. Argument errors as in the two calls it combines, plus
  * FP8T_ERR_INVALID_ARG for a NULL or shared scale-inverse pointer.
  */
 fp8t_status fp8_cast_transpose_amax_update_multi(const fp8t_cast_tensor* tensors,
@@ -249,10 +252,11 @@ fp8t_status fp8_gemm_multi(const fp8t_gemm_desc* gemms, int32_t n_gemms, void* s
  * one pass in index order), so S is the same on every run; it may differ from a sequential
  * FP64 sum in the last bits.
  *   sumsq_of        HOST array of n_gemms int32: nonzero = include this problem's D.
- *   d_sumsq_out     1 double (device), overwritten; NaN if a bounded wait of the call expired.
+ *   d_sumsq_out     1 double (device), overwritten; NaN if a bounded wait of this call expired.
  *   d_workspace     device scratch of fp8_gemm_sumsq_workspace_bytes() bytes, 256-byte aligned,
- *                   ZERO-FILLED before its first use (it holds a ticket counter that every call
- *                   leaves at zero). Calls that may run at the same time need their own.
+ *                   ZERO-FILLED before its first use (it holds a ticket counter and the call's
+ *                   abort word, which every call leaves at zero). Calls that may run at the
+ *                   same time need their own.
  * Errors as in fp8_gemm_multi, plus FP8T_ERR_INVALID_ARG for NULL/misaligned S or workspace,
  * no selected problem, or a workspace that is too small.
  */

@@ -130,19 +130,29 @@ __device__ __forceinline__ uint32_t quantise_segment(const Tensor& T, const uint
   return m;
 }
 
+// Ticket word of a fused cast launch: each CTA adds 1 when it is done, plus kTicketAbort if one
+// of its waits expired (grids stay far below 2^16 CTAs), so the last CTA learns from the value it
+// draws whether this launch, and only this launch, is complete.
+constexpr unsigned kTicketAbort = 1u << 16;
+
 // The last CTA of a launch to finish (ticket counter) updates the scale state of every tensor of
 // the launch, one warp per tensor. Called by every thread of every CTA once its own work, amax
-// atomics included, is issued.
-__device__ __forceinline__ void last_cta_update(const Group& g) {
-  __shared__ int s_last;
+// atomics included, is issued; `aborted` is the same for every thread of the CTA.
+__device__ __forceinline__ void last_cta_update(const Group& g, bool aborted) {
+  __shared__ int s_last, s_complete;
   __threadfence();                                 // this CTA's amax atomics before its ticket
   __syncthreads();
-  if (threadIdx.x == 0) s_last = atomicAdd(g.ticket, 1u) == gridDim.x - 1;
+  if (threadIdx.x == 0) {
+    const unsigned old = atomicAdd(g.ticket, aborted ? 1u + kTicketAbort : 1u);
+    s_last = (old & (kTicketAbort - 1u)) == gridDim.x - 1;
+    s_complete = !aborted && old < kTicketAbort;
+  }
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  // a launch whose waits expired leaves the scale state alone (its amax may be incomplete)
-  const bool ok = *reinterpret_cast<volatile unsigned int*>(&g_error_word) == 0u;
+  // a launch whose own waits expired leaves the scale state alone (its amax may be incomplete);
+  // an expired wait of any other launch does not matter here
+  const bool ok = s_complete != 0;
   const int warp = threadIdx.x >> 5;
   if (ok && warp < g.n) {
     const Tensor& T = g.t[warp];
@@ -310,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_cast_transpose_amax(const __gri
       if (pending & (1u << b)) mbar_wait(smem_u32(&full[b]), (pending_ph >> b) & 1u, kDrainLimitNs);
     bulk_wait_group<0>();                          // stores complete before the CTA exits
   }
-  if (g.update) last_cta_update(g);
+  if (g.update) last_cta_update(g, s_abort != 0);
 }
 
 // Row-major-only casts (no tensor of the launch wants q^T): a plain streaming kernel. Each
@@ -369,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_cast_rowmajor(const __grid_cons
     }
     if (T.scale_inv && blockIdx.x == 0 && tid == 0) *T.scale_inv = __fdiv_rn(1.0f, s);
   }
-  if (g.update) last_cta_update(g);
+  if (g.update) last_cta_update(g, false);        // this kernel has no waits that can expire
 }
 
 }  // namespace cast

@@ -455,7 +455,7 @@ fp8t_status fp8_cast_transpose_amax(const void* x_bf16, int64_t rows, int64_t co
 
 namespace {
 
-constexpr size_t kSumsqHeader = 256;    // ticket, then the partial slots
+constexpr size_t kSumsqHeader = 256;    // ticket and abort words, then the partial slots
 
 // Tile lists of a grouped GEMM launch: every tile costs its problem's K / 128 k-blocks; tiles are
 // handed out longest first, each to the least-loaded cluster, and every cluster then runs its
@@ -555,6 +555,7 @@ fp8t_status gemm_multi(const fp8t_gemm_desc* gemms, int32_t n_gemms, const int32
     group.n = b1 - b0;
     if (sumsq_of) {
       group.ticket = static_cast<unsigned int*>(d_workspace);
+      group.abort_word = static_cast<unsigned int*>(d_workspace) + 1;
       group.partials = reinterpret_cast<double*>(static_cast<char*>(d_workspace) + kSumsqHeader);
       group.sumsq_out = d_sumsq_out;
       group.n_partials = static_cast<int32_t>(n_slots);

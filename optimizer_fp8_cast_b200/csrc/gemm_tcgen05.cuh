@@ -169,6 +169,8 @@ struct alignas(64) Group {
   double* partials;              // every launch's slots (8 per summed tile)
   double* sumsq_out;
   unsigned int* ticket;          // zero on entry, left zero
+  unsigned int* abort_word;      // set by any CTA of the call whose waits expired; zero on entry,
+                                 // left zero
   int32_t n_partials;            // slots of all launches of the call
   int32_t last_launch;           // this launch reduces the slots
 };
@@ -496,7 +498,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc_pair(tmem, kTmemCols);
 
   // ---------------- sum of squares: the last CTA of the last launch adds the slots in order
-  if (!g.sumsq_out || !g.last_launch) return;
+  if (!g.sumsq_out) return;
+  // a CTA whose waits expired left slots unwritten: it marks the call (any of its launches)
+  if (threadIdx.x == 0 && *abort_flag) atomicOr(g.abort_word, 1u);
+  if (!g.last_launch) return;
   __shared__ int s_last;
   __shared__ double s_part[kThreads];
   if (threadIdx.x == 0) {
@@ -513,9 +518,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     double total = 0.0;
     for (int i = 0; i < kThreads; ++i) total = __dadd_rn(total, s_part[i]);
-    // a launch whose waits expired has slots that were never written
-    if (*reinterpret_cast<volatile unsigned int*>(&g_error_word) != 0u) total = __longlong_as_double(0x7FF8000000000000LL);
+    // a launch of this call whose waits expired has slots that were never written (expired waits
+    // of other calls do not matter here)
+    if (*reinterpret_cast<volatile unsigned int*>(g.abort_word) != 0u)
+      total = __longlong_as_double(0x7FF8000000000000LL);
     *g.sumsq_out = total;
+    atomicExch(g.abort_word, 0u);
     atomicExch(g.ticket, 0u);
   }
 }
