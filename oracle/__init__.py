@@ -75,6 +75,10 @@ def lib():
         L.orc_mx_gemm.restype = None
         L.orc_mx_gemm.argtypes = [u8p, u8p, C.c_int, u8p, u8p, C.c_int, C.c_int64, C.c_int64,
                                   C.c_int64, u16p, f64p]
+        L.orc_set_threads.restype = C.c_int
+        L.orc_set_threads.argtypes = [C.c_int]
+        L.orc_get_threads.restype = C.c_int
+        L.orc_get_threads.argtypes = []
         L.orc_mx_gemm_at.restype = None
         L.orc_mx_gemm_at.argtypes = [u8p, u8p, C.c_int, u8p, u8p, C.c_int, C.c_int64, C.c_int64,
                                      i64p, i64p, u16p, f64p]
@@ -87,6 +91,16 @@ def _ptr(a, ctype):
         return None
     assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
     return a.ctypes.data_as(C.POINTER(ctype))
+
+
+def set_threads(n: int) -> int:
+    """Host threads the oracle's loops may use (n <= 0: every core). Results do not depend on
+    it: only independent pieces are split, and sums keep their fixed order. Returns the count."""
+    return int(lib().orc_set_threads(int(n)))
+
+
+def get_threads() -> int:
+    return int(lib().orc_get_threads())
 
 
 # ----------------------------------------------------------------------------- scalars

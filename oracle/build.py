@@ -2,6 +2,7 @@
 
 Test infrastructure: the oracle is the checker, never part of the product path.
 Plain IEEE arithmetic: -O2 -ffp-contract=off, no -ffast-math, no -march (no FMA contraction).
+-fopenmp: the oracle splits independent work over threads (same results for any thread count).
 """
 import os
 import subprocess
@@ -17,7 +18,7 @@ def build_oracle(force: bool = False) -> str:
         return LIB
     tmp = LIB + ".tmp.%d" % os.getpid()
     cmd = ["gcc", "-std=c11", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
-           "-Wall", "-Wextra", "-o", tmp, SRC, "-lm"]
+           "-fopenmp", "-Wall", "-Wextra", "-o", tmp, SRC, "-lm"]
     subprocess.run(cmd, check=True)
     os.replace(tmp, LIB)
     return LIB

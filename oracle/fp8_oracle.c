@@ -5,8 +5,12 @@
  * library computes. Only the test suite, the package smoke check and the benchmark's CPU
  * baseline load it; the product path never does. It shares no code, header, table or constant
  * generator with the CUDA library: every FP8 value is encoded and decoded here from the bit
- * fields, by integer manipulation written out below. Build: gcc -O2 -ffp-contract=off (plain
- * IEEE single/double arithmetic, no fused multiply-add, no fast-math). Single-threaded.
+ * fields, by integer manipulation written out below. Build: gcc -O2 -ffp-contract=off -fopenmp
+ * (plain IEEE single/double arithmetic, no fused multiply-add, no fast-math).
+ * Threads (OpenMP) only split work whose pieces are independent (output elements, rows, the
+ * fixed chunks of the norm sum) or combine integer counts and maxima, so every result is the
+ * same bit for bit whatever the thread count (orc_set_threads; 1 gives the plain sequential
+ * program).
  *
  * Sources, cited by page title and section:
  *   [P1] "算子与编译器：FP8 训练与优化器 Kernel"
@@ -20,11 +24,36 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define ORC_E4M3 0
 #define ORC_E5M2 1
 #define ORC_AMAX_MAX 0
 #define ORC_AMAX_MOST_RECENT 1
+
+/* Threads used by the functions below (0 or less: all the host offers). Returns the count now
+ * in effect. */
+int orc_set_threads(int n)
+{
+#ifdef _OPENMP
+    omp_set_num_threads(n > 0 ? n : omp_get_num_procs());
+    return omp_get_max_threads();
+#else
+    (void)n;
+    return 1;
+#endif
+}
+
+int orc_get_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
 
 static uint32_t f32_bits(float f) { uint32_t b; memcpy(&b, &f, 4); return b; }
 static float bits_f32(uint32_t b) { float f; memcpy(&f, &b, 4); return f; }
@@ -145,6 +174,7 @@ uint8_t orc_fp8_encode(float v, int fmt)
 /* Encode an array of f32 values (the encode above, element by element). */
 void orc_fp8_encode_array(const float* x, int64_t n, int fmt, uint8_t* out)
 {
+#pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < n; ++i) out[i] = orc_fp8_encode(x[i], fmt);
 }
 
@@ -171,6 +201,7 @@ void orc_cast_transpose_amax(const uint16_t* x, int64_t rows, int64_t cols, int 
     const float maxv = fmt_max(fmt);
     uint32_t amax_bits = 0;
     uint64_t nsat = 0, nzero = 0, nnonfinite = 0;
+#pragma omp parallel for schedule(static) reduction(max : amax_bits) reduction(+ : nsat, nzero, nnonfinite)
     for (int64_t i = 0; i < rows; ++i) {
         for (int64_t j = 0; j < cols; ++j) {
             const uint16_t h = x[i * cols + j];
@@ -298,6 +329,7 @@ void orc_gemm(const uint8_t* A, int afmt, const uint8_t* B, int bfmt, int64_t M,
               int64_t K, float a_scale_inv, float b_scale_inv, uint16_t* D, double* abs_out)
 {
     const float alpha = a_scale_inv * b_scale_inv;
+#pragma omp parallel for schedule(dynamic, 1)
     for (int64_t i = 0; i < M; ++i)
         for (int64_t j = 0; j < N; ++j)
             gemm_element(A + i * K, afmt, B + j * K, bfmt, K, alpha, D + i * N + j,
@@ -310,6 +342,7 @@ void orc_gemm_at(const uint8_t* A, int afmt, const uint8_t* B, int bfmt, int64_t
                  const int64_t* jj, uint16_t* out, double* abs_out)
 {
     const float alpha = a_scale_inv * b_scale_inv;
+#pragma omp parallel for schedule(static)
     for (int64_t s = 0; s < n; ++s)
         gemm_element(A + ii[s] * K, afmt, B + jj[s] * K, bfmt, K, alpha, out + s,
                      abs_out ? abs_out + s : NULL);
@@ -318,18 +351,51 @@ void orc_gemm_at(const uint8_t* A, int afmt, const uint8_t* B, int bfmt, int64_t
 /* ---------------------------------------------------------------------------------------
  * Global gradient norm for clipping [P1 FP8 训练主路径图: unscale / clip before the fused
  * optimizer; P2 §四: gradients of the loss-scaled loss are divided by the loss scale].
- * Reading (pages give no formula): G = sum over tensors, then elements, in order, of f32(g)^2
- * in double; norm = float(sqrt(G) * (1 / loss_scale)), the norm of the unscaled gradient.
+ * Reading (pages give no formula): G = sum of f32(g)^2 in double over every element; each
+ * tensor is cut into fixed chunks of 65,536 elements, each chunk summed in order, and the chunk
+ * sums (tensor by tensor, chunk by chunk) combined by pairwise summation; norm =
+ * float(sqrt(G) * (1 / loss_scale)), the norm of the unscaled gradient. (Any FP64 order agrees
+ * to far below an f32 ulp here; this one is fixed, so it does not depend on the thread count.)
  * ------------------------------------------------------------------------------------- */
+#define ORC_NORM_CHUNK 65536
+
+static double pairwise_sum(const double* v, int64_t n)
+{
+    if (n == 1) return v[0];
+    const int64_t h = n / 2;
+    return pairwise_sum(v, h) + pairwise_sum(v + h, n - h);
+}
+
 float orc_global_norm(int32_t n, const uint16_t* const* grads, const int64_t* numel,
                       float loss_scale)
 {
-    double G = 0.0;
+    int64_t nchunks = 0;
+    for (int32_t t = 0; t < n; ++t) nchunks += (numel[t] + ORC_NORM_CHUNK - 1) / ORC_NORM_CHUNK;
+    if (nchunks == 0) return 0.0f;
+    double* part = (double*)malloc((size_t)nchunks * sizeof(double));
+    int64_t* tens = (int64_t*)malloc((size_t)nchunks * sizeof(int64_t));
+    int64_t* first = (int64_t*)malloc((size_t)nchunks * sizeof(int64_t));
+    int64_t c = 0;
     for (int32_t t = 0; t < n; ++t)
-        for (int64_t i = 0; i < numel[t]; ++i) {
-            const double g = (double)orc_bf16_to_f32(grads[t][i]);
-            G += g * g;
+        for (int64_t i = 0; i < numel[t]; i += ORC_NORM_CHUNK) {
+            tens[c] = t;
+            first[c++] = i;
         }
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t k = 0; k < nchunks; ++k) {
+        const int64_t t = tens[k], i0 = first[k];
+        const int64_t i1 = i0 + ORC_NORM_CHUNK < numel[t] ? i0 + ORC_NORM_CHUNK : numel[t];
+        double acc = 0.0;
+        for (int64_t i = i0; i < i1; ++i) {
+            const double g = (double)orc_bf16_to_f32(grads[t][i]);
+            acc += g * g;
+        }
+        part[k] = acc;
+    }
+    const double G = pairwise_sum(part, nchunks);
+    free(part);
+    free(tens);
+    free(first);
     return (float)(sqrt(G) * (1.0 / (double)loss_scale));
 }
 
@@ -360,6 +426,7 @@ int orc_adamw_update(int32_t n, float* const* master, float* const* m, float* co
     const float step_size = (float)((double)lr / (1.0 - pow((double)beta1, (double)step)));
     const float bc2_sqrt = (float)sqrt(1.0 - pow((double)beta2, (double)step));
     for (int32_t t = 0; t < n; ++t) {
+#pragma omp parallel for schedule(static)
         for (int64_t i = 0; i < numel[t]; ++i) {
             const float gg = orc_bf16_to_f32(g[t][i]) * f;
             const float mm = beta1 * m[t][i] + omb1 * gg;
@@ -459,10 +526,12 @@ void orc_mx_quantise(const uint16_t* x, int64_t rows, int64_t cols, int axis, in
                      uint8_t* q, uint8_t* sf)
 {
     if (axis == 0) {
+#pragma omp parallel for schedule(static)
         for (int64_t r = 0; r < rows; ++r)
             for (int64_t b = 0; b < cols / 32; ++b)
                 sf[r * (cols / 32) + b] = mx_block(x + r * cols + 32 * b, 1, fmt, q + r * cols + 32 * b, 1);
     } else {
+#pragma omp parallel for schedule(static)
         for (int64_t b = 0; b < rows / 32; ++b)
             for (int64_t c = 0; c < cols; ++c)
                 sf[b * cols + c] = mx_block(x + 32 * b * cols + c, cols, fmt, q + 32 * b * cols + c, cols);
@@ -513,6 +582,7 @@ void orc_mx_gemm(const uint8_t* A, const uint8_t* sfa, int afmt, const uint8_t* 
                  const uint8_t* sfb, int bfmt, int64_t M, int64_t N, int64_t K, uint16_t* D,
                  double* abs_out)
 {
+#pragma omp parallel for schedule(dynamic, 1)
     for (int64_t i = 0; i < M; ++i)
         for (int64_t j = 0; j < N; ++j)
             mx_element(A + i * K, sfa + i * (K / 32), afmt, B + j * K, sfb + j * (K / 32), bfmt, K,
@@ -524,6 +594,7 @@ void orc_mx_gemm_at(const uint8_t* A, const uint8_t* sfa, int afmt, const uint8_
                     const uint8_t* sfb, int bfmt, int64_t K, int64_t n, const int64_t* ii,
                     const int64_t* jj, uint16_t* out, double* abs_out)
 {
+#pragma omp parallel for schedule(static)
     for (int64_t s = 0; s < n; ++s)
         mx_element(A + ii[s] * K, sfa + ii[s] * (K / 32), afmt, B + jj[s] * K, sfb + jj[s] * (K / 32),
                    bfmt, K, out + s, abs_out ? abs_out + s : NULL);
