@@ -4,20 +4,33 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 A step is one pass of the whole hot path over one batch of the 4096 x 4096 Linear with 8192
-tokens (batch 4 x sequence 2048): three casts (X, W to E4M3, dY to E5M2, each with its
-transposed copy and amax), fprop / dgrad / wgrad FP8 GEMMs, the amax-history roll and scale
-update (history 1024, algo max, margin 0), and one fused AdamW over dW. Inputs are synthetic
-(seeded normals of the stated shapes), resident in HBM when timing starts; L2 is flushed (a
-256 MiB write) before every timed step.
+tokens (batch 4 x sequence 2048), three launches captured in one CUDA graph:
+  1. the cast launch: X -> E4M3 and dY -> E5M2 (row-major codes, amax, inverse scales used; the
+     GEMMs read the codes MN-major where they need the transpose, so no transposed copy is
+     written), and in its last CTA the amax-history roll and scale update of X, W and dY
+     (history 1024, algo max, margin 0);
+  2. one grouped GEMM launch: fprop, dgrad and wgrad (FP8 operands, FP32 accumulation, BF16
+     out), the wgrad epilogue also summing dW^2 for the global norm;
+  3. one fused AdamW launch over dW (unscale, clip, m, v, master, BF16 weight) that also casts
+     the new weight to E4M3 codes for the next step.
+Inputs are synthetic (seeded normals of the stated shapes), resident in HBM when timing starts.
+Before every timed step L2 is flushed by writing a 256 MiB buffer (its dirty lines are written
+back while the next step runs, as the previous step's AdamW writes would be in a training loop);
+a second, shorter loop also reads a 256 MiB buffer after the write, so that the step starts with
+clean lines, and reports each launch's time without that write-back.
 
 Prints one JSON line (rank 0). `value` is the GEMM work of all ranks (3 x 2 x 8192 x 4096 x 4096
 FLOP per step per rank) divided by the max over ranks of the summed device time of the K steps.
 With N > 1 every rank runs an independent replica (the path has no data-path collective);
-the barrier and the max-over-ranks reduction use NCCL.
+the barrier and the max-over-ranks reduction use NCCL. `rooflines` lists the three launches
+(GEMM against the FP8 tensor peak, cast and AdamW against HBM), `roofline` is the GEMM's.
 
---impl reference times the CPU oracle (single thread, as it stands) on a bounded sample of the
-same workload: each step runs every stage on 1/4096 of its rows and the sample's share of the
-GEMM work is scaled to the same TFLOP/s unit. Only rank 0 runs it.
+`cpu_baseline` times the CPU oracle (the correctness reference, as it stands) on this host, on
+one thread and on all of them, stage by stage on samples of about two seconds each; the step
+throughput it reports is the step's work over the sum of the stage times that the measured
+rates give for the whole step. --impl reference times the oracle on all host threads on a
+bounded sample of the workload (the GEMMs at seeded output positions, the other stages on
+slices), scaled to the same TFLOP/s unit. Only rank 0 runs either.
 """
 import argparse
 import json
@@ -36,6 +49,7 @@ METRIC = "FP8 Linear fwd+bwd TFLOP/s; cast+amax & fused AdamW GB/s vs HBM peak"
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP8_OVER_BF16 = 2.0        # nominal dense FP8 / BF16 tensor-core ratio (4.5 / 2.25 PFLOP/s)
+DATASHEET_FP8_TFLOPS = 4500.0   # B200 dense FP8 datasheet figure (context denominator)
 L2_FLUSH_BYTES = 256 << 20
 CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -167,6 +181,16 @@ def run_ours(args, rank, world, local_rank):
                        recipe=args.recipe)
     batches = [list(zip(*[synth.linear_inputs(wl, k, t, dev) for k in range(nl)])) for t in range(2)]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    sweep = torch.ones(L2_FLUSH_BYTES // 8, dtype=torch.int64, device=dev)
+    sweep_out = torch.empty((), dtype=torch.int64, device=dev)
+
+    def flush_dirty():                    # L2 full of dirty lines of another buffer
+        flush.zero_()
+
+    def flush_clean():                    # the same write, then a read: L2 full of clean lines
+        flush.zero_()
+        torch.sum(sweep, dim=0, out=sweep_out)
+
     # one timing window per kernel launch of the step (the scale update runs in the last CTA of
     # the cast launch unless --separate-scale-update)
     stages = [("cast", None), ("gemm", None), ("adamw", None)]
@@ -199,7 +223,7 @@ def run_ours(args, rank, world, local_rank):
             rec(i + 1)
 
     for w in range(args.warmup):
-        flush.zero_()
+        flush_dirty()
         one_step(*batches[w % 2])
     torch.cuda.synchronize()
     fp8.fp8t_check_device_error()
@@ -217,21 +241,18 @@ def run_ours(args, rank, world, local_rank):
                 one_step(*batches[b], ev=evs)
             graphs.append((g, evs))
         for g, _ in graphs:
-            flush.zero_()
+            flush_dirty()
             g.replay()
         torch.cuda.synchronize()
         fp8.fp8t_check_device_error()
 
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(NEV)] for _ in range(args.steps)]
-    gpu_id = gpu_uuid(dev, local_rank)
-    stage_ms, step_ms = [], []
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    wall0 = time.perf_counter()
-    with ClockSampler(gpu_id) as clocks:
-        for t in range(args.steps):
-            flush.zero_()
+    def timed_loop(pre, n):
+        """n steps, each after `pre` (outside the events); per-launch and per-step ms."""
+        stage_ms, step_ms = [], []
+        events = None if graphs else [[torch.cuda.Event(enable_timing=True) for _ in range(NEV)]
+                                      for _ in range(n)]
+        for t in range(n):
+            pre()
             if graphs:
                 g, ev = graphs[t % 2]
                 g.replay()
@@ -241,20 +262,34 @@ def run_ours(args, rank, world, local_rank):
             else:
                 one_step(*batches[t % 2], ev=events[t])
         torch.cuda.synchronize()
+        if events is not None:
+            stage_ms = [[events[t][i].elapsed_time(events[t][i + 1]) for i in range(NEV - 1)]
+                        for t in range(n)]
+            step_ms = [events[t][0].elapsed_time(events[t][NEV - 1]) for t in range(n)]
+        return stage_ms, step_ms
+
+    gpu_id = gpu_uuid(dev, local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    with ClockSampler(gpu_id) as clocks:
+        stage_ms, step_ms = timed_loop(flush_dirty, args.steps)
     wall = time.perf_counter() - wall0
     if world > 1:
         dist.barrier()
     fp8.fp8t_check_device_error()
-    if not graphs:
-        stage_ms = [[events[t][i].elapsed_time(events[t][i + 1]) for i in range(NEV - 1)]
-                    for t in range(args.steps)]
-        step_ms = [events[t][0].elapsed_time(events[t][NEV - 1]) for t in range(args.steps)]
     total_ms = reduce_max(sum(step_ms), world, dev)
     flop_step = 3 * sum(nums["gemm_flop"])
     value = throughput(flop_step, args.steps, world, total_ms)
+    # the same steps after a clean flush: each launch without the write-back of the flush's lines
+    n_clean = min(args.steps, 200)
+    clean_stage_ms, clean_step_ms = timed_loop(flush_clean, n_clean)
+    fp8.fp8t_check_device_error()
 
     # per-kernel figures (this rank), averaged over the timed steps
     avg = {name: statistics.mean(s[i] for s in stage_ms) for i, (name, _) in enumerate(stages)}
+    avg_clean = {name: statistics.mean(s[i] for s in clean_stage_ms) for i, (name, _) in enumerate(stages)}
     gemm_achieved = flop_step / (avg["gemm"] * 1e-3) / 1e12
     # algorithmic bytes of the launches as configured: a cast moves 2 B in and 1 B of codes out
     # per element (+1 B with the transposed copy); the W cast moves from the cast launch into
@@ -267,11 +302,42 @@ def run_ours(args, rank, world, local_rank):
                    + (0 if st.fused_norm else 2 * nums["params"]))
     cast_gbs = cast_bytes / (avg["cast"] * 1e-3) / 1e9
     adamw_gbs = adamw_bytes / (avg["adamw"] * 1e-3) / 1e9
+    cast_gbs_clean = cast_bytes / (avg_clean["cast"] * 1e-3) / 1e9
+    adamw_gbs_clean = adamw_bytes / (avg_clean["adamw"] * 1e-3) / 1e9
     fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
     hbm = peaks["hbm_gbs"]
-    # the committed counters are of the default configuration's GEMM launch
-    default_cfg = (args.recipe == "delayed" and not args.transposes and not args.separate_norm_pass)
-    traffic = gemm_traffic_from_profile(wl.name) if default_cfg else None
+    # DRAM traffic per launch from the committed ncu counters, when they were taken on the
+    # current sources of that kernel and on this configuration
+    default_cfg = (args.recipe == "delayed" and not args.transposes and not args.separate_norm_pass
+                   and not args.separate_weight_cast and not args.separate_scale_update)
+    traffic = {k: (measured_traffic(wl.name, k) if default_cfg else None)
+               for k in ("gemm", "cast", "adamw")}
+    gemm_name = ("k_fp8_gemm<true> block-scaled" if st.recipe == "mxfp8" else "k_fp8_gemm") + \
+        " (one grouped launch: every fprop, dgrad, wgrad)"
+    cast_name = ("k_mx_cast" if st.recipe == "mxfp8" else
+                 "k_current_amax + k_cast_rowmajor" if st.recipe == "current" else
+                 "k_cast_transpose_amax" if st.transposes else "k_cast_rowmajor") + " (cast launch)"
+    adamw_name = "k_adamw_update" + ("<cast>" if st.fused_wcast else "") + \
+        ("" if st.fused_norm else " + k_adamw_sumsq")
+    rooflines = [
+        {"kernel": gemm_name, "bound": "tensor", "achieved": round(gemm_achieved, 1),
+         "peak": round(fp8_peak, 1), "unit": "TFLOP/s", "frac": round(gemm_achieved / fp8_peak, 4),
+         "traffic": traffic["gemm"], "work_per_launch": flop_step,
+         "ms_per_launch": round(avg["gemm"], 5),
+         "frac_of_datasheet_fp8": round(gemm_achieved / DATASHEET_FP8_TFLOPS, 4),
+         "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {FP8_OVER_BF16} "
+                        f"(nominal FP8/BF16 ratio); datasheet dense FP8 {DATASHEET_FP8_TFLOPS} TFLOP/s"},
+        {"kernel": cast_name, "bound": "hbm", "achieved": round(cast_gbs, 1), "peak": hbm,
+         "unit": "GB/s", "frac": round(cast_gbs / hbm, 4), "traffic": traffic["cast"],
+         "work_per_launch": cast_bytes, "ms_per_launch": round(avg["cast"], 5),
+         "achieved_clean_l2": round(cast_gbs_clean, 1), "frac_clean_l2": round(cast_gbs_clean / hbm, 4),
+         "peak_source": f"{peaks['source']} HBM copy"},
+        {"kernel": adamw_name, "bound": "hbm", "achieved": round(adamw_gbs, 1), "peak": hbm,
+         "unit": "GB/s", "frac": round(adamw_gbs / hbm, 4), "traffic": traffic["adamw"],
+         "work_per_launch": adamw_bytes, "ms_per_launch": round(avg["adamw"], 5),
+         "achieved_clean_l2": round(adamw_gbs_clean, 1), "frac_clean_l2": round(adamw_gbs_clean / hbm, 4),
+         "peak_source": f"{peaks['source']} HBM copy"},
+    ]
 
     for g, _ in graphs:
         del g
@@ -325,18 +391,16 @@ def run_ours(args, rank, world, local_rank):
                    "operands": "K-major only (transposed FP8 copies written by the casts)"
                                if st.transposes else "no transposed copies (wgrad A, B and fprop B "
                                                      "read MN-major by tcgen05)",
-                   "l2": "flushed before every timed step (256 MiB write)"},
+                   "l2": "flushed before every timed step (256 MiB write; its dirty lines are "
+                         "written back during the step); kernels.clean_l2: a 256 MiB read after "
+                         "the write"},
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": nums["h2d"],
                 "d2h_bytes_per_step": nums["d2h"], "ms_per_step": round(e2e_total / n_e2e, 4),
                 "how": "pinned host X, dY in and Y, dX out every step; copies overlapped with "
                        "the previous/next step's kernels on separate streams"},
         "gpu_launches": args.steps * st.kernels_per_step(),
-        "roofline": {"kernel": ("k_fp8_gemm<true> block-scaled" if st.recipe == "mxfp8" else "k_fp8_gemm")
-                               + " (one grouped launch: every fprop, dgrad, wgrad)", "bound": "tensor",
-                     "achieved": round(gemm_achieved, 1), "peak": round(fp8_peak, 1),
-                     "unit": "TFLOP/s", "frac": round(gemm_achieved / fp8_peak, 4),
-                     "traffic": traffic,
-                     "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {FP8_OVER_BF16} (nominal FP8/BF16 ratio)"},
+        "roofline": dict(rooflines[0]),
+        "rooflines": rooflines,
         "kernels": {
             "stage_ms": {n: round(a, 4) for n, a in avg.items()},
             "gemm_tflops": round(gemm_achieved, 1),
@@ -344,13 +408,23 @@ def run_ours(args, rank, world, local_rank):
             "cast_bytes_per_step": cast_bytes, "adamw_bytes_per_step": adamw_bytes,
             "adamw_gbs": round(adamw_gbs, 1), "adamw_frac_of_hbm": round(adamw_gbs / hbm, 4),
             "hbm_peak_gbs": hbm, "peak_source": peaks["source"],
+            "clean_l2": {"steps": n_clean,
+                         "stage_ms": {n: round(a, 4) for n, a in avg_clean.items()},
+                         "ms_per_step": round(statistics.mean(clean_step_ms), 4),
+                         "cast_gbs": round(cast_gbs_clean, 1),
+                         "cast_frac_of_hbm": round(cast_gbs_clean / hbm, 4),
+                         "adamw_gbs": round(adamw_gbs_clean, 1),
+                         "adamw_frac_of_hbm": round(adamw_gbs_clean / hbm, 4),
+                         "gemm_tflops": round(flop_step / (avg_clean["gemm"] * 1e-3) / 1e12, 1),
+                         "how": "256 MiB write then 256 MiB read before each step (outside the "
+                                "events): L2 holds clean lines, nothing is written back during the step"},
         },
         "clocks": clocks.summary(),
         "wall_s_timed_region": round(wall, 3),
     }
     if rank == 0 and world == 1 and nl == 1 and not args.no_cpu_baseline:
         b0 = (batches[0][0][0], batches[0][1][0])
-        result["cpu_baseline"] = cpu_baseline(st, wl, nums, b0, frac_rows=1024)
+        result["cpu_baseline"] = cpu_baseline(st, wl, nums, b0)
     return result
 
 
@@ -483,63 +557,122 @@ def gpu_uuid(dev, fallback):
     return s if s.startswith("GPU-") else "GPU-" + s
 
 
-def gemm_traffic_from_profile(workload):
-    """DRAM bytes (read + write) per GEMM launch from the committed ncu summary, or None when the
-    summary is missing or was taken on different kernel sources."""
-    import re
-    path = os.path.join(ROOT, "profiles", f"k_fp8_gemm_{workload}.md")
-    if not os.path.exists(path):
-        return None
-    text = open(path).read()
-    t = re.search(r"traffic_bytes_per_launch[^:]*:\s*(\d+)", text)
-    sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text)
-    if not t or not sha or sha.group(1) != kernel_source_sha():
-        return None
-    return int(t.group(1))
+# source files whose change invalidates a kernel's committed DRAM counters
+KERNEL_SOURCES = {
+    "gemm": ("gemm_tcgen05.cuh", "ptx.cuh", "fp8train.cu"),
+    "cast": ("cast_transpose_amax.cuh", "scale_update.cuh", "ptx.cuh", "fp8train.cu"),
+    "adamw": ("fused_adamw.cuh", "ptx.cuh", "fp8train.cu"),
+}
 
 
-def kernel_source_sha(files=("gemm_tcgen05.cuh", "ptx.cuh")):
-    """Hash of the GEMM kernel's source files (what the committed counters were taken on)."""
+def kernel_source_sha(kernel):
+    """Hash of the sources a kernel's launches are built from."""
     import hashlib
     h = hashlib.sha256()
     d = os.path.join(ROOT, "optimizer_fp8_cast_b200", "csrc")
-    for f in files:
+    for f in KERNEL_SOURCES[kernel]:
         with open(os.path.join(d, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
 
 
+def measured_traffic(workload, kernel):
+    """DRAM bytes (read + write) per launch of a kernel of the default step, from the ncu counters
+    committed in profiles/traffic_<workload>.json, or None when there are none or they were taken
+    on other sources of that kernel."""
+    path = os.path.join(ROOT, "profiles", f"traffic_{workload}.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        entry = json.load(f).get("kernels", {}).get(kernel)
+    if not entry or entry.get("source_sha") != kernel_source_sha(kernel):
+        return None
+    return int(entry["dram_bytes_per_launch"])
+
+
 # ----------------------------------------------------------------------------- CPU oracle
-def oracle_sample_step(oracle, host, wl, rows_div):
-    """Every stage of one step on a 1/rows_div row sample of the workload (CPU oracle).
-    Returns (seconds, GEMM FLOP of the sample)."""
+def cpu_host():
+    """The host the CPU figures were taken on."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "nproc": os.cpu_count()}
+
+
+CPU_STAGE_S = 1.5      # oracle seconds per stage and thread setting, about
+
+
+def _calibrated(run, unit_max, budget_s, probe_units):
+    """Run `run(units)` once on a probe, then on as many units as fill about budget_s (at most
+    unit_max); returns (seconds, units) of the second run."""
+    t0 = time.perf_counter()
+    run(probe_units)
+    dt = max(time.perf_counter() - t0, 1e-6)
+    units = int(min(unit_max, max(probe_units, probe_units * budget_s / dt)))
+    t0 = time.perf_counter()
+    run(units)
+    return time.perf_counter() - t0, units
+
+
+def oracle_stage_rates(oracle, host, wl, threads, budget_s=CPU_STAGE_S):
+    """The CPU oracle, stage by stage, on samples of the workload sized to about budget_s each:
+    casts of X (E4M3) and dY (E5M2) rows, the three GEMMs at seeded output positions, the scale
+    update of X, W and dY (history H), AdamW (norm pass and update) on a slice of the parameters.
+    Returns the rates and what each sample was."""
     import numpy as np
+    oracle.set_threads(threads)
     _, fin, fout = wl.layers[0]
     T = wl.tokens
-    rt, rw = max(1, T // rows_div), max(1, fin // rows_div)
-    t0 = time.perf_counter()
-    # casts of the sampled rows (q, q^T of the sample, amax, counters)
-    oracle.cast_transpose_amax(host["X"][:rt], oracle.E4M3, 1.0)
-    oracle.cast_transpose_amax(host["W"][:rw], oracle.E4M3, 1.0)
-    oracle.cast_transpose_amax(host["dY"][:rt], oracle.E5M2, 1.0)
-    # GEMMs: rt (resp. rw) full output rows each
-    oracle.gemm(host["Xq"][:rt], 0, host["WqT"], 0, 1.0, 1.0)
-    oracle.gemm(host["dYq"][:rt], 1, host["Wq"], 0, 1.0, 1.0)
-    oracle.gemm(host["XqT"][:rw], 0, host["dYqT"], 1, 1.0, 1.0)
-    # scale update (whole: it is tiny) and AdamW on the sample's share of the parameters
-    hist = np.zeros((3, wl.history_len), np.float32)
-    sc = np.ones(3, np.float32)
-    si = np.ones(3, np.float32)
-    oracle.scale_update(np.ones(3, np.float32), hist, [448.0, 448.0, 57344.0], 0, 0, sc, si)
-    n = max(1, fin * fout // rows_div)
-    p = [host["master"][:n].copy()]
-    m = [np.zeros(n, np.float32)]
-    v = [np.zeros(n, np.float32)]
-    w = [np.zeros(n, np.uint16)]
-    oracle.fused_adamw(p, m, v, [host["dW"][:n]], w, dict(wl.adamw, step=1))
-    dt = time.perf_counter() - t0
-    flop = 2 * (rt * fout * fin + rt * fin * fout + rw * fout * T)   # the sampled GEMM rows
-    return dt, flop
+    out = {}
+    # casts: 3 B per element (2 read, 1 code written), as the GPU cast's algorithmic bytes
+    def cast(rows):
+        oracle.cast_transpose_amax(host["X"][:rows], oracle.E4M3, 1.0, True, False)
+        oracle.cast_transpose_amax(host["dY"][:rows], oracle.E5M2, 1.0, True, False)
+    dt, rows = _calibrated(cast, T, budget_s, 4)
+    out["cast"] = {"gbs": 3 * rows * (fin + fout) / dt / 1e9, "sample": f"{rows} rows of X and dY"}
+    # GEMMs: n outputs of each (fprop K = in, dgrad K = out, wgrad K = tokens)
+    rng = np.random.default_rng(7)
+    gemms = ((host["Xq"], 0, host["WqT"], 0, fin), (host["dYq"], 1, host["Wq"], 0, fout),
+             (host["XqT"], 0, host["dYqT"], 1, T))
+    def gemm(n):
+        for A, af, B, bf, _ in gemms:
+            oracle.gemm_at(A, af, B, bf, 1.0, 1.0, rng.integers(0, A.shape[0], n),
+                           rng.integers(0, B.shape[0], n))
+    dt, n = _calibrated(gemm, 1 << 22, budget_s, 8 * max(1, threads))
+    out["gemm"] = {"tflops": 2 * n * (fin + fout + T) / dt / 1e12,
+                   "sample": f"{n} outputs of each of the three GEMMs"}
+    # scale update of the three tensors (median of 9)
+    times = []
+    for _ in range(9):
+        hist = np.zeros((3, wl.history_len), np.float32)
+        sc, si = np.ones(3, np.float32), np.ones(3, np.float32)
+        t0 = time.perf_counter()
+        oracle.scale_update(np.ones(3, np.float32), hist, [448.0, 448.0, 57344.0], 0, 0, sc, si)
+        times.append(time.perf_counter() - t0)
+    out["scale_update"] = {"us": statistics.median(times) * 1e6, "sample": f"3 tensors, H = {wl.history_len}"}
+    # AdamW: norm pass (2 B/param) + update (28 B/param)
+    def adamw(n):
+        oracle.fused_adamw([host["master"][:n].copy()], [np.zeros(n, np.float32)],
+                           [np.zeros(n, np.float32)], [host["dW"][:n]], [np.zeros(n, np.uint16)],
+                           dict(wl.adamw, step=1))
+    dt, n = _calibrated(adamw, host["master"].size, budget_s, 1 << 16)
+    out["adamw"] = {"gbs": 30 * n / dt / 1e9, "sample": f"{n} parameters"}
+    return out
+
+
+def oracle_step_value(rates, nums, flop_step):
+    """Step throughput (TFLOP/s) the measured stage rates give for one whole step."""
+    t = (nums["cast_bytes"] // 4 * 3 / (rates["cast"]["gbs"] * 1e9)
+         + flop_step / (rates["gemm"]["tflops"] * 1e12)
+         + rates["scale_update"]["us"] * 1e-6
+         + 30 * nums["params"] / (rates["adamw"]["gbs"] * 1e9))
+    return flop_step / t / 1e12, t
 
 
 def oracle_output_sample_step(oracle, host, wl, n_out, rng):
@@ -564,7 +697,7 @@ def oracle_output_sample_step(oracle, host, wl, n_out, rng):
     sc = np.ones(3, np.float32)
     si = np.ones(3, np.float32)
     oracle.scale_update(np.ones(3, np.float32), hist, [448.0, 448.0, 57344.0], 0, 0, sc, si)
-    n = 16 * n_out
+    n = min(16 * n_out, host["master"].size)
     oracle.fused_adamw([host["master"][:n].copy()], [np.zeros(n, np.float32)], [np.zeros(n, np.float32)],
                        [host["dW"][:n]], [np.zeros(n, np.uint16)], dict(wl.adamw, step=1))
     return time.perf_counter() - t0, flop
@@ -582,13 +715,26 @@ def host_copies(st, batch):
                 dW=bf16_bits(L.dW).reshape(-1))
 
 
-def cpu_baseline(st, wl, nums, batch, frac_rows):
+def cpu_baseline(st, wl, nums, batch):
     import oracle
     host = host_copies(st, batch)
-    dt, flop = oracle_sample_step(oracle, host, wl, frac_rows)
-    return {"value": round(flop / dt / 1e12, 9), "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"every stage on 1/{frac_rows} of its rows ({flop / 1e9:.3f} GFLOP of GEMM "
-                      f"work, {dt:.1f} s), single-threaded C oracle on the host"}
+    flop_step = 3 * sum(nums["gemm_flop"])
+    t0 = time.perf_counter()
+    one = oracle_stage_rates(oracle, host, wl, 1)
+    n_all = oracle.set_threads(0)
+    every = oracle_stage_rates(oracle, host, wl, n_all)
+    spent = time.perf_counter() - t0
+    v1, t1 = oracle_step_value(one, nums, flop_step)
+    va, ta = oracle_step_value(every, nums, flop_step)
+    stages = {k: {"one_thread": {m: (round(x, 6) if isinstance(x, float) else x) for m, x in one[k].items()},
+                  "all_threads": {m: (round(x, 6) if isinstance(x, float) else x) for m, x in every[k].items()}}
+              for k in one}
+    return {"value": round(va, 9), "unit": UNIT, "cores": n_all, "kind": "oracle",
+            "sample": f"each stage on a sample of about {CPU_STAGE_S} s per thread setting "
+                      f"({spent:.0f} s in all); value = the step's GEMM FLOP over the whole-step "
+                      f"time the {n_all}-thread stage rates give ({ta:.1f} s)",
+            "host": cpu_host(), "one_thread": {"value": round(v1, 9), "step_s": round(t1, 2)},
+            "all_threads_step_s": round(ta, 2), "stages": stages}
 
 
 REFERENCE_BUDGET_S = 90.0       # the reference arm's warm-up plus timed steps, about
@@ -616,11 +762,13 @@ def run_reference(args):
     host["master"] = W.float().numpy().reshape(-1)
     host["dW"] = synth.bf16_bits(torch.randn(fin * fout, generator=torch.Generator().manual_seed(1)).to(torch.bfloat16))
     host = {k: np.ascontiguousarray(v) for k, v in host.items()}
+    threads = oracle.set_threads(0)          # every host core
     # size each step's sample so that warm-up plus timed steps take about REFERENCE_BUDGET_S
     rng = np.random.default_rng(0)
-    probe, _ = oracle_output_sample_step(oracle, host, wl, 64, rng)
+    probe_n = 64 * threads
+    probe, _ = oracle_output_sample_step(oracle, host, wl, probe_n, rng)
     per_step = REFERENCE_BUDGET_S / max(1, args.steps + args.warmup)
-    n_out = int(min(16384, max(8, 64 * per_step / max(probe, 1e-6))))
+    n_out = int(min(1 << 20, max(8, probe_n * per_step / max(probe, 1e-6))))
     for _ in range(args.warmup):
         oracle_output_sample_step(oracle, host, wl, n_out, rng)
     times, flops = [], []
@@ -632,7 +780,7 @@ def run_reference(args):
     value = sum(flops) / total / 1e12
     sample = (f"every stage on a sample per step: casts of one row of X, W, dY; each GEMM at {n_out} "
               f"seeded outputs ({flops[0] / 1e9:.3f} GFLOP); scale update; AdamW on {16 * n_out} "
-              f"parameters; single-threaded C oracle")
+              f"parameters; C oracle on {threads} host threads")
     return {
         "metric": METRIC, "value": round(value, 9), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 3),
@@ -641,8 +789,8 @@ def run_reference(args):
         "config": {"workload": wl.name, "tokens": wl.tokens, "in_features": fin,
                    "out_features": fout, "history_len": wl.history_len},
         "impl": "reference",
-        "cpu_baseline": {"value": round(value, 9), "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": sample},
+        "cpu_baseline": {"value": round(value, 9), "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample, "host": cpu_host()},
         "e2e": {"value": round(value, 9), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
         "gpu_launches": 0,

@@ -140,6 +140,10 @@ constexpr unsigned kTicketAbort = 1u << 16;
 // atomics included, is issued; `aborted` is the same for every thread of the CTA.
 __device__ __forceinline__ void last_cta_update(const Group& g, bool aborted) {
   __shared__ int s_last, s_complete;
+  const int warp = threadIdx.x >> 5;
+  // every CTA pulls its warps' scale state (a few KB) into its SM's L1 ahead of its ticket, so
+  // the CTA that turns out to be last does not wait for HBM or L2 there
+  if (warp < g.n) scale::warp_prefetch_state(g.t[warp].hist, g.H, g.t[warp].scale);
   __threadfence();                                 // this CTA's amax atomics before its ticket
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -153,7 +157,6 @@ __device__ __forceinline__ void last_cta_update(const Group& g, bool aborted) {
   // a launch whose own waits expired leaves the scale state alone (its amax may be incomplete);
   // an expired wait of any other launch does not matter here
   const bool ok = s_complete != 0;
-  const int warp = threadIdx.x >> 5;
   if (ok && warp < g.n) {
     const Tensor& T = g.t[warp];
     scale::warp_update(reinterpret_cast<float*>(T.amax_bits), T.hist, g.H,

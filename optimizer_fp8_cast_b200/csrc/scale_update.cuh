@@ -28,6 +28,17 @@ __device__ __forceinline__ float next_scale(uint32_t rep, float fmax, int margin
   return s;
 }
 
+// Pull a tensor's history and scale into this SM's L1 (non-binding prefetches, one 128-byte
+// line per lane and step). Kernels that finish with an update issue it ahead of their ticket, so
+// the CTA that turns out to be last reads its state from L1; nothing but that update writes these
+// words during the launch, and L1 holds no older copy of them (it starts each launch empty).
+__device__ __forceinline__ void warp_prefetch_state(const float* h, int H, const float* scale) {
+  const int lane = threadIdx.x & 31;
+  for (int i = 32 * lane; i < H; i += 32 * 32)
+    asm volatile("prefetch.global.L1 [%0];" ::"l"(h + i));
+  if (lane == 0) asm volatile("prefetch.global.L1 [%0];" ::"l"(scale));
+}
+
 // The same update for one tensor, done by one warp (used inside other kernels once their amax
 // is complete). The roll goes from the top down in chunks of 32 x kPer entries: every lane
 // reads its kPer entries (all loads in flight at once), the warp synchronises, then writes them
@@ -61,7 +72,7 @@ __device__ __forceinline__ void warp_update(float* amax, float* h, int H, float 
   if (lane == 0) {
     const uint32_t rep = algo_max ? m : (__float_as_uint(a) & 0x7FFFFFFFu);
     h[0] = a;
-    const float s = next_scale(rep, fmax, margin, *reinterpret_cast<volatile float*>(scale));
+    const float s = next_scale(rep, fmax, margin, *scale);
     *scale = s;
     *scale_inv = __fdiv_rn(1.0f, s);
     *amax = 0.0f;
