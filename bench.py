@@ -422,6 +422,13 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clocks.summary(),
         "wall_s_timed_region": round(wall, 3),
     }
+    if world == 1 and nl == 1 and not args.no_comparator:
+        _, fin, fout = wl.layers[0]
+        result["comparator"] = {
+            "what": "torch._scaled_mm (cuBLAS FP8) vs this library's fp8_gemm, the step's three GEMM "
+                    "shapes with K-major E4M3 operands, back-to-back launches, L2 warm; not the step",
+            "shapes": gemm_comparator(fp8, dev, [(wl.tokens, fout, fin), (wl.tokens, fin, fout),
+                                                 (fin, fout, wl.tokens)])}
     if rank == 0 and world == 1 and nl == 1 and not args.no_cpu_baseline:
         b0 = (batches[0][0][0], batches[0][1][0])
         result["cpu_baseline"] = cpu_baseline(st, wl, nums, b0)
@@ -555,6 +562,39 @@ def gpu_uuid(dev, fallback):
         return fallback
     s = str(u)
     return s if s.startswith("GPU-") else "GPU-" + s
+
+
+def gemm_comparator(fp8, dev, shapes, seconds=0.3):
+    """cuBLAS FP8 (torch._scaled_mm, E4M3 x E4M3 -> BF16, unit scales) beside this library's GEMM
+    on the same shapes and K-major operands, back-to-back launches (L2 warm), each timed for about
+    `seconds`. A comparator only: nothing on the measured path calls a library GEMM."""
+    import torch
+    out = []
+    one_t = torch.ones((), device=dev)
+    one = torch.ones(1, device=dev)
+    for M, N, K in shapes:
+        A = torch.randint(0, 120, (M, K), dtype=torch.uint8, device=dev)
+        B = torch.randint(0, 120, (N, K), dtype=torch.uint8, device=dev)
+        D = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        a8, b8 = A.view(torch.float8_e4m3fn), B.view(torch.float8_e4m3fn)
+        row = {"M": M, "N": N, "K": K}
+        for name, fn in (("ours", lambda: fp8.fp8_gemm_multi([dict(A=A, a_fmt=0, B=B, b_fmt=0, a_scale_inv=one,
+                                                                     b_scale_inv=one, D=D)])),
+                         ("cublas", lambda: torch._scaled_mm(a8, b8.t(), scale_a=one_t, scale_b=one_t,
+                                                             out_dtype=torch.bfloat16))):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            n = max(10, int(seconds / (2.0 * M * N * K / 3.0e15)))
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(n):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            row[name + "_tflops"] = round(2.0 * M * N * K * n / (e0.elapsed_time(e1) * 1e-3) / 1e12, 1)
+        out.append(row)
+    return out
 
 
 # source files whose change invalidates a kernel's committed DRAM counters
@@ -807,6 +847,8 @@ def main(argv=None):
                     help="linear4096_t8192 (default), linear256_t512, block7b_t16384, "
                          "adamw4e9_512t, stress1024_t2048")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-comparator", action="store_true",
+                    help="skip the cuBLAS FP8 comparator timing of the step's GEMM shapes")
     ap.add_argument("--eager", action="store_true", help="time eager launches, not CUDA graphs")
     ap.add_argument("--recipe", choices=("delayed", "current", "mxfp8"), default="delayed",
                     help="current: each scale from its own tensor's amax (an extra read); "
