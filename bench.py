@@ -367,6 +367,7 @@ def run_ours(args, rank, world, local_rank):
     e2e_value = throughput(flop_step, n_e2e, world, e2e_total)
 
     shapes = {lname: [fin, fout] for lname, fin, fout in wl.layers}
+    clk = clocks.summary()             # step_kcycles = ms per step x median SM MHz (clock-free)
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
@@ -419,7 +420,8 @@ def run_ours(args, rank, world, local_rank):
                          "how": "256 MiB write then 256 MiB read before each step (outside the "
                                 "events): L2 holds clean lines, nothing is written back during the step"},
         },
-        "clocks": clocks.summary(),
+        "clocks": clk,
+        "step_kcycles": (round(total_ms / args.steps * clk["sm_mhz"], 1) if clk.get("sm_mhz") else None),
         "wall_s_timed_region": round(wall, 3),
     }
     if world == 1 and nl == 1 and not args.no_comparator:

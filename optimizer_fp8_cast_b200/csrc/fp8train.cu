@@ -657,6 +657,8 @@ fp8t_status fp8_mx_cast_multi(const fp8t_mx_cast_tensor* tensors, int32_t n_tens
   DeviceInfo* dev = nullptr;
   fp8t_status st = current_device(&dev);
   if (st != FP8T_OK) return st;
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(FP8T_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   using namespace fp8t::mx;
   static thread_local Group group;
   for (int32_t b0 = 0; b0 < n_tensors; b0 += kMaxTensors) {
@@ -667,7 +669,15 @@ fp8t_status fp8_mx_cast_multi(const fp8t_mx_cast_tensor* tensors, int32_t n_tens
     for (int32_t i = b0; i < b1; ++i) {
       const fp8t_mx_cast_tensor& t = tensors[i];
       Tensor& T = group.t[i - b0];
-      T.x = static_cast<const uint4*>(t.x_bf16);
+      // BF16 [rows][cols] read as 128-row x 64-column boxes (128 bytes per row: 128-byte swizzle)
+      cuuint64_t dims[2] = {static_cast<cuuint64_t>(t.cols), static_cast<cuuint64_t>(t.rows)};
+      cuuint64_t strides[1] = {static_cast<cuuint64_t>(t.cols) * 2};
+      cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kTile)};
+      cuuint32_t es[2] = {1, 1};
+      CUresult r = fn(&T.x_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(t.x_bf16),
+                      dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (r != CUDA_SUCCESS) return fail(FP8T_ERR_CUDA, "cuTensorMapEncodeTiled (MX cast input) failed (%d)", (int)r);
       T.q_row = static_cast<uint8_t*>(t.q_row);
       T.sf_row = static_cast<uint8_t*>(t.scales_row);
       T.q_col = static_cast<uint8_t*>(t.q_col);

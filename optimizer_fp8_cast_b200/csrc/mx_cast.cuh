@@ -13,13 +13,17 @@
 // rows (M or N) x 4 blocks (128 K values): byte (i % 32) * 16 + (i / 32) * 4 + kb holds row i,
 // block kb, which is the order the tensor-core scale copy (tcgen05.cp 32x128b, replicated to
 // the four lane quarters) expects; atoms are stored [MN / 128][K / 128].
-// A CTA reads its tiles into a double-buffered shared tile with 16-byte asynchronous copies (the
-// next tile's copies are in flight while the current one is quantised; 16-byte chunk c of row r
-// is stored at c ^ (r % 8), so that the row-wise and the column-wise reads are free of bank
-// conflicts),
-// quantises the row-wise blocks
-// straight to global memory, the column-wise blocks into a staged tile that it then writes out
-// row by row, and writes each atom with 16-byte stores.
+// Persistent CTAs; thread 0 keeps two tiles in flight: each tile arrives as two TMA boxes of
+// 128 rows x 64 columns (128-byte swizzle: 16-byte chunk c of a row's 128 bytes at c ^ (row % 8))
+// into a double buffer, completion on one mbarrier per buffer. Then, in parallel,
+//   warps 0-3 quantise the column-wise blocks: a thread takes 4 adjacent columns of one block of
+//     32 rows (32 eight-byte shared loads), forms their four scales and stores each row's four
+//     codes as one 4-byte word into a staged code tile;
+//   warps 4-7 quantise the row-wise blocks straight to global memory: a quarter-warp takes the
+//     same block of 8 consecutive rows, so its shared loads hit 8 different bank groups;
+// and after a barrier all threads write the staged column-wise codes out row by row with 16-byte
+// stores, and the two scale atoms. Every wait on an mbarrier is bounded: on expiry the CTA
+// records the timeout in the device error word, stops, and waits (bounded) for its loads.
 #pragma once
 
 #include "ptx.cuh"
@@ -30,10 +34,12 @@ namespace mx {
 constexpr int kTile = 128;
 constexpr int kThreads = 256;
 constexpr int kMaxTensors = 8;
-constexpr int kSmemBytes = 2 * kTile * kTile * 2 + kTile * kTile + 2 * 512 + 128;
+constexpr int kHalfBytes = kTile * 64 * 2;                 // one 128-row x 64-column BF16 box
+constexpr int kXBytes = 2 * kHalfBytes;                    // one 128 x 128 BF16 tile
+constexpr int kSmemBytes = 2 * kXBytes + kTile * kTile + 2 * 512 + 64 + 1024 /*alignment*/;
 
-struct Tensor {
-  const uint4* x;                  // BF16 [rows][cols]
+struct alignas(64) Tensor {
+  CUtensorMap x_map;               // BF16 [rows][cols], 64 x 128 boxes, 128-byte swizzle
   uint8_t* q_row;                  // codes, blocks along rows (may be null)
   uint8_t* sf_row;                 // atoms [rows/128][cols/128]
   uint8_t* q_col;                  // codes, blocks down columns (may be null)
@@ -42,7 +48,7 @@ struct Tensor {
   int32_t fmt;
 };
 
-struct Group {
+struct alignas(64) Group {
   Tensor t[kMaxTensors];
   int32_t n;
   int64_t total_tiles;
@@ -78,10 +84,10 @@ __device__ __forceinline__ uint32_t q4(uint32_t w0, uint32_t w1, float inv) {
   return r;
 }
 
-// position of 16-byte chunk c16 of tile row `row` in the swizzled BF16 tile (uint4 units)
-__device__ __forceinline__ int xchunk(int row, int c16) { return row * 16 + (c16 ^ (row & 7)); }
-// position of BF16 element (row, col) of the tile (uint16 units)
-__device__ __forceinline__ int xelem(int row, int col) { return xchunk(row, col >> 3) * 8 + (col & 7); }
+// Byte offset of BF16 element (row, col) in a tile as the two swizzled TMA boxes lay it out.
+__device__ __forceinline__ uint32_t xoff(int row, int col) {
+  return (col >> 6) * kHalfBytes + row * 128 + ((((col >> 3) & 7) ^ (row & 7)) << 4) + (col & 7) * 2;
+}
 
 __device__ __forceinline__ int tensor_of(const Group& g, int64_t tile) {
   int ti = 0;
@@ -89,57 +95,122 @@ __device__ __forceinline__ int tensor_of(const Group& g, int64_t tile) {
   return ti;
 }
 
-// Issue the 16-byte copies of one 128 x 128 BF16 tile (128 rows x 256 bytes) into xs.
-__device__ __forceinline__ void prefetch_tile(const Group& g, int64_t tile, uint16_t* xs) {
+__device__ __forceinline__ void issue_tile(const Group& g, int64_t tile, uint32_t dst, uint32_t bar) {
   const Tensor& T = g.t[tensor_of(g, tile)];
   const int64_t local = tile - T.tile_start;
-  const int64_t r0 = (local / T.tiles_c) * kTile, c0 = (local % T.tiles_c) * kTile;
-#pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    const int v = u * kThreads + threadIdx.x, row = v >> 4, c16 = v & 15;
-    cp_async_16(smem_u32(reinterpret_cast<uint4*>(xs) + xchunk(row, c16)),
-                T.x + ((r0 + row) * T.cols + c0) / 8 + c16);
-  }
+  const int32_t r0 = static_cast<int32_t>((local / T.tiles_c) * kTile);
+  const int32_t c0 = static_cast<int32_t>((local % T.tiles_c) * kTile);
+  mbar_arrive_expect_tx(bar, kXBytes);
+  tma_load_2d(dst, &T.x_map, c0, r0, bar);
+  tma_load_2d(dst + kHalfBytes, &T.x_map, c0 + 64, r0, bar);
 }
 
-__global__ void __launch_bounds__(kThreads) k_mx_cast(const __grid_constant__ Group g) {
+__device__ __forceinline__ uint8_t scale_code(uint32_t m, int X) {
+  return m > 0x7F80u ? 0xFF : static_cast<uint8_t>(X + 127);
+}
+
+__global__ void __launch_bounds__(kThreads, 2) k_mx_cast(const __grid_constant__ Group g) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);
-  // [2][128][128] BF16 tiles at smem and smem + kXBytes
-  constexpr int kXBytes = kTile * kTile * 2;
-  auto xbuf = [&](int b) { return reinterpret_cast<uint16_t*>(smem + b * kXBytes); };
-  uint8_t* qs = smem + 2 * kTile * kTile * 2;                       // [128][128] column-wise codes
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* xbuf = smem;                                             // [2][2 boxes][128][128 B]
+  uint8_t* qs = smem + 2 * kXBytes;                                 // [128][128] column-wise codes
   uint8_t* atom_r = qs + kTile * kTile;                             // 512 B
   uint8_t* atom_c = atom_r + 512;                                   // 512 B
-  const int tid = threadIdx.x;
+  uint64_t* full = reinterpret_cast<uint64_t*>(atom_c + 512);       // 2 mbarriers
+  __shared__ int s_abort;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t stride = gridDim.x;
+  uint32_t pending = 0, pending_ph = 0;      // thread 0: loads not yet consumed, their phases
 
-  if (static_cast<int64_t>(blockIdx.x) < g.total_tiles) prefetch_tile(g, blockIdx.x, xbuf(0));
-  cp_async_commit();
-  int k = 0;
-  for (int64_t tile = blockIdx.x; tile < g.total_tiles; tile += gridDim.x, ++k) {
+  if (tid == 0) {
+    mbar_init(smem_u32(&full[0]), 1);
+    mbar_init(smem_u32(&full[1]), 1);
+    fence_mbar_init();
+    s_abort = 0;
+    for (int b = 0; b < 2; ++b) {
+      const int64_t tile = blockIdx.x + b * stride;
+      if (tile < g.total_tiles) {
+        issue_tile(g, tile, smem_u32(xbuf + b * kXBytes), smem_u32(&full[b]));
+        pending |= 1u << b;
+      }
+    }
+  }
+  __syncthreads();
+  const uint64_t limit = wait_limit_ns();
+  const bool expire = expire_mode() == kExpireAll;
+
+  for (int64_t i = 0;; ++i) {
+    const int64_t tile = blockIdx.x + i * stride;
+    if (tile >= g.total_tiles) break;
+    const int buf = static_cast<int>(i & 1);
+    if (tid == 0) {
+      if (!mbar_wait(smem_u32(&full[buf]), static_cast<uint32_t>((i >> 1) & 1), limit, expire)) {
+        record_error(kErrTimeout);
+        s_abort = 1;
+      } else {
+        pending &= ~(1u << buf);
+      }
+    }
+    __syncthreads();                          // tile landed; the previous tile's outputs written
+    if (s_abort) break;
     const Tensor& T = g.t[tensor_of(g, tile)];
     const int64_t local = tile - T.tile_start;
     const int64_t r0 = (local / T.tiles_c) * kTile, c0 = (local % T.tiles_c) * kTile;
     const int emax = T.fmt == 0 ? 8 : 15;
-    uint16_t* xs = xbuf(k & 1);
+    const uint8_t* xs = xbuf + buf * kXBytes;
 
-    // ---- the next tile's copies go out; this tile's have landed
-    if (tile + gridDim.x < g.total_tiles) prefetch_tile(g, tile + gridDim.x, xbuf((k + 1) & 1));
-    cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
-
-    // ---- row-wise blocks: 128 rows x 4 blocks, two per thread
-    if (T.q_row) {
+    if (warp < 4) {
+      // ---- column-wise blocks: columns 4cq .. 4cq+3, rows 32rb .. 32rb+31
+      if (T.q_col) {
+        const int cq = lane, rb = warp, col = 4 * cq;
+        uint2 v[32];
+        uint32_t ma = 0, mb = 0;
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int j = u * kThreads + tid, row = j >> 2, b = j & 3;
-        const uint4* src = reinterpret_cast<const uint4*>(xs);
+        for (int r = 0; r < 32; ++r) {
+          v[r] = *reinterpret_cast<const uint2*>(xs + xoff(32 * rb + r, col));
+          ma = __vmaxu2(ma, v[r].x & 0x7FFF7FFFu);
+          mb = __vmaxu2(mb, v[r].y & 0x7FFF7FFFu);
+        }
+        const uint32_t m[4] = {ma & 0xFFFFu, ma >> 16, mb & 0xFFFFu, mb >> 16};
+        int X[4];
+        float inv[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          X[c] = m[c] > 0x7F80u ? 0 : block_exponent(m[c], emax);
+          inv[c] = pow2_neg(X[c]);
+        }
+        const bool nan_block = max(max(m[0], m[1]), max(m[2], m[3])) > 0x7F80u;
+#pragma unroll
+        for (int r = 0; r < 32; ++r) {
+          const float p0 = __fmul_rn(__uint_as_float(v[r].x << 16), inv[0]);
+          const float p1 = __fmul_rn(__uint_as_float(v[r].x & 0xFFFF0000u), inv[1]);
+          const float p2 = __fmul_rn(__uint_as_float(v[r].y << 16), inv[2]);
+          const float p3 = __fmul_rn(__uint_as_float(v[r].y & 0xFFFF0000u), inv[3]);
+          uint32_t c = T.fmt == 0 ? cvt_fp8x2<0>(p0, p1) | (cvt_fp8x2<0>(p2, p3) << 16)
+                                  : cvt_fp8x2<1>(p0, p1) | (cvt_fp8x2<1>(p2, p3) << 16);
+          if (nan_block) {                       // only a NaN input gives a NaN product
+            if (p0 != p0) c = (c & 0xFFFFFF00u) | 0x7Fu;
+            if (p1 != p1) c = (c & 0xFFFF00FFu) | 0x7F00u;
+            if (p2 != p2) c = (c & 0xFF00FFFFu) | 0x7F0000u;
+            if (p3 != p3) c = (c & 0x00FFFFFFu) | 0x7F000000u;
+          }
+          *reinterpret_cast<uint32_t*>(qs + (32 * rb + r) * kTile + col) = c;
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          atom_c[((col + c) & 31) * 16 + ((col + c) >> 5) * 4 + rb] = scale_code(m[c], X[c]);
+      }
+    } else if (T.q_row) {
+      // ---- row-wise blocks: a quarter-warp takes block b of 8 consecutive rows
+      const int wr = warp - 4, b = lane >> 3;
+#pragma unroll 1
+      for (int u = 0; u < 4; ++u) {
+        const int row = 32 * u + 8 * wr + (lane & 7);
         uint4 w[4];
         uint32_t m2 = 0;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          w[k] = src[xchunk(row, 4 * b + k)];
+          w[k] = *reinterpret_cast<const uint4*>(xs + xoff(row, 32 * b + 8 * k));
           m2 = __vmaxu2(m2, __vmaxu2(__vmaxu2(w[k].x & 0x7FFF7FFFu, w[k].y & 0x7FFF7FFFu),
                                      __vmaxu2(w[k].z & 0x7FFF7FFFu, w[k].w & 0x7FFF7FFFu)));
         }
@@ -169,41 +240,18 @@ __global__ void __launch_bounds__(kThreads) k_mx_cast(const __grid_constant__ Gr
         uint4* dst = reinterpret_cast<uint4*>(T.q_row + (r0 + row) * T.cols + c0 + 32 * b);
         dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
         dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
-        atom_r[(row & 31) * 16 + (row >> 5) * 4 + b] = m > 0x7F80u ? 0xFF : static_cast<uint8_t>(X + 127);
+        atom_r[(row & 31) * 16 + (row >> 5) * 4 + b] = scale_code(m, X);
       }
     }
-    // ---- column-wise blocks: 128 columns x 4 blocks of 32 rows; each thread takes a column
-    //      pair of one block: 32 four-byte reads (two BF16 each) and 32 two-byte code stores
-    if (T.q_col) {
-      const int cp = tid & 63, rb = tid >> 6, col = 2 * cp;
-      uint32_t v[32];
-      uint32_t m2 = 0;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        v[i] = *reinterpret_cast<const uint32_t*>(xs + xelem(32 * rb + i, col));
-        m2 = __vmaxu2(m2, v[i] & 0x7FFF7FFFu);
+    __syncthreads();                          // input tile consumed; staged codes, atoms complete
+    if (tid == 0) {                           // refill the buffer just consumed
+      const int64_t next = tile + 2 * stride;
+      if (next < g.total_tiles) {
+        issue_tile(g, next, smem_u32(xbuf + buf * kXBytes), smem_u32(&full[buf]));
+        pending |= 1u << buf;
+        pending_ph = (pending_ph & ~(1u << buf)) | (static_cast<uint32_t>(((i + 2) >> 1) & 1) << buf);
       }
-      const uint32_t m0 = m2 & 0xFFFFu, m1 = m2 >> 16;   // column col, column col + 1
-      const int X0 = m0 > 0x7F80u ? 0 : block_exponent(m0, emax);
-      const int X1 = m1 > 0x7F80u ? 0 : block_exponent(m1, emax);
-      const float inv0 = pow2_neg(X0), inv1 = pow2_neg(X1);
-      const bool nan_block = max(m0, m1) > 0x7F80u;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float p0 = __fmul_rn(__uint_as_float(v[i] << 16), inv0);
-        const float p1 = __fmul_rn(__uint_as_float(v[i] & 0xFFFF0000u), inv1);
-        uint32_t c = T.fmt == 0 ? cvt_fp8x2<0>(p0, p1) : cvt_fp8x2<1>(p0, p1);
-        if (nan_block) {                       // only a NaN input gives a NaN product
-          if (p0 != p0) c = (c & 0xFF00u) | 0x7Fu;
-          if (p1 != p1) c = (c & 0x00FFu) | 0x7F00u;
-        }
-        *reinterpret_cast<uint16_t*>(qs + (32 * rb + i) * kTile + col) = static_cast<uint16_t>(c);
-      }
-      atom_c[(col & 31) * 16 + (col >> 5) * 4 + rb] = m0 > 0x7F80u ? 0xFF : static_cast<uint8_t>(X0 + 127);
-      atom_c[((col + 1) & 31) * 16 + ((col + 1) >> 5) * 4 + rb] =
-          m1 > 0x7F80u ? 0xFF : static_cast<uint8_t>(X1 + 127);
     }
-    __syncthreads();                                   // staged codes and both atoms complete
     if (T.q_col) {
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
@@ -218,7 +266,11 @@ __global__ void __launch_bounds__(kThreads) k_mx_cast(const __grid_constant__ Gr
     if (tid >= 32 && tid < 64 && T.q_col)
       reinterpret_cast<uint4*>(T.sf_col + ((c0 / kTile) * (T.rows / kTile) + r0 / kTile) * 512)[tid - 32] =
           reinterpret_cast<const uint4*>(atom_c)[tid - 32];
-    __syncthreads();                                   // shared buffers free for the next tile
+  }
+  if (tid == 0) {
+    // loads still in flight after an abort must land before shared memory is released
+    for (int b = 0; b < 2; ++b)
+      if (pending & (1u << b)) mbar_wait(smem_u32(&full[b]), (pending_ph >> b) & 1u, kDrainLimitNs);
   }
 }
 
