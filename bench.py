@@ -178,7 +178,7 @@ def run_ours(args, rank, world, local_rank):
                        dev, device_step=True, fused_update=not args.separate_scale_update,
                        fused_norm=not args.separate_norm_pass,
                        fused_wcast=not args.separate_weight_cast, transposes=args.transposes,
-                       recipe=args.recipe)
+                       recipe=args.recipe, side_update=args.side_update)
     batches = [list(zip(*[synth.linear_inputs(wl, k, t, dev) for k in range(nl)])) for t in range(2)]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     sweep = torch.ones(L2_FLUSH_BYTES // 8, dtype=torch.int64, device=dev)
@@ -212,8 +212,12 @@ def run_ours(args, rank, world, local_rank):
                 st.cast_all_current(xs, dys)      # amax launch, then the grouped cast
             elif name == "cast":                  # grouped: X, W -> E4M3, dY -> E5M2
                 st.cast_all(xs, dys, update=st.fused_update)
+                if st.side_update:                # the scale update, on a side stream
+                    st.side_update_begin()
             elif name == "gemm":                  # grouped: every fprop, dgrad and wgrad
                 st.gemm_all(sumsq=st.fused_norm)
+                if st.side_update:
+                    st.side_update_end()
             elif name == "scale update":
                 st.scale_update()
             elif name == "adamw":
@@ -384,6 +388,8 @@ def run_ours(args, rank, world, local_rank):
                    "scale_update": "none (MX block scales)" if args.recipe == "mxfp8"
                                    else "none (current scaling)" if args.recipe == "current"
                                    else "separate launch" if args.separate_scale_update
+                                   else "own launch on a side stream, concurrent with the GEMMs"
+                                   if st.side_update
                                    else "in the last CTA of the cast launch",
                    "grad_sum_of_squares": "AdamW norm pass" if args.separate_norm_pass
                                           else "in the wgrad GEMM epilogue",
@@ -863,6 +869,9 @@ def main(argv=None):
                     help="run AdamW's own norm pass instead of summing dW^2 in the wgrad epilogue")
     ap.add_argument("--separate-scale-update", action="store_true",
                     help="run the scale update as its own launch instead of in the cast launch")
+    ap.add_argument("--side-update", action="store_true",
+                    help="run the scale update as its own launch on a second stream, concurrently "
+                         "with the GEMM launch, instead of in the cast launch's last CTA")
     ap.add_argument("--out", default=None, help="stress sweep: write the per-step table here")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":

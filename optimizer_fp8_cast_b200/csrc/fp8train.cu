@@ -48,6 +48,7 @@ struct DeviceInfo {
   int adamw_blocks_per_sm = 0;
   int adamw_cast_blocks_per_sm = 0;
   int gemm_clusters = 0;       // co-resident 2-CTA clusters of the GEMM kernel
+  int gemm_wide_clusters = 0;  // ... of its wide-tile form
   int gemm_mx_clusters = 0;    // ... of its MXFP8 variant
   int mx_cast_blocks_per_sm = 0;
   int cast_blocks_per_sm = 0;
@@ -88,6 +89,9 @@ fp8t_status current_device(DeviceInfo** out) {
         e = cudaFuncSetAttribute(fp8t::gemm::k_fp8_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  fp8t::gemm::kSmemBytesMX);
       if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(fp8t::gemm::k_fp8_gemm_wide, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 fp8t::gemm::kSmemBytesW);
+      if (e == cudaSuccess)
         e = cudaFuncSetAttribute(fp8t::mx::k_mx_cast, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  fp8t::mx::kSmemBytes);
       if (e != cudaSuccess) {
@@ -105,6 +109,16 @@ fp8t_status current_device(DeviceInfo** out) {
         clusters = sms / 2;
       }
       d.gemm_clusters = clusters;
+      cfg.blockDim = dim3(fp8t::gemm::kThreadsW, 1, 1);
+      cfg.dynamicSmemBytes = fp8t::gemm::kSmemBytesW;
+      clusters = 0;
+      e = cudaOccupancyMaxActiveClusters(&clusters, fp8t::gemm::k_fp8_gemm_wide, &cfg);
+      if (e != cudaSuccess || clusters < 1) {
+        (void)cudaGetLastError();
+        clusters = sms / 2;
+      }
+      d.gemm_wide_clusters = clusters;
+      cfg.blockDim = dim3(fp8t::gemm::kThreads, 1, 1);
       cfg.dynamicSmemBytes = fp8t::gemm::kSmemBytesMX;
       clusters = 0;
       e = cudaOccupancyMaxActiveClusters(&clusters, fp8t::gemm::k_fp8_gemm<true>, &cfg);
@@ -457,51 +471,95 @@ namespace {
 
 constexpr size_t kSumsqHeader = 256;    // ticket and abort words, then the partial slots
 
-// Tile lists of a grouped GEMM launch: every tile costs its problem's K / 128 k-blocks; tiles are
-// handed out longest first, each to the least-loaded cluster, and every cluster then runs its
-// tiles in index order. Launches with more tiles than the table holds keep round-robin (with
-// thousands of tiles it is balanced already).
-void build_schedule(fp8t::gemm::Group& g, int clusters) {
+// Tile lists of a grouped GEMM launch: every tile costs its problem's K / 128 k-blocks (twice
+// that for a wide tile); tiles are handed out longest first, each to the least-loaded cluster.
+// A wide launch with fewer tiles than clusters then splits tiles into their two 256-column
+// halves, one half moving to the least busy cluster, while the busiest cluster is more than half
+// a tile above it. (With at least as many tiles as clusters splitting does not pay: a half tile
+// reloads A for half the MMAs, the operand-starved pattern the wide tile avoids; measured on the
+// 4096 step, splitting there to balance the clusters left the launch no faster.) Every cluster
+// then runs its items in index order. Items are 3 * tile + part.
+// Launches with more tiles than the table holds keep round-robin (with thousands of tiles it is
+// balanced already).
+void build_schedule(fp8t::gemm::Group& g, int clusters, bool wide) {
   using namespace fp8t::gemm;
   g.scheduled = 0;
   if (g.total_tiles > kMaxSchedTiles || clusters > kMaxClusters || clusters < 2) return;
-  std::vector<std::pair<int, int>> tiles;                  // (-cost, tile)
-  tiles.reserve(g.total_tiles);
+  struct Item { int64_t cost; int tile, part; };
+  std::vector<Item> items;
+  items.reserve(g.total_tiles);
   for (int p = 0; p < g.n; ++p) {
     const int end = p + 1 < g.n ? g.p[p + 1].tile_start : g.total_tiles;
-    const int cost = (g.p[p].K + kBK - 1) / kBK;
-    for (int t = g.p[p].tile_start; t < end; ++t) tiles.emplace_back(-cost, t);
+    const int64_t cost = ((g.p[p].K + kBK - 1) / kBK) * (wide ? 2 : 1);
+    for (int t = g.p[p].tile_start; t < end; ++t) items.push_back({cost, t, 0});
   }
-  std::stable_sort(tiles.begin(), tiles.end(),
-                   [](const std::pair<int, int>& a, const std::pair<int, int>& b) { return a.first < b.first; });
+  std::stable_sort(items.begin(), items.end(),
+                   [](const Item& a, const Item& b) { return a.cost > b.cost; });
   std::vector<int64_t> load(clusters, 0);
-  std::vector<std::vector<int>> own(clusters);
-  for (const auto& t : tiles) {
+  std::vector<std::vector<Item>> own(clusters);
+  for (const auto& it : items) {
     int best = 0;
     for (int c = 1; c < clusters; ++c)
       if (load[c] < load[best]) best = c;
-    load[best] -= t.first;
-    own[best].push_back(t.second);
+    load[best] += it.cost;
+    own[best].push_back(it);
+  }
+  int n_items = g.total_tiles;
+  while (wide && g.total_tiles < clusters && n_items < kMaxSchedTiles) {
+    int hi = 0, lo = 0;
+    for (int c = 1; c < clusters; ++c) {
+      if (load[c] > load[hi]) hi = c;
+      if (load[c] < load[lo]) lo = c;
+    }
+    int pick = -1;                    // the whole tile of `hi` whose half moves best
+    for (int k = 0; k < static_cast<int>(own[hi].size()); ++k) {
+      const Item& it = own[hi][k];
+      if (it.part == 0 && 2 * (it.cost / 2) == it.cost && it.cost / 2 < load[hi] - load[lo] &&
+          (pick < 0 || it.cost > own[hi][pick].cost))
+        pick = k;
+    }
+    if (pick < 0) break;
+    Item& it = own[hi][pick];
+    const int64_t half = it.cost / 2;
+    it.cost = half;
+    it.part = 1;
+    own[lo].push_back({half, it.tile, 2});
+    load[hi] -= half;
+    load[lo] += half;
+    ++n_items;
   }
   int k = 0;
   for (int c = 0; c < clusters; ++c) {
-    std::sort(own[c].begin(), own[c].end());
+    std::sort(own[c].begin(), own[c].end(), [](const Item& a, const Item& b) {
+      return a.tile != b.tile ? a.tile < b.tile : a.part < b.part;
+    });
     g.start[c] = static_cast<uint16_t>(k);
-    for (int t : own[c]) g.order[k++] = static_cast<uint16_t>(t);
+    for (const auto& it : own[c]) g.order[k++] = static_cast<uint16_t>(3 * it.tile + it.part);
   }
   g.start[clusters] = static_cast<uint16_t>(k);
   g.scheduled = 1;
 }
 
-int64_t gemm_tiles(const fp8t_gemm_desc& d) {
+// Wide tiles (256 x 512 per pair) when every problem of the call is at least 512 wide; the choice
+// is made for the whole call, so every launch of it numbers its sum-of-squares slots alike.
+bool use_wide(const fp8t_gemm_desc* gemms, int32_t n) {
+  for (int32_t i = 0; i < n; ++i)
+    if (gemms[i].N < fp8t::gemm::kBNw) return false;
+  return true;
+}
+
+int64_t gemm_tiles(const fp8t_gemm_desc& d, bool wide) {
   using namespace fp8t::gemm;
-  return ((d.M + kBM - 1) / kBM) * ((d.N + kBN - 1) / kBN);
+  const int64_t bn = wide ? kBNw : kBN;
+  return ((d.M + kBM - 1) / kBM) * ((d.N + bn - 1) / bn);
 }
 
 int64_t sumsq_slots(const fp8t_gemm_desc* gemms, int32_t n, const int32_t* sumsq_of) {
+  const bool wide = use_wide(gemms, n);
+  const int64_t per_tile = wide ? fp8t::gemm::kSumsqPerTileW : fp8t::gemm::kSumsqPerTile;
   int64_t slots = 0;
   for (int32_t i = 0; i < n; ++i)
-    if (sumsq_of[i]) slots += gemm_tiles(gemms[i]) * fp8t::gemm::kSumsqPerTile;
+    if (sumsq_of[i]) slots += gemm_tiles(gemms[i], wide) * per_tile;
   return slots;
 }
 
@@ -549,6 +607,8 @@ fp8t_status gemm_multi(const fp8t_gemm_desc* gemms, int32_t n_gemms, const int32
   using namespace fp8t::gemm;
   static thread_local Group group;
   int64_t slot = 0;
+  const bool wide = use_wide(gemms, n_gemms);
+  const int bn = wide ? kBNw : kBN;
   for (int32_t b0 = 0; b0 < n_gemms; b0 += kMaxProblems) {
     const int32_t b1 = std::min<int32_t>(n_gemms, b0 + kMaxProblems);
     std::memset(&group, 0, sizeof(group));
@@ -588,21 +648,27 @@ fp8t_status gemm_multi(const fp8t_gemm_desc* gemms, int32_t n_gemms, const int32
       P.N = static_cast<int32_t>(d.N);
       P.K = static_cast<int32_t>(d.K);
       P.idesc = make_idesc(d.a_fmt, d.b_fmt, P.a_mn, P.b_mn);
-      P.tiles_n = static_cast<int32_t>((d.N + kBN - 1) / kBN);
+      P.tiles_n = static_cast<int32_t>((d.N + bn - 1) / bn);
       P.tile_start = static_cast<int32_t>(tiles);
       P.sumsq_slot = -1;
       if (sumsq_of && sumsq_of[i]) {
         P.sumsq_slot = static_cast<int32_t>(slot);
-        slot += gemm_tiles(d) * kSumsqPerTile;
+        slot += gemm_tiles(d, wide) * (wide ? kSumsqPerTileW : kSumsqPerTile);
       }
-      tiles += ((d.M + kBM - 1) / kBM) * P.tiles_n;            // 256 x 256 tiles, one per pair
+      tiles += ((d.M + kBM - 1) / kBM) * P.tiles_n;            // one tile per pair
       if (tiles >= (int64_t(1) << 30))
         return fail(FP8T_ERR_UNSUPPORTED_SHAPE, "fp8_gemm: too many tiles in one launch");
     }
     group.total_tiles = static_cast<int32_t>(tiles);
-    const int64_t grid = 2 * std::min<int64_t>(tiles, dev->gemm_clusters);   // persistent pairs
-    build_schedule(group, static_cast<int>(grid / 2));
-    k_fp8_gemm<false><<<static_cast<unsigned>(grid), kThreads, kSmemBytes, as_stream(stream)>>>(group);
+    // persistent pairs: wide tiles may be split in two, so a wide launch may use up to twice as
+    // many clusters as it has tiles
+    const int64_t grid = wide ? 2 * std::min<int64_t>(2 * tiles, dev->gemm_wide_clusters)
+                              : 2 * std::min<int64_t>(tiles, dev->gemm_clusters);
+    build_schedule(group, static_cast<int>(grid / 2), wide);   // round-robin: extra pairs idle
+    if (wide)
+      k_fp8_gemm_wide<<<static_cast<unsigned>(grid), kThreadsW, kSmemBytesW, as_stream(stream)>>>(group);
+    else
+      k_fp8_gemm<false><<<static_cast<unsigned>(grid), kThreads, kSmemBytes, as_stream(stream)>>>(group);
     if ((st = after_launch("fp8_gemm launch")) != FP8T_OK) return st;
   }
   return FP8T_OK;
@@ -778,7 +844,7 @@ fp8t_status fp8_mx_gemm_multi(const fp8t_mx_gemm_desc* gemms, int32_t n_gemms, v
     }
     group.total_tiles = static_cast<int32_t>(tiles);
     const int64_t grid = 2 * std::min<int64_t>(tiles, dev->gemm_mx_clusters);
-    build_schedule(group, static_cast<int>(grid / 2));
+    build_schedule(group, static_cast<int>(grid / 2), false);
     k_fp8_gemm<true><<<static_cast<unsigned>(grid), kThreads, kSmemBytesMX, as_stream(stream)>>>(group);
     if ((st = after_launch("fp8_mx_gemm launch")) != FP8T_OK) return st;
   }

@@ -24,6 +24,9 @@
 // longest-first greedy assignment balances the clusters (a grouped step mixes K = T wgrad tiles
 // with K = features fprop/dgrad tiles, which round-robin leaves several percent apart). Two TMEM
 // accumulators (2 x 256 columns) let the epilogue of one tile overlap the main loop of the next.
+// Launches whose every problem has N >= 512 use the wide form (k_fp8_gemm_wide, below): 256 x 512
+// tiles, a quarter fewer operand bytes per FLOP; its host schedule may run a tile as its two
+// 256-column halves on different clusters to even out the clusters' loads.
 // Warp roles (192 threads per CTA):
 //   warp 0, lane 0  TMA producer (both CTAs)
 //   warp 1, lane 0  MMA issuer (even CTA only); warp 1 also owns the TMEM allocation
@@ -164,7 +167,8 @@ struct alignas(64) Group {
   int32_t n, total_tiles;
   int32_t scheduled;             // 1: cluster c runs order[start[c] .. start[c+1])
   uint16_t start[kMaxClusters + 1];
-  uint16_t order[kMaxSchedTiles];
+  uint16_t order[kMaxSchedTiles];  // 3 * tile + part; part 0: whole tile, 1 / 2: the first / second
+                                   // 256-column half of a wide tile
   // sum of squares (sumsq_out null: off)
   double* partials;              // every launch's slots (8 per summed tile)
   double* sumsq_out;
@@ -176,13 +180,16 @@ struct alignas(64) Group {
 };
 constexpr int kSumsqPerTile = 8; // 2 CTAs x 4 epilogue warps
 
-// Number of tiles cluster c runs, and its i-th tile.
+// Number of work items cluster c runs, and the tile and part of its i-th.
 __device__ __forceinline__ int tiles_of(const Group& g, int c, int n_clusters) {
   return g.scheduled ? g.start[c + 1] - g.start[c]
                      : (g.total_tiles > c ? (g.total_tiles - c + n_clusters - 1) / n_clusters : 0);
 }
 __device__ __forceinline__ int tile_at(const Group& g, int c, int n_clusters, int i) {
-  return g.scheduled ? g.order[g.start[c] + i] : c + i * n_clusters;
+  return g.scheduled ? g.order[g.start[c] + i] / 3 : c + i * n_clusters;
+}
+__device__ __forceinline__ int part_at(const Group& g, int c, int i) {
+  return g.scheduled ? g.order[g.start[c] + i] % 3 : 0;
 }
 
 __device__ __forceinline__ int find_problem(const Group& g, int tile) {
@@ -520,6 +527,300 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kThreads; ++i) total = __dadd_rn(total, s_part[i]);
     // a launch of this call whose waits expired has slots that were never written (expired waits
     // of other calls do not matter here)
+    if (*reinterpret_cast<volatile unsigned int*>(g.abort_word) != 0u)
+      total = __longlong_as_double(0x7FF8000000000000LL);
+    *g.sumsq_out = total;
+    atomicExch(g.abort_word, 0u);
+    atomicExch(g.ticket, 0u);
+  }
+}
+
+// ---------------------------------------------------------------- wide tiles (N = 512 per pair)
+// For launches whose every problem has N >= 512: a pair computes a 256 x 512 tile, each k-step
+// two N = 256 MMAs into one 512-column accumulator (the whole of tensor memory). Per SM and
+// k-block that is 48 KB of operands (A 16 KB, two B boxes 32 KB) for 1024 tensor-core cycles,
+// three quarters of the bytes per FLOP of the 256 x 256 tile: the narrow tile needs about 64 B
+// per SM-cycle from L2, at the limit of what an SM's TMA loads bring in, and its MMAs waited for
+// operands about a sixth of the time. With a single accumulator the next tile's MMAs wait until
+// the epilogue has read this one, so eight epilogue warps (two per TMEM lane quarter, one per
+// 256-column half) pull the accumulator into registers as packed BF16 (128 registers a thread),
+// release it, and only then store it. A work item may also be one 256-column half of a tile
+// (part 1 or 2): only that half's B box is loaded, one MMA per k-step runs, and only that half's
+// epilogue warps store; the host uses such halves to balance the clusters' loads.
+constexpr int kBNw = 512;
+constexpr int kStagesW = 4;
+constexpr int kBBytesW = 2 * kHalf * kBK;                  // two 128-row B boxes per CTA
+constexpr int kStageBytesW = kABytes + kBBytesW;
+constexpr uint32_t kPairTxBytesW = 2 * kStageBytesW;
+constexpr int kEpiWarpsW = 8;
+constexpr int kThreadsW = 64 + 32 * kEpiWarpsW;            // producer, MMA issuer, 8 epilogue warps
+constexpr int kEpiBytesW = kEpiWarpsW * 2 * kEpiChunkBytes;
+constexpr int kSmemBytesW = kStagesW * kStageBytesW + kEpiBytesW + 1024 + 256;
+constexpr int kSumsqPerTileW = 16;                         // 2 CTAs x 8 epilogue warps
+
+struct SmemW {
+  uint64_t full[kStagesW];
+  uint64_t empty[kStagesW];
+  uint64_t acc_full;          // both CTAs: the accumulator holds a finished tile
+  uint64_t acc_empty;         // even CTA: every epilogue warp of both CTAs has read it
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsW, 1)
+    k_fp8_gemm_wide(const __grid_constant__ Group g) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  uint8_t* sA = smem;                                        // [stage][128 rows][128 B]
+  uint8_t* sB = smem + kStagesW * kABytes;                   // [stage][2 boxes][128 rows][128 B]
+  uint8_t* sEpi = smem + kStagesW * kStageBytesW;
+  SmemW* S = reinterpret_cast<SmemW*>(sEpi + kEpiBytesW);
+  volatile int* abort_flag = &S->abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
+  const int my_tiles = tiles_of(g, cluster, n_clusters);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStagesW; ++s) {
+      mbar_init(smem_u32(&S->full[s]), 1);
+      mbar_init(smem_u32(&S->empty[s]), 1);
+    }
+    mbar_init(smem_u32(&S->acc_full), 1);
+    mbar_init(smem_u32(&S->acc_empty), 2 * kEpiWarpsW);
+    mbar_init(smem_u32(&S->mma_done), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    for (int p = 0; p < g.n && p < 8; ++p) {
+      tma_prefetch_desc(&g.p[p].a);
+      tma_prefetch_desc(&g.p[p].b);
+      tma_prefetch_desc(&g.p[p].d);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(&S->tmem_base), kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = S->tmem_base;
+  const uint64_t limit = wait_limit_ns();
+  const int expire = expire_mode();
+  const bool expire_main = expire == kExpireAll;
+  const bool expire_epi = expire == kExpireAll || expire == kExpireGemmEpilogue;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer (both CTAs): A box and two B boxes per stage
+      uint32_t it = 0, issued = 0;
+      for (int i = 0; i < my_tiles && !*abort_flag; ++i) {
+        const int tile = tile_at(g, cluster, n_clusters, i), part = part_at(g, cluster, i);
+        const Problem& P = g.p[find_problem(g, tile)];
+        const int local = tile - P.tile_start;
+        const int m0 = (local / P.tiles_n) * kBM + static_cast<int>(rank) * kHalf;
+        const int n0 = (local % P.tiles_n) * kBNw + static_cast<int>(rank) * kHalf;
+        const int num_kb = (P.K + kBK - 1) / kBK;
+        const int h0 = part == 2 ? 1 : 0, h1 = part == 1 ? 1 : 2;   // B halves [h0, h1)
+        const uint32_t tx = 2u * (kABytes + (h1 - h0) * kBBytes);    // both CTAs' boxes
+        for (int kb = 0; kb < num_kb; ++kb, ++it) {
+          const uint32_t s = it % kStagesW, ph = (it / kStagesW) & 1;
+          if (*abort_flag) break;
+          if (!mbar_wait(smem_u32(&S->empty[s]), ph ^ 1, limit, expire_main)) {
+            *abort_flag = 1;
+            record_error(kErrTimeout);
+            break;
+          }
+          const uint32_t full_leader = mapa_shared(smem_u32(&S->full[s]), 0);
+          if (leader) mbar_arrive_expect_tx(smem_u32(&S->full[s]), tx);
+          const uint32_t a_dst = smem_u32(sA + s * kABytes), b_dst = smem_u32(sB + s * kBBytesW);
+          if (P.a_mn) tma_load_2d_pair(a_dst, &P.a, m0, kb * kBK, full_leader);
+          else        tma_load_2d_pair(a_dst, &P.a, kb * kBK, m0, full_leader);
+          for (int h = h0; h < h1; ++h) {
+            const uint32_t dst = b_dst + h * kBBytes;
+            if (P.b_mn) tma_load_2d_pair(dst, &P.b, n0 + h * kBN, kb * kBK, full_leader);
+            else        tma_load_2d_pair(dst, &P.b, kb * kBK, n0 + h * kBN, full_leader);
+          }
+          ++issued;
+        }
+      }
+      if (leader) {
+        const uint64_t t0 = globaltimer_ns();
+        for (uint32_t i = issued > kStagesW ? issued - kStagesW : 0; i < issued; ++i) {
+          const uint64_t spent = globaltimer_ns() - t0;
+          if (spent >= kPairDrainNs) break;
+          mbar_wait(smem_u32(&S->full[i % kStagesW]), (i / kStagesW) & 1, kPairDrainNs - spent);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ---------------- MMA issuer (even CTA): two N = 256 MMAs per k-step
+      uint32_t it = 0, local = 0;
+      for (int i = 0; i < my_tiles && !*abort_flag; ++i, ++local) {
+        const int tile = tile_at(g, cluster, n_clusters, i), part = part_at(g, cluster, i);
+        const Problem& P = g.p[find_problem(g, tile)];
+        const int num_kb = (P.K + kBK - 1) / kBK;
+        const uint32_t idesc = P.idesc;
+        const bool a_mn = P.a_mn != 0, b_mn = P.b_mn != 0;
+        const int h0 = part == 2 ? 1 : 0, h1 = part == 1 ? 1 : 2;
+        if (!mbar_wait(smem_u32(&S->acc_empty), (local & 1) ^ 1, limit, expire_main)) {
+          *abort_flag = 1;
+          record_error(kErrTimeout);
+          break;
+        }
+        tc_fence_after();
+        bool ok = true;
+        for (int kb = 0; kb < num_kb; ++kb, ++it) {
+          const uint32_t s = it % kStagesW, ph = (it / kStagesW) & 1;
+          if (*abort_flag || !mbar_wait(smem_u32(&S->full[s]), ph, limit, expire_main)) {
+            if (!*abort_flag) record_error(kErrTimeout);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sA + s * kABytes);
+          const uint32_t b_base = smem_u32(sB + s * kBBytesW);
+#pragma unroll
+          for (int k = 0; k < kBK / kUmmaK; ++k) {
+            const uint64_t adesc = a_mn ? make_sw128_desc_mn(a_base + k * kUmmaK * 128)
+                                        : make_sw128_desc(a_base + k * kUmmaK);
+            for (int h = h0; h < h1; ++h) {
+              const uint32_t bb = b_base + h * kBBytes;
+              tc_mma_f8_pair(tmem + h * kAccCols, adesc,
+                             b_mn ? make_sw128_desc_mn(bb + k * kUmmaK * 128)
+                                  : make_sw128_desc(bb + k * kUmmaK),
+                             idesc, (kb | k) != 0 ? 1u : 0u);
+            }
+          }
+          tc_commit_pair_mc(smem_u32(&S->empty[s]), 0x3);
+        }
+        if (!ok) break;
+        tc_commit_pair_mc(smem_u32(&S->acc_full), 0x3);
+      }
+      tc_commit_pair(smem_u32(&S->mma_done));
+      mbar_wait(smem_u32(&S->mma_done), 0, kDrainLimitNs);
+    }
+  } else {
+    // ---------------- epilogue warps 2..9 (both CTAs): TMEM lane quarter warp % 4, column half
+    const int quad = warp & 3, half = (warp - 2) >> 2;
+    uint8_t* my_buf = sEpi + (warp - 2) * 2 * kEpiChunkBytes;
+    uint32_t local = 0, chunk_count = 0;
+    for (int i = 0; i < my_tiles; ++i, ++local) {
+      const int tile = tile_at(g, cluster, n_clusters, i), part = part_at(g, cluster, i);
+      if (*abort_flag) break;
+      if (!mbar_wait(smem_u32(&S->acc_full), local & 1, limit, expire_epi)) {
+        *abort_flag = 1;
+        record_error(kErrTimeout);
+        break;
+      }
+      tc_fence_after();
+      if (part != 0 && part != half + 1) {        // the other half of a split tile: nothing here
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&S->acc_empty), 0));
+        continue;
+      }
+      const Problem& P = g.p[find_problem(g, tile)];
+      const int M = P.M, N = P.N, local_tile = tile - P.tile_start;
+      const float alpha = P.sa ? __fmul_rn(__ldg(P.sa), __ldg(P.sb)) : 1.0f;
+      const int row0 = (local_tile / P.tiles_n) * kBM + static_cast<int>(rank) * kHalf + quad * 32;
+      const int n0 = (local_tile % P.tiles_n) * kBNw + half * kAccCols;
+      const uint32_t t_base = tmem + (static_cast<uint32_t>(quad * 32) << 16) + half * kAccCols;
+      // the whole half-row of this lane into registers as packed BF16, then release the
+      // accumulator so the next tile's MMAs can start while these values are stored
+      uint32_t w[kAccCols / 32][16];
+#pragma unroll
+      for (int c = 0; c < kAccCols / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(t_base + c * 32, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          w[c][j] = pack_bf16x2(__fmul_rn(__uint_as_float(r[2 * j]), alpha),
+                                __fmul_rn(__uint_as_float(r[2 * j + 1]), alpha));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&S->acc_empty), 0));
+      const bool sumsq = P.sumsq_slot >= 0;
+      double ss = 0.0;
+#pragma unroll
+      for (int c = 0; c < kAccCols / 32; ++c) {
+        if (n0 + c * 32 >= N || row0 >= M) continue;       // chunk entirely outside the matrix
+        uint8_t* buf = my_buf + (chunk_count & 1) * kEpiChunkBytes;
+        ++chunk_count;
+        if (lane == 0) bulk_wait_group_read<1>();
+        __syncwarp();
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          if (sumsq) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint32_t v = w[c][4 * p + q];
+              const double lo = __uint_as_float(v << 16), hi = __uint_as_float(v & 0xFFFF0000u);
+              ss = __fma_rn(lo, lo, ss);
+              ss = __fma_rn(hi, hi, ss);
+            }
+          }
+          const int pp = p ^ ((lane >> 1) & 3);
+          *reinterpret_cast<uint4*>(buf + lane * 64 + pp * 16) =
+              make_uint4(w[c][4 * p], w[c][4 * p + 1], w[c][4 * p + 2], w[c][4 * p + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&P.d, smem_u32(buf), n0 + c * 32, row0);
+          bulk_commit_group();
+        }
+      }
+      if (sumsq) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, o));
+        if (lane == 0) {
+          g.partials[P.sumsq_slot + local_tile * kSumsqPerTileW + static_cast<int>(rank) * kEpiWarpsW +
+                     half * 4 + quad] = ss;
+          __threadfence();
+        }
+      }
+    }
+    if (lane == 0) bulk_wait_group<0>();
+  }
+  __syncwarp();
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) {
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < kSettleNs) {
+    }
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem, kTmemCols);
+
+  if (!g.sumsq_out) return;
+  if (threadIdx.x == 0 && *abort_flag) atomicOr(g.abort_word, 1u);
+  if (!g.last_launch) return;
+  __shared__ int s_last;
+  double* s_part = reinterpret_cast<double*>(sA);  // the stage buffers are idle by now
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(g.ticket, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  double acc = 0.0;
+  for (int i = threadIdx.x; i < g.n_partials; i += kThreadsW) acc = __dadd_rn(acc, __ldcg(g.partials + i));
+  s_part[threadIdx.x] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double total = 0.0;
+    for (int i = 0; i < kThreadsW; ++i) total = __dadd_rn(total, s_part[i]);
     if (*reinterpret_cast<volatile unsigned int*>(g.abort_word) != 0u)
       total = __longlong_as_double(0x7FF8000000000000LL);
     *g.sumsq_out = total;

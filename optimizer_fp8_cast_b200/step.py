@@ -14,7 +14,9 @@ then, for all layers at once, the amax-history roll and next scales, and one fus
 every dW (loss-scale unscale, global-norm clip, FP32 master/m/v, BF16 weight for the next step).
 With fused_update (the default) the roll and next scales run in the last CTA of the cast launch,
 which is possible because the GEMMs read the inverse scales the casts used (sinv_used), not the
-next ones (scale_inv). With fused_norm (the default) the wgrad epilogues also form the gradient
+next ones (scale_inv). With side_update the same update runs as its own small kernel on a second
+stream, concurrently with the GEMM launch (whose one CTA per SM leaves room for it), and AdamW
+waits for it: the cast launch then ends without the update's tail. With fused_norm (the default) the wgrad epilogues also form the gradient
 sum of squares, and AdamW runs without its norm pass, so each dW is read once. With fused_wcast
 (the default when both are on and no counters are kept) AdamW also casts each new BF16 weight
 for the next step with that step's scale, which the cast launch's update has already formed;
@@ -63,7 +65,8 @@ class Fp8LinearStep:
 
     def __init__(self, layer_shapes, tokens, history_len, algo="max", margin=0, adamw=None,
                  w_init=None, device="cuda", counters=False, device_step=False, fused_update=True,
-                 fused_norm=True, fused_wcast=True, transposes=False, recipe="delayed"):
+                 fused_norm=True, fused_wcast=True, transposes=False, recipe="delayed",
+                 side_update=False):
         self.device = torch.device(device)
         self.tokens = tokens
         self.algo = AMAX_MAX if algo == "max" else AMAX_MOST_RECENT
@@ -76,7 +79,9 @@ class Fp8LinearStep:
         self.scale = torch.ones(n, **f32)
         self.scale_inv = torch.ones(n, **f32)          # 1 / next scale (scale update output)
         self.sinv_used = torch.ones(n, **f32)          # 1 / scale the casts used (GEMM input)
-        self.fused_update = fused_update
+        # side_update: the scale update on a second stream, concurrent with the GEMMs
+        self.side_update = bool(side_update) and recipe == "delayed"
+        self.fused_update = fused_update and not self.side_update
         self.ticket = torch.zeros(1, dtype=torch.int32, device=self.device)
         self.fp8_max = torch.tensor([FP8_MAX[ROLE_FMT[i % 3]] for i in range(n)], **f32)
         self.counters = torch.zeros(n, 3, dtype=torch.int64, device=self.device) if counters else None
@@ -118,7 +123,12 @@ class Fp8LinearStep:
         # the W cast inside AdamW needs the in-launch scale update and the presummed AdamW, and
         # writes row-major codes only; the saturation / zero counters of W are only kept by the
         # separate cast
-        self.fused_wcast = fused_wcast and fused_update and fused_norm and not counters and not transposes
+        self.fused_wcast = (fused_wcast and (self.fused_update or self.side_update) and fused_norm
+                            and not counters and not transposes)
+        if self.side_update and self.device.type == "cuda":
+            self._side = torch.cuda.Stream(device=self.device)
+            self._cast_done = torch.cuda.Event()
+            self._update_done = torch.cuda.Event()
         if self.fused_wcast and self.device.type == "cuda":
             self.prime()
 
@@ -152,13 +162,16 @@ class Fp8LinearStep:
         update, each launch's last CTA also performs those tensors' scale update."""
         descs = []
         for k, L in enumerate(self.layers):
-            w = (self.cast_desc(k, ROLE_W, None, None, None) if update and self.fused_wcast
-                 else self.cast_desc(k, ROLE_W, L.W, L.Wq, L.WqT))   # None: scale update only
-            descs += [self.cast_desc(k, ROLE_X, xs[k], L.Xq, L.XqT), w,
-                      self.cast_desc(k, ROLE_DY, dys[k], L.dYq, L.dYqT)]
+            # with the W cast inside AdamW, W has no cast here: an update-only entry when the
+            # launch updates the scales, nothing otherwise
+            w = ([self.cast_desc(k, ROLE_W, None, None, None)] if update else []) if self.fused_wcast \
+                else [self.cast_desc(k, ROLE_W, L.W, L.Wq, L.WqT)]
+            descs += [self.cast_desc(k, ROLE_X, xs[k], L.Xq, L.XqT)] + w + \
+                     [self.cast_desc(k, ROLE_DY, dys[k], L.dYq, L.dYqT)]
         if update:
             ups = [dict(history=self.history[i], scale_inv_next=self._slot(self.scale_inv, i))
                    for i in range(len(descs))]
+            assert len(descs) == 3 * len(self.layers)
             fp8_cast_transpose_amax_update_multi(descs, ups, self.algo, self.margin, self.ticket,
                                                  stream=stream)
         else:
@@ -291,10 +304,27 @@ class Fp8LinearStep:
             self.cast_all_current(xs, dys, stream)
         else:
             self.cast_all(xs, dys, stream, update=self.fused_update)
+        if self.side_update:
+            self.side_update_begin(stream)
         self.gemm_all(stream, sumsq=self.fused_norm)
-        if not self.fused_update and self.recipe == "delayed":
+        if self.side_update:
+            self.side_update_end(stream)
+        elif not self.fused_update and self.recipe == "delayed":
             self.scale_update(stream)
         self.adamw(stream, presummed=self.fused_norm)
+
+    def side_update_begin(self, stream=None):
+        """After the cast launch: the scale update of every tensor on the side stream."""
+        main = torch.cuda.current_stream(self.device) if stream is None else stream
+        self._cast_done.record(main)
+        self._side.wait_event(self._cast_done)
+        self.scale_update(self._side)
+        self._update_done.record(self._side)
+
+    def side_update_end(self, stream=None):
+        """Before AdamW (which reads the next W scale and accumulates W's amax): join."""
+        main = torch.cuda.current_stream(self.device) if stream is None else stream
+        main.wait_event(self._update_done)
 
     # ------------------------------------------------------------------ training state
     def state_dict(self):
@@ -327,11 +357,14 @@ class Fp8LinearStep:
     # launches of the library's kernels per step (for the benchmark's launch count)
     def kernels_per_step(self):
         n_adamw_batches = (len(self.layers) + 255) // 256
-        n_cast_launches = (3 * len(self.layers) + 7) // 8
+        # a cast launch carries up to 8 entries: X and dY of every layer, and W unless AdamW casts
+        # it and no update in the cast launch needs its (update-only) entry
+        per_layer = 2 if self.fused_wcast and not self.fused_update else 3
+        n_cast_launches = (per_layer * len(self.layers) + 7) // 8
         n_gemm_launches = (3 * len(self.layers) + 23) // 24
         if self.recipe == "mxfp8":
             return (3 * len(self.layers) + 7) // 8 + (3 * len(self.layers) + 23) // 24 + 2 * n_adamw_batches
-        n_scale_launches = 0 if self.fused_update or self.recipe == "current" else 1
+        n_scale_launches = 0 if (self.fused_update and not self.side_update) or self.recipe == "current" else 1
         if self.recipe == "current":
             n_cast_launches *= 2                   # an amax launch before each cast launch
         n_adamw_launches = (1 if self.fused_norm else 2) * n_adamw_batches

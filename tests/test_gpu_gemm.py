@@ -210,3 +210,46 @@ def test_step_layouts_full_size_sampled(cuda_lib):
         ii, jj = sample_positions(D.shape[0], D.shape[1], 4096, seed=D.shape[1])
         R, ab = oracle.gemm_at(np.ascontiguousarray(A), af, np.ascontiguousarray(B), bf, sa, sb, ii, jj)
         assert gemm_within_tolerance(bf16_bits(D)[ii, jj], R, ab).all()
+
+
+@pytest.mark.parametrize("shapes", [[(256, 512, 256)], [(400, 528, 1040)],
+                                    [(512, 1024, 4096), (256, 768, 128), (1040, 1552, 272),
+                                     (128, 512, 64)]],
+                         ids=["one-tile-in-halves", "ragged", "grouped"])
+def test_wide_tiles_with_sum_of_squares(cuda_lib, shapes):
+    """Launches whose every problem is at least 512 wide run 256 x 512 tiles, and the schedule
+    splits tiles into their two 256-column halves on different clusters where that evens out the
+    load (a launch with fewer tiles than clusters is split throughout). Every output against the
+    oracle, mixed formats and operand layouts, and the FP64 sum of squares of the flagged
+    problems against numpy's; a repeat gives identical bits and leaves the workspace at zero."""
+    rng = np.random.default_rng(len(shapes) * 7)
+    probs = []
+    for i, (M, N, K) in enumerate(shapes):
+        af, bf = PAIRS[(i + 1) % 4]
+        A = random_codes(M, K, af, 500 + i)
+        B = random_codes(N, K, bf, 600 + i)
+        a_mn, b_mn = bool(i % 2), bool((i // 2) % 2)
+        sa, sb = float(rng.uniform(0.01, 1)), float(rng.uniform(0.01, 1))
+        probs.append(dict(A=A.t().contiguous() if a_mn else A, a_mn=a_mn, a_fmt=af,
+                          B=B.t().contiguous() if b_mn else B, b_mn=b_mn, b_fmt=bf,
+                          a_scale_inv=dev_scalar(sa), b_scale_inv=dev_scalar(sb), sumsq=i != 1,
+                          D=torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda"),
+                          sa=sa, sb=sb, Ah=u8(A), Bh=u8(B)))
+    descs = [{k: v for k, v in p.items() if k not in ("sa", "sb", "Ah", "Bh")} for p in probs]
+    ws = torch.zeros(cuda_lib.fp8_gemm_sumsq_workspace_bytes(descs), dtype=torch.uint8, device="cuda")
+    out = torch.zeros(1, dtype=torch.float64, device="cuda")
+    cuda_lib.fp8_gemm_multi_sumsq(descs, out, ws)
+    cuda_lib.fp8t_check_device_error()
+    first = out.item()
+    for p in probs:
+        R, ab = oracle.gemm(p["Ah"], p["a_fmt"], p["Bh"], p["b_fmt"], p["sa"], p["sb"], want_abs=True)
+        ok = gemm_within_tolerance(bf16_bits(p["D"]), R, ab)
+        assert ok.all(), f"{(~ok).sum()} of {ok.size} outside tolerance"
+    squares = np.concatenate([np.square(f32(p["D"].float()).astype(np.float64)).reshape(-1)
+                              for p in probs if p["sumsq"]])
+    exact = float(np.sum(np.sort(squares)))
+    assert abs(first - exact) <= 1e-13 * exact
+    assert not ws[:8].any()
+    cuda_lib.fp8_gemm_multi_sumsq(descs, out, ws)
+    cuda_lib.fp8t_check_device_error()
+    assert np.float64(out.item()).view(np.uint64) == np.float64(first).view(np.uint64)

@@ -23,16 +23,18 @@ pytestmark = pytest.mark.gpu
 FMT = (oracle.E4M3, oracle.E4M3, oracle.E5M2)
 
 
-def make_step(wl, algo=None, margin=None, H=None, counters=True, fused=True, transposes=False):
+def make_step(wl, algo=None, margin=None, H=None, counters=True, fused=True, transposes=False,
+              side=False):
     """fused: scale update in the cast launch, dW sum of squares in the wgrad epilogue and (when
     no counters are kept) the next W cast inside AdamW; False: every stage its own launch.
-    transposes: the casts also write q^T and the GEMMs read K-major operands only."""
+    transposes: the casts also write q^T and the GEMMs read K-major operands only.
+    side: the scale update as its own launch on a second stream, beside the GEMMs."""
     w0 = [synth.linear_weight(wl, k, "cuda") for k in range(len(wl.layers))]
     return Fp8LinearStep([(i, o) for _, i, o in wl.layers], wl.tokens,
                          H or wl.history_len, algo or wl.algo,
                          wl.margin if margin is None else margin, wl.adamw, w0, "cuda",
                          counters=counters, fused_update=fused, fused_norm=fused, fused_wcast=fused,
-                         transposes=transposes)
+                         transposes=transposes, side_update=side)
 
 
 def tr(q):
@@ -153,19 +155,23 @@ def _check_adamw_on_gpu_grad(st, pre_opt, t):
         assert np.abs(wg - Wref[k].astype(np.int32)).max() <= 1
 
 
-@pytest.mark.parametrize("fused,counters,transposes",
-                         [(True, False, False), (True, True, False), (False, True, False),
-                          (True, False, True), (False, True, True)],
-                         ids=["all-fused", "fused-with-counters", "separate-launches",
+@pytest.mark.parametrize("fused,counters,transposes,side",
+                         [(True, False, False, False), (True, False, False, True),
+                          (True, True, False, False), (False, True, False, False),
+                          (True, False, True, False), (False, True, True, False)],
+                         ids=["all-fused", "side-update", "fused-with-counters", "separate-launches",
                               "all-fused-transposes", "separate-launches-transposes"])
-def test_linear256_three_steps(cuda_lib, fused, counters, transposes):
+def test_linear256_three_steps(cuda_lib, fused, counters, transposes, side):
     """Three steps in full. all-fused: scale update in the cast launch, dW sum of squares in the
-    wgrad epilogue, next W cast in AdamW (three launches per step); with counters the W cast
-    stays in the cast launch; separate-launches: every stage its own kernel. Without transposes
-    the GEMMs read Xq, Wq, dYq MN-major where needed; with them, the K-major transposed copies."""
+    wgrad epilogue, next W cast in AdamW (three launches per step); side-update: the same with
+    the scale update as its own launch on a second stream beside the GEMMs; with counters the W
+    cast stays in the cast launch; separate-launches: every stage its own kernel. Without
+    transposes the GEMMs read Xq, Wq, dYq MN-major where needed; with them, the K-major
+    transposed copies."""
     wl = synth.LINEAR256
-    st = make_step(wl, fused=fused, counters=counters, transposes=transposes)
+    st = make_step(wl, fused=fused, counters=counters, transposes=transposes, side=side)
     assert st.fused_wcast == (fused and not counters and not transposes)
+    assert st.side_update == side and st.kernels_per_step() == (4 if side else 3 if fused else 5)
     for t in range(wl.steps):
         xs, dys = zip(*[synth.linear_inputs(wl, k, t, "cuda") for k in range(len(wl.layers))])
         pre = snapshot(st)
@@ -174,16 +180,18 @@ def test_linear256_three_steps(cuda_lib, fused, counters, transposes):
         check_step(st, pre, xs, dys)
 
 
-def test_linear256_step_in_cuda_graph(cuda_lib):
-    """The whole step captured once into a CUDA graph (device step counter) and replayed three
-    times; after every replay each stage is compared with the oracle fed the same inputs: casts,
-    scales and history bit for bit, GEMMs within tolerance, AdamW within 4 ulp with the oracle's
-    host bias corrections for t = 1, 2, 3 (the graph forms them on the device from the counter)."""
+@pytest.mark.parametrize("side", [False, True], ids=["update-in-cast", "side-update"])
+def test_linear256_step_in_cuda_graph(cuda_lib, side):
+    """The whole step captured once into a CUDA graph (device step counter; with side-update the
+    graph forks the scale update onto a second stream and joins it before AdamW) and replayed
+    three times; after every replay each stage is compared with the oracle fed the same inputs:
+    casts, scales and history bit for bit, GEMMs within tolerance, AdamW within 4 ulp with the
+    oracle's host bias corrections for t = 1, 2, 3 (the graph forms them on the device)."""
     wl = synth.LINEAR256
     xs, dys = zip(*[synth.linear_inputs(wl, k, 0, "cuda") for k in range(len(wl.layers))])
     graphed = Fp8LinearStep([(i, o) for _, i, o in wl.layers], wl.tokens, wl.history_len, wl.algo,
                             wl.margin, wl.adamw, [synth.linear_weight(wl, 0, "cuda")], "cuda",
-                            device_step=True)
+                            device_step=True, side_update=side)
     assert graphed.fused_wcast
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
