@@ -4,15 +4,17 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 A step is one pass of the whole hot path over one batch of the 4096 x 4096 Linear with 8192
-tokens (batch 4 x sequence 2048), three launches captured in one CUDA graph:
+tokens (batch 4 x sequence 2048), four launches captured in one CUDA graph:
   1. the cast launch: X -> E4M3 and dY -> E5M2 (row-major codes, amax, inverse scales used; the
      GEMMs read the codes MN-major where they need the transpose, so no transposed copy is
-     written), and in its last CTA the amax-history roll and scale update of X, W and dY
-     (history 1024, algo max, margin 0);
-  2. one grouped GEMM launch: fprop, dgrad and wgrad (FP8 operands, FP32 accumulation, BF16
+     written);
+  2. the amax-history roll and scale update of X, W and dY (history 1024, algo max, margin 0),
+     its own small launch on a second stream, running beside
+  3. one grouped GEMM launch: fprop, dgrad and wgrad (FP8 operands, FP32 accumulation, BF16
      out), the wgrad epilogue also summing dW^2 for the global norm;
-  3. one fused AdamW launch over dW (unscale, clip, m, v, master, BF16 weight) that also casts
-     the new weight to E4M3 codes for the next step.
+  4. one fused AdamW launch over dW (unscale, clip, m, v, master, BF16 weight) that also casts
+     the new weight to E4M3 codes for the next step (it waits for the scale update).
+(--update-in-cast: the update runs in the cast launch's last CTA instead, three launches.)
 Inputs are synthetic (seeded normals of the stated shapes), resident in HBM when timing starts.
 Before every timed step L2 is flushed by writing a 256 MiB buffer (its dirty lines are written
 back while the next step runs, as the previous step's AdamW writes would be in a training loop);
@@ -178,7 +180,8 @@ def run_ours(args, rank, world, local_rank):
                        dev, device_step=True, fused_update=not args.separate_scale_update,
                        fused_norm=not args.separate_norm_pass,
                        fused_wcast=not args.separate_weight_cast, transposes=args.transposes,
-                       recipe=args.recipe, side_update=args.side_update)
+                       recipe=args.recipe,
+                       side_update=not (args.update_in_cast or args.separate_scale_update))
     batches = [list(zip(*[synth.linear_inputs(wl, k, t, dev) for k in range(nl)])) for t in range(2)]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     sweep = torch.ones(L2_FLUSH_BYTES // 8, dtype=torch.int64, device=dev)
@@ -869,9 +872,9 @@ def main(argv=None):
                     help="run AdamW's own norm pass instead of summing dW^2 in the wgrad epilogue")
     ap.add_argument("--separate-scale-update", action="store_true",
                     help="run the scale update as its own launch instead of in the cast launch")
-    ap.add_argument("--side-update", action="store_true",
-                    help="run the scale update as its own launch on a second stream, concurrently "
-                         "with the GEMM launch, instead of in the cast launch's last CTA")
+    ap.add_argument("--update-in-cast", action="store_true",
+                    help="run the scale update in the cast launch's last CTA instead of as its own "
+                         "launch on a second stream, concurrently with the GEMM launch (default)")
     ap.add_argument("--out", default=None, help="stress sweep: write the per-step table here")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":

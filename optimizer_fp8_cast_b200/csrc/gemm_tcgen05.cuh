@@ -640,7 +640,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsW, 1)
           const uint32_t a_dst = smem_u32(sA + s * kABytes), b_dst = smem_u32(sB + s * kBBytesW);
           if (P.a_mn) tma_load_2d_pair(a_dst, &P.a, m0, kb * kBK, full_leader);
           else        tma_load_2d_pair(a_dst, &P.a, kb * kBK, m0, full_leader);
-          for (int h = h0; h < h1; ++h) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if (h < h0 || h >= h1) continue;     // the other half of a split tile
             const uint32_t dst = b_dst + h * kBBytes;
             if (P.b_mn) tma_load_2d_pair(dst, &P.b, n0 + h * kBN, kb * kBK, full_leader);
             else        tma_load_2d_pair(dst, &P.b, kb * kBK, n0 + h * kBN, full_leader);
@@ -690,7 +692,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsW, 1)
           for (int k = 0; k < kBK / kUmmaK; ++k) {
             const uint64_t adesc = a_mn ? make_sw128_desc_mn(a_base + k * kUmmaK * 128)
                                         : make_sw128_desc(a_base + k * kUmmaK);
-            for (int h = h0; h < h1; ++h) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              if (h < h0 || h >= h1) continue;   // the other half of a split tile
               const uint32_t bb = b_base + h * kBBytes;
               tc_mma_f8_pair(tmem + h * kAccCols, adesc,
                              b_mn ? make_sw128_desc_mn(bb + k * kUmmaK * 128)
