@@ -473,12 +473,13 @@ constexpr size_t kSumsqHeader = 256;    // ticket and abort words, then the part
 
 // Tile lists of a grouped GEMM launch: every tile costs its problem's K / 128 k-blocks (twice
 // that for a wide tile); tiles are handed out longest first, each to the least-loaded cluster.
-// A wide launch with fewer tiles than clusters then splits tiles into their two 256-column
-// halves, one half moving to the least busy cluster, while the busiest cluster is more than half
-// a tile above it. (With at least as many tiles as clusters splitting does not pay: a half tile
-// reloads A for half the MMAs, the operand-starved pattern the wide tile avoids; measured on the
-// 4096 step, splitting there to balance the clusters left the launch no faster.) Every cluster
-// then runs its items in index order. Items are 3 * tile + part.
+// A wide launch then splits tiles into their two 256-column halves, one half moving to the least
+// busy cluster, while that lowers the busiest cluster's load. A half tile is costed at 0.58 of a
+// whole one, not 0.5: it runs half the MMAs but loads all of A, the operand-starved pattern the
+// wide tile avoids. (On the 4096 step this takes the busiest cluster from 704 to 678 k-block
+// units with 28 splits, and the launch from ~0.295 to ~0.292 ms; costing halves at 0.5 split
+// more and gained less.) Every cluster then runs its items in index order. Items are
+// 3 * tile + part.
 // Launches with more tiles than the table holds keep round-robin (with thousands of tiles it is
 // balanced already).
 void build_schedule(fp8t::gemm::Group& g, int clusters, bool wide) {
@@ -504,28 +505,35 @@ void build_schedule(fp8t::gemm::Group& g, int clusters, bool wide) {
     load[best] += it.cost;
     own[best].push_back(it);
   }
+  // a half tile runs about 0.58 of a whole one: half the MMAs, but all of A's loads
+  auto half_cost = [](int64_t whole) { return (whole * 29 + 49) / 50; };
   int n_items = g.total_tiles;
-  while (wide && g.total_tiles < clusters && n_items < kMaxSchedTiles) {
+  while (wide && n_items < kMaxSchedTiles) {
     int hi = 0, lo = 0;
     for (int c = 1; c < clusters; ++c) {
       if (load[c] > load[hi]) hi = c;
       if (load[c] < load[lo]) lo = c;
     }
-    int pick = -1;                    // the whole tile of `hi` whose half moves best
+    int pick = -1;                    // the whole tile of `hi` whose split lowers `hi` most
+    int64_t best = load[hi];
     for (int k = 0; k < static_cast<int>(own[hi].size()); ++k) {
       const Item& it = own[hi][k];
-      if (it.part == 0 && 2 * (it.cost / 2) == it.cost && it.cost / 2 < load[hi] - load[lo] &&
-          (pick < 0 || it.cost > own[hi][pick].cost))
+      if (it.part != 0) continue;
+      const int64_t h = half_cost(it.cost);
+      const int64_t after = std::max(load[hi] - it.cost + h, load[lo] + h);
+      if (after < best) {
+        best = after;
         pick = k;
+      }
     }
     if (pick < 0) break;
     Item& it = own[hi][pick];
-    const int64_t half = it.cost / 2;
-    it.cost = half;
+    const int64_t h = half_cost(it.cost);
+    load[hi] += h - it.cost;
+    load[lo] += h;
+    it.cost = h;
     it.part = 1;
-    own[lo].push_back({half, it.tile, 2});
-    load[hi] -= half;
-    load[lo] += half;
+    own[lo].push_back({h, it.tile, 2});
     ++n_items;
   }
   int k = 0;
