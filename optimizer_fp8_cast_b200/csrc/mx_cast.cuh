@@ -13,17 +13,19 @@
 // rows (M or N) x 4 blocks (128 K values): byte (i % 32) * 16 + (i / 32) * 4 + kb holds row i,
 // block kb, which is the order the tensor-core scale copy (tcgen05.cp 32x128b, replicated to
 // the four lane quarters) expects; atoms are stored [MN / 128][K / 128].
-// Persistent CTAs; thread 0 keeps two tiles in flight: each tile arrives as two TMA boxes of
-// 128 rows x 64 columns (128-byte swizzle: 16-byte chunk c of a row's 128 bytes at c ^ (row % 8))
-// into a double buffer, completion on one mbarrier per buffer. Then, in parallel,
+// Persistent CTAs (three per SM); thread 0 keeps two tiles in flight: each tile arrives as two
+// TMA boxes of 128 rows x 64 columns (128-byte swizzle: 16-byte chunk c of a row's 128 bytes at
+// c ^ (row % 8)) into a double buffer, completion on one mbarrier per buffer. Then, in parallel,
 //   warps 0-3 quantise the column-wise blocks: a thread takes 4 adjacent columns of one block of
-//     32 rows (32 eight-byte shared loads), forms their four scales and stores each row's four
-//     codes as one 4-byte word into a staged code tile;
+//     32 rows, reads them once (eight-byte shared loads) for the four scales and again to
+//     quantise, and stores each row's four codes as one 4-byte word straight to global memory
+//     (the warp's 32 lanes cover the row's 128 columns, so each store instruction writes one
+//     whole 128-byte line);
 //   warps 4-7 quantise the row-wise blocks straight to global memory: a quarter-warp takes the
 //     same block of 8 consecutive rows, so its shared loads hit 8 different bank groups;
-// and after a barrier all threads write the staged column-wise codes out row by row with 16-byte
-// stores, and the two scale atoms. Every wait on an mbarrier is bounded: on expiry the CTA
-// records the timeout in the device error word, stops, and waits (bounded) for its loads.
+// and after a barrier the two 512-byte scale atoms, gathered in shared memory, go out. Every wait
+// on an mbarrier is bounded: on expiry the CTA records the timeout in the device error word,
+// stops, and waits (bounded) for its loads.
 #pragma once
 
 #include "ptx.cuh"
@@ -36,7 +38,7 @@ constexpr int kThreads = 256;
 constexpr int kMaxTensors = 8;
 constexpr int kHalfBytes = kTile * 64 * 2;                 // one 128-row x 64-column BF16 box
 constexpr int kXBytes = 2 * kHalfBytes;                    // one 128 x 128 BF16 tile
-constexpr int kSmemBytes = 2 * kXBytes + kTile * kTile + 2 * 512 + 64 + 1024 /*alignment*/;
+constexpr int kSmemBytes = 2 * kXBytes + 2 * 512 + 64 + 1024 /*alignment*/;
 
 struct alignas(64) Tensor {
   CUtensorMap x_map;               // BF16 [rows][cols], 64 x 128 boxes, 128-byte swizzle
@@ -109,12 +111,11 @@ __device__ __forceinline__ uint8_t scale_code(uint32_t m, int X) {
   return m > 0x7F80u ? 0xFF : static_cast<uint8_t>(X + 127);
 }
 
-__global__ void __launch_bounds__(kThreads, 2) k_mx_cast(const __grid_constant__ Group g) {
+__global__ void __launch_bounds__(kThreads, 3) k_mx_cast(const __grid_constant__ Group g) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* xbuf = smem;                                             // [2][2 boxes][128][128 B]
-  uint8_t* qs = smem + 2 * kXBytes;                                 // [128][128] column-wise codes
-  uint8_t* atom_r = qs + kTile * kTile;                             // 512 B
+  uint8_t* atom_r = smem + 2 * kXBytes;                             // 512 B
   uint8_t* atom_c = atom_r + 512;                                   // 512 B
   uint64_t* full = reinterpret_cast<uint64_t*>(atom_c + 512);       // 2 mbarriers
   __shared__ int s_abort;
@@ -151,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_mx_cast(const __grid_constant__
         pending &= ~(1u << buf);
       }
     }
-    __syncthreads();                          // tile landed; the previous tile's outputs written
+    __syncthreads();                          // tile landed; the previous tile's atoms written
     if (s_abort) break;
     const Tensor& T = g.t[tensor_of(g, tile)];
     const int64_t local = tile - T.tile_start;
@@ -163,13 +164,12 @@ __global__ void __launch_bounds__(kThreads, 2) k_mx_cast(const __grid_constant__
       // ---- column-wise blocks: columns 4cq .. 4cq+3, rows 32rb .. 32rb+31
       if (T.q_col) {
         const int cq = lane, rb = warp, col = 4 * cq;
-        uint2 v[32];
         uint32_t ma = 0, mb = 0;
-#pragma unroll
+#pragma unroll 8
         for (int r = 0; r < 32; ++r) {
-          v[r] = *reinterpret_cast<const uint2*>(xs + xoff(32 * rb + r, col));
-          ma = __vmaxu2(ma, v[r].x & 0x7FFF7FFFu);
-          mb = __vmaxu2(mb, v[r].y & 0x7FFF7FFFu);
+          const uint2 v = *reinterpret_cast<const uint2*>(xs + xoff(32 * rb + r, col));
+          ma = __vmaxu2(ma, v.x & 0x7FFF7FFFu);
+          mb = __vmaxu2(mb, v.y & 0x7FFF7FFFu);
         }
         const uint32_t m[4] = {ma & 0xFFFFu, ma >> 16, mb & 0xFFFFu, mb >> 16};
         int X[4];
@@ -180,12 +180,14 @@ __global__ void __launch_bounds__(kThreads, 2) k_mx_cast(const __grid_constant__
           inv[c] = pow2_neg(X[c]);
         }
         const bool nan_block = max(max(m[0], m[1]), max(m[2], m[3])) > 0x7F80u;
-#pragma unroll
+        uint8_t* dst = T.q_col + (r0 + 32 * rb) * T.cols + c0 + col;
+#pragma unroll 8
         for (int r = 0; r < 32; ++r) {
-          const float p0 = __fmul_rn(__uint_as_float(v[r].x << 16), inv[0]);
-          const float p1 = __fmul_rn(__uint_as_float(v[r].x & 0xFFFF0000u), inv[1]);
-          const float p2 = __fmul_rn(__uint_as_float(v[r].y << 16), inv[2]);
-          const float p3 = __fmul_rn(__uint_as_float(v[r].y & 0xFFFF0000u), inv[3]);
+          const uint2 v = *reinterpret_cast<const uint2*>(xs + xoff(32 * rb + r, col));
+          const float p0 = __fmul_rn(__uint_as_float(v.x << 16), inv[0]);
+          const float p1 = __fmul_rn(__uint_as_float(v.x & 0xFFFF0000u), inv[1]);
+          const float p2 = __fmul_rn(__uint_as_float(v.y << 16), inv[2]);
+          const float p3 = __fmul_rn(__uint_as_float(v.y & 0xFFFF0000u), inv[3]);
           uint32_t c = T.fmt == 0 ? cvt_fp8x2<0>(p0, p1) | (cvt_fp8x2<0>(p2, p3) << 16)
                                   : cvt_fp8x2<1>(p0, p1) | (cvt_fp8x2<1>(p2, p3) << 16);
           if (nan_block) {                       // only a NaN input gives a NaN product
@@ -194,7 +196,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_mx_cast(const __grid_constant__
             if (p2 != p2) c = (c & 0xFF00FFFFu) | 0x7F0000u;
             if (p3 != p3) c = (c & 0x00FFFFFFu) | 0x7F000000u;
           }
-          *reinterpret_cast<uint32_t*>(qs + (32 * rb + r) * kTile + col) = c;
+          *reinterpret_cast<uint32_t*>(dst + r * T.cols) = c;
         }
 #pragma unroll
         for (int c = 0; c < 4; ++c)
@@ -243,21 +245,13 @@ __global__ void __launch_bounds__(kThreads, 2) k_mx_cast(const __grid_constant__
         atom_r[(row & 31) * 16 + (row >> 5) * 4 + b] = scale_code(m, X);
       }
     }
-    __syncthreads();                          // input tile consumed; staged codes, atoms complete
+    __syncthreads();                          // input tile consumed; both atoms complete
     if (tid == 0) {                           // refill the buffer just consumed
       const int64_t next = tile + 2 * stride;
       if (next < g.total_tiles) {
         issue_tile(g, next, smem_u32(xbuf + buf * kXBytes), smem_u32(&full[buf]));
         pending |= 1u << buf;
         pending_ph = (pending_ph & ~(1u << buf)) | (static_cast<uint32_t>(((i + 2) >> 1) & 1) << buf);
-      }
-    }
-    if (T.q_col) {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int v = u * kThreads + tid, row = v >> 3, c16 = v & 7;
-        *reinterpret_cast<uint4*>(T.q_col + (r0 + row) * T.cols + c0 + 16 * c16) =
-            reinterpret_cast<const uint4*>(qs)[v];
       }
     }
     if (tid < 32 && T.q_row)
