@@ -447,6 +447,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           uint32_t r[32];
           tmem_ld_32x32b_x32(t_base + c * 32, r);
           tmem_ld_wait();
+          tmem_reg_fence(r);
           if (step == 0) {
             tc_fence_before();
             __syncwarp();
@@ -469,6 +470,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           uint32_t r[32];
           tmem_ld_32x32b_x32(t_base + c * 32, r);
           tmem_ld_wait();
+          tmem_reg_fence(r);
           if (n0 + c * 32 >= N || row0 >= M) continue;  // chunk entirely outside the matrix
           uint32_t w16[16];
 #pragma unroll
@@ -743,6 +745,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsW, 1)
         uint32_t r[32];
         tmem_ld_32x32b_x32(t_base + c * 32, r);
         tmem_ld_wait();
+        tmem_reg_fence(r);
 #pragma unroll
         for (int j = 0; j < 16; ++j)
           w[c][j] = pack_bf16x2(__fmul_rn(__uint_as_float(r[2 * j]), alpha),

@@ -174,6 +174,13 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+// After tmem_ld_wait: registers a tcgen05.ld wrote are only valid once the wait has returned,
+// but the compiler sees them as written by the load itself. Passing each through an empty asm
+// placed after the wait makes every later use depend on it, so no use is moved above the wait.
+__device__ __forceinline__ void tmem_reg_fence(uint32_t (&r)[32]) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) asm volatile("" : "+r"(r[i]));
+}
 
 // ------------------------------------------------------------------ CTA pairs (cluster of 2)
 __device__ __forceinline__ uint32_t cluster_ctarank() {
