@@ -273,6 +273,29 @@ def test_host_streamed_steps_match_eager(cuda_lib):
     assert torch.equal(eager.history, streamed.history)
 
 
+def test_host_streamed_steps_against_the_oracle(cuda_lib):
+    """The runner on the step the benchmark times (scale update on a side stream), one step at a
+    time so that each step's codes are still on the device: every stage against the oracle fed
+    the same inputs (casts, scales and history bit for bit, GEMMs within tolerance, AdamW within
+    4 ulp), and the Y and dX that reached host memory equal the device's."""
+    from optimizer_fp8_cast_b200.host_stream import HostStreamedStep
+    wl = synth.LINEAR256
+    st = make_step(wl, counters=False, side=True)
+    runner = HostStreamedStep(st)
+    for t in range(3):
+        X, dY = synth.linear_inputs(wl, 0, t, "cpu")
+        hy = torch.empty(wl.tokens, 256, dtype=torch.bfloat16).pin_memory()
+        hdx = torch.empty(wl.tokens, 256, dtype=torch.bfloat16).pin_memory()
+        pre = snapshot(st)
+        runner.step([X.pin_memory()], [dY.pin_memory()], [hy], [hdx])
+        runner.finish()
+        cuda_lib.fp8t_check_device_error()
+        check_step(st, pre, [X.cuda()], [dY.cuda()])
+        L = st.layers[0]
+        assert torch.equal(hy.view(torch.int16), L.Y.cpu().view(torch.int16))
+        assert torch.equal(hdx.view(torch.int16), L.dX.cpu().view(torch.int16))
+
+
 def test_checkpoint_resume_is_bit_exact(cuda_lib):
     """Six steps straight equal three steps, a save of the full training state (weights,
     master/m/v, amax history, scales, step counters) into a fresh step object, and three more.
