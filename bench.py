@@ -319,7 +319,10 @@ def run_ours(args, rank, world, local_rank):
                    and not args.separate_weight_cast and not args.separate_scale_update)
     traffic = {k: (measured_traffic(wl.name, k) if default_cfg else None)
                for k in ("gemm", "cast", "adamw")}
-    gemm_name = ("k_fp8_gemm<true> block-scaled" if st.recipe == "mxfp8" else "k_fp8_gemm") + \
+    # the block-scaled launch runs 256 x 384 tiles when every GEMM output is at least 512 wide
+    mx_kernel = ("k_fp8_gemm_mx_wide" if min(min(i, o) for _, i, o in wl.layers) >= 512
+                 else "k_fp8_gemm<true>")
+    gemm_name = (mx_kernel + " block-scaled" if st.recipe == "mxfp8" else "k_fp8_gemm") + \
         " (one grouped launch: every fprop, dgrad, wgrad)"
     cast_name = ("k_mx_cast" if st.recipe == "mxfp8" else
                  "k_current_amax + k_cast_rowmajor" if st.recipe == "current" else

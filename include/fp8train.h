@@ -319,7 +319,9 @@ typedef struct fp8t_mx_gemm_desc {
 /*
  * fp8_mx_gemm_multi — several MXFP8 GEMMs in one persistent launch on the block-scaled tensor
  * cores (FP32 accumulation, BF16 output, no per-tensor scale). HOST array of n_gemms (1..4096)
- * descriptors. Errors as fp8_gemm_multi; dimensions must be multiples of 128.
+ * descriptors. Errors as fp8_gemm_multi; dimensions must be multiples of 128. The call runs
+ * 256 x 384 output tiles when every N is at least 512, else 256 x 256 tiles; the results do not
+ * depend on the choice.
  */
 fp8t_status fp8_mx_gemm_multi(const fp8t_mx_gemm_desc* gemms, int32_t n_gemms, void* stream);
 

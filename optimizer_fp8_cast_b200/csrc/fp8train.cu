@@ -20,6 +20,7 @@
 #include "current_scaling.cuh"
 #include "fused_adamw.cuh"
 #include "gemm_tcgen05.cuh"
+#include "gemm_mx_wide.cuh"
 #include "mx_cast.cuh"
 #include "scale_update.cuh"
 
@@ -50,6 +51,7 @@ struct DeviceInfo {
   int gemm_clusters = 0;       // co-resident 2-CTA clusters of the GEMM kernel
   int gemm_wide_clusters = 0;  // ... of its wide-tile form
   int gemm_mx_clusters = 0;    // ... of its MXFP8 variant
+  int gemm_mxw_clusters = 0;   // ... of the MXFP8 256 x 384 kernel
   int mx_cast_blocks_per_sm = 0;
   int cast_blocks_per_sm = 0;
   int cast_rowmajor_blocks_per_sm = 0;
@@ -127,6 +129,21 @@ fp8t_status current_device(DeviceInfo** out) {
         clusters = sms / 2;
       }
       d.gemm_mx_clusters = clusters;
+      e = cudaFuncSetAttribute(fp8t::gemm::k_fp8_gemm_mx_wide,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, fp8t::gemm::kSmemBytesX);
+      if (e != cudaSuccess) {
+        d.state = 0;
+        return fail(FP8T_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+      }
+      cfg.blockDim = dim3(fp8t::gemm::kThreadsX, 1, 1);
+      cfg.dynamicSmemBytes = fp8t::gemm::kSmemBytesX;
+      clusters = 0;
+      e = cudaOccupancyMaxActiveClusters(&clusters, fp8t::gemm::k_fp8_gemm_mx_wide, &cfg);
+      if (e != cudaSuccess || clusters < 1) {
+        (void)cudaGetLastError();
+        clusters = sms / 2;
+      }
+      d.gemm_mxw_clusters = clusters;
       e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.mx_cast_blocks_per_sm, fp8t::mx::k_mx_cast,
                                                         fp8t::mx::kThreads, fp8t::mx::kSmemBytes);
       if (e != cudaSuccess || d.mx_cast_blocks_per_sm < 1) {
@@ -201,6 +218,22 @@ fp8t_status encode_kmajor(CUtensorMap* map, const void* ptr, int64_t rows, int64
                   es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(FP8T_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return FP8T_OK;
+}
+
+// K rows x N bytes, row-major, read as an MN-major operand in boxes of 64 columns x 128 K rows with
+// the 64-byte swizzle, zero fill.
+fp8t_status encode_mn64(CUtensorMap* map, const void* ptr, int64_t K, int64_t N) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(FP8T_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(K)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(N)};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(fp8t::gemm::kBK)};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box,
+                  es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FP8T_ERR_CUDA, "cuTensorMapEncodeTiled (64-column box) failed (%d)", (int)r);
   return FP8T_OK;
 }
 
@@ -482,7 +515,7 @@ constexpr size_t kSumsqHeader = 256;    // ticket and abort words, then the part
 // 3 * tile + part.
 // Launches with more tiles than the table holds keep round-robin (with thousands of tiles it is
 // balanced already).
-void build_schedule(fp8t::gemm::Group& g, int clusters, bool wide) {
+void build_schedule(fp8t::gemm::Group& g, int clusters, bool wide, bool mx_wide = false) {
   using namespace fp8t::gemm;
   g.scheduled = 0;
   if (g.total_tiles > kMaxSchedTiles || clusters > kMaxClusters || clusters < 2) return;
@@ -491,8 +524,14 @@ void build_schedule(fp8t::gemm::Group& g, int clusters, bool wide) {
   items.reserve(g.total_tiles);
   for (int p = 0; p < g.n; ++p) {
     const int end = p + 1 < g.n ? g.p[p + 1].tile_start : g.total_tiles;
-    const int64_t cost = ((g.p[p].K + kBK - 1) / kBK) * (wide ? 2 : 1);
-    for (int t = g.p[p].tile_start; t < end; ++t) items.push_back({cost, t, 0});
+    const int64_t kbs = (g.p[p].K + kBK - 1) / kBK;
+    const int64_t cost = kbs * (wide ? 2 : 1);
+    for (int t = g.p[p].tile_start; t < end; ++t) {
+      // MX 256 x 384 tiles: three 128-column MMAs per k-step, two where N ends within the tile
+      const int nt = (t - g.p[p].tile_start) % g.p[p].tiles_n;
+      const int64_t c = mx_wide ? kbs * (nt * kBNx + 256 < g.p[p].N ? 3 : 2) : cost;
+      items.push_back({c, t, 0});
+    }
   }
   std::stable_sort(items.begin(), items.end(),
                    [](const Item& a, const Item& b) { return a.cost > b.cost; });
@@ -797,13 +836,17 @@ fp8t_status fp8_mx_gemm_multi(const fp8t_mx_gemm_desc* gemms, int32_t n_gemms, v
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(FP8T_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   using namespace fp8t::gemm;
-  // scale atoms viewed as [atoms * 2][256] bytes, read 512 bytes (one atom) at a time
+  // 256 x 384 tiles when every output is at least 512 wide (the choice holds for the whole call)
+  bool mxw = true;
+  for (int32_t i = 0; i < n_gemms; ++i)
+    if (gemms[i].N < 512) mxw = false;
+  // scale atoms viewed as [atoms][512] bytes, read one atom at a time
   auto encode_sf = [&](CUtensorMap* map, const void* ptr, int64_t atoms) -> fp8t_status {
-    cuuint64_t dims[2] = {256, static_cast<cuuint64_t>(atoms * 2)};
-    cuuint64_t strides[1] = {256};
-    cuuint32_t box[2] = {256, 2};
+    cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(atoms)};
+    cuuint64_t strides[1] = {512};
+    cuuint32_t box[2] = {128, 1};
     cuuint32_t es[2] = {1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, es,
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(ptr), dims, strides, box, es,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(FP8T_ERR_CUDA, "cuTensorMapEncodeTiled (scales) failed (%d)", (int)r);
@@ -844,16 +887,21 @@ fp8t_status fp8_mx_gemm_multi(const fp8t_mx_gemm_desc* gemms, int32_t n_gemms, v
       P.b_fmt = d.b_fmt;
       P.kb128 = static_cast<int32_t>(d.K / 128);
       P.sumsq_slot = -1;
-      P.tiles_n = static_cast<int32_t>((d.N + kBN - 1) / kBN);
+      if (mxw && (st = b_mn ? encode_mn64(&P.b64, d.B, d.K, d.N)
+                            : encode_kmajor(&P.b64, d.B, d.N, d.K, kHalf / 2)) != FP8T_OK) return st;
+      P.tiles_n = static_cast<int32_t>((d.N + (mxw ? kBNx : kBN) - 1) / (mxw ? kBNx : kBN));
       P.tile_start = static_cast<int32_t>(tiles);
       tiles += ((d.M + kBM - 1) / kBM) * P.tiles_n;
       if (tiles >= (int64_t(1) << 30))
         return fail(FP8T_ERR_UNSUPPORTED_SHAPE, "fp8_mx_gemm: too many tiles in one launch");
     }
     group.total_tiles = static_cast<int32_t>(tiles);
-    const int64_t grid = 2 * std::min<int64_t>(tiles, dev->gemm_mx_clusters);
-    build_schedule(group, static_cast<int>(grid / 2), false);
-    k_fp8_gemm<true><<<static_cast<unsigned>(grid), kThreads, kSmemBytesMX, as_stream(stream)>>>(group);
+    const int64_t grid = 2 * std::min<int64_t>(tiles, mxw ? dev->gemm_mxw_clusters : dev->gemm_mx_clusters);
+    build_schedule(group, static_cast<int>(grid / 2), false, mxw);
+    if (mxw)
+      k_fp8_gemm_mx_wide<<<static_cast<unsigned>(grid), kThreadsX, kSmemBytesX, as_stream(stream)>>>(group);
+    else
+      k_fp8_gemm<true><<<static_cast<unsigned>(grid), kThreads, kSmemBytesMX, as_stream(stream)>>>(group);
     if ((st = after_launch("fp8_mx_gemm launch")) != FP8T_OK) return st;
   }
   return FP8T_OK;

@@ -148,9 +148,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // One GEMM of a grouped launch. Tiles are numbered problem by problem.
 constexpr int kMaxProblems = 24;
 struct alignas(64) Problem {
+  CUtensorMap b64;               // MX 256 x 384 tiles: B boxes of 64 rows (K-major) or columns
   CUtensorMap a, b, d;           // A [M][K] or [K][M], B [N][K] or [K][N] (128 x 128-byte boxes),
                                  // D [M][N] (32 x 32)
-  CUtensorMap sfa, sfb;          // MX: scale atoms as [atoms * 2][256] bytes, 512-byte boxes
+  CUtensorMap sfa, sfb;          // MX: scale atoms as [atoms][128] 32-bit words, one-atom boxes
   const float* sa;
   const float* sb;
   int32_t M, N, K;
@@ -286,11 +287,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int mt = (local / P.tiles_n), nt = (local % P.tiles_n);
             uint8_t* sf = sSF + s * kSfStageBytes;
             tma_load_2d_pair(smem_u32(sf), &P.sfa, 0,
-                             2 * ((2 * mt + static_cast<int>(rank)) * P.kb128 + kb), full_leader);
-            tma_load_2d_pair(smem_u32(sf + kSfaBytes), &P.sfb, 0, 2 * ((2 * nt) * P.kb128 + kb),
+                             (2 * mt + static_cast<int>(rank)) * P.kb128 + kb, full_leader);
+            tma_load_2d_pair(smem_u32(sf + kSfaBytes), &P.sfb, 0, (2 * nt) * P.kb128 + kb,
                              full_leader);
             tma_load_2d_pair(smem_u32(sf + kSfaBytes + 512), &P.sfb, 0,
-                             2 * ((2 * nt + 1) * P.kb128 + kb), full_leader);
+                             (2 * nt + 1) * P.kb128 + kb, full_leader);
           }
           if (P.a_mn) tma_load_2d_pair(smem_u32(sA + s * kABytes), &P.a, m0, kb * kBK, full_leader);
           else        tma_load_2d_pair(smem_u32(sA + s * kABytes), &P.a, kb * kBK, m0, full_leader);

@@ -87,8 +87,12 @@ def mx_operands(rows, cols, fmt, seed, spread=8.0):
 
 
 @pytest.mark.parametrize("a_mn,b_mn", [(False, False), (False, True), (True, False), (True, True)])
-@pytest.mark.parametrize("M,N,K", [(128, 128, 128), (256, 256, 256), (384, 640, 512)])
+@pytest.mark.parametrize("M,N,K", [(128, 128, 128), (256, 256, 256), (384, 640, 512),
+                                   (256, 512, 256), (128, 896, 384), (256, 1152, 128)])
 def test_mx_gemm_small_full(cuda_lib, a_mn, b_mn, M, N, K):
+    """Every output against the oracle. N < 512 runs the 256 x 256 kernel; N >= 512 the 256 x 384
+    one, whose last column tile may have no rows for its N = 128 MMA (640, 896: 256 and 128 rows
+    left) or only part of its N = 256 MMA's rows (512, 896), and 1152 = 3 x 384 has no such tile."""
     for bf in (oracle.E4M3, oracle.E5M2):
         (qa_r, sa_r), (qa_c, sa_c) = mx_operands(M, K, oracle.E4M3, M + K) if not a_mn else \
             mx_operands(K, M, oracle.E4M3, M + K)
