@@ -18,7 +18,8 @@
 // c ^ (row % 8)) into a double buffer, completion on one mbarrier per buffer. Then, in parallel,
 //   warps 0-3 quantise the column-wise blocks: a thread takes 4 adjacent columns of one block of
 //     32 rows, reads them once (eight-byte shared loads) for the four scales and again to
-//     quantise, and stores each row's four codes as one 4-byte word straight to global memory
+//     quantise (a loop compiled per format and per NaN case, so neither choice is made per
+//     element), and stores each row's four codes as one 4-byte word straight to global memory
 //     (the warp's 32 lanes cover the row's 128 columns, so each store instruction writes one
 //     whole 128-byte line);
 //   warps 4-7 quantise the row-wise blocks straight to global memory: a quarter-warp takes the
@@ -111,6 +112,29 @@ __device__ __forceinline__ uint8_t scale_code(uint32_t m, int X) {
   return m > 0x7F80u ? 0xFF : static_cast<uint8_t>(X + 127);
 }
 
+// Column-wise codes of 4 adjacent columns x 32 rows of a tile (one format per instantiation),
+// each row's four codes stored as one 4-byte word.
+template <int FMT, bool NAN_CHECK>
+__device__ __forceinline__ void col_codes(const uint8_t* xs, int rb, int col, const float (&inv)[4],
+                                          uint8_t* dst, int64_t cols) {
+#pragma unroll 8
+  for (int r = 0; r < 32; ++r) {
+    const uint2 v = *reinterpret_cast<const uint2*>(xs + xoff(32 * rb + r, col));
+    const float p0 = __fmul_rn(__uint_as_float(v.x << 16), inv[0]);
+    const float p1 = __fmul_rn(__uint_as_float(v.x & 0xFFFF0000u), inv[1]);
+    const float p2 = __fmul_rn(__uint_as_float(v.y << 16), inv[2]);
+    const float p3 = __fmul_rn(__uint_as_float(v.y & 0xFFFF0000u), inv[3]);
+    uint32_t c = cvt_fp8x2<FMT>(p0, p1) | (cvt_fp8x2<FMT>(p2, p3) << 16);
+    if (NAN_CHECK) {                       // only a NaN input gives a NaN product
+      if (p0 != p0) c = (c & 0xFFFFFF00u) | 0x7Fu;
+      if (p1 != p1) c = (c & 0xFFFF00FFu) | 0x7F00u;
+      if (p2 != p2) c = (c & 0xFF00FFFFu) | 0x7F0000u;
+      if (p3 != p3) c = (c & 0x00FFFFFFu) | 0x7F000000u;
+    }
+    *reinterpret_cast<uint32_t*>(dst + r * cols) = c;
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 3) k_mx_cast(const __grid_constant__ Group g) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -181,23 +205,11 @@ __global__ void __launch_bounds__(kThreads, 3) k_mx_cast(const __grid_constant__
         }
         const bool nan_block = max(max(m[0], m[1]), max(m[2], m[3])) > 0x7F80u;
         uint8_t* dst = T.q_col + (r0 + 32 * rb) * T.cols + c0 + col;
-#pragma unroll 8
-        for (int r = 0; r < 32; ++r) {
-          const uint2 v = *reinterpret_cast<const uint2*>(xs + xoff(32 * rb + r, col));
-          const float p0 = __fmul_rn(__uint_as_float(v.x << 16), inv[0]);
-          const float p1 = __fmul_rn(__uint_as_float(v.x & 0xFFFF0000u), inv[1]);
-          const float p2 = __fmul_rn(__uint_as_float(v.y << 16), inv[2]);
-          const float p3 = __fmul_rn(__uint_as_float(v.y & 0xFFFF0000u), inv[3]);
-          uint32_t c = T.fmt == 0 ? cvt_fp8x2<0>(p0, p1) | (cvt_fp8x2<0>(p2, p3) << 16)
-                                  : cvt_fp8x2<1>(p0, p1) | (cvt_fp8x2<1>(p2, p3) << 16);
-          if (nan_block) {                       // only a NaN input gives a NaN product
-            if (p0 != p0) c = (c & 0xFFFFFF00u) | 0x7Fu;
-            if (p1 != p1) c = (c & 0xFFFF00FFu) | 0x7F00u;
-            if (p2 != p2) c = (c & 0xFF00FFFFu) | 0x7F0000u;
-            if (p3 != p3) c = (c & 0x00FFFFFFu) | 0x7F000000u;
-          }
-          *reinterpret_cast<uint32_t*>(dst + r * T.cols) = c;
-        }
+        if (nan_block)
+          T.fmt == 0 ? col_codes<0, true>(xs, rb, col, inv, dst, T.cols)
+                     : col_codes<1, true>(xs, rb, col, inv, dst, T.cols);
+        else if (T.fmt == 0) col_codes<0, false>(xs, rb, col, inv, dst, T.cols);
+        else                 col_codes<1, false>(xs, rb, col, inv, dst, T.cols);
 #pragma unroll
         for (int c = 0; c < 4; ++c)
           atom_c[((col + c) & 31) * 16 + ((col + c) >> 5) * 4 + rb] = scale_code(m[c], X[c]);
