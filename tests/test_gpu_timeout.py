@@ -107,3 +107,50 @@ def test_expired_gemm_sum_of_squares_is_nan(cuda_lib):
     cuda_lib.fp8t_check_device_error()
     d = g[0]["D"].float().double()
     assert abs(out.item() - float((d * d).sum())) <= 1e-12 * float((d * d).sum())
+
+
+def _mx_problem(M, N, K, seed):
+    """K-major E4M3 codes and atom-ordered scales of A [M, K] and B [N, K] (plain copies too)."""
+    rng = np.random.default_rng(seed)
+    qa = rng.integers(0x20, 0x48, (M, K)).astype(np.uint8)
+    qb = rng.integers(0x20, 0x48, (N, K)).astype(np.uint8)
+    sa = rng.integers(120, 134, (M, K // 32)).astype(np.uint8)
+    sb = rng.integers(120, 134, (N, K // 32)).astype(np.uint8)
+
+    def atoms(plain):
+        mn, kk = plain.shape
+        a = plain.reshape(mn // 128, 4, 32, kk // 4, 4).transpose(0, 3, 2, 1, 4)
+        return torch.from_numpy(np.ascontiguousarray(a).reshape(-1)).cuda()
+    return qa, qb, sa, sb, atoms(sa), atoms(sb)
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+@pytest.mark.parametrize("N", [1024, 256])
+def test_mx_gemm_waits_expire_and_context_survives(cuda_lib, mode, N):
+    """Both block-scaled kernels (256 x 384 tiles for N >= 512, 256 x 256 below): expired waits,
+    then a correct launch."""
+    M, K = 1024, 2048
+    qa, qb, sa, sb, sa_d, sb_d = _mx_problem(M, N, K, 40 + mode + N)
+    D = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    g = [dict(A=torch.from_numpy(qa).cuda(), a_sf=sa_d, a_fmt=oracle.E4M3,
+              B=torch.from_numpy(qb).cuda(), b_sf=sb_d, b_fmt=oracle.E4M3, D=D)]
+    _run_expired(cuda_lib, mode, lambda: cuda_lib.fp8_mx_gemm_multi(g))
+    cuda_lib.fp8_mx_gemm_multi(g)
+    cuda_lib.fp8t_check_device_error()
+    rng = np.random.default_rng(7)
+    ii = rng.integers(0, M, 512); jj = rng.integers(0, N, 512)
+    R, ab = oracle.mx_gemm_at(qa, sa, oracle.E4M3, qb, sb, oracle.E4M3, ii, jj)
+    assert gemm_within_tolerance(bf16_bits(D)[ii, jj], R, ab).all()
+
+
+def test_mx_cast_waits_expire_and_context_survives(cuda_lib):
+    x = (torch.randn(1024, 2048) * 3).to(torch.bfloat16)
+    xd = x.cuda()
+    q = torch.empty(1024, 2048, dtype=torch.uint8, device="cuda")
+    sf = torch.empty(cuda_lib.mx_scale_bytes(1024, 2048), dtype=torch.uint8, device="cuda")
+    cast = lambda: cuda_lib.fp8_mx_cast_multi([dict(x=xd, fmt=oracle.E4M3, q_row=q, sf_row=sf)])
+    _run_expired(cuda_lib, 1, cast)
+    cast()
+    cuda_lib.fp8t_check_device_error()
+    rq, _ = oracle.mx_quantise(bf16_bits(x), 0, oracle.E4M3)
+    assert np.array_equal(u8(q), rq)
