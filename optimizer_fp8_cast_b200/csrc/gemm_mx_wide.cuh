@@ -12,8 +12,10 @@
 // TMEM per CTA: accumulator 0..383, A scales 384..387, the scales of MMA 0's 256 B rows 388..395,
 // of MMA 1's 128 rows 396..399. Per stage each CTA loads the A box (128 rows), a 128-row and a
 // 64-row B box (MN-major: the 64-column box uses the 64-byte swizzle) and four 512-byte scale
-// atoms: 42 KB, four stages. A column tile that starts within 256 of N's end runs MMA 0 only
-// (N is a multiple of 128, so such a tile has no rows for MMA 1).
+// atoms: 42 KB, four stages; the MMA thread copies the atoms to TMEM (tcgen05.cp 32x128b,
+// replicated to the four lane quarters) before the k-block's MMAs, which select each 32-deep
+// sub-block's scale byte through the descriptor. A column tile that starts within 256 of N's end
+// runs MMA 0 only (N is a multiple of 128, so such a tile has no rows for MMA 1).
 // As in the per-tensor 256 x 512 kernel there is one accumulator: eight epilogue warps (a TMEM
 // lane quarter and a 192-column half each) read it into registers as packed BF16, release it,
 // then store. Waits are bounded as in the other kernels.
