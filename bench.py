@@ -209,7 +209,7 @@ def run_ours(args, rank, world, local_rank):
             if name == "cast" and st.recipe == "mxfp8":
                 st.mx_cast_all(xs, dys)           # X, W, dY: both orientations + block scales
             elif name == "gemm" and st.recipe == "mxfp8":
-                st.mx_gemm_all()                  # grouped block-scaled fprop, dgrad, wgrad
+                st.mx_gemm_all(sumsq=st.fused_norm)   # grouped block-scaled fprop, dgrad, wgrad
             elif name == "cast" and st.recipe == "current":
                 st.amax.zero_()
                 st.cast_all_current(xs, dys)      # amax launch, then the grouped cast

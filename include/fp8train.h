@@ -326,6 +326,25 @@ typedef struct fp8t_mx_gemm_desc {
 fp8t_status fp8_mx_gemm_multi(const fp8t_mx_gemm_desc* gemms, int32_t n_gemms, void* stream);
 
 /*
+ * fp8_mx_gemm_multi_sumsq — fp8_mx_gemm_multi that also leaves in *d_sumsq_out the FP64 sum of
+ * f32(D)^2 over the problems whose sumsq_of entry is nonzero (the wgrad outputs of a step, so
+ * AdamW's global norm needs no pass over the gradients [P1 Fused Optimizer 的意义; 优化器 kernel
+ * 的带宽账]), with the same fixed summation order, workspace rules, zero-on-entry / zero-on-exit
+ * ticket words and NaN result on an expired wait as fp8_gemm_multi_sumsq.
+ *   sumsq_of         HOST array of n_gemms int32 flags.
+ *   d_sumsq_out      1 double (device), written by the launch that finishes the call.
+ *   d_workspace      device scratch of fp8_mx_gemm_sumsq_workspace_bytes, 256-byte aligned,
+ *                    zero-filled once before its first use (the call leaves it zero again).
+ */
+fp8t_status fp8_mx_gemm_multi_sumsq(const fp8t_mx_gemm_desc* gemms, int32_t n_gemms,
+                                    const int32_t* sumsq_of, double* d_sumsq_out,
+                                    void* d_workspace, size_t workspace_bytes, void* stream);
+
+/* Scratch bytes fp8_mx_gemm_multi_sumsq needs (0 on invalid input or no problem selected). */
+size_t fp8_mx_gemm_sumsq_workspace_bytes(const fp8t_mx_gemm_desc* gemms, int32_t n_gemms,
+                                         const int32_t* sumsq_of);
+
+/*
  * fp8_scale_update — roll each tensor's amax history and compute the next scale
  * [P3 核心原理, Scale 决定数值是否进入可表示区间 (scale = (FP8_MAX / amax) / 2^margin) and
  *  Delayed Scaling 用历史换取稳定性 (history window; max / most_recent; used next iteration)].

@@ -19,6 +19,7 @@ __all__ = ["fp8_cast_transpose_amax", "fp8_cast_transpose_amax_multi",
            "fused_adamw_workspace_bytes", "fused_adamw_multi_tensor_noalloc",
            "fp8_gemm_multi_sumsq", "fp8_gemm_sumsq_workspace_bytes",
            "fused_adamw_multi_tensor_presummed", "fp8_mx_cast_multi", "fp8_mx_gemm_multi",
+           "fp8_mx_gemm_multi_sumsq", "fp8_mx_gemm_sumsq_workspace_bytes",
            "mx_scale_bytes",
            "fp8t_check_device_error", "fp8t_debug_expire_waits", "fp8t_set_wait_timeout_ns",
            "Fp8TrainError", "E4M3", "E5M2", "K_MAJOR", "MN_MAJOR", "AMAX_MAX", "AMAX_MOST_RECENT", "FP8_MAX", "load",
@@ -213,9 +214,7 @@ def fp8_mx_cast_multi(casts, stream=None):
     _check(load().fp8_mx_cast_multi(arr, len(casts), _stream(stream)), "fp8_mx_cast_multi")
 
 
-def fp8_mx_gemm_multi(gemms, stream=None):
-    """Block-scaled FP8 GEMMs in one launch: dicts with A, a_sf, a_fmt, (a_mn), B, b_sf, b_fmt,
-    (b_mn), D; D = bf16(A . B^T) with the operands' block scales (no per-tensor scale)."""
+def _mx_gemm_array(gemms):
     arr = (_abi.MxGemmDesc * len(gemms))()
     for i, g in enumerate(gemms):
         M, N, K = _gemm_shape(g)
@@ -225,7 +224,35 @@ def fp8_mx_gemm_multi(gemms, stream=None):
                                  MN_MAJOR if g.get("a_mn") else K_MAJOR, _ptr(g["B"]), _ptr(g["b_sf"]),
                                  int(g["b_fmt"]), MN_MAJOR if g.get("b_mn") else K_MAJOR, M, N, K,
                                  _ptr(D))
-    _check(load().fp8_mx_gemm_multi(arr, len(gemms), _stream(stream)), "fp8_mx_gemm_multi")
+    return arr
+
+
+def fp8_mx_gemm_multi(gemms, stream=None):
+    """Block-scaled FP8 GEMMs in one launch: dicts with A, a_sf, a_fmt, (a_mn), B, b_sf, b_fmt,
+    (b_mn), D; D = bf16(A . B^T) with the operands' block scales (no per-tensor scale)."""
+    _check(load().fp8_mx_gemm_multi(_mx_gemm_array(gemms), len(gemms), _stream(stream)),
+           "fp8_mx_gemm_multi")
+
+
+def fp8_mx_gemm_sumsq_workspace_bytes(gemms):
+    """Scratch bytes of fp8_mx_gemm_multi_sumsq for these problems (dicts with a ``sumsq`` flag;
+    only their shapes are read)."""
+    flags = (C.c_int32 * len(gemms))(*[1 if g.get("sumsq") else 0 for g in gemms])
+    arr = (_abi.MxGemmDesc * len(gemms))()
+    for i, g in enumerate(gemms):
+        arr[i].M, arr[i].N, arr[i].K = _gemm_shape(g)
+    return int(load().fp8_mx_gemm_sumsq_workspace_bytes(arr, len(gemms), flags))
+
+
+def fp8_mx_gemm_multi_sumsq(gemms, sumsq_out, workspace, stream=None):
+    """fp8_mx_gemm_multi that also writes into ``sumsq_out`` (float64 [1]) the FP64 sum of
+    f32(D)^2 over the problems whose dict has ``sumsq=True``. ``workspace``: uint8 CUDA tensor of
+    fp8_mx_gemm_sumsq_workspace_bytes, zero-filled once before its first use."""
+    flags = (C.c_int32 * len(gemms))(*[1 if g.get("sumsq") else 0 for g in gemms])
+    assert sumsq_out.dtype == torch.float64
+    _check(load().fp8_mx_gemm_multi_sumsq(_mx_gemm_array(gemms), len(gemms), flags, _ptr(sumsq_out),
+                                          _ptr(workspace), workspace.numel(), _stream(stream)),
+           "fp8_mx_gemm_multi_sumsq")
 
 
 def fp8_scale_update(amax, history, fp8_max, algo, margin, scale, scale_inv, stream=None):

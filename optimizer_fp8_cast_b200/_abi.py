@@ -85,6 +85,11 @@ def declare(L):
     L.fp8_mx_cast_multi.argtypes = [C.POINTER(MxCastTensor), i32, vp]
     L.fp8_mx_gemm_multi.restype = C.c_int
     L.fp8_mx_gemm_multi.argtypes = [C.POINTER(MxGemmDesc), i32, vp]
+    L.fp8_mx_gemm_multi_sumsq.restype = C.c_int
+    L.fp8_mx_gemm_multi_sumsq.argtypes = [C.POINTER(MxGemmDesc), i32, C.POINTER(C.c_int32), vp, vp,
+                                          C.c_size_t, vp]
+    L.fp8_mx_gemm_sumsq_workspace_bytes.restype = C.c_size_t
+    L.fp8_mx_gemm_sumsq_workspace_bytes.argtypes = [C.POINTER(MxGemmDesc), i32, C.POINTER(C.c_int32)]
     L.fp8_gemm.restype = C.c_int
     L.fp8_gemm.argtypes = [vp, C.c_int, vp, C.c_int, i64, i64, i64, vp, vp, vp, vp]
     L.fp8_scale_update.restype = C.c_int

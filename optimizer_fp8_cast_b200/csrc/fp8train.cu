@@ -810,7 +810,30 @@ fp8t_status fp8_mx_cast_multi(const fp8t_mx_cast_tensor* tensors, int32_t n_tens
   return FP8T_OK;
 }
 
-fp8t_status fp8_mx_gemm_multi(const fp8t_mx_gemm_desc* gemms, int32_t n_gemms, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// MX launches use 256 x 384 tiles when every output is at least 512 wide (for the whole call).
+bool mx_use_wide(const fp8t_mx_gemm_desc* gemms, int32_t n) {
+  for (int32_t i = 0; i < n; ++i)
+    if (gemms[i].N < 512) return false;
+  return true;
+}
+
+int64_t mx_sumsq_slots(const fp8t_mx_gemm_desc* gemms, int32_t n, const int32_t* sumsq_of) {
+  using namespace fp8t::gemm;
+  const bool wide = mx_use_wide(gemms, n);
+  const int64_t bn = wide ? kBNx : kBN, per_tile = wide ? kSumsqPerTileW : kSumsqPerTile;
+  int64_t slots = 0;
+  for (int32_t i = 0; i < n; ++i)
+    if (sumsq_of[i]) slots += ((gemms[i].M + kBM - 1) / kBM) * ((gemms[i].N + bn - 1) / bn) * per_tile;
+  return slots;
+}
+
+fp8t_status mx_gemm_multi(const fp8t_mx_gemm_desc* gemms, int32_t n_gemms, const int32_t* sumsq_of,
+                          double* d_sumsq_out, void* d_workspace, size_t workspace_bytes,
+                          void* stream) {
   t_last_error.clear();
   if (!gemms || n_gemms < 1 || n_gemms > 4096)
     return fail(FP8T_ERR_INVALID_ARG, "fp8_mx_gemm: gemms NULL or n_gemms out of range");
@@ -830,6 +853,17 @@ fp8t_status fp8_mx_gemm_multi(const fp8t_mx_gemm_desc* gemms, int32_t n_gemms, v
         !aligned(d.B_scales, 16))
       return fail(FP8T_ERR_MISALIGNED, "fp8_mx_gemm: problem %d: pointers must be 16-byte aligned", i);
   }
+  int64_t n_slots = 0;
+  if (sumsq_of) {
+    if (!d_sumsq_out || !aligned(d_sumsq_out, 8) || !d_workspace || !aligned(d_workspace, 256))
+      return fail(FP8T_ERR_INVALID_ARG, "fp8_mx_gemm_multi_sumsq: NULL or misaligned sumsq_out or workspace");
+    n_slots = mx_sumsq_slots(gemms, n_gemms, sumsq_of);
+    if (n_slots < 1 || n_slots >= (int64_t(1) << 31))
+      return fail(FP8T_ERR_INVALID_ARG, "fp8_mx_gemm_multi_sumsq: no problem (or too many tiles) selected");
+    const size_t need = kSumsqHeader + static_cast<size_t>(n_slots) * 8;
+    if (workspace_bytes < need)
+      return fail(FP8T_ERR_INVALID_ARG, "fp8_mx_gemm_multi_sumsq: workspace of %zu bytes needed", need);
+  }
   DeviceInfo* dev = nullptr;
   fp8t_status st = current_device(&dev);
   if (st != FP8T_OK) return st;
@@ -837,9 +871,8 @@ fp8t_status fp8_mx_gemm_multi(const fp8t_mx_gemm_desc* gemms, int32_t n_gemms, v
   if (!fn) return fail(FP8T_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   using namespace fp8t::gemm;
   // 256 x 384 tiles when every output is at least 512 wide (the choice holds for the whole call)
-  bool mxw = true;
-  for (int32_t i = 0; i < n_gemms; ++i)
-    if (gemms[i].N < 512) mxw = false;
+  const bool mxw = mx_use_wide(gemms, n_gemms);
+  int64_t slot = 0;
   // scale atoms viewed as [atoms][512] bytes, read one atom at a time
   auto encode_sf = [&](CUtensorMap* map, const void* ptr, int64_t atoms) -> fp8t_status {
     cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(atoms)};
@@ -857,6 +890,14 @@ fp8t_status fp8_mx_gemm_multi(const fp8t_mx_gemm_desc* gemms, int32_t n_gemms, v
     const int32_t b1 = std::min<int32_t>(n_gemms, b0 + kMaxProblems);
     std::memset(&group, 0, sizeof(group));
     group.n = b1 - b0;
+    if (sumsq_of) {
+      group.ticket = static_cast<unsigned int*>(d_workspace);
+      group.abort_word = static_cast<unsigned int*>(d_workspace) + 1;
+      group.partials = reinterpret_cast<double*>(static_cast<char*>(d_workspace) + kSumsqHeader);
+      group.sumsq_out = d_sumsq_out;
+      group.n_partials = static_cast<int32_t>(n_slots);
+      group.last_launch = b1 == n_gemms ? 1 : 0;
+    }
     int64_t tiles = 0;
     for (int32_t i = b0; i < b1; ++i) {
       const fp8t_mx_gemm_desc& d = gemms[i];
@@ -891,7 +932,12 @@ fp8t_status fp8_mx_gemm_multi(const fp8t_mx_gemm_desc* gemms, int32_t n_gemms, v
                             : encode_kmajor(&P.b64, d.B, d.N, d.K, kHalf / 2)) != FP8T_OK) return st;
       P.tiles_n = static_cast<int32_t>((d.N + (mxw ? kBNx : kBN) - 1) / (mxw ? kBNx : kBN));
       P.tile_start = static_cast<int32_t>(tiles);
-      tiles += ((d.M + kBM - 1) / kBM) * P.tiles_n;
+      const int64_t p_tiles = ((d.M + kBM - 1) / kBM) * P.tiles_n;
+      if (sumsq_of && sumsq_of[i]) {
+        P.sumsq_slot = static_cast<int32_t>(slot);
+        slot += p_tiles * (mxw ? kSumsqPerTileW : kSumsqPerTile);
+      }
+      tiles += p_tiles;
       if (tiles >= (int64_t(1) << 30))
         return fail(FP8T_ERR_UNSUPPORTED_SHAPE, "fp8_mx_gemm: too many tiles in one launch");
     }
@@ -905,6 +951,34 @@ fp8t_status fp8_mx_gemm_multi(const fp8t_mx_gemm_desc* gemms, int32_t n_gemms, v
     if ((st = after_launch("fp8_mx_gemm launch")) != FP8T_OK) return st;
   }
   return FP8T_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+fp8t_status fp8_mx_gemm_multi(const fp8t_mx_gemm_desc* gemms, int32_t n_gemms, void* stream) {
+  return mx_gemm_multi(gemms, n_gemms, nullptr, nullptr, nullptr, 0, stream);
+}
+
+size_t fp8_mx_gemm_sumsq_workspace_bytes(const fp8t_mx_gemm_desc* gemms, int32_t n_gemms,
+                                         const int32_t* sumsq_of) {
+  if (!gemms || !sumsq_of || n_gemms < 1 || n_gemms > 4096) return 0;
+  for (int32_t i = 0; i < n_gemms; ++i)
+    if (gemms[i].M <= 0 || gemms[i].N <= 0) return 0;
+  const int64_t slots = mx_sumsq_slots(gemms, n_gemms, sumsq_of);
+  if (slots < 1) return 0;
+  return kSumsqHeader + static_cast<size_t>(slots) * 8;
+}
+
+fp8t_status fp8_mx_gemm_multi_sumsq(const fp8t_mx_gemm_desc* gemms, int32_t n_gemms,
+                                    const int32_t* sumsq_of, double* d_sumsq_out,
+                                    void* d_workspace, size_t workspace_bytes, void* stream) {
+  if (!sumsq_of) {
+    t_last_error.clear();
+    return fail(FP8T_ERR_INVALID_ARG, "fp8_mx_gemm_multi_sumsq: sumsq_of NULL");
+  }
+  return mx_gemm_multi(gemms, n_gemms, sumsq_of, d_sumsq_out, d_workspace, workspace_bytes, stream);
 }
 
 fp8t_status fp8_gemm(const void* A, fp8t_format a_fmt, const void* B, fp8t_format b_fmt, int64_t M,

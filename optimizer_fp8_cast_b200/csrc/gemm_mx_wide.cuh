@@ -18,7 +18,9 @@
 // runs MMA 0 only (N is a multiple of 128, so such a tile has no rows for MMA 1).
 // As in the per-tensor 256 x 512 kernel there is one accumulator: eight epilogue warps (a TMEM
 // lane quarter and a 192-column half each) read it into registers as packed BF16, release it,
-// then store. Waits are bounded as in the other kernels.
+// then store. Summed problems (the wgrad outputs of a step) also leave f32(bf16(D))^2 per warp and
+// tile in a partial slot, added up in index order by the last CTA, as in the per-tensor kernels.
+// Waits are bounded as in the other kernels.
 #pragma once
 
 #include "gemm_tcgen05.cuh"
@@ -272,6 +274,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsX, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&S->acc_empty), 0));
+      const bool sumsq = P.sumsq_slot >= 0;
+      double ss = 0.0;
 #pragma unroll
       for (int c = 0; c < kAccColsX / 32; ++c) {
         if (n0 + c * 32 >= N || row0 >= M) continue;       // chunk entirely outside the matrix
@@ -281,6 +285,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsX, 1)
         __syncwarp();
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
+          if (sumsq) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint32_t v = w[c][4 * p + q];
+              const double lo = __uint_as_float(v << 16), hi = __uint_as_float(v & 0xFFFF0000u);
+              ss = __fma_rn(lo, lo, ss);
+              ss = __fma_rn(hi, hi, ss);
+            }
+          }
           const int pp = p ^ ((lane >> 1) & 3);
           *reinterpret_cast<uint4*>(buf + lane * 64 + pp * 16) =
               make_uint4(w[c][4 * p], w[c][4 * p + 1], w[c][4 * p + 2], w[c][4 * p + 3]);
@@ -290,6 +303,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsX, 1)
         if (lane == 0) {
           tma_store_2d(&P.d, smem_u32(buf), n0 + c * 32, row0);
           bulk_commit_group();
+        }
+      }
+      if (sumsq) {                       // this warp's rows of the tile: one partial slot
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, o));
+        if (lane == 0) {
+          g.partials[P.sumsq_slot + local_tile * kSumsqPerTileW + static_cast<int>(rank) * kEpiWarpsX +
+                     half * 4 + quad] = ss;
+          __threadfence();
         }
       }
     }
@@ -306,6 +328,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsX, 1)
   cluster_sync();
   tc_fence_after();
   if (warp == 1) tmem_dealloc_pair(tmem, kTmemCols);
+
+  // ---------------- sum of squares: the last CTA of the last launch adds the slots in order
+  if (!g.sumsq_out) return;
+  if (threadIdx.x == 0 && *abort_flag) atomicOr(g.abort_word, 1u);
+  if (!g.last_launch) return;
+  __shared__ int s_last;
+  double* s_part = reinterpret_cast<double*>(sStage);   // the stage buffers are idle by now
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(g.ticket, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  double acc = 0.0;
+  for (int i = threadIdx.x; i < g.n_partials; i += kThreadsX) acc = __dadd_rn(acc, __ldcg(g.partials + i));
+  s_part[threadIdx.x] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double total = 0.0;
+    for (int i = 0; i < kThreadsX; ++i) total = __dadd_rn(total, s_part[i]);
+    if (*reinterpret_cast<volatile unsigned int*>(g.abort_word) != 0u)
+      total = __longlong_as_double(0x7FF8000000000000LL);
+    *g.sumsq_out = total;
+    atomicExch(g.abort_word, 0u);
+    atomicExch(g.ticket, 0u);
+  }
 }
 
 }  // namespace gemm

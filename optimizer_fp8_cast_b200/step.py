@@ -30,7 +30,8 @@ from . import (AMAX_MAX, AMAX_MOST_RECENT, CURRENT_WORKSPACE_BYTES, E4M3, E5M2, 
                fp8_cast_transpose_amax, fp8_cast_transpose_amax_current_multi,
                fp8_cast_transpose_amax_multi, fp8_cast_transpose_amax_update_multi,
                fp8_gemm_multi, fp8_gemm_multi_sumsq, fp8_gemm_sumsq_workspace_bytes,
-               fp8_mx_cast_multi, fp8_mx_gemm_multi, mx_scale_bytes,
+               fp8_mx_cast_multi, fp8_mx_gemm_multi, fp8_mx_gemm_multi_sumsq,
+               fp8_mx_gemm_sumsq_workspace_bytes, mx_scale_bytes,
                fp8_scale_update, fused_adamw_multi_tensor, fused_adamw_multi_tensor_presummed,
                fused_adamw_workspace_bytes)
 
@@ -111,7 +112,6 @@ class Fp8LinearStep:
             fused_update = fused_wcast = False
             self.fused_update = False
         if recipe == "mxfp8":
-            self.fused_norm = fused_norm = False
             u8 = dict(dtype=torch.uint8, device=self.device)
             for L in self.layers:
                 shapes = dict(X=(tokens, L.fin), W=(L.fin, L.fout), dY=(tokens, L.fout))
@@ -120,6 +120,9 @@ class Fp8LinearStep:
                     L.mx[name] = dict(q_row=torch.empty(r, c, **u8), q_col=torch.empty(r, c, **u8),
                                       sf_row=torch.empty(mx_scale_bytes(r, c), **u8),
                                       sf_col=torch.empty(mx_scale_bytes(c, r), **u8))
+            if self.fused_norm:            # the wgrad epilogues of the block-scaled launch sum dW^2
+                mws = fp8_mx_gemm_sumsq_workspace_bytes(self.mx_gemm_descs(sumsq=True))
+                self.mx_gemm_workspace = torch.zeros(mws, **u8)
         # the W cast inside AdamW needs the in-launch scale update and the presummed AdamW, and
         # writes row-major codes only; the saturation / zero counters of W are only kept by the
         # separate cast
@@ -186,7 +189,7 @@ class Fp8LinearStep:
                 casts.append(dict(x=src, fmt=E4M3, **L.mx[name]))
         fp8_mx_cast_multi(casts, stream=stream)
 
-    def mx_gemm_descs(self):
+    def mx_gemm_descs(self, sumsq=False):
         out = []
         for L in self.layers:
             X, W, dY = L.mx["X"], L.mx["W"], L.mx["dY"]
@@ -195,12 +198,17 @@ class Fp8LinearStep:
                     dict(A=dY["q_row"], a_sf=dY["sf_row"], a_fmt=E4M3, B=W["q_row"], b_sf=W["sf_row"],
                          b_fmt=E4M3, D=L.dX),
                     dict(A=X["q_col"], a_sf=X["sf_col"], a_mn=True, a_fmt=E4M3, B=dY["q_col"],
-                         b_sf=dY["sf_col"], b_mn=True, b_fmt=E4M3, D=L.dW)]
+                         b_sf=dY["sf_col"], b_mn=True, b_fmt=E4M3, D=L.dW, sumsq=sumsq)]
         return out
 
-    def mx_gemm_all(self, stream=None):
-        """The block-scaled fprop, dgrad and wgrad of every layer in one grouped launch."""
-        fp8_mx_gemm_multi(self.mx_gemm_descs(), stream=stream)
+    def mx_gemm_all(self, stream=None, sumsq=False):
+        """The block-scaled fprop, dgrad and wgrad of every layer in one grouped launch; with sumsq
+        the wgrad epilogues also leave the FP64 sum of dW^2 in self.sumsq."""
+        if sumsq:
+            fp8_mx_gemm_multi_sumsq(self.mx_gemm_descs(sumsq=True), self.sumsq, self.mx_gemm_workspace,
+                                    stream=stream)
+        else:
+            fp8_mx_gemm_multi(self.mx_gemm_descs(), stream=stream)
 
     def cast_all_current(self, xs, dys, stream=None):
         """Current scaling: the X, W and dY scales from their own amax, then the casts."""
@@ -296,8 +304,8 @@ class Fp8LinearStep:
         self.t += 1
         if self.recipe == "mxfp8":
             self.mx_cast_all(xs, dys, stream)
-            self.mx_gemm_all(stream)
-            self.adamw(stream)
+            self.mx_gemm_all(stream, sumsq=self.fused_norm)
+            self.adamw(stream, presummed=self.fused_norm)
             return
         if self.recipe == "current":
             self.amax.zero_()                  # amax slots report this step's tensors only
@@ -363,7 +371,8 @@ class Fp8LinearStep:
         n_cast_launches = (per_layer * len(self.layers) + 7) // 8
         n_gemm_launches = (3 * len(self.layers) + 23) // 24
         if self.recipe == "mxfp8":
-            return (3 * len(self.layers) + 7) // 8 + (3 * len(self.layers) + 23) // 24 + 2 * n_adamw_batches
+            return ((3 * len(self.layers) + 7) // 8 + (3 * len(self.layers) + 23) // 24 +
+                    (1 if self.fused_norm else 2) * n_adamw_batches)
         n_scale_launches = 0 if (self.fused_update and not self.side_update) or self.recipe == "current" else 1
         if self.recipe == "current":
             n_cast_launches *= 2                   # an amax launch before each cast launch

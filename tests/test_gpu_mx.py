@@ -147,3 +147,46 @@ def test_mx_step_gemms_full_size_sampled(cuda_lib):
         ii, jj = sample_positions(D.shape[0], D.shape[1], 4096, seed=D.shape[0] + 7)
         R, ab = oracle.mx_gemm_at(np.ascontiguousarray(A), sa, E, np.ascontiguousarray(B), sb, E, ii, jj)
         assert gemm_within_tolerance(bf16_bits(D)[ii, jj], R, ab).all()
+
+
+@pytest.mark.parametrize("shapes", [[(256, 768, 512), (384, 512, 256), (256, 1152, 384)],
+                                    [(256, 256, 512), (128, 384, 256)]])
+def test_mx_gemm_sum_of_squares(cuda_lib, shapes):
+    """fp8_mx_gemm_multi_sumsq: the first list runs the 256 x 384 kernel (every N >= 512), the
+    second the 256 x 256 one. Every output against the oracle, the FP64 sum of f32(D)^2 over the
+    flagged problems against numpy's, a repeat with identical bits, the workspace left at zero."""
+    probs = []
+    for i, (M, N, K) in enumerate(shapes):
+        a_mn, b_mn = bool(i % 2), bool((i // 2) % 2) or i == 0
+        (qa_r, sa_r), (qa_c, sa_c) = mx_operands(M, K, oracle.E4M3, 900 + i) if not a_mn else \
+            mx_operands(K, M, oracle.E4M3, 900 + i)
+        (qb_r, sb_r), (qb_c, sb_c) = mx_operands(N, K, oracle.E4M3, 950 + i) if not b_mn else \
+            mx_operands(K, N, oracle.E4M3, 950 + i)
+        A_dev, A_log, sa_log = (qa_c, qa_c.T, sa_c.T) if a_mn else (qa_r, qa_r, sa_r)
+        B_dev, B_log, sb_log = (qb_c, qb_c.T, sb_c.T) if b_mn else (qb_r, qb_r, sb_r)
+        probs.append(dict(
+            desc=dict(A=torch.from_numpy(np.ascontiguousarray(A_dev)).cuda(), a_mn=a_mn,
+                      a_sf=to_atoms(np.ascontiguousarray(sa_log)), a_fmt=oracle.E4M3,
+                      B=torch.from_numpy(np.ascontiguousarray(B_dev)).cuda(), b_mn=b_mn,
+                      b_sf=to_atoms(np.ascontiguousarray(sb_log)), b_fmt=oracle.E4M3, sumsq=i != 1,
+                      D=torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")),
+            ref=(A_log, sa_log, B_log, sb_log)))
+    descs = [p["desc"] for p in probs]
+    ws = torch.zeros(cuda_lib.fp8_mx_gemm_sumsq_workspace_bytes(descs), dtype=torch.uint8, device="cuda")
+    out = torch.zeros(1, dtype=torch.float64, device="cuda")
+    cuda_lib.fp8_mx_gemm_multi_sumsq(descs, out, ws)
+    cuda_lib.fp8t_check_device_error()
+    first = out.item()
+    for p in probs:
+        A_log, sa_log, B_log, sb_log = p["ref"]
+        R, ab = oracle.mx_gemm(A_log, sa_log, oracle.E4M3, B_log, sb_log, oracle.E4M3, want_abs=True)
+        ok = gemm_within_tolerance(bf16_bits(p["desc"]["D"]), R, ab)
+        assert ok.all(), f"{(~ok).sum()} of {ok.size} outside tolerance"
+    squares = np.concatenate([np.square(p["desc"]["D"].float().cpu().numpy().astype(np.float64)).reshape(-1)
+                              for p in probs if p["desc"]["sumsq"]])
+    exact = float(np.sum(np.sort(squares)))
+    assert abs(first - exact) <= 1e-13 * exact
+    assert not ws[:8].any()
+    cuda_lib.fp8_mx_gemm_multi_sumsq(descs, out, ws)
+    cuda_lib.fp8t_check_device_error()
+    assert np.float64(out.item()).view(np.uint64) == np.float64(first).view(np.uint64)

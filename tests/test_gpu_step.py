@@ -377,16 +377,22 @@ def test_current_scaling_steps(cuda_lib):
         _check_adamw_on_gpu_grad(st, pre_opt, t + 1)
 
 
-def test_mxfp8_steps(cuda_lib):
-    """Two steps of the 256 x 256 / 512-token Linear with the MXFP8 recipe: X, W, dY quantised
-    with E4M3 codes and E8M0 block scales in both orientations (oracle mx_quantise, bit for bit),
-    the three block-scaled GEMMs in one launch (oracle mx_gemm on every output) and AdamW on the
-    GPU's dW (oracle fused_adamw: norm within 2 ulp, master, m, v within 4 ulp)."""
+@pytest.mark.parametrize("fin,fout,fused_norm", [(256, 256, True), (256, 256, False), (512, 640, True)],
+                         ids=["256x256-fused-norm", "256x256-norm-pass", "512x640-fused-norm"])
+def test_mxfp8_steps(cuda_lib, fin, fout, fused_norm):
+    """Two steps of a Linear (512 tokens) with the MXFP8 recipe: X, W, dY quantised with E4M3
+    codes and E8M0 block scales in both orientations (oracle mx_quantise, bit for bit), the three
+    block-scaled GEMMs in one launch (oracle mx_gemm on every output; 512 x 640 runs the 256 x 384
+    tiles, 256 x 256 the 256 x 256 ones), the sum of dW^2 from the wgrad epilogue (against numpy's)
+    or AdamW's norm pass, and AdamW on the GPU's dW (oracle fused_adamw: norm within 2 ulp,
+    master, m, v within 4 ulp)."""
+    import dataclasses
     from tests.test_gpu_mx import from_atoms
-    wl = synth.LINEAR256
-    st = Fp8LinearStep([(256, 256)], wl.tokens, wl.history_len, wl.algo, 0, wl.adamw,
-                       [synth.linear_weight(wl, 0, "cuda")], "cuda", recipe="mxfp8")
-    assert st.kernels_per_step() == 4 and not st.fused_norm
+    wl = dataclasses.replace(synth.LINEAR256, layers=[("linear", fin, fout)])
+    st = Fp8LinearStep([(fin, fout)], wl.tokens, wl.history_len, wl.algo, 0, wl.adamw,
+                       [synth.linear_weight(wl, 0, "cuda")], "cuda", recipe="mxfp8",
+                       fused_norm=fused_norm)
+    assert st.kernels_per_step() == (3 if fused_norm else 4) and st.fused_norm == fused_norm
     E = oracle.E4M3
     T = wl.tokens
     for t in range(2):
@@ -412,6 +418,10 @@ def test_mxfp8_steps(cuda_lib):
                                 (L.dW, tr(xc), tr(xcs), tr(dc), tr(dcs))):
             R, ab = oracle.mx_gemm(A, sa, E, B, sb, E, want_abs=True)
             assert gemm_within_tolerance(bf16_bits(D), R, ab).all()
+        if fused_norm:
+            sq = np.sort(np.square(L.dW.float().cpu().numpy().astype(np.float64)).reshape(-1))
+            exact = float(np.sum(sq))
+            assert abs(st.sumsq.item() - exact) <= 1e-13 * exact
         _check_adamw_on_gpu_grad(st, pre_opt, t + 1)
 
 

@@ -21,7 +21,8 @@ def test_launch_counts_per_configuration():
     assert make(counters=True).kernels_per_step() == 3                    # W cast back in the cast launch
     assert make(fused_update=False, fused_norm=False, fused_wcast=False).kernels_per_step() == 5
     assert make(recipe="current").kernels_per_step() == 4                 # amax launch + cast
-    assert make(recipe="mxfp8").kernels_per_step() == 4                   # MX cast, GEMM, AdamW x2
+    assert make(recipe="mxfp8").kernels_per_step() == 3                   # MX cast, GEMM (+ dW^2), AdamW
+    assert make(recipe="mxfp8", fused_norm=False).kernels_per_step() == 4  # AdamW with its norm pass
     assert make(layers=3).kernels_per_step() == 4                         # 9 casts: two cast launches
     assert make(layers=9).kernels_per_step() == 4 + 2 + 1                 # 27 casts, 27 GEMMs: 4 + 2 launches
 
