@@ -11,8 +11,10 @@
 // warp max-accumulates into a per-tensor word of a small workspace; the CTA that finishes last
 // (ticket counter in the same workspace) turns every amax into its scale and zeroes the words
 // again. The cast itself then runs as usual with that scale (and records the amax in the
-// caller's slot). Traffic: 2 B read per element (the cast reads the tensor again; for tensors that
-// fit in L2 that second read is served there).
+// caller's slot). Traffic: 2 B read per element, and the cast reads the tensors again. This pass
+// takes them last to first with loads of normal L2 priority, so the cast, going first to last,
+// starts on what the pass read most recently: on the 4096 step (X, W, dY: 168 MB) that part is
+// still in L2 and the cast launch pair takes 80.6 instead of 85.4 µs.
 #pragma once
 
 #include "ptx.cuh"
@@ -37,21 +39,23 @@ struct Group {
 __global__ void __launch_bounds__(kThreads) k_current_amax(const __grid_constant__ Group g) {
   const int tid = threadIdx.x;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
-  for (int t = 0; t < g.n; ++t) {
+  // last tensor first: the cast launch that follows reads the tensors first to last, so it starts
+  // on the ones this pass read most recently, still in L2
+  for (int t = g.n - 1; t >= 0; --t) {
     const uint4* __restrict__ x = g.x[t];
     uint32_t m2 = 0;
     int64_t v = static_cast<int64_t>(blockIdx.x) * kThreads + tid;
     for (; v + 3 * stride < g.nvec[t]; v += 4 * stride) {      // four 16-byte loads in flight
       uint4 a[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) a[u] = ld_stream_u4(x + v + u * stride);
+      for (int u = 0; u < 4; ++u) a[u] = __ldg(x + v + u * stride);   // kept in L2 for the cast
 #pragma unroll
       for (int u = 0; u < 4; ++u)
         m2 = __vmaxu2(__vmaxu2(m2, __vmaxu2(a[u].x & 0x7FFF7FFFu, a[u].y & 0x7FFF7FFFu)),
                       __vmaxu2(a[u].z & 0x7FFF7FFFu, a[u].w & 0x7FFF7FFFu));
     }
     for (; v < g.nvec[t]; v += stride) {
-      const uint4 a = ld_stream_u4(x + v);
+      const uint4 a = __ldg(x + v);
       m2 = __vmaxu2(__vmaxu2(m2, __vmaxu2(a.x & 0x7FFF7FFFu, a.y & 0x7FFF7FFFu)),
                     __vmaxu2(a.z & 0x7FFF7FFFu, a.w & 0x7FFF7FFFu));
     }

@@ -511,8 +511,10 @@ constexpr size_t kSumsqHeader = 256;    // ticket and abort words, then the part
 // whole one, not 0.5: it runs half the MMAs but loads all of A, the operand-starved pattern the
 // wide tile avoids. (On the 4096 step this takes the busiest cluster from 704 to 678 k-block
 // units with 28 splits, and the launch from ~0.295 to ~0.292 ms; costing halves at 0.5 split
-// more and gained less.) Every cluster then runs its items in index order. Items are
-// 3 * tile + part.
+// more and gained less. Timed per cluster, a half tile's k-block costs 0.76 of a whole one's and
+// wgrad's k-blocks 8% more than dgrad's; costing the items that way, or running halves last,
+// changed the launch by less than its run-to-run spread.) Every cluster then runs its items in
+// index order. Items are 3 * tile + part.
 // Launches with more tiles than the table holds keep round-robin (with thousands of tiles it is
 // balanced already).
 void build_schedule(fp8t::gemm::Group& g, int clusters, bool wide, bool mx_wide = false) {
