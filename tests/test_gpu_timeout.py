@@ -154,3 +154,22 @@ def test_mx_cast_waits_expire_and_context_survives(cuda_lib):
     cuda_lib.fp8t_check_device_error()
     rq, _ = oracle.mx_quantise(bf16_bits(x), 0, oracle.E4M3)
     assert np.array_equal(u8(q), rq)
+
+
+@pytest.mark.parametrize("N", [1024, 256])
+def test_expired_mx_gemm_sum_of_squares_is_nan(cuda_lib, N):
+    """fp8_mx_gemm_multi_sumsq (both block-scaled kernels) with expired epilogue waits reports a
+    NaN sum and leaves its workspace words at zero; the next call gives the exact sum again."""
+    M, K = 1024, 1024
+    qa, qb, sa, sb, sa_d, sb_d = _mx_problem(M, N, K, 60 + N)
+    g = [dict(A=torch.from_numpy(qa).cuda(), a_sf=sa_d, a_fmt=oracle.E4M3,
+              B=torch.from_numpy(qb).cuda(), b_sf=sb_d, b_fmt=oracle.E4M3, sumsq=True,
+              D=torch.empty(M, N, dtype=torch.bfloat16, device="cuda"))]
+    ws = torch.zeros(cuda_lib.fp8_mx_gemm_sumsq_workspace_bytes(g), dtype=torch.uint8, device="cuda")
+    out = torch.zeros(1, dtype=torch.float64, device="cuda")
+    _run_expired(cuda_lib, 2, lambda: cuda_lib.fp8_mx_gemm_multi_sumsq(g, out, ws))
+    assert np.isnan(out.item()) and not ws[:8].any()
+    cuda_lib.fp8_mx_gemm_multi_sumsq(g, out, ws)
+    cuda_lib.fp8t_check_device_error()
+    d = g[0]["D"].float().double()
+    assert abs(out.item() - float((d * d).sum())) <= 1e-12 * float((d * d).sum())
