@@ -190,3 +190,44 @@ def test_mx_gemm_sum_of_squares(cuda_lib, shapes):
     cuda_lib.fp8_mx_gemm_multi_sumsq(descs, out, ws)
     cuda_lib.fp8t_check_device_error()
     assert np.float64(out.item()).view(np.uint64) == np.float64(first).view(np.uint64)
+
+
+def test_mx_grouped_launch_7b_block_shapes_sampled(cuda_lib):
+    """One block-scaled launch with the fprop, dgrad and wgrad of three 7B-block projections
+    (q 4096 -> 4096, gate 4096 -> 11008, down 11008 -> 4096) at 256 tokens: nine problems with
+    4096- and 11008-wide outputs (11008 leaves a column tile with no rows for the N = 128 MMA) and
+    K of 256, 4096 and 11008, codes and scales from the library's MX cast. 1024 sampled outputs of
+    each against the oracle, and the sum of squares of the three wgrad outputs against numpy's."""
+    T, E = 256, oracle.E4M3
+    layers = [(4096, 4096), (4096, 11008), (11008, 4096)]
+    gen = torch.Generator(device="cuda").manual_seed(77)
+    descs, refs = [], []
+    for li, (fin, fout) in enumerate(layers):
+        X = (torch.randn(T, fin, generator=gen, device="cuda") * 2).to(torch.bfloat16)
+        W = (torch.randn(fin, fout, generator=gen, device="cuda") * 0.02).to(torch.bfloat16)
+        dY = (torch.randn(T, fout, generator=gen, device="cuda") * 1e-3).to(torch.bfloat16)
+        xq, wq, dq = (mx_cast(cuda_lib, bf16_bits(t), E) for t in (X, W, dY))
+        Y = torch.empty(T, fout, dtype=torch.bfloat16, device="cuda")
+        dX = torch.empty(T, fin, dtype=torch.bfloat16, device="cuda")
+        dW = torch.empty(fin, fout, dtype=torch.bfloat16, device="cuda")
+        descs += [dict(A=xq[0], a_sf=xq[1], a_fmt=E, B=wq[2], b_sf=wq[3], b_mn=True, b_fmt=E, D=Y),
+                  dict(A=dq[0], a_sf=dq[1], a_fmt=E, B=wq[0], b_sf=wq[1], b_fmt=E, D=dX),
+                  dict(A=xq[2], a_sf=xq[3], a_mn=True, a_fmt=E, B=dq[2], b_sf=dq[3], b_mn=True,
+                       b_fmt=E, D=dW, sumsq=True)]
+        hx = (u8(xq[0]), from_atoms(xq[1], T, fin), u8(xq[2]), from_atoms(xq[3], fin, T))
+        hw = (u8(wq[0]), from_atoms(wq[1], fin, fout), u8(wq[2]), from_atoms(wq[3], fout, fin))
+        hd = (u8(dq[0]), from_atoms(dq[1], T, fout), u8(dq[2]), from_atoms(dq[3], fout, T))
+        refs += [(Y, hx[0], hx[1], hw[2].T, hw[3]), (dX, hd[0], hd[1], hw[0], hw[1]),
+                 (dW, hx[2].T, hx[3], hd[2].T, hd[3])]
+    ws = torch.zeros(cuda_lib.fp8_mx_gemm_sumsq_workspace_bytes(descs), dtype=torch.uint8, device="cuda")
+    out = torch.zeros(1, dtype=torch.float64, device="cuda")
+    cuda_lib.fp8_mx_gemm_multi_sumsq(descs, out, ws)
+    cuda_lib.fp8t_check_device_error()
+    for k, (D, A, sa, B, sb) in enumerate(refs):
+        ii, jj = sample_positions(D.shape[0], D.shape[1], 1024, seed=300 + k)
+        R, ab = oracle.mx_gemm_at(np.ascontiguousarray(A), sa, E, np.ascontiguousarray(B), sb, E, ii, jj)
+        assert gemm_within_tolerance(bf16_bits(D)[ii, jj], R, ab).all(), f"problem {k}"
+    squares = np.concatenate([np.square(d["D"].float().cpu().numpy().astype(np.float64)).reshape(-1)
+                              for d in descs if d.get("sumsq")])
+    exact = float(np.sum(np.sort(squares)))
+    assert abs(out.item() - exact) <= 1e-13 * exact and not ws[:8].any()
