@@ -231,3 +231,33 @@ def test_mx_grouped_launch_7b_block_shapes_sampled(cuda_lib):
                               for d in descs if d.get("sumsq")])
     exact = float(np.sum(np.sort(squares)))
     assert abs(out.item() - exact) <= 1e-13 * exact and not ws[:8].any()
+
+
+@pytest.mark.parametrize("wide", [True, False], ids=["256x384-tiles", "256x256-tiles"])
+def test_mx_gemm_26_problems_two_launches_with_sum_of_squares(cuda_lib, wide):
+    """26 block-scaled problems are more than one launch table holds: two launches share one sum
+    of squares (slots numbered over the call, the second launch reduces them). Every output
+    against the oracle, the sum against numpy's, the workspace left at zero."""
+    shapes = [(128, 512, 256), (256, 640, 128), (128, 1152, 128)] if wide else \
+             [(128, 512, 256), (256, 256, 128), (128, 384, 128)]
+    descs, refs = [], []
+    for i in range(26):
+        M, N, K = shapes[i % 3]
+        (qa, sa), _ = mx_operands(M, K, oracle.E4M3, 1300 + i)
+        (qb, sb), _ = mx_operands(N, K, oracle.E4M3, 1400 + i)
+        descs.append(dict(A=torch.from_numpy(qa).cuda(), a_sf=to_atoms(sa), a_fmt=oracle.E4M3,
+                          B=torch.from_numpy(qb).cuda(), b_sf=to_atoms(sb), b_fmt=oracle.E4M3,
+                          sumsq=(i % 3 == 1) or i == 25,
+                          D=torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")))
+        refs.append((qa, sa, qb, sb))
+    ws = torch.zeros(cuda_lib.fp8_mx_gemm_sumsq_workspace_bytes(descs), dtype=torch.uint8, device="cuda")
+    out = torch.zeros(1, dtype=torch.float64, device="cuda")
+    cuda_lib.fp8_mx_gemm_multi_sumsq(descs, out, ws)
+    cuda_lib.fp8t_check_device_error()
+    for d, (qa, sa, qb, sb) in zip(descs, refs):
+        R, ab = oracle.mx_gemm(qa, sa, oracle.E4M3, qb, sb, oracle.E4M3, want_abs=True)
+        assert gemm_within_tolerance(bf16_bits(d["D"]), R, ab).all()
+    squares = np.concatenate([np.square(d["D"].float().cpu().numpy().astype(np.float64)).reshape(-1)
+                              for d in descs if d["sumsq"]])
+    exact = float(np.sum(np.sort(squares)))
+    assert abs(out.item() - exact) <= 1e-13 * exact and not ws[:8].any()
