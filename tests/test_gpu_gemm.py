@@ -253,3 +253,53 @@ def test_wide_tiles_with_sum_of_squares(cuda_lib, shapes):
     cuda_lib.fp8_gemm_multi_sumsq(descs, out, ws)
     cuda_lib.fp8t_check_device_error()
     assert np.float64(out.item()).view(np.uint64) == np.float64(first).view(np.uint64)
+
+
+def tile_samples(M, N, per_tile, seed):
+    """per_tile positions inside every 256 x 512 output tile (so split tiles are always hit)."""
+    rng = np.random.default_rng(seed)
+    ti, tj = np.meshgrid(np.arange(-(-M // 256)), np.arange(-(-N // 512)), indexing="ij")
+    ti, tj = np.repeat(ti.reshape(-1), per_tile), np.repeat(tj.reshape(-1), per_tile)
+    ii = np.minimum(ti * 256 + rng.integers(0, 256, ti.size), M - 1)
+    jj = np.minimum(tj * 512 + rng.integers(0, 512, tj.size), N - 1)
+    return ii, jj
+
+
+def test_step_gemms_summed_full_size_every_tile_sampled(cuda_lib):
+    """The 4096-class step's three GEMMs as the step issues them with the wgrad sum of squares
+    (fp8_gemm_multi_sumsq): the schedule gives some clusters 256-column halves of tiles, so
+    eight outputs of every 256 x 512 tile of every problem are checked against the oracle, and
+    the sum of squares against numpy's over the whole of dW. A second call with other X codes
+    gives the same agreement (nothing carried over from the first)."""
+    T, fin, fout = 8192, 4096, 4096
+    Wq = random_codes(fin, fout, oracle.E4M3, 2)
+    dYq = random_codes(T, fout, oracle.E5M2, 3)
+    s = [dev_scalar(v) for v in (0.011, 0.023, 0.5)]
+    Y = torch.empty(T, fout, dtype=torch.bfloat16, device="cuda")
+    dX = torch.empty(T, fin, dtype=torch.bfloat16, device="cuda")
+    dW = torch.empty(fin, fout, dtype=torch.bfloat16, device="cuda")
+    ws, out = None, torch.zeros(1, dtype=torch.float64, device="cuda")
+    hW, hdY = u8(Wq), u8(dYq)
+    for call, xseed in enumerate((1, 11)):
+        Xq = random_codes(T, fin, oracle.E4M3, xseed)
+        descs = [
+            dict(A=Xq, a_fmt=0, B=Wq, b_mn=True, b_fmt=0, a_scale_inv=s[0], b_scale_inv=s[1], D=Y),
+            dict(A=dYq, a_fmt=1, B=Wq, b_fmt=0, a_scale_inv=s[2], b_scale_inv=s[1], D=dX),
+            dict(A=Xq, a_mn=True, a_fmt=0, B=dYq, b_mn=True, b_fmt=1, a_scale_inv=s[0],
+                 b_scale_inv=s[2], D=dW, sumsq=True)]
+        if ws is None:
+            ws = torch.zeros(cuda_lib.fp8_gemm_sumsq_workspace_bytes(descs), dtype=torch.uint8,
+                             device="cuda")
+        cuda_lib.fp8_gemm_multi_sumsq(descs, out, ws)
+        cuda_lib.fp8t_check_device_error()
+        hX = u8(Xq)
+        for D, A, af, B, bf, sa, sb in ((Y, hX, 0, hW.T, 0, 0.011, 0.023), (dX, hdY, 1, hW, 0, 0.5, 0.023),
+                                        (dW, hX.T, 0, hdY.T, 1, 0.011, 0.5)):
+            ii, jj = tile_samples(D.shape[0], D.shape[1], 8, seed=D.shape[1] + call)
+            R, ab = oracle.gemm_at(np.ascontiguousarray(A), af, np.ascontiguousarray(B), bf, sa, sb, ii, jj)
+            ok = gemm_within_tolerance(bf16_bits(D)[ii, jj], R, ab)
+            assert ok.all(), f"call {call}: {(~ok).sum()} of {ok.size} outside tolerance"
+        sq = np.square(f32(dW.float()).astype(np.float64)).reshape(-1)
+        exact = float(np.sum(np.sort(sq)))
+        assert abs(out.item() - exact) <= 1e-13 * exact
+        assert ws[:8].view(torch.int32).eq(0).all()
